@@ -1,0 +1,199 @@
+/*
+ * ttq.h — C ABI of libttq, the sm_100a hot path of TTQ (activation-aware
+ * test-time quantization).
+ *
+ * Source of the method: "TTQ: Activation-Aware Test-Time Quantization to
+ * Accelerate LLM Inference On The Fly" (Koike-Akino, Liu, Wang; arXiv
+ * 2603.19296), as summarised by the nubint.ai review of that paper (cited
+ * below as "TTQ review"), section "Proposed method" (제안 방법), bullets 1-7:
+ *   1  weights are quantized on the fly with group-wise RTN and QDQ;
+ *   2  AWQ with a closed form built on a diagonal approximation of the input
+ *      covariance;
+ *   3  activation statistics are estimated online per prompt, the covariance
+ *      is shrunk (C_lambda), the target is L = E_X ||(W - W_hat) X||^2;
+ *   4  alpha, lambda, p are fixed (no search at test time);
+ *   5  optional low-rank factors: W = W_q + B A;
+ *   6  the overhead vanishes as d' and T grow;
+ *   7  a CUDA GEMM kernel runs the quantized projection.
+ *
+ * Per prompt and per linear layer the hot path is four calls on one stream:
+ *   ttq_act_stats -> ttq_awq_scales -> ttq_quantize_rtn_grouped
+ *   -> ttq_w_lowbit_gemm (optionally with the low-rank term).
+ *
+ * Notation. X is [T, K] (tokens x input channels, row-major, row pitch ldx
+ * elements). W is [N, K] (output x input, the PyTorch Linear layout, row
+ * pitch ldw). Y = X diag(1/s) W_hat^T is [T, N] (row pitch ldy). A group is
+ * g consecutive input channels of one weight row.
+ *
+ * Conventions shared by every call.
+ *   - Pointers named X, W, Y, sum, s, inv_s, codes, delta, zero, A, B,
+ *     workspace are DEVICE pointers owned by the caller. The library
+ *     allocates nothing, frees nothing and keeps no pointer after a call
+ *     returns.
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Every call only enqueues work; none synchronises the host.
+ *   - Argument checks happen before any launch. A bad argument returns
+ *     TTQ_ERR_INVALID_ARG (or TTQ_ERR_UNSUPPORTED for a valid but
+ *     unimplemented combination) and enqueues nothing. A failed launch
+ *     returns TTQ_ERR_CUDA. The library never aborts the process.
+ *   - Faults found on the device (a bounded wait that gave up, an fp16 range
+ *     overflow) set a sticky device error word; ttq_device_error() reads it.
+ *   - All device pointers must be 16-byte aligned; ldx, ldw, ldy must make
+ *     every row start 16-byte aligned.
+ */
+#ifndef TTQ_H_
+#define TTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTQ_OK = 0,
+  TTQ_ERR_INVALID_ARG = 1, /* bad pointer, size, pitch, alignment or enum  */
+  TTQ_ERR_UNSUPPORTED = 2, /* valid request this build does not implement */
+  TTQ_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed         */
+  TTQ_ERR_TIMEOUT = 4,     /* a device-side bounded wait gave up           */
+  TTQ_ERR_RANGE = 5        /* an fp16 operand overflowed on the device     */
+} ttq_status;
+
+typedef enum { TTQ_F32 = 0, TTQ_BF16 = 1, TTQ_F16 = 2 } ttq_dtype;
+
+/* Fixed hyperparameters of one layer (TTQ review, Proposed method, bullet 4:
+ * alpha, lambda, p are fixed; bullet 1: b bits, group g). */
+typedef struct {
+  int bits;     /* b, 2..8                                     */
+  int group;    /* g, one of 16, 32, 64, 128                   */
+  float alpha;  /* AWQ exponent, >= 0                          */
+  float lambda; /* shrinkage weight, in [0, 1]                 */
+  float p;      /* moment order of the channel statistic, > 0  */
+} ttq_params;
+
+/* Sticky device error bits (read with ttq_device_error). */
+#define TTQ_DEVERR_TIMEOUT 0x1u    /* a bounded wait inside a kernel gave up */
+#define TTQ_DEVERR_FP16_RANGE 0x2u /* |x / s| exceeded the fp16 range        */
+
+/* ---------------------------------------------------------------------
+ * Packed code layout (TTQ review, Proposed method, bullet 1: group-wise
+ * RTN; the pages fix no storage format, this one is ours).
+ *
+ * Row n of the codes array holds K/32 blocks; block k holds the codes of
+ * input channels 32k .. 32k+31 in `bits` consecutive uint32 words. Inside a
+ * block the codes form a little-endian bit stream: the code of channel
+ * 32k + c occupies bits [c*bits, c*bits + bits) of the block, where bit i of
+ * the block is bit (i % 32) of word (i / 32). A row therefore spans
+ * K*bits/32 words and the array is [N][K*bits/32] uint32, row-major, dense.
+ *
+ * delta is [N][K/g] float32 (row-major, dense), zero is [N][K/g] uint8.
+ * The scaled-domain weight of channel j in row n is
+ *     W_hat_s[n][j] = (q[n][j] - zero[n][j/g]) * delta[n][j/g]
+ * and the effective weight is W_hat_s[n][j] / s[j].
+ * ------------------------------------------------------------------- */
+
+/* Step 1, online activation statistics (TTQ review, Proposed method,
+ * bullets 2-3: the diagonal of the input covariance, estimated per prompt).
+ *
+ * sum_out[j] (+)= sum_t |X[t][j]|^p, accumulated in fp32, for j < K.
+ *   X      [T, K] of dtype xt (F32, BF16 or F16), row pitch ldx elements.
+ *   p      > 0. p == 2 gives the diagonal of the uncentred X^T X.
+ *   accumulate  0: overwrite sum_out; 1: add to it (chunked long prompts).
+ * Requires K % 8 == 0 and T >= 1. The reduction order is fixed, so the
+ * result is bit-reproducible run to run. */
+ttq_status ttq_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                         int64_t ldx, float p, int accumulate, float* sum_out,
+                         void* stream);
+
+/* Step 2, AWQ scales from the shrunk diagonal covariance (TTQ review,
+ * Proposed method, bullets 2-4).
+ *   m_j   = sum[j] / T_total
+ *   mbar  = (1/K) sum_j m_j
+ *   c_j   = (1 - lambda) m_j + lambda mbar        (shrink toward the mean)
+ *   s_j   = c_j^(alpha/p); s_j = 1 when alpha == 0 or c_j <= 0 or not finite
+ *   inv_s_j = 1 / s_j
+ * Computed in fp64 on the device and stored as fp32. Only prm->alpha,
+ * prm->lambda and prm->p are read. */
+ttq_status ttq_awq_scales(const float* sum, int64_t T_total, int64_t K,
+                          const ttq_params* prm, float* s, float* inv_s,
+                          void* stream);
+
+/* Step 3, group-wise RTN of the scaled weights (TTQ review, Proposed
+ * method, bullet 1). For row n and group G, in fp32 with IEEE round-to-
+ * nearest-even for every operation and no fused multiply-add:
+ *   w_j  = float(W[n][j]) * s_j                  (s == NULL means s_j = 1)
+ *   mn   = min(0, min_G w_j),  mx = max(0, max_G w_j)
+ *   D    = (mx - mn) / (2^b - 1);  D = 1 when it is 0
+ *   r    = 1 / D
+ *   z    = clamp(rint(-mn * r), 0, 2^b - 1)
+ *   q_j  = clamp(rint(w_j * r) + z, 0, 2^b - 1)
+ * Outputs codes (layout above), delta = D, zero = z.
+ *   W      [N, K] of dtype wt, row pitch ldw.
+ * Requires 2 <= bits <= 8, group in {16,32,64,128}, K % 32 == 0,
+ * K % group == 0. Bit-exact and deterministic. */
+ttq_status ttq_quantize_rtn_grouped(const void* W, ttq_dtype wt, int64_t N,
+                                    int64_t K, int64_t ldw, const float* s,
+                                    int bits, int group, uint32_t* codes,
+                                    float* delta, uint8_t* zero, void* stream);
+
+/* Bytes of workspace ttq_w_lowbit_gemm needs for a T x K input. */
+size_t ttq_w_lowbit_gemm_workspace_size(int64_t T, int64_t K, int r);
+
+/* Step 4, the quantized projection with dequantisation inside the GEMM
+ * (TTQ review, Proposed method, bullets 1 and 7; bullet 5 for the optional
+ * low-rank term):
+ *   Y[t][n] = sum_j (X[t][j] * inv_s[j]) * (q[n][j] - z) * D
+ *             + sum_rho (sum_j X[t][j] A[rho][j]) * B[n][rho]   (if r > 0)
+ *   X      [T, K] of dtype xt, row pitch ldx.
+ *   inv_s  [K] float32 (from ttq_awq_scales).
+ *   codes, delta, zero: from ttq_quantize_rtn_grouped for an [N, K] weight.
+ *   A      [r, K], B [N, r], dtype xt, dense; NULL with r == 0 for none.
+ *   Y      [T, N] of dtype yt (F32, BF16 or F16), row pitch ldy.
+ *   workspace  device buffer of at least
+ *              ttq_w_lowbit_gemm_workspace_size(T, K, r) bytes; its contents
+ *              are scratch and are overwritten.
+ * The tensor cores take fp16 operands: X / s is rounded once to fp16 and
+ * each weight (q - z) * D once to fp16; products accumulate in fp32.
+ * |X / s| must stay below 65504 (else TTQ_DEVERR_FP16_RANGE is raised).
+ * T <= 16 runs the decode (skinny) configuration, larger T the prefill one.
+ * Requires K % 32 == 0, K % group == 0, 0 <= r <= 64. */
+ttq_status ttq_w_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
+                             int64_t K, int64_t ldx, const float* inv_s,
+                             const uint32_t* codes, const float* delta,
+                             const uint8_t* zero, int64_t N, int bits,
+                             int group, const void* A, const void* B, int r,
+                             void* Y, ttq_dtype yt, int64_t ldy,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* The low-rank term alone (TTQ review, Proposed method, bullet 5; Main
+ * results, bullet 4): Y[t][n] += sum_rho (sum_j X[t][j] A[rho][j]) B[n][rho].
+ * X [T, K], A [r, K], B [N, r] of dtype xt; Y [T, N] of dtype yt, pitch ldy.
+ * Accumulates in fp32; 1 <= r <= 64. */
+ttq_status ttq_lowrank_add(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                           int64_t ldx, const void* A, const void* B, int r,
+                           int64_t N, void* Y, ttq_dtype yt, int64_t ldy,
+                           void* stream);
+
+/* Expand packed codes to one uint8 per weight: q_out [N][K] (device).
+ * Inverse of the packing in ttq_quantize_rtn_grouped. */
+ttq_status ttq_unpack_codes(const uint32_t* codes, int64_t N, int64_t K,
+                            int bits, uint8_t* q_out, void* stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char* ttq_status_string(ttq_status status);
+
+/* Reads the sticky device error word of the current device (a
+ * synchronising copy; call it outside the hot loop). Clears it when clear
+ * is non-zero. Returns the TTQ_DEVERR_* bits, or -1 if the copy failed. */
+int ttq_device_error(int clear);
+
+/* ABI version of this header. */
+int ttq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTQ_H_ */
