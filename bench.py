@@ -1,0 +1,546 @@
+#!/usr/bin/env python3
+"""Throughput of the TTQ hot path: prompt tokens/s per layer, including the
+on-the-fly quantization.
+
+One step is one pass of the whole path over one prompt of the workload: for
+every distinct layer input, statistics -> scales -> prepared fp16 operand;
+for every layer, group RTN of its weight -> tensor-core low-bit projection.
+The default workload is an OPT-125M-shaped block (q, k, v, o 768x768, fc1
+3072x768, fc2 768x3072; q, k, v share one input), T = 2048, b = 3, g = 32.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs an independent replica
+(the path has no exchange step), the timed region is bracketed by a barrier
+and a device synchronisation, and the slowest rank's time counts.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs  # noqa
+
+METRIC = "prompt tokens/s per layer incl. on-the-fly quant"
+L2_BYTES = 126 * 1024 * 1024
+ORACLE_SAMPLE_TOKENS = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="opt125m-block",
+                    choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained",
+                                               d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------ workload ----
+
+class Step:
+    """Device buffers and the launch sequence of one step."""
+
+    def __init__(self, ttq, wl, data, device, replicas):
+        self.ttq, self.wl = ttq, wl
+        self.T = wl.T
+        self.inputs = sorted(data["X"])
+        self.layers = list(wl.layers)
+        self.R = replicas
+        self.X = [{k: v.to(device) for k, v in data["X"].items()}
+                  for _ in range(replicas)]
+        self.W = [{k: v.to(device) for k, v in data["W"].items()}
+                  for _ in range(replicas)]
+        self.A = {k: v.to(device) for k, v in data["A"].items()}
+        self.B = {k: v.to(device) for k, v in data["B"].items()}
+        f32 = dict(dtype=torch.float32, device=device)
+        self.sums = {k: torch.empty(self.X[0][k].shape[1], **f32)
+                     for k in self.inputs}
+        self.s = {k: torch.empty_like(v) for k, v in self.sums.items()}
+        self.inv = {k: torch.empty_like(v) for k, v in self.sums.items()}
+        self.Xs = {k: torch.empty(self.X[0][k].shape, dtype=torch.float16,
+                                  device=device) for k in self.inputs}
+        r = wl.rank
+        self.U = {k: torch.empty((self.T, 64), dtype=torch.float16,
+                                 device=device) for k in self.inputs} if r \
+            else {}
+        b, g = wl.bits, wl.group
+        self.codes, self.delta, self.zero, self.Y = {}, {}, {}, {}
+        for L in self.layers:
+            self.codes[L.name] = torch.empty((L.N, L.K * b // 32),
+                                             dtype=torch.int32, device=device)
+            self.delta[L.name] = torch.empty((L.N, L.K // g), **f32)
+            self.zero[L.name] = torch.empty((L.N, L.K // g), dtype=torch.uint8,
+                                            device=device)
+            self.Y[L.name] = torch.empty((self.T, L.N), dtype=wl.dtype,
+                                         device=device)
+
+    def input_bytes(self):
+        return sum(v.numel() * v.element_size() for v in self.X[0].values()) + \
+            sum(v.numel() * v.element_size() for v in self.W[0].values())
+
+    def calls(self, rep):
+        """(kind, callable) in launch order for replica ``rep``."""
+        t, wl = self.ttq, self.wl
+        X, W = self.X[rep], self.W[rep]
+        out = []
+        for k in self.inputs:
+            A = None
+            if wl.rank:
+                # the low-rank factors belong to a layer; layers that share
+                # an input in these workloads never both carry factors
+                owners = [L.name for L in self.layers if L.input_name == k]
+                A = self.A[owners[0]]
+            out.append(("stats", lambda k=k: t.act_stats(X[k], wl.p,
+                                                         out=self.sums[k])))
+            out.append(("scales", lambda k=k: t.awq_scales(
+                self.sums[k], self.T, wl.alpha, wl.lam, wl.p, self.s[k],
+                self.inv[k])))
+            out.append(("prepare", lambda k=k, A=A: t.prepare_activations(
+                X[k], self.inv[k], A, self.Xs[k], self.U.get(k))))
+        for L in self.layers:
+            k, n = L.input_name, L.name
+            out.append(("quantize", lambda k=k, n=n: t.quantize_rtn_grouped(
+                W[n], self.s[k], wl.bits, wl.group, self.codes[n],
+                self.delta[n], self.zero[n])))
+            out.append(("gemm", lambda k=k, n=n, L=L: t.w_lowbit_gemm_prepared(
+                self.Xs[k], self.U.get(k), self.codes[n], self.delta[n],
+                self.zero[n], L.N, wl.bits, wl.group,
+                self.B.get(n) if wl.rank else None, out=self.Y[n])))
+        return out
+
+    def run(self, rep, events=None):
+        for i, (kind, fn) in enumerate(self.calls(rep)):
+            if events is not None:
+                events[i][0].record()
+            fn()
+            if events is not None:
+                events[i][1].record()
+
+
+def algorithmic_work(wl):
+    """Bytes (HBM-bound steps) and flops (projection) per step, from the
+    algorithmic minimum: every input read once, every output written once."""
+    T, b, g = wl.T, wl.bits, wl.group
+    xb = 2 if wl.dtype != torch.float32 else 4
+    seen, w = set(), {"stats": 0, "scales": 0, "prepare": 0, "quantize": 0,
+                      "gemm": 0, "gemm_flops": 0}
+    for L in wl.layers:
+        if L.input_name not in seen:
+            seen.add(L.input_name)
+            w["stats"] += T * L.K * xb + L.K * 4
+            w["scales"] += L.K * 12
+            w["prepare"] += T * L.K * (xb + 2) + L.K * 4
+        w["quantize"] += L.N * L.K * xb + L.K * 4 + L.N * L.K * b // 8 + \
+            5 * L.N * L.K // g
+        w["gemm"] += T * L.K * 2 + L.N * L.K * b // 8 + 5 * L.N * L.K // g + \
+            T * L.N * xb
+        w["gemm_flops"] += 2 * T * L.N * L.K + 2 * T * wl.rank * (L.K + L.N)
+    return w
+
+
+# -------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu),
+                 f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "samples": len(rows),
+                "reasons": reasons}
+
+
+# ------------------------------------------------------------- oracle -----
+
+def oracle_step(wl, data, sample_tokens):
+    """The CPU oracle on a bounded sample of one step: statistics, scales and
+    quantization at full size, the projection on the first ``sample_tokens``
+    tokens, scaled linearly to T. Returns (seconds per step, description)."""
+    import numpy as np
+    import oracle
+    T = wl.T
+    Ts = min(sample_tokens, T)
+    Xn = {k: v.float().numpy() for k, v in data["X"].items()}
+    t0 = time.perf_counter()
+    s, inv = {}, {}
+    for k, X in Xn.items():
+        sums = oracle.act_sums(X, wl.p)
+        s[k], inv[k] = oracle.awq_scales(sums, T, wl.alpha, wl.lam, wl.p)
+    t_full = time.perf_counter() - t0
+    t_gemm = 0.0
+    for L in wl.layers:
+        W = data["W"][L.name].float().numpy()
+        t1 = time.perf_counter()
+        c, d, z = oracle.quantize(W, s[L.input_name].astype(np.float32),
+                                  wl.bits, wl.group)
+        t_full += time.perf_counter() - t1
+        A = B = None
+        if wl.rank:
+            A = data["A"][L.name].float().numpy()
+            B = data["B"][L.name].float().numpy()
+        t2 = time.perf_counter()
+        oracle.lowbit_gemm(Xn[L.input_name][:Ts], inv[L.input_name], c, d, z,
+                           L.N, wl.bits, wl.group, A, B)
+        t_gemm += time.perf_counter() - t2
+    est = t_full + t_gemm * (T / Ts)
+    desc = (f"stats, scales and quantize at full size; projection on {Ts} of "
+            f"{T} tokens scaled x{T / Ts:g}; 1 thread")
+    return est, desc
+
+
+# ---------------------------------------------------------------- main ----
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_reference(args, wl):
+    """The oracle as it stands, on the host cores, each step a bounded
+    sample of the workload."""
+    torch.set_num_threads(1)
+    data = make_inputs(wl)
+    sample = 16
+    for _ in range(args.warmup):
+        oracle_step(wl, data, sample)
+    times = []
+    desc = ""
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        est, desc = oracle_step(wl, data, sample)
+        times.append(est)
+    wall = time.perf_counter() - t0
+    per_step = sum(times) / len(times)
+    value = len(wl.layers) * wl.T / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "T": wl.T, "bits": wl.bits,
+                   "group": wl.group, "layers": len(wl.layers)},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "test_weight_quantization_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def traffic_from_profiles(kind, workload):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or
+    None when absent or taken on a different kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kind}/{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_step")
+
+
+def main():
+    args = parse()
+    wl = WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, wl)
+        return
+    from test_weight_quantization_b200 import ttq
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    data = make_inputs(wl)
+
+    probe = Step(ttq, wl, data, device, 1)
+    rep = max(2, math.ceil(2.5 * L2_BYTES / probe.input_bytes()))
+    del probe
+    step = Step(ttq, wl, data, device, rep)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+
+    # eager warm-up (loads kernels, sets attributes), then capture
+    with torch.cuda.stream(stream):
+        for r in range(rep):
+            step.run(r)
+    stream.synchronize()
+    ttq.device_error(clear=True)
+    calls = step.calls(0)
+    kinds = [k for k, _ in calls]
+    graphs, igraphs = [], []
+    # external events record timestamps when replayed inside a graph
+    ev = [[[torch.cuda.Event(enable_timing=True, external=True)
+            for _ in range(2)] for _ in calls] for _ in range(rep)]
+    for r in range(rep):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step.run(r)
+        graphs.append(g)
+        gi = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gi, stream=stream):
+            step.run(r, ev[r])
+        igraphs.append(gi)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            graphs[i % rep].replay()
+    stream.synchronize()
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            start.record()
+            for i in range(args.steps):
+                graphs[i % rep].replay()
+            end.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    clocks = clk.summary()
+    ms_per_step = ms / args.steps
+    value = world * len(wl.layers) * wl.T / (ms_per_step / 1e3)
+
+    # per-kernel times: event-instrumented replays of the same step
+    with torch.cuda.stream(stream):
+        for r in range(rep):
+            igraphs[r].replay()
+    torch.cuda.synchronize()
+    per_kind = {}
+    for r in range(rep):
+        for i, kind in enumerate(kinds):
+            per_kind.setdefault(kind, 0.0)
+            per_kind[kind] += ev[r][i][0].elapsed_time(ev[r][i][1]) / rep
+    derr = ttq.device_error(clear=True)
+    if derr:
+        raise SystemExit(f"device error bits {derr:#x} raised during bench")
+
+    pk = peaks()
+    work = algorithmic_work(wl)
+    kernels = {}
+    for kind, msk in per_kind.items():
+        e = {"ms_per_step": msk, "launches_per_step": kinds.count(kind)}
+        if kind == "gemm":
+            e["tflops"] = work["gemm_flops"] / (msk / 1e3) / 1e12
+        e["gbs"] = work[kind] / (msk / 1e3) / 1e9
+        kernels[kind] = e
+    dom = max(per_kind, key=per_kind.get)
+    if dom == "gemm":
+        peak = pk["bf16_tflops_sustained"]
+        achieved = kernels["gemm"]["tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_kind": f"{pk['source']} bf16 sustained (fp16 dense rate "
+                             "= bf16 nominal)"}
+    else:
+        peak = pk["hbm_gbs"]
+        achieved = kernels[dom]["gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak,
+                "peak_kind": f"{pk['source']} HBM copy"}
+    roof["kernel"] = dom
+    roof["traffic"] = traffic_from_profiles(dom, wl.name)
+
+    # end to end through the binding: host buffers in, host buffers out
+    e2e = None
+    if not args.no_e2e:
+        e2e = end_to_end(ttq, wl, data, device, args, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS)
+        cpu = {"value": len(wl.layers) * wl.T / est, "unit": "tokens/s",
+               "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {
+                "workload": wl.name, "T": wl.T, "bits": wl.bits,
+                "group": wl.group,
+                "layers": ", ".join(f"{L.name} {L.N}x{L.K}"
+                                    for L in wl.layers),
+                "operands": "fp16 x fp16 -> fp32 (tensor cores); quantizer "
+                            "fp32; statistics fp32",
+                "l2": f"inputs rotate over {rep} replicas "
+                      f"({rep * step.input_bytes() / 2**20:.0f} MiB > L2)",
+                "parallelism": f"replicas x{world}", "graph": "CUDA graph per "
+                "replica"},
+            "roofline": roof, "kernels": kernels,
+            "gpu_launches": len(kinds) * args.steps,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs, igraphs
+        dist.destroy_process_group()
+
+
+def end_to_end(ttq, wl, data, device, args, stream, world):
+    """Same metric through the Python binding with host buffers: each step
+    copies its prompt activations from pinned host memory, runs the path
+    (eager calls, one per step of the method) and copies every output back.
+    The layer weights are the model's resident parameters and stay on the
+    device."""
+    step = Step(ttq, wl, data, device, 1)
+    hx = {k: v.pin_memory() for k, v in data["X"].items()}
+    hy = {L.name: torch.empty((wl.T, L.N), dtype=wl.dtype).pin_memory()
+          for L in wl.layers}
+    h2d = sum(v.numel() * v.element_size() for v in hx.values())
+    d2h = sum(v.numel() * v.element_size() for v in hy.values())
+
+    def one():
+        for k, v in hx.items():
+            step.X[0][k].copy_(v, non_blocking=True)
+        step.run(0)
+        for n, v in hy.items():
+            v.copy_(step.Y[n], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            one()
+    stream.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    steps = max(5, args.steps // 2)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        a.record()
+        for _ in range(steps):
+            one()
+        b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * len(wl.layers) * wl.T / (ms / 1e3),
+            "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+if __name__ == "__main__":
+    main()

@@ -167,6 +167,34 @@ ttq_status ttq_w_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
                              void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* The two halves of ttq_w_lowbit_gemm, for callers that reuse one prepared
+ * input across several projections of the same X (q, k, v share X and s)
+ * or time the tensor-core kernel alone.
+ *
+ * ttq_prepare_activations: the activation side of step 4.
+ *   Xs[t][j] = fp16(X[t][j] * inv_s[j])        Xs [T, K] fp16, dense
+ *   U[t][rho] = fp16(sum_j X[t][j] A[rho][j])  U [T, 64] fp16, dense, zero
+ *                                               for rho >= r (r > 0 only)
+ * A is [r, K] of dtype xt; pass A = U = NULL with r = 0.
+ * Raises TTQ_DEVERR_FP16_RANGE if |X * inv_s| reaches the fp16 range. */
+ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt, int64_t T,
+                                   int64_t K, int64_t ldx, const float* inv_s,
+                                   const void* A, int r, void* Xs, void* U,
+                                   void* stream);
+
+/* ttq_w_lowbit_gemm_prepared: the tensor-core projection on prepared
+ * operands, one kernel launch:
+ *   Y[t][n] = sum_j Xs[t][j] (q[n][j] - z) D + sum_rho U[t][rho] B[n][rho].
+ * Xs, U as written by ttq_prepare_activations; B [N, r] of dtype bt. */
+ttq_status ttq_w_lowbit_gemm_prepared(const void* Xs, const void* U,
+                                      int64_t T, int64_t K,
+                                      const uint32_t* codes,
+                                      const float* delta, const uint8_t* zero,
+                                      int64_t N, int bits, int group,
+                                      const void* B, ttq_dtype bt, int r,
+                                      void* Y, ttq_dtype yt, int64_t ldy,
+                                      void* stream);
+
 /* The low-rank term alone (TTQ review, Proposed method, bullet 5; Main
  * results, bullet 4): Y[t][n] += sum_rho (sum_j X[t][j] A[rho][j]) B[n][rho].
  * X [T, K], A [r, K], B [N, r] of dtype xt; Y [T, N] of dtype yt, pitch ldy.

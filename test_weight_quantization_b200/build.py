@@ -1,0 +1,106 @@
+"""Builds libttq.so (the CUDA kernels behind include/ttq.h) for sm_100a.
+
+    python -m test_weight_quantization_b200.build [--force] [--verbose]
+
+Each ``csrc/*.cu`` is compiled by nvcc into ``_build/`` and linked into
+``test_weight_quantization_b200/libttq.so`` (in-tree, so the built library
+travels with the source tree). A file is recompiled only when it, a header it
+may include, or the flags changed. nvcc cross-compiles: no GPU is needed.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import glob
+import hashlib
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+BUILD = os.path.join(ROOT, "_build")
+LIB = os.path.join(PKG, "libttq.so")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+                     "-Xcompiler", "-fvisibility=hidden",
+                     "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"),
+                 "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: set NVCC or add CUDA to PATH")
+
+
+def _digest(paths, extra) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(extra).encode())
+    return h.hexdigest()[:16]
+
+
+def _compile(src: str, headers, flags, verbose: bool) -> str:
+    stem = os.path.splitext(os.path.basename(src))[0]
+    digest = _digest([src] + headers, flags)
+    obj = os.path.join(BUILD, f"{stem}.{digest}.o")
+    if not os.path.exists(obj):
+        cmd = [nvcc(), *flags, "-c", src, "-o", obj + ".tmp"]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"nvcc failed on {src}:\n{res.stderr}")
+        if verbose and res.stderr:
+            sys.stderr.write(res.stderr)
+        os.replace(obj + ".tmp", obj)
+    return obj
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) +
+                     glob.glob(os.path.join(CSRC, "*.h")) +
+                     glob.glob(os.path.join(INCLUDE, "*.h")))
+    if force:
+        for o in glob.glob(os.path.join(BUILD, "*.o")):
+            os.remove(o)
+    with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        objs = list(ex.map(lambda s: _compile(s, headers, NVCC_FLAGS, verbose),
+                           sources))
+    link_key = _digest(objs, ["link"])
+    stamp = LIB + ".stamp"
+    if (force or not os.path.exists(LIB) or not os.path.exists(stamp)
+            or open(stamp).read() != link_key):
+        tmp = LIB + ".tmp"
+        cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp,
+               *objs, "-ldl", "-lrt", "-lpthread"]
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"link failed:\n{res.stderr}")
+        os.replace(tmp, LIB)
+        with open(stamp, "w") as f:
+            f.write(link_key)
+    return LIB
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true",
+                    help="print ptxas register/spill/shared-memory usage")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose))
+
+
+if __name__ == "__main__":
+    main()

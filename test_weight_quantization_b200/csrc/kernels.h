@@ -1,0 +1,55 @@
+// kernels.h — internal launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ttq.h"
+
+namespace ttq {
+
+ttq_status launch_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                            int64_t ldx, float p, int accumulate,
+                            float* sum_out, cudaStream_t st);
+
+ttq_status launch_awq_scales(const float* sum, int64_t T_total, int64_t K,
+                             double alpha, double lambda, double p, float* s,
+                             float* inv_s, cudaStream_t st);
+
+ttq_status launch_quantize(const void* W, ttq_dtype wt, int64_t N, int64_t K,
+                           int64_t ldw, const float* s, int bits, int group,
+                           uint32_t* codes, float* delta, uint8_t* zero,
+                           cudaStream_t st);
+
+ttq_status launch_unpack(const uint32_t* codes, int64_t N, int64_t K, int bits,
+                         uint8_t* q_out, cudaStream_t st);
+
+// Workspace carve-up of the projection.
+size_t gemm_workspace_bytes(int64_t T, int64_t K, int r);
+
+ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
+                              int64_t K, int64_t ldx, const float* inv_s,
+                              const uint32_t* codes, const float* delta,
+                              const uint8_t* zero, int64_t N, int bits,
+                              int group, const void* A, const void* B, int r,
+                              void* Y, ttq_dtype yt, int64_t ldy,
+                              void* workspace, cudaStream_t st);
+
+ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                          int64_t ldx, const float* inv_s, const void* A,
+                          int r, void* Xs, void* U, cudaStream_t st);
+
+ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
+                                int64_t K, const uint32_t* codes,
+                                const float* delta, const uint8_t* zero,
+                                int64_t N, int bits, int group, const void* B,
+                                ttq_dtype bt, int r, void* Y, ttq_dtype yt,
+                                int64_t ldy, cudaStream_t st);
+
+ttq_status launch_lowrank_add(const void* X, ttq_dtype xt, int64_t T,
+                              int64_t K, int64_t ldx, const void* A,
+                              const void* B, int r, int64_t N, void* Y,
+                              ttq_dtype yt, int64_t ldy, cudaStream_t st);
+
+}  // namespace ttq

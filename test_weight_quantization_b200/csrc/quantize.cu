@@ -1,0 +1,189 @@
+// quantize.cu — step 3 of TTQ: group-wise RTN of the scaled weights.
+//
+// TTQ review, "Proposed method", bullet 1: weights are quantized on the fly
+// with group-wise round-to-nearest. Per group of g input channels of one
+// weight row, in fp32 with explicit round-to-nearest-even operations (no
+// contraction into FMA), exactly as ttq.h states:
+//   w = W*s;  mn = min(0, min w);  mx = max(0, max w);
+//   D = (mx - mn)/(2^b - 1) (1 if 0);  r = 1/D;
+//   z = clamp(rint(-mn*r));  q = clamp(rint(w*r) + z).
+//
+// Design (HBM-bound): one warp per 256-channel segment of a row; a lane owns
+// 8 consecutive channels loaded as one 16-byte vector. A group spans g/8
+// lanes and its min/max is a butterfly shuffle inside that lane segment.
+// Four lanes hold one 32-code block; they exchange their 8*b-bit chunks by
+// shuffles and each lane stores the one or two packed words it owns, so a
+// warp writes 8*b consecutive words. Delta and zero go out from the first
+// lane of each group.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ttq {
+namespace {
+
+constexpr int kWarpsPerCta = 8;
+
+template <typename TW, int BITS>
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+    quantize_kernel(const TW* __restrict__ W, int64_t N, int64_t K,
+                    int64_t ldw, const float* __restrict__ s, int group,
+                    uint32_t* __restrict__ codes, float* __restrict__ delta,
+                    uint8_t* __restrict__ zero) {
+  const int lane = threadIdx.x & 31;
+  const int64_t segs = (K + 255) / 256;
+  const int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (item >= N * segs) return;  // whole warp exits together
+  const int64_t n = item / segs;
+  const int64_t col0 = (item % segs) * 256 + lane * 8;
+  const bool active = col0 < K;  // K % 32 == 0: whole blocks/groups agree
+
+  const float qmax = (float)((1 << BITS) - 1);
+  float w[8];
+  if (active) {
+    load8<TW>(W + n * ldw + col0, w);
+    if (s != nullptr) {
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + col0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + col0 + 4));
+      w[0] = __fmul_rn(w[0], s0.x); w[1] = __fmul_rn(w[1], s0.y);
+      w[2] = __fmul_rn(w[2], s0.z); w[3] = __fmul_rn(w[3], s0.w);
+      w[4] = __fmul_rn(w[4], s1.x); w[5] = __fmul_rn(w[5], s1.y);
+      w[6] = __fmul_rn(w[6], s1.z); w[7] = __fmul_rn(w[7], s1.w);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = 0.f;
+  }
+
+  // group range, widened to contain 0
+  float mn = 0.f, mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    mn = fminf(mn, w[i]);
+    mx = fmaxf(mx, w[i]);
+  }
+  const int lanes_per_group = group >> 3;
+  for (int o = 1; o < lanes_per_group; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  float d = __fdiv_rn(__fsub_rn(mx, mn), qmax);
+  if (d == 0.f) d = 1.f;
+  const float r = __frcp_rn(d);
+  const float z = fminf(fmaxf(rintf(__fmul_rn(-mn, r)), 0.f), qmax);
+
+  uint64_t chunk = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float v = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(w[i], r)), z), 0.f),
+                          qmax);
+    chunk |= (uint64_t)(uint32_t)v << (BITS * i);
+  }
+
+  // gather the four 8*BITS-bit chunks of this lane's 32-code block
+  const int qbase = lane & ~3;
+  const int qpos = lane & 3;
+  uint64_t c[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)chunk, qbase + j);
+    const uint32_t hi =
+        __shfl_sync(0xffffffffu, (uint32_t)(chunk >> 32), qbase + j);
+    c[j] = ((uint64_t)hi << 32) | lo;
+  }
+  if (active) {
+    const int64_t row_words = K * BITS / 32;
+    uint32_t* out = codes + n * row_words + (col0 / 32) * BITS;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int wi = qpos + 4 * half;  // word index inside the block
+      if (wi >= BITS) continue;
+      uint32_t word = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int lo_bit = 8 * BITS * j;  // chunk j spans [lo_bit, +8*BITS)
+        const int shift = lo_bit - 32 * wi;
+        if (lo_bit + 8 * BITS <= 32 * wi || lo_bit >= 32 * wi + 32) continue;
+        word |= shift >= 0 ? (uint32_t)(c[j] << shift)
+                           : (uint32_t)(c[j] >> (-shift));
+      }
+      out[wi] = word;
+    }
+    if ((lane & (lanes_per_group - 1)) == 0) {
+      const int64_t gi = n * (K / group) + col0 / group;
+      delta[gi] = d;
+      zero[gi] = (uint8_t)z;
+    }
+  }
+}
+
+template <typename TW>
+ttq_status launch_bits(const void* W, int64_t N, int64_t K, int64_t ldw,
+                       const float* s, int bits, int group, uint32_t* codes,
+                       float* delta, uint8_t* zero, cudaStream_t st) {
+  const int64_t items = N * ((K + 255) / 256);
+  const dim3 grid((unsigned)((items + kWarpsPerCta - 1) / kWarpsPerCta));
+  const dim3 block(kWarpsPerCta * 32);
+  const TW* w = static_cast<const TW*>(W);
+#define TTQ_Q(B)                                                              \
+  case B:                                                                     \
+    quantize_kernel<TW, B><<<grid, block, 0, st>>>(w, N, K, ldw, s, group,    \
+                                                   codes, delta, zero);       \
+    break;
+  switch (bits) {
+    TTQ_Q(2) TTQ_Q(3) TTQ_Q(4) TTQ_Q(5) TTQ_Q(6) TTQ_Q(7) TTQ_Q(8)
+    default:
+      return TTQ_ERR_INVALID_ARG;
+  }
+#undef TTQ_Q
+  return launch_status();
+}
+
+// q_out[n][j] = code of channel j; one thread per 32-code block.
+__global__ void unpack_kernel(const uint32_t* __restrict__ codes, int64_t N,
+                              int64_t K, int bits,
+                              uint8_t* __restrict__ q_out) {
+  const int64_t blocks = K / 32;
+  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= N * blocks) return;
+  const int64_t n = id / blocks, b = id % blocks;
+  const uint32_t* w = codes + n * (K * bits / 32) + b * bits;
+  const uint32_t mask = (1u << bits) - 1u;
+  uint8_t* out = q_out + n * K + b * 32;
+  for (int c = 0; c < 32; ++c) {
+    const int bit = c * bits, wi = bit >> 5, sh = bit & 31;
+    uint64_t v = w[wi] >> sh;
+    if (sh + bits > 32) v |= (uint64_t)w[wi + 1] << (32 - sh);
+    out[c] = (uint8_t)(v & mask);
+  }
+}
+
+}  // namespace
+
+ttq_status launch_quantize(const void* W, ttq_dtype wt, int64_t N, int64_t K,
+                           int64_t ldw, const float* s, int bits, int group,
+                           uint32_t* codes, float* delta, uint8_t* zero,
+                           cudaStream_t st) {
+  switch (wt) {
+    case TTQ_F32:
+      return launch_bits<float>(W, N, K, ldw, s, bits, group, codes, delta,
+                                zero, st);
+    case TTQ_BF16:
+      return launch_bits<__nv_bfloat16>(W, N, K, ldw, s, bits, group, codes,
+                                        delta, zero, st);
+    case TTQ_F16:
+      return launch_bits<__half>(W, N, K, ldw, s, bits, group, codes, delta,
+                                 zero, st);
+  }
+  return TTQ_ERR_INVALID_ARG;
+}
+
+ttq_status launch_unpack(const uint32_t* codes, int64_t N, int64_t K, int bits,
+                         uint8_t* q_out, cudaStream_t st) {
+  const int64_t total = N * (K / 32);
+  const int threads = 256;
+  unpack_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0,
+                  st>>>(codes, N, K, bits, q_out);
+  return launch_status();
+}
+
+}  // namespace ttq

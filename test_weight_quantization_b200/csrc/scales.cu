@@ -1,0 +1,56 @@
+// scales.cu — step 2 of TTQ: AWQ scales from the shrunk diagonal covariance.
+//
+// TTQ review, "Proposed method", bullets 2-4: AWQ with a closed form on the
+// diagonal input covariance, shrunk by lambda, hyperparameters fixed. With
+// m_j = sum_j / T:
+//   c_j = (1 - lambda) m_j + lambda mean_k(m_k),   s_j = c_j^(alpha/p).
+// O(K) work: one CTA, fp64 arithmetic (the result is stored as fp32), the
+// mean reduced in a fixed order.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ttq {
+namespace {
+
+constexpr int kThreads = 1024;
+
+__global__ void __launch_bounds__(kThreads)
+    awq_scales_kernel(const float* __restrict__ sum, int64_t T_total,
+                      int64_t K, double alpha, double lambda, double p,
+                      float* __restrict__ s, float* __restrict__ inv_s) {
+  __shared__ double warp_sums[kThreads / 32];
+  const double invT = 1.0 / (double)T_total;
+  double local = 0.0;
+  for (int64_t j = threadIdx.x; j < K; j += kThreads)
+    local += (double)sum[j] * invT;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+    local += __shfl_xor_sync(0xffffffffu, local, o);
+  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = local;
+  __syncthreads();
+  double total = 0.0;
+  for (int w = 0; w < kThreads / 32; ++w) total += warp_sums[w];
+  const double mbar = total / (double)K;
+  const double expo = alpha / p;
+
+  for (int64_t j = threadIdx.x; j < K; j += kThreads) {
+    const double m = (double)sum[j] * invT;
+    const double c = (1.0 - lambda) * m + lambda * mbar;
+    double sj = 1.0;
+    if (alpha != 0.0 && c > 0.0 && isfinite(c)) sj = pow(c, expo);
+    s[j] = (float)sj;
+    inv_s[j] = (float)(1.0 / sj);
+  }
+}
+
+}  // namespace
+
+ttq_status launch_awq_scales(const float* sum, int64_t T_total, int64_t K,
+                             double alpha, double lambda, double p, float* s,
+                             float* inv_s, cudaStream_t st) {
+  awq_scales_kernel<<<1, kThreads, 0, st>>>(sum, T_total, K, alpha, lambda, p,
+                                            s, inv_s);
+  return launch_status();
+}
+
+}  // namespace ttq

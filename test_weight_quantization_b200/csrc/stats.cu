@@ -1,0 +1,170 @@
+// stats.cu — step 1 of TTQ: per-input-channel activation statistics.
+//
+// TTQ review, "Proposed method", bullets 2-3: the per-prompt activation
+// statistic is the diagonal of the input covariance; here the kernel emits
+// sum_t |x_tj|^p (p = 2: the diagonal of X^T X) and the scales kernel
+// divides by the token count.
+//
+// Design (HBM-bound column reduction):
+//   - a thread owns 8 consecutive channels and loads them as one 16-byte
+//     vector (two for fp32); CW/8 threads cover a row segment of CW channels
+//     and the 256-thread CTA covers 256/(CW/8) rows per pass;
+//   - each CTA walks a contiguous range of rows with 8 independent loads in
+//     flight per thread, accumulating in fp32 registers;
+//   - rows split across a thread-block cluster of up to 8 CTAs; partial sums
+//     are reduced through distributed shared memory by cluster rank 0 in a
+//     fixed order, so the result is deterministic and no global scratch is
+//     needed.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace ttq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 8;
+
+template <int PK>
+__device__ __forceinline__ float moment(float x, float p) {
+  if (PK == 2) return x * x;
+  if (PK == 1) return fabsf(x);
+  return powf(fabsf(x), p);
+}
+
+// grid = (column tiles, cluster size); cluster = (1, C, 1).
+template <typename TX, int PK>
+__global__ void __launch_bounds__(kThreads)
+    act_stats_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
+                     int64_t ldx, float p, int accumulate, int cw,
+                     float* __restrict__ sum_out) {
+  extern __shared__ float smem[];  // [rows_per_pass][cw] then part[cw]
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tpr = cw / 8;                 // threads per row segment
+  const int rows_per_pass = kThreads / tpr;
+  const int tid = threadIdx.x;
+  const int lane_col = tid % tpr;
+  const int row_in_pass = tid / tpr;
+  const int64_t col0 = (int64_t)blockIdx.x * cw + lane_col * 8;
+  const bool col_ok = col0 < K;
+
+  const int C = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int64_t rows_per_cta = (T + C - 1) / C;
+  const int64_t r_begin = rank * rows_per_cta;
+  const int64_t r_end = min(T, r_begin + rows_per_cta);
+
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+
+  if (col_ok) {
+    int64_t r = r_begin + row_in_pass;
+    for (; r + (int64_t)(kUnroll - 1) * rows_per_pass < r_end;
+         r += (int64_t)kUnroll * rows_per_pass) {
+      float v[kUnroll][8];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        load8<TX>(X + (r + (int64_t)u * rows_per_pass) * ldx + col0, v[u]);
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(v[u][i], p);
+    }
+    for (; r < r_end; r += rows_per_pass) {
+      float v[8];
+      load8<TX>(X + r * ldx + col0, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(v[i], p);
+    }
+  }
+
+  // CTA reduction over the rows of a pass, fixed order.
+  float* red = smem;
+  float* part = smem + rows_per_pass * cw;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[row_in_pass * cw + lane_col * 8 + i] = acc[i];
+  __syncthreads();
+  for (int c = tid; c < cw; c += kThreads) {
+    float s = 0.f;
+    for (int rr = 0; rr < rows_per_pass; ++rr) s += red[rr * cw + c];
+    part[c] = s;
+  }
+  cluster.sync();
+
+  // Cluster reduction by rank 0, ranks in order.
+  if (rank == 0) {
+    for (int c = tid; c < cw; c += kThreads) {
+      const int64_t col = (int64_t)blockIdx.x * cw + c;
+      if (col >= K) continue;
+      float s = 0.f;
+      for (int q = 0; q < C; ++q) s += cluster.map_shared_rank(part, q)[c];
+      sum_out[col] = accumulate ? sum_out[col] + s : s;
+    }
+  }
+  cluster.sync();  // keep every CTA's shared memory alive until read
+}
+
+template <typename TX, int PK>
+ttq_status launch_typed(const void* X, int64_t T, int64_t K, int64_t ldx,
+                        float p, int accumulate, float* sum_out,
+                        cudaStream_t st) {
+  const int cw = K >= 1024 ? 128 : 64;
+  const int64_t col_tiles = (K + cw - 1) / cw;
+  const int target = 2 * sm_count();
+  int C = (int)std::min<int64_t>(
+      8, std::max<int64_t>(1, (target + col_tiles - 1) / col_tiles));
+  // keep at least 32 rows per CTA
+  C = (int)std::min<int64_t>(C, std::max<int64_t>(1, (T + 31) / 32));
+  const int rows_per_pass = kThreads / (cw / 8);
+  const size_t smem = sizeof(float) * ((size_t)rows_per_pass * cw + cw);
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)col_tiles, (unsigned)C, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = C;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, act_stats_kernel<TX, PK>,
+                                        static_cast<const TX*>(X), T, K, ldx,
+                                        p, accumulate, cw, sum_out));
+}
+
+template <typename TX>
+ttq_status launch_p(const void* X, int64_t T, int64_t K, int64_t ldx, float p,
+                    int accumulate, float* sum_out, cudaStream_t st) {
+  if (p == 2.0f)
+    return launch_typed<TX, 2>(X, T, K, ldx, p, accumulate, sum_out, st);
+  if (p == 1.0f)
+    return launch_typed<TX, 1>(X, T, K, ldx, p, accumulate, sum_out, st);
+  return launch_typed<TX, 0>(X, T, K, ldx, p, accumulate, sum_out, st);
+}
+
+}  // namespace
+
+ttq_status launch_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                            int64_t ldx, float p, int accumulate,
+                            float* sum_out, cudaStream_t st) {
+  switch (xt) {
+    case TTQ_F32:
+      return launch_p<float>(X, T, K, ldx, p, accumulate, sum_out, st);
+    case TTQ_BF16:
+      return launch_p<__nv_bfloat16>(X, T, K, ldx, p, accumulate, sum_out, st);
+    case TTQ_F16:
+      return launch_p<__half>(X, T, K, ldx, p, accumulate, sum_out, st);
+  }
+  return TTQ_ERR_INVALID_ARG;
+}
+
+}  // namespace ttq

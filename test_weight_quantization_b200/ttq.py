@@ -1,0 +1,314 @@
+"""ctypes binding of libttq (include/ttq.h): same call names, marshalling only.
+
+Every function takes torch tensors that already live on a CUDA device,
+passes their device pointers and the current torch stream to the C ABI, and
+raises :class:`TTQError` on a non-OK status. No step of the computation runs
+in Python; if ``libttq.so`` is missing or cannot be loaded, importing this
+module raises, so there is no silent fallback.
+
+Paper: "TTQ: Activation-Aware Test-Time Quantization to Accelerate LLM
+Inference On The Fly" (TTQ review, section "Proposed method", bullets 1-7).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                         "libttq.so")
+
+TTQ_OK = 0
+DEVERR_TIMEOUT = 0x1
+DEVERR_FP16_RANGE = 0x2
+
+_DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+
+
+class TTQError(RuntimeError):
+    pass
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is missing: build it with "
+            "`python -m test_weight_quantization_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I64, I, F, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                        ctypes.c_float, ctypes.c_size_t)
+    sig = {
+        "ttq_act_stats": [P, I, I64, I64, I64, F, I, P, P],
+        "ttq_awq_scales": [P, I64, I64, P, P, P, P],
+        "ttq_quantize_rtn_grouped": [P, I, I64, I64, I64, P, I, I, P, P, P, P],
+        "ttq_w_lowbit_gemm_workspace_size": [I64, I64, I],
+        "ttq_w_lowbit_gemm": [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P,
+                              I, P, I, I64, P, SZ, P],
+        "ttq_prepare_activations": [P, I, I64, I64, I64, P, P, I, P, P, P],
+        "ttq_w_lowbit_gemm_prepared": [P, P, I64, I64, P, P, P, I64, I, I, P,
+                                       I, I, P, I, I64, P],
+        "ttq_lowrank_add": [P, I, I64, I64, I64, P, P, I, I64, P, I, I64, P],
+        "ttq_unpack_codes": [P, I64, I64, I, P, P],
+        "ttq_status_string": [I],
+        "ttq_device_error": [I],
+        "ttq_abi_version": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = I
+    lib.ttq_status_string.restype = ctypes.c_char_p
+    lib.ttq_w_lowbit_gemm_workspace_size.restype = SZ
+    return lib
+
+
+_lib = _load()
+
+# Names the C ABI exports (include/ttq.h).
+EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_quantize_rtn_grouped",
+           "ttq_w_lowbit_gemm_workspace_size", "ttq_w_lowbit_gemm",
+           "ttq_prepare_activations", "ttq_w_lowbit_gemm_prepared",
+           "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
+           "ttq_device_error", "ttq_abi_version")
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group", ctypes.c_int),
+                ("alpha", ctypes.c_float), ("lambda_", ctypes.c_float),
+                ("p", ctypes.c_float)]
+
+
+@dataclass(frozen=True)
+class TTQParams:
+    """Fixed per-layer hyperparameters (Proposed method, bullet 4)."""
+    bits: int = 4
+    group: int = 128
+    alpha: float = 0.5
+    lam: float = 0.1
+    p: float = 2.0
+
+
+def _check(status: int, what: str) -> None:
+    if status != TTQ_OK:
+        raise TTQError(f"{what}: {_lib.ttq_status_string(status).decode()}")
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TTQError(f"{name} must be a CUDA tensor")
+
+
+def _rows(t: torch.Tensor, name: str) -> int:
+    """Row pitch (elements) of a 2D tensor whose rows are contiguous."""
+    _dev(t, name)
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise TTQError(f"{name} must be 2D with contiguous rows")
+    return t.stride(0)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def abi_version() -> int:
+    return int(_lib.ttq_abi_version())
+
+
+def device_error(clear: bool = True) -> int:
+    """Sticky device error bits (synchronising read)."""
+    return int(_lib.ttq_device_error(1 if clear else 0))
+
+
+def act_stats(X: torch.Tensor, p: float = 2.0, out: torch.Tensor | None = None,
+              accumulate: bool = False) -> torch.Tensor:
+    """Step 1: out[j] (+)= sum_t |X[t, j]|^p, fp32 [K]."""
+    ldx = _rows(X, "X")
+    T, K = X.shape
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=X.device)
+    _dev(out, "out")
+    _check(_lib.ttq_act_stats(X.data_ptr(), _DTYPE[X.dtype], T, K, ldx,
+                              float(p), 1 if accumulate else 0,
+                              out.data_ptr(), _stream()), "ttq_act_stats")
+    return out
+
+
+def awq_scales(sums: torch.Tensor, T_total: int, alpha: float = 0.5,
+               lam: float = 0.1, p: float = 2.0, s=None, inv_s=None):
+    """Step 2: (s, inv_s) fp32 [K] from the channel sums."""
+    _dev(sums, "sums")
+    K = sums.shape[0]
+    s = torch.empty(K, dtype=torch.float32, device=sums.device) if s is None \
+        else s
+    inv_s = torch.empty_like(s) if inv_s is None else inv_s
+    prm = _Params(0, 0, alpha, lam, p)
+    _check(_lib.ttq_awq_scales(sums.data_ptr(), int(T_total), K,
+                               ctypes.addressof(prm), s.data_ptr(),
+                               inv_s.data_ptr(), _stream()), "ttq_awq_scales")
+    return s, inv_s
+
+
+def quantize_rtn_grouped(W: torch.Tensor, s: torch.Tensor | None, bits: int,
+                         group: int, codes=None, delta=None, zero=None):
+    """Step 3: packed codes [N, K*bits/32] u32 (as int32), delta [N, K/g]
+    fp32, zero [N, K/g] u8."""
+    ldw = _rows(W, "W")
+    N, K = W.shape
+    dev = W.device
+    if codes is None:
+        codes = torch.empty((N, K * bits // 32), dtype=torch.int32, device=dev)
+    if delta is None:
+        delta = torch.empty((N, K // group), dtype=torch.float32, device=dev)
+    if zero is None:
+        zero = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+    _check(_lib.ttq_quantize_rtn_grouped(
+        W.data_ptr(), _DTYPE[W.dtype], N, K, ldw, _ptr(s), bits, group,
+        codes.data_ptr(), delta.data_ptr(), zero.data_ptr(), _stream()),
+        "ttq_quantize_rtn_grouped")
+    return codes, delta, zero
+
+
+def workspace_size(T: int, K: int, r: int = 0) -> int:
+    return int(_lib.ttq_w_lowbit_gemm_workspace_size(T, K, r))
+
+
+def w_lowbit_gemm(X: torch.Tensor, inv_s: torch.Tensor, codes: torch.Tensor,
+                  delta: torch.Tensor, zero: torch.Tensor, N: int, bits: int,
+                  group: int, A: torch.Tensor | None = None,
+                  B: torch.Tensor | None = None,
+                  out: torch.Tensor | None = None, out_dtype=None,
+                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Step 4: Y = (X diag(inv_s)) W_hat^T [+ (X A^T) B^T], [T, N]."""
+    ldx = _rows(X, "X")
+    T, K = X.shape
+    r = 0 if A is None else A.shape[0]
+    if out is None:
+        out = torch.empty((T, N), dtype=out_dtype or X.dtype, device=X.device)
+    ldy = _rows(out, "out")
+    need = workspace_size(T, K, r)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(_lib.ttq_w_lowbit_gemm(
+        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(),
+        codes.data_ptr(), delta.data_ptr(), zero.data_ptr(), N, bits, group,
+        _ptr(A), _ptr(B), r, out.data_ptr(), _DTYPE[out.dtype], ldy,
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream()), "ttq_w_lowbit_gemm")
+    return out
+
+
+def prepare_activations(X: torch.Tensor, inv_s: torch.Tensor,
+                        A: torch.Tensor | None = None, Xs=None, U=None):
+    """Activation side of step 4: Xs = fp16(X diag(inv_s)) [T, K] and, with
+    low-rank factors, U = fp16(X A^T) zero-padded to [T, 64]."""
+    ldx = _rows(X, "X")
+    T, K = X.shape
+    r = 0 if A is None else A.shape[0]
+    if Xs is None:
+        Xs = torch.empty((T, K), dtype=torch.float16, device=X.device)
+    if r and U is None:
+        U = torch.empty((T, 64), dtype=torch.float16, device=X.device)
+    _check(_lib.ttq_prepare_activations(
+        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(), _ptr(A), r,
+        Xs.data_ptr(), _ptr(U) if r else None, _stream()),
+        "ttq_prepare_activations")
+    return Xs, (U if r else None)
+
+
+def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
+                           codes: torch.Tensor, delta: torch.Tensor,
+                           zero: torch.Tensor, N: int, bits: int, group: int,
+                           B: torch.Tensor | None = None,
+                           out: torch.Tensor | None = None,
+                           out_dtype=torch.bfloat16) -> torch.Tensor:
+    """Tensor-core projection on prepared operands (one kernel launch)."""
+    _dev(Xs, "Xs")
+    T, K = Xs.shape
+    r = 0 if B is None else B.shape[1]
+    if out is None:
+        out = torch.empty((T, N), dtype=out_dtype, device=Xs.device)
+    ldy = _rows(out, "out")
+    _check(_lib.ttq_w_lowbit_gemm_prepared(
+        Xs.data_ptr(), _ptr(U) if r else None, T, K, codes.data_ptr(),
+        delta.data_ptr(), zero.data_ptr(), N, bits, group, _ptr(B),
+        _DTYPE[B.dtype] if r else 0, r, out.data_ptr(), _DTYPE[out.dtype],
+        ldy, _stream()), "ttq_w_lowbit_gemm_prepared")
+    return out
+
+
+def lowrank_add(X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                Y: torch.Tensor) -> torch.Tensor:
+    """Y += (X A^T) B^T in place."""
+    ldx = _rows(X, "X")
+    ldy = _rows(Y, "Y")
+    T, K = X.shape
+    r = A.shape[0]
+    N = B.shape[0]
+    _check(_lib.ttq_lowrank_add(X.data_ptr(), _DTYPE[X.dtype], T, K, ldx,
+                                A.data_ptr(), B.data_ptr(), r, N, Y.data_ptr(),
+                                _DTYPE[Y.dtype], ldy, _stream()),
+           "ttq_lowrank_add")
+    return Y
+
+
+def unpack_codes(codes: torch.Tensor, K: int, bits: int) -> torch.Tensor:
+    """One uint8 per weight, [N, K]."""
+    _dev(codes, "codes")
+    N = codes.shape[0]
+    q = torch.empty((N, K), dtype=torch.uint8, device=codes.device)
+    _check(_lib.ttq_unpack_codes(codes.data_ptr(), N, K, bits, q.data_ptr(),
+                                 _stream()), "ttq_unpack_codes")
+    return q
+
+
+class TTQLinear:
+    """One linear layer run the TTQ way: per prompt, statistics -> scales ->
+    quantize -> low-bit projection (+ optional static low-rank term).
+
+    ``W`` is the stored weight ([N, K], or the residual W - B A when ``A`` and
+    ``B`` are given). Buffers are allocated once per (T) and reused.
+    """
+
+    def __init__(self, W: torch.Tensor, params: TTQParams, A=None, B=None):
+        self.W, self.A, self.B, self.prm = W, A, B, params
+        N, K = W.shape
+        dev = W.device
+        self.sums = torch.empty(K, dtype=torch.float32, device=dev)
+        self.s = torch.empty(K, dtype=torch.float32, device=dev)
+        self.inv_s = torch.empty(K, dtype=torch.float32, device=dev)
+        self.codes = torch.empty((N, K * params.bits // 32), dtype=torch.int32,
+                                 device=dev)
+        self.delta = torch.empty((N, K // params.group), dtype=torch.float32,
+                                 device=dev)
+        self.zero = torch.empty((N, K // params.group), dtype=torch.uint8,
+                                device=dev)
+        self._ws = None
+
+    def calibrate(self, X: torch.Tensor) -> None:
+        """Online statistics and quantization from this prompt's input."""
+        p = self.prm
+        act_stats(X, p.p, out=self.sums)
+        awq_scales(self.sums, X.shape[0], p.alpha, p.lam, p.p, self.s,
+                   self.inv_s)
+        quantize_rtn_grouped(self.W, self.s, p.bits, p.group, self.codes,
+                             self.delta, self.zero)
+
+    def project(self, X: torch.Tensor, out: torch.Tensor | None = None):
+        T, K = X.shape
+        r = 0 if self.A is None else self.A.shape[0]
+        need = workspace_size(T, K, r)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=X.device)
+        return w_lowbit_gemm(X, self.inv_s, self.codes, self.delta, self.zero,
+                             self.W.shape[0], self.prm.bits, self.prm.group,
+                             self.A, self.B, out=out, workspace=self._ws)
+
+    def __call__(self, X: torch.Tensor, out: torch.Tensor | None = None):
+        self.calibrate(X)
+        return self.project(X, out)

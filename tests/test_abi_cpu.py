@@ -1,0 +1,102 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/ttq.h declares, and rejects bad arguments before
+touching the device. Also checks that the oracle and the CUDA path share no
+code."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ttq.h")
+LIB = os.path.join(ROOT, "test_weight_quantization_b200", "libttq.so")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from test_weight_quantization_b200 import build
+        build.build()
+    return ctypes.CDLL(LIB)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("ttq_act_stats", "ttq_awq_scales", "ttq_quantize_rtn_grouped",
+              "ttq_w_lowbit_gemm", "ttq_lowrank_add"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    lib.ttq_status_string.restype = ctypes.c_char_p
+    assert lib.ttq_status_string(0) == b"TTQ_OK"
+    assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
+    assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
+    assert lib.ttq_abi_version() == 1
+
+
+def test_workspace_size(lib):
+    f = lib.ttq_w_lowbit_gemm_workspace_size
+    f.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+    f.restype = ctypes.c_size_t
+    assert f(16, 4096, 0) >= 16 * 4096 * 2
+    assert f(16, 4096, 16) >= f(16, 4096, 0) + 16 * 64 * 2
+    assert f(0, 4096, 0) == 0
+
+
+def test_bad_arguments_are_rejected_before_launch(lib):
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fake = ctypes.c_void_p(0x100000)  # never dereferenced: checks fail first
+    lib.ttq_act_stats.argtypes = [P, I, I64, I64, I64, F, I, P, P]
+    assert lib.ttq_act_stats(None, 1, 8, 64, 64, 2.0, 0, fake, None) == 1
+    assert lib.ttq_act_stats(fake, 1, 8, 60, 64, 2.0, 0, fake, None) == 1  # K%8
+    assert lib.ttq_act_stats(fake, 1, 8, 64, 64, -1.0, 0, fake, None) == 1
+    assert lib.ttq_act_stats(fake, 7, 8, 64, 64, 2.0, 0, fake, None) == 1
+    lib.ttq_quantize_rtn_grouped.argtypes = [P, I, I64, I64, I64, P, I, I, P,
+                                             P, P, P]
+    q = lib.ttq_quantize_rtn_grouped
+    assert q(fake, 1, 4, 64, 64, None, 9, 32, fake, fake, fake, None) == 1
+    assert q(fake, 1, 4, 64, 64, None, 4, 24, fake, fake, fake, None) == 1
+    assert q(fake, 1, 4, 48, 48, None, 4, 16, fake, fake, fake, None) == 1
+    lib.ttq_w_lowbit_gemm.argtypes = [P, I, I64, I64, I64, P, P, P, P, I64, I,
+                                      I, P, P, I, P, I, I64, P, ctypes.c_size_t,
+                                      P]
+    g = lib.ttq_w_lowbit_gemm
+    # workspace too small
+    assert g(fake, 1, 16, 64, 64, fake, fake, fake, fake, 32, 4, 32, None,
+             None, 0, fake, 1, 32, fake, 16, None) == 1
+    # low-rank rank without factors
+    assert g(fake, 1, 16, 64, 64, fake, fake, fake, fake, 32, 4, 32, None,
+             None, 8, fake, 1, 32, fake, 1 << 20, None) == 1
+    lib.ttq_unpack_codes.argtypes = [P, I64, I64, I, P, P]
+    assert lib.ttq_unpack_codes(None, 4, 64, 4, fake, None) == 1
+
+
+def test_oracle_and_cuda_path_share_no_code():
+    csrc = glob.glob(os.path.join(ROOT, "test_weight_quantization_b200",
+                                  "**", "*.*"), recursive=True)
+    for path in csrc:
+        if path.endswith((".cu", ".cuh", ".h", ".py")):
+            text = open(path, errors="ignore").read()
+            assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), \
+                path
+            assert "ttq_oracle" not in text, path
+    osrc = open(os.path.join(ROOT, "oracle", "ttq_oracle.c")).read()
+    includes = re.findall(r"^\s*#\s*include\s*[<\"]([^>\"]+)", osrc, re.M)
+    assert all(i in ("math.h", "stdint.h", "stdlib.h", "string.h")
+               for i in includes), includes
+    opy = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    assert "test_weight_quantization_b200" not in opy

@@ -1,0 +1,279 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the CPU oracle on the same seeded inputs.
+
+Small shapes span several tiles and a ragged tail; the oracle is always fed
+the GPU's own upstream outputs (sums -> scales -> codes) so each step is
+compared on identical inputs. Tolerances: see parity_util.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import (assert_gemm_close, assert_rel_close, gemm_errors,
+                         np32)
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
+
+
+@pytest.fixture(scope="module")
+def ttq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from test_weight_quantization_b200 import ttq as mod
+    mod.device_error(clear=True)
+    yield mod
+    assert mod.device_error(clear=True) == 0
+
+
+def acts(T, K, seed, dtype, frac=0.02, factor=20.0):
+    from test_weight_quantization_b200.inputs import activations
+    X = activations(T, K, seed, "student_t", outlier_frac=frac,
+                    outlier_factor=factor)
+    return torch.from_numpy(X).to(dtype)
+
+
+def weights(N, K, seed, dtype):
+    from test_weight_quantization_b200.inputs import weights as w
+    return torch.from_numpy(w(N, K, seed)).to(dtype)
+
+
+# ------------------------------------------------------------- stats ----
+
+@pytest.mark.parametrize("dt", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("T,K", [(1, 8), (37, 264), (300, 1000), (1000, 2056)])
+@pytest.mark.parametrize("p", [2.0, 1.0, 3.0])
+def test_stats(ttq, dt, T, K, p):
+    X = acts(T, K, T + K, DT[dt])
+    got = ttq.act_stats(X.cuda(), p)
+    ref = oracle.act_sums(np32(X), p)
+    assert_rel_close(np32(got), ref, what="sums")
+
+
+def test_stats_accumulate_and_pitch(ttq):
+    X = acts(700, 512, 5, torch.bfloat16)
+    big = torch.zeros(700, 640, dtype=torch.bfloat16)
+    big[:, :512] = X
+    Xg = big.cuda()[:, :512]  # row pitch 640
+    out = ttq.act_stats(Xg[:300])
+    ttq.act_stats(Xg[300:], out=out, accumulate=True)
+    assert_rel_close(np32(out), oracle.act_sums(np32(X)), what="chunked")
+
+
+def test_stats_deterministic(ttq):
+    Xg = acts(2048, 768, 6, torch.bfloat16).cuda()
+    a = ttq.act_stats(Xg)
+    b = ttq.act_stats(Xg)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------ scales ----
+
+@pytest.mark.parametrize("alpha,lam,p", [(0.5, 0.1, 2.0), (0.0, 0.1, 2.0),
+                                         (0.7, 1.0, 2.0), (0.4, 0.0, 1.0)])
+def test_scales(ttq, alpha, lam, p):
+    X = acts(512, 1024, 7, torch.bfloat16)
+    sums = ttq.act_stats(X.cuda(), p)
+    s, inv = ttq.awq_scales(sums, 512, alpha, lam, p)
+    rs, rinv = oracle.awq_scales(np32(sums).astype(np.float64), 512, alpha,
+                                 lam, p)
+    assert_rel_close(np32(s), rs, what="s")
+    assert_rel_close(np32(inv), rinv, what="inv_s")
+
+
+def test_scales_zero_statistic(ttq):
+    sums = torch.zeros(256, device="cuda")
+    s, inv = ttq.awq_scales(sums, 10, 0.5, 0.0, 2.0)
+    assert torch.all(s == 1) and torch.all(inv == 1)
+
+
+# ---------------------------------------------------------- quantize ----
+
+def quantize_both(ttq, W, s, bits, group):
+    c, d, z = ttq.quantize_rtn_grouped(W.cuda(), None if s is None else
+                                       s.cuda(), bits, group)
+    s_np = None if s is None else np32(s)
+    rc, rd, rz = oracle.quantize(np32(W), s_np, bits, group)
+    return (c.cpu().numpy().view(np.uint32), d.cpu().numpy(), z.cpu().numpy(),
+            rc, rd, rz)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("group", [16, 32, 64, 128])
+def test_quantize_bit_exact(ttq, bits, group):
+    N, K = 37, 1152  # ragged rows; K not a multiple of 256
+    W = weights(N, K, 100 + bits, torch.bfloat16)
+    s = torch.from_numpy(np.exp(np.random.default_rng(bits).standard_normal(K)
+                                * 0.7).astype(np.float32))
+    c, d, z, rc, rd, rz = quantize_both(ttq, W, s, bits, group)
+    np.testing.assert_array_equal(d, rd)
+    np.testing.assert_array_equal(z, rz)
+    np.testing.assert_array_equal(c, rc)
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16"])
+def test_quantize_dtypes_and_no_scale(ttq, dt):
+    W = weights(20, 96, 9, DT[dt])
+    c, d, z, rc, rd, rz = quantize_both(ttq, W, None, 4, 32)
+    np.testing.assert_array_equal(c, rc)
+    np.testing.assert_array_equal(d, rd)
+    np.testing.assert_array_equal(z, rz)
+
+
+def test_quantize_degenerate_groups(ttq):
+    W = torch.zeros(4, 64)
+    W[1, :16] = torch.linspace(0.1, 1.0, 16)
+    W[2, 16:32] = -torch.linspace(0.1, 1.0, 16)
+    W[3] = 0.5  # constant row
+    c, d, z, rc, rd, rz = quantize_both(ttq, W, None, 3, 16)
+    np.testing.assert_array_equal(c, rc)
+    np.testing.assert_array_equal(d, rd)
+    np.testing.assert_array_equal(z, rz)
+
+
+def test_unpack(ttq):
+    W = weights(9, 160, 3, torch.bfloat16)
+    for bits in (2, 3, 5, 8):
+        c, _, _ = ttq.quantize_rtn_grouped(W.cuda(), None, bits, 32)
+        q = ttq.unpack_codes(c, 160, bits).cpu().numpy()
+        np.testing.assert_array_equal(
+            q, oracle.unpack_codes(c.cpu().numpy().view(np.uint32), 160, bits))
+
+
+# -------------------------------------------------------------- gemm ----
+
+def run_path(ttq, X, W, bits, group, A=None, B=None, out_dtype=None,
+             alpha=0.5, lam=0.1, p=2.0):
+    """GPU path: stats -> scales -> quantize -> projection."""
+    Xg, Wg = X.cuda(), W.cuda()
+    sums = ttq.act_stats(Xg, p)
+    s, inv = ttq.awq_scales(sums, X.shape[0], alpha, lam, p)
+    c, d, z = ttq.quantize_rtn_grouped(Wg, s, bits, group)
+    Y = ttq.w_lowbit_gemm(Xg, inv, c, d, z, W.shape[0], bits, group,
+                          None if A is None else A.cuda(),
+                          None if B is None else B.cuda(),
+                          out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    return Y, inv, c, d, z
+
+
+def oracle_y(X, inv, c, d, z, N, bits, group, A=None, B=None, rows=None):
+    return oracle.lowbit_gemm(np32(X), np32(inv), c.cpu().numpy().view(
+        np.uint32), d.cpu().numpy(), z.cpu().numpy(), N, bits, group,
+        None if A is None else np32(A), None if B is None else np32(B),
+        rows=rows)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 17, 100, 300])
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 32), (2, 16), (5, 64)])
+def test_gemm_shapes(ttq, T, bits, group):
+    N, K = 300, 640  # 3 weight tiles (ragged), 10 K steps
+    X = acts(T, K, 11 + T, torch.bfloat16)
+    W = weights(N, K, 12, torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, bits, group)
+    ref = oracle_y(X, inv, c, d, z, N, bits, group)
+    assert_gemm_close(np32(Y), ref, f"T={T} b={bits} g={group}", Y.dtype)
+
+
+@pytest.mark.parametrize("bits", [6, 7, 8])
+def test_gemm_wide_codes(ttq, bits):
+    X = acts(64, 256, 13, torch.bfloat16)
+    W = weights(160, 256, 14, torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, bits, 32)
+    assert_gemm_close(np32(Y), oracle_y(X, inv, c, d, z, 160, bits, 32),
+                      dtype=Y.dtype)
+
+
+@pytest.mark.parametrize("K", [32, 96, 160])
+def test_gemm_ragged_k(ttq, K):
+    # K not a multiple of the 64-wide K step: the tail step is half empty
+    X = acts(40, K, 15, torch.bfloat16)
+    W = weights(130, K, 16, torch.bfloat16)
+    for T in (40, 3):
+        Y, inv, c, d, z = run_path(ttq, X[:T], W, 4, 32)
+        assert_gemm_close(np32(Y), oracle_y(X[:T], inv, c, d, z, 130, 4, 32),
+                          dtype=Y.dtype)
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("xin", ["f32", "bf16", "f16"])
+def test_gemm_dtypes(ttq, xin, out):
+    X = acts(50, 256, 17, DT[xin])
+    W = weights(144, 256, 18, DT[xin])
+    Y, inv, c, d, z = run_path(ttq, X, W, 4, 32, out_dtype=DT[out])
+    assert Y.dtype == DT[out]
+    assert_gemm_close(np32(Y), oracle_y(X, inv, c, d, z, 144, 4, 32),
+                      dtype=Y.dtype)
+
+
+def test_gemm_fp32_output_error_is_operand_rounding_only(ttq):
+    # fp32 Y isolates the fp16 operand roundings (X/s and (q-z)D): far
+    # below the bar
+    X = acts(256, 512, 19, torch.bfloat16)
+    W = weights(256, 512, 20, torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, 4, 64, out_dtype=torch.float32)
+    fro, rowmax = gemm_errors(np32(Y), oracle_y(X, inv, c, d, z, 256, 4, 64))
+    assert fro < 7e-4 and rowmax < 1e-2
+
+
+@pytest.mark.parametrize("T", [1, 16, 200])
+@pytest.mark.parametrize("r", [16, 7])
+def test_gemm_lowrank(ttq, T, r):
+    N, K = 272, 384
+    X = acts(T, K, 21, torch.bfloat16)
+    rng = np.random.default_rng(22)
+    A = torch.from_numpy(rng.standard_normal((r, K)).astype(np.float32) *
+                         0.05).to(torch.bfloat16)
+    B = torch.from_numpy(rng.standard_normal((N, r)).astype(np.float32) *
+                         0.05).to(torch.bfloat16)
+    W = weights(N, K, 23, torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, 4, 64, A, B)
+    assert_gemm_close(np32(Y), oracle_y(X, inv, c, d, z, N, 4, 64, A, B),
+                      dtype=Y.dtype)
+
+
+def test_lowrank_add_alone(ttq):
+    T, K, N, r = 33, 200, 150, 16
+    X = acts(T, K, 24, torch.float32)
+    rng = np.random.default_rng(25)
+    A = torch.from_numpy(rng.standard_normal((r, K)).astype(np.float32))
+    B = torch.from_numpy(rng.standard_normal((N, r)).astype(np.float32))
+    Y0 = torch.from_numpy(rng.standard_normal((T, N)).astype(np.float32))
+    Y = ttq.lowrank_add(X.cuda(), A.cuda(), B.cuda(), Y0.clone().cuda())
+    ref = Y0.double().numpy() + (X.double().numpy() @ A.double().numpy().T) @ \
+        B.double().numpy().T
+    assert_gemm_close(np32(Y), ref)
+
+
+def test_gemm_deterministic_and_reusable_workspace(ttq):
+    X = acts(8, 1024, 26, torch.bfloat16).cuda()
+    W = weights(512, 1024, 27, torch.bfloat16).cuda()
+    sums = ttq.act_stats(X)
+    s, inv = ttq.awq_scales(sums, 8)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, 4, 128)
+    ws = torch.empty(ttq.workspace_size(8, 1024), dtype=torch.uint8,
+                     device="cuda")
+    y1 = ttq.w_lowbit_gemm(X, inv, c, d, z, 512, 4, 128, workspace=ws)
+    y2 = ttq.w_lowbit_gemm(X, inv, c, d, z, 512, 4, 128, workspace=ws)
+    assert torch.equal(y1, y2)
+
+
+def test_fp16_range_flag(ttq):
+    X = torch.full((4, 64), 60000.0, dtype=torch.float32).cuda()
+    inv = torch.full((64,), 2.0, device="cuda")
+    W = weights(128, 64, 28, torch.float32).cuda()
+    c, d, z = ttq.quantize_rtn_grouped(W, None, 4, 32)
+    ttq.device_error(clear=True)
+    ttq.w_lowbit_gemm(X, inv, c, d, z, 128, 4, 32)
+    assert ttq.device_error(clear=True) & ttq.DEVERR_FP16_RANGE
+
+
+def test_layer_object_matches_calls(ttq):
+    X = acts(64, 256, 29, torch.bfloat16).cuda()
+    W = weights(96, 256, 30, torch.bfloat16).cuda()
+    layer = ttq.TTQLinear(W, ttq.TTQParams(bits=3, group=32))
+    y = layer(X)
+    Y, *_ = run_path(ttq, X.cpu(), W.cpu(), 3, 32)
+    assert torch.equal(y, Y)
