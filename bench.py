@@ -50,6 +50,9 @@ def parse():
                     choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the step directly instead of replaying a "
+                         "CUDA graph (for profilers)")
     return ap.parse_args()
 
 
@@ -97,10 +100,11 @@ class Step:
         b, g = wl.bits, wl.group
         self.codes, self.delta, self.zero, self.Y = {}, {}, {}, {}
         for L in self.layers:
-            self.codes[L.name] = torch.empty((L.N, L.K * b // 32),
+            self.codes[L.name] = torch.empty((L.N, ttq.codes_ld(L.K, b)),
                                              dtype=torch.int32, device=device)
-            self.delta[L.name] = torch.empty((L.N, L.K // g), **f32)
-            self.zero[L.name] = torch.empty((L.N, L.K // g), dtype=torch.uint8,
+            gl = ttq.groups_ld(L.K, g)
+            self.delta[L.name] = torch.empty((L.N, gl), **f32)
+            self.zero[L.name] = torch.empty((L.N, gl), dtype=torch.uint8,
                                             device=device)
             self.Y[L.name] = torch.empty((self.T, L.N), dtype=wl.dtype,
                                          device=device)
@@ -368,11 +372,23 @@ def main():
     ttq.device_error(clear=True)
     calls = step.calls(0)
     kinds = [k for k, _ in calls]
-    graphs, igraphs = [], []
     # external events record timestamps when replayed inside a graph
-    ev = [[[torch.cuda.Event(enable_timing=True, external=True)
+    ev = [[[torch.cuda.Event(enable_timing=True, external=not args.eager)
             for _ in range(2)] for _ in calls] for _ in range(rep)]
+
+    class Eager:
+        def __init__(self, r, events=None):
+            self.r, self.events = r, events
+
+        def replay(self):
+            step.run(self.r, self.events)
+
+    graphs, igraphs = [], []
     for r in range(rep):
+        if args.eager:
+            graphs.append(Eager(r))
+            igraphs.append(Eager(r, ev[r]))
+            continue
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             step.run(r)
@@ -481,8 +497,8 @@ def main():
                             "fp32; statistics fp32",
                 "l2": f"inputs rotate over {rep} replicas "
                       f"({rep * step.input_bytes() / 2**20:.0f} MiB > L2)",
-                "parallelism": f"replicas x{world}", "graph": "CUDA graph per "
-                "replica"},
+                "parallelism": f"replicas x{world}",
+                "launch": "eager" if args.eager else "CUDA graph per replica"},
             "roofline": roof, "kernels": kernels,
             "gpu_launches": len(kinds) * args.steps,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,

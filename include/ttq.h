@@ -84,14 +84,23 @@ typedef struct {
  * input channels 32k .. 32k+31 in `bits` consecutive uint32 words. Inside a
  * block the codes form a little-endian bit stream: the code of channel
  * 32k + c occupies bits [c*bits, c*bits + bits) of the block, where bit i of
- * the block is bit (i % 32) of word (i / 32). A row therefore spans
- * K*bits/32 words and the array is [N][K*bits/32] uint32, row-major, dense.
+ * the block is bit (i % 32) of word (i / 32). A row holds K*bits/32 words
+ * followed by zero padding up to its pitch ttq_codes_ld(K, bits) (a multiple
+ * of 4 words), so the array is [N][ttq_codes_ld(K, bits)] uint32.
  *
- * delta is [N][K/g] float32 (row-major, dense), zero is [N][K/g] uint8.
- * The scaled-domain weight of channel j in row n is
+ * delta is [N][ttq_groups_ld(K, g)] float32 and zero is
+ * [N][ttq_groups_ld(K, g)] uint8: entry [n][G] for the K/g groups of row n,
+ * then zero padding up to the pitch (a multiple of 16 entries). The pitches
+ * keep every row 16-byte aligned, which tensor-memory-accelerator copies
+ * need. The scaled-domain weight of channel j in row n is
  *     W_hat_s[n][j] = (q[n][j] - zero[n][j/g]) * delta[n][j/g]
  * and the effective weight is W_hat_s[n][j] / s[j].
  * ------------------------------------------------------------------- */
+
+/* Row pitches of the packed layout: words per codes row, entries per
+ * delta/zero row. Both return 0 for invalid arguments. */
+int64_t ttq_codes_ld(int64_t K, int bits);
+int64_t ttq_groups_ld(int64_t K, int group);
 
 /* Step 1, online activation statistics (TTQ review, Proposed method,
  * bullets 2-3: the diagonal of the input covariance, estimated per prompt).
@@ -128,7 +137,7 @@ ttq_status ttq_awq_scales(const float* sum, int64_t T_total, int64_t K,
  *   r    = 1 / D
  *   z    = clamp(rint(-mn * r), 0, 2^b - 1)
  *   q_j  = clamp(rint(w_j * r) + z, 0, 2^b - 1)
- * Outputs codes (layout above), delta = D, zero = z.
+ * Outputs codes (layout above), delta = D, zero = z; padding is zeroed.
  *   W      [N, K] of dtype wt, row pitch ldw.
  * Requires 2 <= bits <= 8, group in {16,32,64,128}, K % 32 == 0,
  * K % group == 0. Bit-exact and deterministic. */

@@ -84,7 +84,17 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 1; }
+TTQ_EXPORT int ttq_abi_version(void) { return 2; }
+
+TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
+  if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
+  return codes_ld(K, bits);
+}
+
+TTQ_EXPORT int64_t ttq_groups_ld(int64_t K, int group) {
+  if (K < 1 || !valid_group(group) || K % group != 0) return 0;
+  return groups_ld(K, group);
+}
 
 TTQ_EXPORT const char* ttq_status_string(ttq_status s) {
   switch (s) {

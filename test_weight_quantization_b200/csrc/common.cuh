@@ -15,6 +15,17 @@
 
 namespace ttq {
 
+// ------------------------------------------------------ packed layout ---
+
+// Row pitch of the codes array in uint32 words (16-byte aligned rows).
+__host__ __device__ inline int64_t codes_ld(int64_t K, int bits) {
+  return (K * bits / 32 + 3) / 4 * 4;
+}
+// Row pitch of the delta / zero arrays in entries (16-entry aligned rows).
+__host__ __device__ inline int64_t groups_ld(int64_t K, int group) {
+  return (K / group + 15) / 16 * 16;
+}
+
 // ---------------------------------------------------------------- host ---
 
 // Device address of the sticky error word of the current device (defined in

@@ -12,17 +12,19 @@
 // (prescale_kernel), each weight (q - z) * D is rounded once to fp16 in the
 // dequantiser; products accumulate in fp32 in TMEM.
 //
-// CTA = 6 warps:
-//   warp 0      TMA producer: fp16 activation tiles (64 x BN, 128B swizzle)
-//   warp 1      TMEM owner and single-thread tcgen05.mma issuer
-//   warps 2-5   dequantisers (one weight row per thread: codes, delta, zero
-//               arrive by cp.async into a private ring; fp16 pairs are built
-//               with the 1024+q exponent trick and written in the 128B
-//               swizzled K-major layout), then the epilogue (TMEM -> Y)
-// Decode (T <= 16) splits K over a cluster of up to 8 CTAs; partial tiles
-// are summed by cluster rank 0 through distributed shared memory in a fixed
-// order. The rank-r low-rank term is one extra K stage: [X~ | U] [W | B]^T
-// with U = X A^T (fp16, computed by lowrank_u_kernel).
+// CTA = 10 warps, four shared-memory rings filled by the tensor memory
+// accelerator (TMA) and drained in K order:
+//   X~ ring      64-channel fp16 activation tiles (128B swizzle)      warp 0
+//   codes ring   128 rows x 128 channels of packed codes                warp 0
+//   params ring  128 rows x 16 groups of delta (fp32) and zero (u8)     warp 0
+//   A ring       64-channel fp16 weight tiles (128B swizzle)       warps 2-9
+// warp 1 owns TMEM and issues tcgen05.mma from one thread; warps 2-9 are
+// the dequantisers (two threads per weight row, one 32-code block each:
+// fp16 pairs built with the 1024+q exponent trick) and then the epilogue
+// (TMEM -> Y). Decode (T <= 16) splits K over a cluster of up to 8 CTAs
+// whose partial tiles rank 0 sums through distributed shared memory in a
+// fixed order. The rank-r low-rank term is one extra K stage,
+// [X~ | U] [W_hat | B]^T with U = X A^T (fp16, from lowrank_u_kernel).
 // Every wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds down).
 #include <cooperative_groups.h>
 
@@ -37,48 +39,53 @@ namespace cg = cooperative_groups;
 namespace ttq {
 namespace {
 
-constexpr int kBM = 128;       // weight rows per CTA
-constexpr int kBK = 64;        // K per stage: one 128-byte fp16 row
-constexpr int kThreads = 192;  // 6 warps
+constexpr int kBM = 128;           // weight rows per CTA (TMEM lanes)
+constexpr int kBK = 64;            // channels per MMA stage (128 B of fp16)
+constexpr int kCodeCols = 128;     // channels per codes chunk
+constexpr int kParamGroups = 16;   // groups per params chunk
+constexpr int kDequantWarps = 8;
+constexpr int kDq = 32 * kDequantWarps;  // dequantiser threads
+constexpr int kThreads = 64 + kDq;       // + producer warp + MMA warp
 constexpr int kATileBytes = kBM * kBK * 2;
-constexpr int kMaxStages = 8;
-constexpr int kSmemBudget = 220 * 1024;
-
-// Words each dequantiser thread stages per K step: 2 blocks of codes,
-// up to 4 deltas, 2 words holding the zero bytes.
-__host__ __device__ constexpr int ring_words(int bits) { return 2 * bits + 6; }
+constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
+constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
+constexpr int kMaxSmem = 225 * 1024;
 
 struct GemmArgs {
-  const uint32_t* codes;
-  const float* delta;
-  const uint8_t* zero;
   const void* Blr;  // low-rank B [N][r] in dtype blr_t, or null
-  int blr_t;        // ttq_dtype of Blr
+  int blr_t;
   int r;
-  int64_t N, K, T;
+  int N, K, T;
   void* Y;
   int yt;  // ttq_dtype of Y
-  int64_t ldy;
-  int bn;      // tokens per tile (MMA N)
-  int stages;  // pipeline depth
+  long long ldy;
+  int bn;              // tokens per tile (MMA N)
+  int sx, sa, sc;      // ring depths: activations, weight tiles, codes
   int group;
-  int64_t k_steps;  // ceil(K / 64)
+  int k_steps;         // ceil(K / 64)
+  int per;             // K steps per split rank
   uint32_t* err;
 };
 
-struct SmemLayout {
-  uint32_t a, b, ring, bars, tmem_slot, abort_flag, total;
+__host__ __device__ inline uint32_t code_chunk_bytes(int bits) {
+  return (uint32_t)(kBM * 16 * bits);  // 128 rows x 4*bits words
+}
+
+struct Layout {
+  uint32_t x, a, c, p, bars, tmem, abort_flag, total;
 };
 
-__host__ __device__ inline SmemLayout smem_layout(int bits, int bn,
-                                                  int stages) {
-  SmemLayout L;
-  L.a = 0;
-  L.b = L.a + stages * kATileBytes;
-  L.ring = L.b + stages * bn * 128;
-  L.bars = L.ring + stages * ring_words(bits) * 128 * 4;
-  L.tmem_slot = L.bars + (3 * stages + 1) * 8;
-  L.abort_flag = L.tmem_slot + 4;
+__host__ __device__ inline Layout make_layout(int bits, int bn, int sx, int sa,
+                                              int sc) {
+  Layout L;
+  L.x = 0;
+  L.a = L.x + (uint32_t)(sx * bn * 128);
+  L.c = L.a + (uint32_t)(sa * kATileBytes);
+  L.p = L.c + (uint32_t)sc * code_chunk_bytes(bits);
+  L.bars = L.p + 2u * kParamBytes;
+  const int nbars = 2 * sx + 2 * sa + 2 * sc + 4 + 1;
+  L.tmem = L.bars + 8u * nbars;
+  L.abort_flag = L.tmem + 4;
   L.total = L.abort_flag + 4;
   return L;
 }
@@ -90,25 +97,37 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a,
                "r"(b), "r"(c), "r"(d)
                : "memory");
 }
-__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
 }
+__device__ __forceinline__ uint32_t ld_shared_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 
-__device__ __forceinline__ void cp_async_wait_dyn(int n) {
-  switch (n) {
-    case 0: cp_async_wait<0>(); break;
-    case 1: cp_async_wait<1>(); break;
-    case 2: cp_async_wait<2>(); break;
-    case 3: cp_async_wait<3>(); break;
-    case 4: cp_async_wait<4>(); break;
-    case 5: cp_async_wait<5>(); break;
-    case 6: cp_async_wait<6>(); break;
-    default: cp_async_wait<7>(); break;
+// The BITS words of one 32-code block, with the widest aligned loads.
+template <int BITS>
+__device__ __forceinline__ void load_block(uint32_t addr, uint32_t (&w)[BITS]) {
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int k = 0; k < BITS; k += 4)
+      asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                   : "=r"(w[k]), "=r"(w[k + 1]), "=r"(w[k + 2]), "=r"(w[k + 3])
+                   : "r"(addr + 4 * k)
+                   : "memory");
+  } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int k = 0; k < BITS; k += 2)
+      asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];"
+                   : "=r"(w[k]), "=r"(w[k + 1])
+                   : "r"(addr + 4 * k)
+                   : "memory");
+  } else {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) w[k] = ld_shared_u32(addr + 4 * k);
   }
 }
 
@@ -119,7 +138,7 @@ __device__ __forceinline__ __half2 bits_h2(uint32_t u) {
   return *reinterpret_cast<__half2*>(&u);
 }
 
-__device__ __forceinline__ void store_y(void* Y, int yt, int64_t idx,
+__device__ __forceinline__ void store_y(void* Y, int yt, long long idx,
                                         float v) {
   if (yt == TTQ_BF16)
     static_cast<__nv_bfloat16*>(Y)[idx] = __float2bfloat16_rn(v);
@@ -129,68 +148,81 @@ __device__ __forceinline__ void store_y(void* Y, int yt, int64_t idx,
     static_cast<float*>(Y)[idx] = v;
 }
 
-__device__ __forceinline__ float load_any(const void* p, int t, int64_t idx) {
+__device__ __forceinline__ float load_any(const void* p, int t, long long idx) {
   if (t == TTQ_BF16)
     return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[idx]);
   if (t == TTQ_F16) return __half2float(static_cast<const __half*>(p)[idx]);
   return static_cast<const float*>(p)[idx];
 }
 
-// GMODE: 0 -> g = 16 (4 groups per K step), 1 -> g = 32 (2 groups),
-// 2 -> g >= 64 (one group per K step).
+// GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
 template <int BITS, int GMODE>
 __global__ void __launch_bounds__(kThreads, 1)
-    lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
-                       const __grid_constant__ CUtensorMap tmap_u,
+    lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
+                       const __grid_constant__ CUtensorMap tm_u,
+                       const __grid_constant__ CUtensorMap tm_c,
+                       const __grid_constant__ CUtensorMap tm_d,
+                       const __grid_constant__ CUtensorMap tm_z,
                        const GemmArgs p) {
-  constexpr int GPS = GMODE == 0 ? 4 : (GMODE == 1 ? 2 : 1);
-  constexpr int RW = ring_words(BITS);
   constexpr uint32_t QMASK = (1u << BITS) - 1u;
+  constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
   const uint32_t base = (raw_base + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - raw_base);
 
-  const int stages = p.stages;
-  const SmemLayout L = smem_layout(BITS, p.bn, stages);
-  const uint32_t bar_full_x = base + L.bars;
-  const uint32_t bar_full_a = bar_full_x + 8 * stages;
-  const uint32_t bar_empty = bar_full_a + 8 * stages;
-  const uint32_t bar_accum = bar_empty + 8 * stages;
+  const int sx = p.sx, sa = p.sa, sc = p.sc, bn = p.bn;
+  const Layout L = make_layout(BITS, bn, sx, sa, sc);
+  const uint32_t b_full_x = base + L.bars;
+  const uint32_t b_empty_x = b_full_x + 8 * sx;
+  const uint32_t b_full_a = b_empty_x + 8 * sx;
+  const uint32_t b_empty_a = b_full_a + 8 * sa;
+  const uint32_t b_full_c = b_empty_a + 8 * sa;
+  const uint32_t b_empty_c = b_full_c + 8 * sc;
+  const uint32_t b_full_p = b_empty_c + 8 * sc;
+  const uint32_t b_empty_p = b_full_p + 16;
+  const uint32_t b_accum = b_empty_p + 16;
   volatile uint32_t* tmem_slot =
-      reinterpret_cast<volatile uint32_t*>(gbase + L.tmem_slot);
+      reinterpret_cast<volatile uint32_t*>(gbase + L.tmem);
   volatile int* aborted = reinterpret_cast<volatile int*>(gbase + L.abort_flag);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t m0 = (int64_t)blockIdx.x * kBM;
-  const int64_t t0 = (int64_t)blockIdx.y * p.bn;
+  const int m0 = blockIdx.x * kBM;
+  const int t0 = blockIdx.y * bn;
   const int split = (int)gridDim.z;
   const int rank = (int)blockIdx.z;
-
-  // K steps of this split; rank 0 also runs the low-rank stage.
-  const int64_t per = (p.k_steps + split - 1) / split;
-  const int64_t ks_begin =
-      rank * per < p.k_steps ? rank * per : p.k_steps;
-  const int64_t ks_end =
-      ks_begin + per < p.k_steps ? ks_begin + per : p.k_steps;
-  const int n_main = (int)(ks_end - ks_begin);
+  const int ks_begin = min(rank * p.per, p.k_steps);
+  const int ks_end = min(ks_begin + p.per, p.k_steps);
+  const int n_main = ks_end - ks_begin;
   const int n_total = n_main + ((p.r > 0 && rank == 0) ? 1 : 0);
-  const uint32_t tmem_cols = p.bn < 32 ? 32u : (uint32_t)p.bn;
+  const int gcols = kParamGroups * p.group;  // channels per params chunk
+  const uint32_t tmem_cols = bn < 32 ? 32u : (uint32_t)bn;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < stages; ++i) {
-      mbar_init(bar_full_x + 8 * i, 1);
-      mbar_init(bar_full_a + 8 * i, kBM);
-      mbar_init(bar_empty + 8 * i, 1);
+    for (int i = 0; i < sx; ++i) {
+      mbar_init(b_full_x + 8 * i, 1);
+      mbar_init(b_empty_x + 8 * i, 1);
     }
-    mbar_init(bar_accum, 1);
+    for (int i = 0; i < sa; ++i) {
+      mbar_init(b_full_a + 8 * i, kDq);
+      mbar_init(b_empty_a + 8 * i, 1);
+    }
+    for (int i = 0; i < sc; ++i) {
+      mbar_init(b_full_c + 8 * i, 1);
+      mbar_init(b_empty_c + 8 * i, kDq);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_full_p + 8 * i, 1);
+      mbar_init(b_empty_p + 8 * i, kDq);
+    }
+    mbar_init(b_accum, 1);
     *aborted = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(base + L.tmem_slot, tmem_cols);
+    tmem_alloc(base + L.tmem, tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -201,188 +233,189 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_x);
-      if (p.r > 0) tma_prefetch_desc(&tmap_u);
-      int issued = 0;
-      const uint32_t tx = (uint32_t)p.bn * 128u;
-      for (int s = 0; s < n_total; ++s) {
-        const int slot = s % stages;
-        const uint32_t it = (uint32_t)(s / stages);
-        if (s >= stages && !mbar_wait(bar_empty + 8 * slot, (it - 1) & 1,
-                                      p.err)) {
-          *aborted = 1;
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_c);
+      tma_prefetch_desc(&tm_d);
+      tma_prefetch_desc(&tm_z);
+      if (p.r > 0) tma_prefetch_desc(&tm_u);
+      int cseq = -1, pseq = -1, last_cc = -1, last_pc = -1, issued = 0;
+      bool ok = true;
+      for (int s = 0; s < n_total && ok; ++s) {
+        if (s < n_main) {
+          const int k0 = (ks_begin + s) * kBK;
+          const int cc = k0 / kCodeCols;
+          if (cc != last_cc) {
+            last_cc = cc;
+            ++cseq;
+            const int slot = cseq % sc;
+            if (cseq >= sc &&
+                !mbar_wait(b_empty_c + 8 * slot, ((cseq / sc) - 1) & 1, p.err)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(b_full_c + 8 * slot, code_chunk_bytes(BITS));
+            tma_load_2d(base + L.c + slot * code_chunk_bytes(BITS), &tm_c,
+                        cc * 4 * BITS, m0, b_full_c + 8 * slot);
+          }
+          const int pc = k0 / gcols;
+          if (pc != last_pc) {
+            last_pc = pc;
+            ++pseq;
+            const int slot = pseq & 1;
+            if (pseq >= 2 &&
+                !mbar_wait(b_empty_p + 8 * slot, ((pseq >> 1) - 1) & 1, p.err)) {
+              ok = false;
+              break;
+            }
+            const uint32_t dst = base + L.p + slot * kParamBytes;
+            mbar_arrive_expect_tx(b_full_p + 8 * slot, kParamBytes);
+            tma_load_2d(dst, &tm_d, pc * kParamGroups, m0, b_full_p + 8 * slot);
+            tma_load_2d(dst + kParamDeltaBytes, &tm_z, pc * kParamGroups, m0,
+                        b_full_p + 8 * slot);
+          }
+        }
+        const int slot = s % sx;
+        if (s >= sx &&
+            !mbar_wait(b_empty_x + 8 * slot, ((s / sx) - 1) & 1, p.err)) {
+          ok = false;
           break;
         }
         if (*aborted) break;
-        const uint32_t dst = base + L.b + slot * p.bn * 128;
-        mbar_arrive_expect_tx(bar_full_x + 8 * slot, tx);
+        mbar_arrive_expect_tx(b_full_x + 8 * slot, (uint32_t)bn * 128u);
         if (s < n_main)
-          tma_load_2d(dst, &tmap_x, (int32_t)((ks_begin + s) * kBK),
-                      (int32_t)t0, bar_full_x + 8 * slot);
+          tma_load_2d(base + L.x + slot * bn * 128, &tm_x,
+                      (ks_begin + s) * kBK, t0, b_full_x + 8 * slot);
         else
-          tma_load_2d(dst, &tmap_u, 0, (int32_t)t0, bar_full_x + 8 * slot);
+          tma_load_2d(base + L.x + slot * bn * 128, &tm_u, 0, t0,
+                      b_full_x + 8 * slot);
         issued = s + 1;
       }
+      if (!ok) *aborted = 1;
       // never leave a bulk copy in flight into shared memory at exit
-      for (int s = max(0, issued - stages); s < issued; ++s)
-        mbar_wait(bar_full_x + 8 * (s % stages), (uint32_t)(s / stages) & 1,
-                  p.err);
+      for (int s = max(0, issued - sx); s < issued; ++s)
+        mbar_wait(b_full_x + 8 * (s % sx), (uint32_t)(s / sx) & 1, p.err);
+      for (int q = max(0, cseq - sc + 1); q <= cseq; ++q)
+        mbar_wait(b_full_c + 8 * (q % sc), (uint32_t)(q / sc) & 1, p.err);
+      for (int q = max(0, pseq - 1); q <= pseq; ++q)
+        mbar_wait(b_full_p + 8 * (q & 1), (uint32_t)(q >> 1) & 1, p.err);
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(kBM, p.bn);
+      const uint32_t idesc = idesc_f16_f32(kBM, bn);
       for (int s = 0; s < n_total; ++s) {
-        const int slot = s % stages;
-        const uint32_t par = (uint32_t)(s / stages) & 1;
-        if (!mbar_wait(bar_full_x + 8 * slot, par, p.err) ||
-            !mbar_wait(bar_full_a + 8 * slot, par, p.err)) {
+        const int sxs = s % sx, sas = s % sa;
+        if (!mbar_wait(b_full_x + 8 * sxs, (uint32_t)(s / sx) & 1, p.err) ||
+            !mbar_wait(b_full_a + 8 * sas, (uint32_t)(s / sa) & 1, p.err)) {
           *aborted = 1;
           break;
         }
         tc_fence_after();
-        const uint64_t ad = smem_desc_sw128(base + L.a + slot * kATileBytes);
-        const uint64_t bd = smem_desc_sw128(base + L.b + slot * p.bn * 128);
+        const uint64_t ad = smem_desc_sw128(base + L.a + sas * kATileBytes);
+        const uint64_t bd = smem_desc_sw128(base + L.x + sxs * bn * 128);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k)
           tc_mma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc,
                      (s > 0 || k > 0) ? 1u : 0u);
-        tc_commit(bar_empty + 8 * slot);
+        tc_commit(b_empty_x + 8 * sxs);
+        tc_commit(b_empty_a + 8 * sas);
       }
-      tc_commit(bar_accum);
+      tc_commit(b_accum);
     }
   } else {
     // ------------------------------------------------ dequantisers ----
-    const int i = 32 * (warp & 3) + lane;  // weight row in the tile = TMEM lane
-    const int64_t n = m0 + i;
+    const int q4 = warp & 3;         // TMEM lane quarter
+    const int h = (warp - 2) >> 2;   // which 32-code block of a 64-col stage
+    const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
+    const int n = m0 + i;
     const bool row_ok = n < p.N;
-    const int64_t row_words = p.K * BITS / 32;
-    const int64_t G = p.K / p.group;
-    const uint32_t* crow = p.codes + (row_ok ? n : 0) * row_words;
-    const float* drow = p.delta + (row_ok ? n : 0) * G;
-    const int64_t zrow = (row_ok ? n : 0) * G;
-    const int64_t zend = p.N * G;
-    const uint32_t ring0 = base + L.ring + 4u * i;
+    int cseq = -1, pseq = -1, last_cc = -1, last_pc = -1;
 
-    auto ring_addr = [&](int slot, int w) -> uint32_t {
-      return ring0 + (uint32_t)((slot * RW + w) * 128 * 4);
-    };
-    auto first_group = [&](int64_t k0) -> int64_t { return k0 / p.group; };
-
-    // Stage s's codes, deltas and zero bytes into ring slot s % stages.
-    auto issue = [&](int s) {
+    for (int s = 0; s < n_total; ++s) {
+      const int k0 = (ks_begin + s) * kBK;
+      const int cc = k0 / kCodeCols, pc = k0 / gcols;
       if (s < n_main) {
-        const int slot = s % stages;
-        const int64_t k0 = (ks_begin + s) * kBK;
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const bool ok = row_ok && (k0 + 32 * b < p.K);
-#pragma unroll
-          for (int w = 0; w < BITS; ++w)
-            cp_async_4(ring_addr(slot, b * BITS + w),
-                       ok ? crow + (k0 / 32 + b) * BITS + w : p.codes,
-                       ok ? 4u : 0u);
+        if (cc != last_cc) {
+          last_cc = cc;
+          ++cseq;
+          if (!mbar_wait(b_full_c + 8 * (cseq % sc), (uint32_t)(cseq / sc) & 1,
+                         p.err)) {
+            *aborted = 1;
+            break;
+          }
         }
-        const int64_t g0 = first_group(k0);
-#pragma unroll
-        for (int j = 0; j < GPS; ++j) {
-          const bool ok = row_ok && (g0 + j) * p.group < p.K;
-          cp_async_4(ring_addr(slot, 2 * BITS + j), ok ? drow + g0 + j : p.delta,
-                     ok ? 4u : 0u);
-        }
-        const int64_t wa = (zrow + g0) & ~(int64_t)3;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int64_t wq = wa + 4 * q;
-          const uint32_t dst = ring_addr(slot, 2 * BITS + 4 + q);
-          if (row_ok && wq + 4 <= zend) {
-            cp_async_4(dst, p.zero + wq, 4u);
-          } else if (row_ok && wq < zend) {
-            uint32_t v = 0;
-            for (int b = 0; b < 4; ++b)
-              if (wq + b < zend) v |= (uint32_t)p.zero[wq + b] << (8 * b);
-            st_shared_u32(dst, v);
-          } else {
-            cp_async_4(dst, p.zero, 0u);
+        if (pc != last_pc) {
+          last_pc = pc;
+          ++pseq;
+          if (!mbar_wait(b_full_p + 8 * (pseq & 1), (uint32_t)(pseq >> 1) & 1,
+                         p.err)) {
+            *aborted = 1;
+            break;
           }
         }
       }
-      cp_async_commit();
-    };
-
-    for (int s = 0; s < stages - 1; ++s) issue(s);
-    for (int s = 0; s < n_total; ++s) {
-      issue(s + stages - 1);
-      cp_async_wait_dyn(stages - 1);
-      const int slot = s % stages;
-      const uint32_t it = (uint32_t)(s / stages);
-      if (s >= stages &&
-          !mbar_wait(bar_empty + 8 * slot, (it - 1) & 1, p.err)) {
+      const int sas = s % sa;
+      if (s >= sa &&
+          !mbar_wait(b_empty_a + 8 * sas, ((s / sa) - 1) & 1, p.err)) {
         *aborted = 1;
         break;
       }
       if (*aborted) break;
-      const uint32_t arow = base + L.a + slot * kATileBytes + i * 128;
+      const uint32_t arow = base + L.a + sas * kATileBytes + i * 128;
       const uint32_t swz = (uint32_t)(i & 7);
 
       if (s < n_main) {
-        const int64_t k0 = (ks_begin + s) * kBK;
-        uint32_t cw[2 * BITS];
+        const int blk = ((k0 % kCodeCols) >> 5) + h;  // block in the chunk
+        uint32_t cw[BITS];
+        load_block<BITS>(base + L.c + (cseq % sc) * code_chunk_bytes(BITS) +
+                             i * 16 * BITS + blk * 4 * BITS,
+                         cw);
+        const uint32_t pb = base + L.p + (pseq & 1) * kParamBytes;
+        const int gl0 = (k0 + 32 * h) / p.group - pc * kParamGroups;
+        __half2 zsub[GPB], dh[GPB];
 #pragma unroll
-        for (int w = 0; w < 2 * BITS; ++w) cw[w] = ld_shared_u32(ring_addr(slot, w));
-        __half2 zsub[GPS], dh[GPS];
-        const int64_t g0 = first_group(k0);
-        const uint64_t zz =
-            (((uint64_t)ld_shared_u32(ring_addr(slot, 2 * BITS + 5)) << 32) |
-             ld_shared_u32(ring_addr(slot, 2 * BITS + 4))) >>
-            (8 * ((zrow + g0) & 3));
-#pragma unroll
-        for (int j = 0; j < GPS; ++j) {
-          const uint32_t zj = (uint32_t)(zz >> (8 * j)) & 0xFFu;
+        for (int j = 0; j < GPB; ++j) {
+          const float dl = __uint_as_float(ld_shared_u32(pb + i * 64 + 4 * (gl0 + j)));
+          const uint32_t zj = ld_shared_u8(pb + kParamDeltaBytes + i * 16 + gl0 + j);
+          dh[j] = __float2half2_rn(dl);
           zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
-          dh[j] = __float2half2_rn(
-              __uint_as_float(ld_shared_u32(ring_addr(slot, 2 * BITS + j))));
         }
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk) {
-          const bool ok = k0 + 32 * blk < p.K;
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t o[4];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t o[4];
-#pragma unroll
-            for (int pp = 0; pp < 4; ++pp) {
-              const int c = 8 * cc + 2 * pp;  // code index in the block
-              const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
-              uint32_t x;
-              if (sh + 2 * BITS <= 32)
-                x = cw[blk * BITS + wd] >> sh;
-              else
-                x = __funnelshift_r(cw[blk * BITS + wd],
-                                    cw[blk * BITS + wd + 1], sh);
-              const uint32_t h = (x & QMASK) |
-                                 ((x << (16 - BITS)) & (QMASK << 16)) |
-                                 0x64006400u;  // fp16 pair (1024+q0, 1024+q1)
-              const int gl = GMODE == 0 ? (32 * blk + c) / 16
-                                        : (GMODE == 1 ? blk : 0);
-              o[pp] = h2_bits(__hmul2(__hsub2(bits_h2(h), zsub[gl]), dh[gl]));
-            }
-            if (!ok) o[0] = o[1] = o[2] = o[3] = 0u;
-            const uint32_t chunk = (uint32_t)(4 * blk + cc);
-            st_shared_v4(arow + ((chunk ^ swz) << 4), o[0], o[1], o[2], o[3]);
+          for (int pp = 0; pp < 4; ++pp) {
+            const int c = 8 * c8 + 2 * pp;  // code index in the block
+            const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
+            uint32_t x;
+            if (sh + 2 * BITS <= 32)
+              x = cw[wd] >> sh;
+            else
+              x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
+            // fp16 pair (1024 + q_c, 1024 + q_c+1)
+            const uint32_t hv = (x & QMASK) |
+                                ((x << (16 - BITS)) & (QMASK << 16)) |
+                                0x64006400u;
+            const int gl = GMODE == 0 ? c / 16 : 0;
+            o[pp] = h2_bits(__hmul2(__hsub2(bits_h2(hv), zsub[gl]), dh[gl]));
           }
+          const uint32_t chunk = (uint32_t)(4 * h + c8);
+          st_shared_v4(arow + ((chunk ^ swz) << 4), o[0], o[1], o[2], o[3]);
         }
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
 #pragma unroll 1
-        for (int chunk = 0; chunk < 8; ++chunk) {
+        for (int c8 = 0; c8 < 4; ++c8) {
+          const int chunk = 4 * h + c8;
           uint32_t o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int rho = chunk * 8 + 2 * e;
             float lo = 0.f, hi = 0.f;
-            if (row_ok && rho < p.r) lo = load_any(p.Blr, p.blr_t, n * p.r + rho);
+            if (row_ok && rho < p.r)
+              lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
             if (row_ok && rho + 1 < p.r)
-              hi = load_any(p.Blr, p.blr_t, n * p.r + rho + 1);
+              hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
             o[e] = h2_bits(__floats2half2_rn(lo, hi));
           }
           st_shared_v4(arow + (((uint32_t)chunk ^ swz) << 4), o[0], o[1], o[2],
@@ -390,31 +423,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar_full_a + 8 * slot);
+      mbar_arrive(b_full_a + 8 * sas);
+      if (s < n_main) {
+        const bool last = s + 1 >= n_main;
+        const int k1 = k0 + kBK;
+        if (last || k1 / kCodeCols != cc) mbar_arrive(b_empty_c + 8 * (cseq % sc));
+        if (last || k1 / gcols != pc) mbar_arrive(b_empty_p + 8 * (pseq & 1));
+      }
     }
-    cp_async_wait_all();
     __syncwarp();
 
     // ------------------------------------------------------ epilogue ----
-    const bool acc_ok = mbar_wait(bar_accum, 0, p.err);
+    const bool acc_ok = mbar_wait(b_accum, 0, p.err);
     tc_fence_after();
     const bool ok = acc_ok && !*aborted && n_total > 0;
-    const uint32_t t_lane = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+    const int half_cols = bn >= 32 ? bn / 2 : (h == 0 ? bn : 0);
+    const int c_begin = bn >= 32 ? h * (bn / 2) : 0;
     if (split == 1) {
-      for (int j = 0; j < p.bn; j += 16) {
+      for (int j = c_begin; j < c_begin + half_cols; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
         if (ok && row_ok) {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const int64_t t = t0 + j + c;
-            if (t < p.T) store_y(p.Y, p.yt, t * p.ldy + n, v[c]);
+            const int t = t0 + j + c;
+            if (t < p.T) store_y(p.Y, p.yt, (long long)t * p.ldy + n, v[c]);
           }
         }
       }
     } else {
       float* part = reinterpret_cast<float*>(gbase + L.a);
-      for (int j = 0; j < p.bn; j += 16) {
+      for (int j = c_begin; j < c_begin + half_cols; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
 #pragma unroll
@@ -427,17 +467,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (rank == 0 && warp >= 2) {
-      const int i = 32 * (warp & 3) + lane;
-      const int64_t n = m0 + i;
+      const int q4 = warp & 3, h = (warp - 2) >> 2;
+      const int i = 32 * q4 + lane;
+      const int n = m0 + i;
+      const int half_cols = bn >= 32 ? bn / 2 : (h == 0 ? bn : 0);
+      const int c_begin = bn >= 32 ? h * (bn / 2) : 0;
       float* part = reinterpret_cast<float*>(gbase + L.a);
       if (n < p.N && !*aborted) {
-        for (int c = 0; c < p.bn; ++c) {
-          const int64_t t = t0 + c;
+        for (int c = c_begin; c < c_begin + half_cols; ++c) {
+          const int t = t0 + c;
           if (t >= p.T) break;
           float acc = 0.f;
           for (int q = 0; q < split; ++q)
             acc += cluster.map_shared_rank(part, q)[c * kBM + i];
-          store_y(p.Y, p.yt, t * p.ldy + n, acc);
+          store_y(p.Y, p.yt, (long long)t * p.ldy + n, acc);
         }
       }
     }
@@ -525,28 +568,33 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2D fp16 tensor [rows][inner] with the given row pitch (elements); box of
-// 64 x box_rows with 128-byte swizzle; out-of-range elements read as zero.
-bool make_tmap_f16(CUtensorMap* m, const void* ptr, uint64_t inner,
-                   uint64_t rows, uint64_t pitch, uint32_t box_rows) {
+// 2D tensor [rows][inner] of `esize`-byte elements with a row pitch of
+// `pitch_bytes`, copied in boxes of box_inner x box_rows; out-of-range
+// elements read as zero.
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr,
+               uint64_t inner, uint64_t rows, uint64_t pitch_bytes,
+               uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {pitch * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr),
-            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+struct Maps {
+  CUtensorMap x, u, c, d, z;
+};
+
 template <int BITS, int GMODE>
-ttq_status launch_kernel(const CUtensorMap& tx, const CUtensorMap& tu,
-                         const GemmArgs& a, dim3 grid, int split,
-                         size_t smem, cudaStream_t st) {
+ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
+                         int split, size_t smem, cudaStream_t st) {
   auto kern = lowbit_gemm_kernel<BITS, GMODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
@@ -563,21 +611,21 @@ ttq_status launch_kernel(const CUtensorMap& tx, const CUtensorMap& tu,
   attr[0].val.clusterDim.z = (unsigned)split;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, tx, tu, a));
+  return cuda_status(
+      cudaLaunchKernelEx(&cfg, kern, m.x, m.u, m.c, m.d, m.z, a));
 }
 
 template <int GMODE>
-ttq_status dispatch_bits(int bits, const CUtensorMap& tx, const CUtensorMap& tu,
-                         const GemmArgs& a, dim3 grid, int split, size_t smem,
-                         cudaStream_t st) {
+ttq_status dispatch_bits(int bits, const Maps& m, const GemmArgs& a, dim3 grid,
+                         int split, size_t smem, cudaStream_t st) {
   switch (bits) {
-    case 2: return launch_kernel<2, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 3: return launch_kernel<3, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 4: return launch_kernel<4, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 5: return launch_kernel<5, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 6: return launch_kernel<6, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 7: return launch_kernel<7, GMODE>(tx, tu, a, grid, split, smem, st);
-    case 8: return launch_kernel<8, GMODE>(tx, tu, a, grid, split, smem, st);
+    case 2: return launch_kernel<2, GMODE>(m, a, grid, split, smem, st);
+    case 3: return launch_kernel<3, GMODE>(m, a, grid, split, smem, st);
+    case 4: return launch_kernel<4, GMODE>(m, a, grid, split, smem, st);
+    case 5: return launch_kernel<5, GMODE>(m, a, grid, split, smem, st);
+    case 6: return launch_kernel<6, GMODE>(m, a, grid, split, smem, st);
+    case 7: return launch_kernel<7, GMODE>(m, a, grid, split, smem, st);
+    case 8: return launch_kernel<8, GMODE>(m, a, grid, split, smem, st);
   }
   return TTQ_ERR_INVALID_ARG;
 }
@@ -630,14 +678,12 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   // token tile that still gives at least one CTA per SM.
   const int sms = sm_count();
   const int64_t tiles_m = (N + kBM - 1) / kBM;
-  const int64_t k_steps = (K + kBK - 1) / kBK;
+  const int k_steps = (int)((K + kBK - 1) / kBK);
   int bn = 16, split = 1;
   if (T <= 16) {
     split = (int)std::min<int64_t>(
         8, std::max<int64_t>(1, (2 * sms + tiles_m - 1) / tiles_m));
-    split = (int)std::min<int64_t>(split, k_steps);
-    const int64_t per = (k_steps + split - 1) / split;
-    split = (int)((k_steps + per - 1) / per);  // every rank gets >= 1 step
+    split = std::min(split, k_steps);
   } else if (T <= 32) {
     bn = 32;
   } else {
@@ -649,49 +695,65 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
         break;
       }
   }
+  int per = (k_steps + split - 1) / split;
+  split = (k_steps + per - 1) / per;  // every rank gets at least one step
   const int64_t tiles_t = (T + bn - 1) / bn;
 
-  const int per_stage = kATileBytes + bn * 128 + ring_words(bits) * 128 * 4;
-  const int stages = std::min(kMaxStages, (kSmemBudget - 2048) / per_stage);
-  if (stages < 2) return TTQ_ERR_UNSUPPORTED;
-  const SmemLayout L = smem_layout(bits, bn, stages);
+  // Ring depths: small token tiles keep two CTAs per SM, wide ones fill
+  // the shared memory with activation stages.
+  int sa = 3, sc = 2, sx;
+  const size_t fixed = (size_t)sa * kATileBytes + sc * code_chunk_bytes(bits) +
+                       2 * kParamBytes + 2048;
+  const size_t xtile = (size_t)bn * 128;
+  sx = (int)std::min<size_t>(8, (kMaxSmem - fixed) / xtile);
+  if (bn <= 64 && fixed + 3 * xtile <= 110 * 1024)  // two CTAs per SM
+    sx = (int)std::min<size_t>(6, (110 * 1024 - fixed) / xtile);
+  if (sx < 2) return TTQ_ERR_UNSUPPORTED;
+  const Layout L = make_layout(bits, bn, sx, sa, sc);
   const size_t smem = L.total + 1024;
+  if (split > 1 && (size_t)bn * kBM * 4 > (size_t)sa * kATileBytes)
+    return TTQ_ERR_UNSUPPORTED;
 
-  CUtensorMap tx, tu;
-  if (!make_tmap_f16(&tx, Xs, (uint64_t)K, (uint64_t)T, (uint64_t)K,
-                     (uint32_t)bn))
-    return TTQ_ERR_CUDA;
-  if (r > 0) {
-    if (!make_tmap_f16(&tu, U, 64, (uint64_t)T, 64, (uint32_t)bn))
-      return TTQ_ERR_CUDA;
-  } else {
-    tu = tx;  // never read without a low-rank stage
-  }
+  Maps m;
+  const int64_t G = K / group;
+  const bool ok =
+      make_tmap(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xs, K, T, K * 2, 64,
+                bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
+      make_tmap(&m.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32, N,
+                codes_ld(K, bits) * 4, 4 * bits, kBM,
+                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_tmap(&m.d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, delta, G, N,
+                groups_ld(K, group) * 4, kParamGroups, kBM,
+                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_tmap(&m.z, CU_TENSOR_MAP_DATA_TYPE_UINT8, zero, G, N,
+                groups_ld(K, group), kParamGroups, kBM,
+                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      (r == 0 || make_tmap(&m.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U, 64, T,
+                           128, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B));
+  if (!ok) return TTQ_ERR_CUDA;
+  if (r == 0) m.u = m.x;  // never read without a low-rank stage
 
   GemmArgs a;
-  a.codes = codes;
-  a.delta = delta;
-  a.zero = zero;
   a.Blr = B;
   a.blr_t = (int)bt;
   a.r = r;
-  a.N = N;
-  a.K = K;
-  a.T = T;
+  a.N = (int)N;
+  a.K = (int)K;
+  a.T = (int)T;
   a.Y = Y;
   a.yt = (int)yt;
   a.ldy = ldy;
   a.bn = bn;
-  a.stages = stages;
+  a.sx = sx;
+  a.sa = sa;
+  a.sc = sc;
   a.group = group;
   a.k_steps = k_steps;
+  a.per = per;
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
-  if (group == 16)
-    return dispatch_bits<0>(bits, tx, tu, a, grid, split, smem, st);
-  if (group == 32)
-    return dispatch_bits<1>(bits, tx, tu, a, grid, split, smem, st);
-  return dispatch_bits<2>(bits, tx, tu, a, grid, split, smem, st);
+  if (group == 16) return dispatch_bits<0>(bits, m, a, grid, split, smem, st);
+  return dispatch_bits<1>(bits, m, a, grid, split, smem, st);
 }
 
 ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,

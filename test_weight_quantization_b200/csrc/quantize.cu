@@ -90,9 +90,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
         __shfl_sync(0xffffffffu, (uint32_t)(chunk >> 32), qbase + j);
     c[j] = ((uint64_t)hi << 32) | lo;
   }
+  const int64_t ldc = codes_ld(K, BITS), ldg = groups_ld(K, group);
   if (active) {
-    const int64_t row_words = K * BITS / 32;
-    uint32_t* out = codes + n * row_words + (col0 / 32) * BITS;
+    uint32_t* out = codes + n * ldc + (col0 / 32) * BITS;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int wi = qpos + 4 * half;  // word index inside the block
@@ -109,9 +109,18 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
       out[wi] = word;
     }
     if ((lane & (lanes_per_group - 1)) == 0) {
-      const int64_t gi = n * (K / group) + col0 / group;
+      const int64_t gi = n * ldg + col0 / group;
       delta[gi] = d;
       zero[gi] = (uint8_t)z;
+    }
+  }
+  // the warp holding the row's first segment zeroes the row's padding
+  if (item % segs == 0) {
+    for (int64_t w = K * BITS / 32 + lane; w < ldc; w += 32)
+      codes[n * ldc + w] = 0u;
+    for (int64_t gi = K / group + lane; gi < ldg; gi += 32) {
+      delta[n * ldg + gi] = 0.f;
+      zero[n * ldg + gi] = 0;
     }
   }
 }
@@ -146,7 +155,7 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ codes, int64_t N,
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= N * blocks) return;
   const int64_t n = id / blocks, b = id % blocks;
-  const uint32_t* w = codes + n * (K * bits / 32) + b * bits;
+  const uint32_t* w = codes + n * codes_ld(K, bits) + b * bits;
   const uint32_t mask = (1u << bits) - 1u;
   uint8_t* out = q_out + n * K + b * 32;
   for (int c = 0; c < 32; ++c) {

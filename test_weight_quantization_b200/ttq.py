@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
         "ttq_status_string": [I],
         "ttq_device_error": [I],
         "ttq_abi_version": [],
+        "ttq_codes_ld": [I64, I],
+        "ttq_groups_ld": [I64, I],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -61,6 +63,8 @@ def _load() -> ctypes.CDLL:
         fn.restype = I
     lib.ttq_status_string.restype = ctypes.c_char_p
     lib.ttq_w_lowbit_gemm_workspace_size.restype = SZ
+    lib.ttq_codes_ld.restype = I64
+    lib.ttq_groups_ld.restype = I64
     return lib
 
 
@@ -71,7 +75,8 @@ EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_quantize_rtn_grouped",
            "ttq_w_lowbit_gemm_workspace_size", "ttq_w_lowbit_gemm",
            "ttq_prepare_activations", "ttq_w_lowbit_gemm_prepared",
            "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
-           "ttq_device_error", "ttq_abi_version")
+           "ttq_device_error", "ttq_abi_version", "ttq_codes_ld",
+           "ttq_groups_ld")
 
 
 class _Params(ctypes.Structure):
@@ -120,6 +125,16 @@ def abi_version() -> int:
     return int(_lib.ttq_abi_version())
 
 
+def codes_ld(K: int, bits: int) -> int:
+    """Row pitch (uint32 words) of the packed codes."""
+    return int(_lib.ttq_codes_ld(K, bits))
+
+
+def groups_ld(K: int, group: int) -> int:
+    """Row pitch (entries) of delta and zero."""
+    return int(_lib.ttq_groups_ld(K, group))
+
+
 def device_error(clear: bool = True) -> int:
     """Sticky device error bits (synchronising read)."""
     return int(_lib.ttq_device_error(1 if clear else 0))
@@ -156,17 +171,20 @@ def awq_scales(sums: torch.Tensor, T_total: int, alpha: float = 0.5,
 
 def quantize_rtn_grouped(W: torch.Tensor, s: torch.Tensor | None, bits: int,
                          group: int, codes=None, delta=None, zero=None):
-    """Step 3: packed codes [N, K*bits/32] u32 (as int32), delta [N, K/g]
-    fp32, zero [N, K/g] u8."""
+    """Step 3: packed codes [N, codes_ld] u32 (held as int32), delta
+    [N, groups_ld] fp32, zero [N, groups_ld] u8 (see ttq.h for the layout)."""
     ldw = _rows(W, "W")
     N, K = W.shape
     dev = W.device
     if codes is None:
-        codes = torch.empty((N, K * bits // 32), dtype=torch.int32, device=dev)
+        codes = torch.empty((N, codes_ld(K, bits)), dtype=torch.int32,
+                            device=dev)
     if delta is None:
-        delta = torch.empty((N, K // group), dtype=torch.float32, device=dev)
+        delta = torch.empty((N, groups_ld(K, group)), dtype=torch.float32,
+                            device=dev)
     if zero is None:
-        zero = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+        zero = torch.empty((N, groups_ld(K, group)), dtype=torch.uint8,
+                           device=dev)
     _check(_lib.ttq_quantize_rtn_grouped(
         W.data_ptr(), _DTYPE[W.dtype], N, K, ldw, _ptr(s), bits, group,
         codes.data_ptr(), delta.data_ptr(), zero.data_ptr(), _stream()),
@@ -282,12 +300,11 @@ class TTQLinear:
         self.sums = torch.empty(K, dtype=torch.float32, device=dev)
         self.s = torch.empty(K, dtype=torch.float32, device=dev)
         self.inv_s = torch.empty(K, dtype=torch.float32, device=dev)
-        self.codes = torch.empty((N, K * params.bits // 32), dtype=torch.int32,
-                                 device=dev)
-        self.delta = torch.empty((N, K // params.group), dtype=torch.float32,
-                                 device=dev)
-        self.zero = torch.empty((N, K // params.group), dtype=torch.uint8,
-                                device=dev)
+        self.codes = torch.empty((N, codes_ld(K, params.bits)),
+                                 dtype=torch.int32, device=dev)
+        gl = groups_ld(K, params.group)
+        self.delta = torch.empty((N, gl), dtype=torch.float32, device=dev)
+        self.zero = torch.empty((N, gl), dtype=torch.uint8, device=dev)
         self._ws = None
 
     def calibrate(self, X: torch.Tensor) -> None:

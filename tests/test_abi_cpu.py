@@ -45,7 +45,7 @@ def test_status_strings_and_version(lib):
     assert lib.ttq_status_string(0) == b"TTQ_OK"
     assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
     assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
-    assert lib.ttq_abi_version() == 1
+    assert lib.ttq_abi_version() == 2
 
 
 def test_workspace_size(lib):
@@ -100,3 +100,17 @@ def test_oracle_and_cuda_path_share_no_code():
                for i in includes), includes
     opy = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
     assert "test_weight_quantization_b200" not in opy
+
+
+def test_packed_pitches(lib):
+    lib.ttq_codes_ld.argtypes = [ctypes.c_int64, ctypes.c_int]
+    lib.ttq_codes_ld.restype = ctypes.c_int64
+    lib.ttq_groups_ld.argtypes = [ctypes.c_int64, ctypes.c_int]
+    lib.ttq_groups_ld.restype = ctypes.c_int64
+    assert lib.ttq_codes_ld(768, 3) == 72        # 72 words, already aligned
+    assert lib.ttq_codes_ld(96, 3) == 12         # 9 words padded to 12
+    assert lib.ttq_codes_ld(4096, 4) == 512
+    assert lib.ttq_groups_ld(768, 32) == 32      # 24 groups padded to 32
+    assert lib.ttq_groups_ld(4096, 128) == 32
+    assert lib.ttq_groups_ld(48, 16) == 16
+    assert lib.ttq_codes_ld(100, 3) == 0 and lib.ttq_groups_ld(96, 24) == 0

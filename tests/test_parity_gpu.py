@@ -91,13 +91,23 @@ def test_scales_zero_statistic(ttq):
 
 # ---------------------------------------------------------- quantize ----
 
+def dense(c, d, z, K, bits, group):
+    """The GPU's padded codes/delta/zero as dense numpy arrays; checks that
+    the padding is zero."""
+    c = c.cpu().numpy().view(np.uint32)
+    d = d.cpu().numpy()
+    z = z.cpu().numpy()
+    w, G = K * bits // 32, K // group
+    assert not c[:, w:].any() and not d[:, G:].any() and not z[:, G:].any()
+    return c[:, :w], d[:, :G], z[:, :G]
+
+
 def quantize_both(ttq, W, s, bits, group):
     c, d, z = ttq.quantize_rtn_grouped(W.cuda(), None if s is None else
                                        s.cuda(), bits, group)
     s_np = None if s is None else np32(s)
     rc, rd, rz = oracle.quantize(np32(W), s_np, bits, group)
-    return (c.cpu().numpy().view(np.uint32), d.cpu().numpy(), z.cpu().numpy(),
-            rc, rd, rz)
+    return (*dense(c, d, z, W.shape[1], bits, group), rc, rd, rz)
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
@@ -138,8 +148,8 @@ def test_unpack(ttq):
     for bits in (2, 3, 5, 8):
         c, _, _ = ttq.quantize_rtn_grouped(W.cuda(), None, bits, 32)
         q = ttq.unpack_codes(c, 160, bits).cpu().numpy()
-        np.testing.assert_array_equal(
-            q, oracle.unpack_codes(c.cpu().numpy().view(np.uint32), 160, bits))
+        cd = c.cpu().numpy().view(np.uint32)[:, :160 * bits // 32]
+        np.testing.assert_array_equal(q, oracle.unpack_codes(cd, 160, bits))
 
 
 # -------------------------------------------------------------- gemm ----
@@ -160,10 +170,10 @@ def run_path(ttq, X, W, bits, group, A=None, B=None, out_dtype=None,
 
 
 def oracle_y(X, inv, c, d, z, N, bits, group, A=None, B=None, rows=None):
-    return oracle.lowbit_gemm(np32(X), np32(inv), c.cpu().numpy().view(
-        np.uint32), d.cpu().numpy(), z.cpu().numpy(), N, bits, group,
-        None if A is None else np32(A), None if B is None else np32(B),
-        rows=rows)
+    cd, dd, zd = dense(c, d, z, X.shape[1], bits, group)
+    return oracle.lowbit_gemm(np32(X), np32(inv), cd, dd, zd, N, bits, group,
+                              None if A is None else np32(A),
+                              None if B is None else np32(B), rows=rows)
 
 
 @pytest.mark.parametrize("T", [1, 4, 16, 17, 100, 300])
