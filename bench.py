@@ -131,7 +131,7 @@ class Step:
                 self.sums[k], self.T, wl.alpha, wl.lam, wl.p, self.s[k],
                 self.inv[k])))
             out.append(("prepare", lambda k=k, A=A: t.prepare_activations(
-                X[k], self.inv[k], A, self.Xs[k], self.U.get(k))))
+                X[k], self.inv[k], wl.bits, A, self.Xs[k], self.U.get(k))))
         for L in self.layers:
             k, n = L.input_name, L.name
             out.append(("quantize", lambda k=k, n=n: t.quantize_rtn_grouped(

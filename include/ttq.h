@@ -181,20 +181,26 @@ ttq_status ttq_w_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
  * or time the tensor-core kernel alone.
  *
  * ttq_prepare_activations: the activation side of step 4.
- *   Xs[t][j] = fp16(X[t][j] * inv_s[j])        Xs [T, K] fp16, dense
+ *   Xs[t][P(j)] = fp16(X[t][j] * inv_s[j])     Xs [T, K] fp16, dense
+ * where P permutes channels inside each aligned span of 16 to match the
+ * order in which the kernel unpacks `bits`-bit codes: for bits = 2, 4, 8
+ * position p of a span holds channel (p>>1) + 8(p&1), 8(p>>3) + ((p&7)>>1)
+ * + 4(p&1), or 4(p>>2) + ((p&3)>>1) + 2(p&1) of that span; for other widths
+ * P is the identity. Xs is therefore only valid for codes of that width.
  *   U[t][rho] = fp16(sum_j X[t][j] A[rho][j])  U [T, 64] fp16, dense, zero
  *                                               for rho >= r (r > 0 only)
  * A is [r, K] of dtype xt; pass A = U = NULL with r = 0.
  * Raises TTQ_DEVERR_FP16_RANGE if |X * inv_s| reaches the fp16 range. */
 ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt, int64_t T,
                                    int64_t K, int64_t ldx, const float* inv_s,
-                                   const void* A, int r, void* Xs, void* U,
-                                   void* stream);
+                                   int bits, const void* A, int r, void* Xs,
+                                   void* U, void* stream);
 
 /* ttq_w_lowbit_gemm_prepared: the tensor-core projection on prepared
  * operands, one kernel launch:
  *   Y[t][n] = sum_j Xs[t][j] (q[n][j] - z) D + sum_rho U[t][rho] B[n][rho].
- * Xs, U as written by ttq_prepare_activations; B [N, r] of dtype bt. */
+ * Xs, U as written by ttq_prepare_activations for the same bits; B [N, r]
+ * of dtype bt. */
 ttq_status ttq_w_lowbit_gemm_prepared(const void* Xs, const void* U,
                                       int64_t T, int64_t K,
                                       const uint32_t* codes,

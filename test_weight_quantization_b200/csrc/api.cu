@@ -192,16 +192,17 @@ TTQ_EXPORT ttq_status ttq_w_lowbit_gemm(
 
 TTQ_EXPORT ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt,
                                               int64_t T, int64_t K, int64_t ldx,
-                                              const float* inv_s,
+                                              const float* inv_s, int bits,
                                               const void* A, int r, void* Xs,
                                               void* U, void* stream) {
-  if (!X || !inv_s || !Xs || !valid_dtype(xt) || T < 1 || K < 8 ||
-      K % 8 != 0 || ldx < K || r < 0 || r > 64 || ((r > 0) != (A && U)) ||
+  if (!X || !inv_s || !Xs || !valid_dtype(xt) || T < 1 || K < 32 ||
+      K % 32 != 0 || bits < 2 || bits > 8 || ldx < K || r < 0 || r > 64 ||
+      ((r > 0) != (A && U)) ||
       (r == 0 && (A || U)) || !rows_aligned(X, xt, ldx) ||
       !aligned(inv_s, 16) || !aligned(Xs, 16) || (U && !aligned(U, 16)) ||
       (r > 0 && !rows_aligned(A, xt, K)))
     return TTQ_ERR_INVALID_ARG;
-  return launch_prepare(X, xt, T, K, ldx, inv_s, A, r, Xs, U,
+  return launch_prepare(X, xt, T, K, ldx, inv_s, bits, A, r, Xs, U,
                         as_stream(stream));
 }
 

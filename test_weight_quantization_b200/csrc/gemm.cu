@@ -155,6 +155,73 @@ __device__ __forceinline__ float load_any(const void* p, int t, long long idx) {
   return static_cast<const float*>(p)[idx];
 }
 
+// Dequantises one 32-code block (BITS words in cw) into four 16-byte fp16
+// chunks (4h .. 4h+3) of a 128B-swizzled weight-tile row: w = (q - z) * D,
+// each pair built as fp16 (1024 + q) by OR-ing the code into the mantissa,
+// then (1024 + q) - (1024 + z), then times D (one fp16 rounding).
+template <int BITS, int GMODE>
+__device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
+                                              const __half2* zsub,
+                                              const __half2* dh, uint32_t arow,
+                                              int h, uint32_t swz) {
+  constexpr uint32_t QMASK = (1u << BITS) - 1u;
+  auto cvt = [&](uint32_t pair, int gl) -> uint32_t {
+    return h2_bits(__hmul2(__hsub2(bits_h2(pair | 0x64006400u), zsub[gl]),
+                           dh[gl]));
+  };
+  if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
+    // codes c and c + 16/BITS sit 16 bits apart in one word: one shift and
+    // mask yield the pair; the chunk order follows k_perm<BITS>
+    constexpr int PER_WORD = 32 / BITS;   // codes per word
+    constexpr int PAIRS = PER_WORD / 2;   // pairs per word
+    constexpr uint32_t PMASK = QMASK | (QMASK << 16);
+    uint32_t o[16];
+#pragma unroll
+    for (int wd = 0; wd < BITS; ++wd)
+#pragma unroll
+      for (int j = 0; j < PAIRS; ++j) {
+        const int gl = GMODE == 0 ? (wd * PER_WORD) / 16 : 0;
+        o[wd * PAIRS + j] = cvt((cw[wd] >> (BITS * j)) & PMASK, gl);
+      }
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8)
+      st_shared_v4(arow + (((uint32_t)(4 * h + c8) ^ swz) << 4), o[4 * c8],
+                   o[4 * c8 + 1], o[4 * c8 + 2], o[4 * c8 + 3]);
+  } else {
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8) {
+      uint32_t o[4];
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp) {
+        const int c = 8 * c8 + 2 * pp;  // code index in the block
+        const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
+        uint32_t x;
+        if (sh + 2 * BITS <= 32)
+          x = cw[wd] >> sh;
+        else
+          x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
+        const uint32_t pair = (x & QMASK) | ((x << (16 - BITS)) & (QMASK << 16));
+        o[pp] = cvt(pair, GMODE == 0 ? c / 16 : 0);
+      }
+      st_shared_v4(arow + (((uint32_t)(4 * h + c8) ^ swz) << 4), o[0], o[1],
+                   o[2], o[3]);
+    }
+  }
+}
+
+// Position in a ring of `depth` slots: the slot and how many times the
+// ring has wrapped (its parity is the mbarrier phase of the slot's use).
+struct Ring {
+  int slot = 0;
+  uint32_t round = 0;
+  __device__ __forceinline__ void next(int depth) {
+    if (++slot == depth) {
+      slot = 0;
+      ++round;
+    }
+  }
+};
+
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
 template <int BITS, int GMODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -166,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const GemmArgs p) {
   constexpr uint32_t QMASK = (1u << BITS) - 1u;
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
+  constexpr uint32_t CHUNK = kBM * 16 * BITS;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -197,7 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ks_end = min(ks_begin + p.per, p.k_steps);
   const int n_main = ks_end - ks_begin;
   const int n_total = n_main + ((p.r > 0 && rank == 0) ? 1 : 0);
-  const int gcols = kParamGroups * p.group;  // channels per params chunk
+  const int lg = 31 - __clz(p.group);            // log2(g)
+  const int pmask = (kParamGroups << lg) - 1;   // channels per params chunk - 1
   const uint32_t tmem_cols = bn < 32 ? 32u : (uint32_t)bn;
 
   if (threadIdx.x == 0) {
@@ -238,87 +307,94 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_d);
       tma_prefetch_desc(&tm_z);
       if (p.r > 0) tma_prefetch_desc(&tm_u);
-      int cseq = -1, pseq = -1, last_cc = -1, last_pc = -1, issued = 0;
+      Ring rx, rc, rp;
+      int nx = 0, nc = 0, np = 0;  // loads issued per ring
       bool ok = true;
-      for (int s = 0; s < n_total && ok; ++s) {
+      int k0 = ks_begin * kBK;
+      for (int s = 0; s < n_total && ok; ++s, k0 += kBK) {
         if (s < n_main) {
-          const int k0 = (ks_begin + s) * kBK;
-          const int cc = k0 / kCodeCols;
-          if (cc != last_cc) {
-            last_cc = cc;
-            ++cseq;
-            const int slot = cseq % sc;
-            if (cseq >= sc &&
-                !mbar_wait(b_empty_c + 8 * slot, ((cseq / sc) - 1) & 1, p.err)) {
+          if (s == 0 || (k0 & (kCodeCols - 1)) == 0) {
+            if (nc >= sc && !mbar_wait(b_empty_c + 8 * rc.slot,
+                                       (rc.round & 1) ^ 1, p.err)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(b_full_c + 8 * slot, code_chunk_bytes(BITS));
-            tma_load_2d(base + L.c + slot * code_chunk_bytes(BITS), &tm_c,
-                        cc * 4 * BITS, m0, b_full_c + 8 * slot);
+            const uint32_t bar = b_full_c + 8 * rc.slot;
+            mbar_arrive_expect_tx(bar, CHUNK);
+            tma_load_2d(base + L.c + rc.slot * CHUNK, &tm_c,
+                        (k0 / kCodeCols) * 4 * BITS, m0, bar);
+            rc.next(sc);
+            ++nc;
           }
-          const int pc = k0 / gcols;
-          if (pc != last_pc) {
-            last_pc = pc;
-            ++pseq;
-            const int slot = pseq & 1;
-            if (pseq >= 2 &&
-                !mbar_wait(b_empty_p + 8 * slot, ((pseq >> 1) - 1) & 1, p.err)) {
+          if (s == 0 || (k0 & pmask) == 0) {
+            if (np >= 2 && !mbar_wait(b_empty_p + 8 * rp.slot,
+                                      (rp.round & 1) ^ 1, p.err)) {
               ok = false;
               break;
             }
-            const uint32_t dst = base + L.p + slot * kParamBytes;
-            mbar_arrive_expect_tx(b_full_p + 8 * slot, kParamBytes);
-            tma_load_2d(dst, &tm_d, pc * kParamGroups, m0, b_full_p + 8 * slot);
-            tma_load_2d(dst + kParamDeltaBytes, &tm_z, pc * kParamGroups, m0,
-                        b_full_p + 8 * slot);
+            const uint32_t bar = b_full_p + 8 * rp.slot;
+            const uint32_t dst = base + L.p + rp.slot * kParamBytes;
+            const int g0 = (k0 >> lg) & ~(kParamGroups - 1);
+            mbar_arrive_expect_tx(bar, kParamBytes);
+            tma_load_2d(dst, &tm_d, g0, m0, bar);
+            tma_load_2d(dst + kParamDeltaBytes, &tm_z, g0, m0, bar);
+            rp.next(2);
+            ++np;
           }
         }
-        const int slot = s % sx;
-        if (s >= sx &&
-            !mbar_wait(b_empty_x + 8 * slot, ((s / sx) - 1) & 1, p.err)) {
+        if (nx >= sx &&
+            !mbar_wait(b_empty_x + 8 * rx.slot, (rx.round & 1) ^ 1, p.err)) {
           ok = false;
           break;
         }
         if (*aborted) break;
-        mbar_arrive_expect_tx(b_full_x + 8 * slot, (uint32_t)bn * 128u);
+        const uint32_t bar = b_full_x + 8 * rx.slot;
+        mbar_arrive_expect_tx(bar, (uint32_t)bn * 128u);
         if (s < n_main)
-          tma_load_2d(base + L.x + slot * bn * 128, &tm_x,
-                      (ks_begin + s) * kBK, t0, b_full_x + 8 * slot);
+          tma_load_2d(base + L.x + rx.slot * bn * 128, &tm_x, k0, t0, bar);
         else
-          tma_load_2d(base + L.x + slot * bn * 128, &tm_u, 0, t0,
-                      b_full_x + 8 * slot);
-        issued = s + 1;
+          tma_load_2d(base + L.x + rx.slot * bn * 128, &tm_u, 0, t0, bar);
+        rx.next(sx);
+        ++nx;
       }
       if (!ok) *aborted = 1;
-      // never leave a bulk copy in flight into shared memory at exit
-      for (int s = max(0, issued - sx); s < issued; ++s)
-        mbar_wait(b_full_x + 8 * (s % sx), (uint32_t)(s / sx) & 1, p.err);
-      for (int q = max(0, cseq - sc + 1); q <= cseq; ++q)
+      // never leave a bulk copy in flight into shared memory at exit: wait
+      // for the last use of every slot that was loaded
+      for (int i = 0; i < sx && i < nx; ++i) {
+        const int q = nx - 1 - i;
+        mbar_wait(b_full_x + 8 * (q % sx), (uint32_t)(q / sx) & 1, p.err);
+      }
+      for (int i = 0; i < sc && i < nc; ++i) {
+        const int q = nc - 1 - i;
         mbar_wait(b_full_c + 8 * (q % sc), (uint32_t)(q / sc) & 1, p.err);
-      for (int q = max(0, pseq - 1); q <= pseq; ++q)
+      }
+      for (int i = 0; i < 2 && i < np; ++i) {
+        const int q = np - 1 - i;
         mbar_wait(b_full_p + 8 * (q & 1), (uint32_t)(q >> 1) & 1, p.err);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kBM, bn);
+      Ring rx, ra;
       for (int s = 0; s < n_total; ++s) {
-        const int sxs = s % sx, sas = s % sa;
-        if (!mbar_wait(b_full_x + 8 * sxs, (uint32_t)(s / sx) & 1, p.err) ||
-            !mbar_wait(b_full_a + 8 * sas, (uint32_t)(s / sa) & 1, p.err)) {
+        if (!mbar_wait(b_full_x + 8 * rx.slot, rx.round & 1, p.err) ||
+            !mbar_wait(b_full_a + 8 * ra.slot, ra.round & 1, p.err)) {
           *aborted = 1;
           break;
         }
         tc_fence_after();
-        const uint64_t ad = smem_desc_sw128(base + L.a + sas * kATileBytes);
-        const uint64_t bd = smem_desc_sw128(base + L.x + sxs * bn * 128);
+        const uint64_t ad = smem_desc_sw128(base + L.a + ra.slot * kATileBytes);
+        const uint64_t bd = smem_desc_sw128(base + L.x + rx.slot * bn * 128);
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k)
           tc_mma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc,
                      (s > 0 || k > 0) ? 1u : 0u);
-        tc_commit(b_empty_x + 8 * sxs);
-        tc_commit(b_empty_a + 8 * sas);
+        tc_commit(b_empty_x + 8 * rx.slot);
+        tc_commit(b_empty_a + 8 * ra.slot);
+        rx.next(sx);
+        ra.next(sa);
       }
       tc_commit(b_accum);
     }
@@ -329,79 +405,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
     const int n = m0 + i;
     const bool row_ok = n < p.N;
-    int cseq = -1, pseq = -1, last_cc = -1, last_pc = -1;
+    const uint32_t swz = (uint32_t)(i & 7);
+    const uint32_t crow = base + L.c + i * 16 * BITS;
+    // delta tile: 64-byte rows in the 64B swizzle (16-byte chunk index XOR
+    // bits 1-2 of the row); zero tile: plain 16-byte rows
+    const uint32_t drow = base + L.p + i * 64;
+    const uint32_t dswz = (uint32_t)((i >> 1) & 3);
+    const uint32_t zrow = base + L.p + kParamDeltaBytes + i * 16;
+    Ring ra, rc, rp;
+    bool first = true;
+    int k0 = ks_begin * kBK;
 
-    for (int s = 0; s < n_total; ++s) {
-      const int k0 = (ks_begin + s) * kBK;
-      const int cc = k0 / kCodeCols, pc = k0 / gcols;
+    for (int s = 0; s < n_total; ++s, k0 += kBK) {
       if (s < n_main) {
-        if (cc != last_cc) {
-          last_cc = cc;
-          ++cseq;
-          if (!mbar_wait(b_full_c + 8 * (cseq % sc), (uint32_t)(cseq / sc) & 1,
-                         p.err)) {
+        if (first || (k0 & (kCodeCols - 1)) == 0) {
+          if (!first) rc.next(sc);
+          if (!mbar_wait(b_full_c + 8 * rc.slot, rc.round & 1, p.err)) {
             *aborted = 1;
             break;
           }
         }
-        if (pc != last_pc) {
-          last_pc = pc;
-          ++pseq;
-          if (!mbar_wait(b_full_p + 8 * (pseq & 1), (uint32_t)(pseq >> 1) & 1,
-                         p.err)) {
+        if (first || (k0 & pmask) == 0) {
+          if (!first) rp.next(2);
+          if (!mbar_wait(b_full_p + 8 * rp.slot, rp.round & 1, p.err)) {
             *aborted = 1;
             break;
           }
         }
+        first = false;
       }
-      const int sas = s % sa;
       if (s >= sa &&
-          !mbar_wait(b_empty_a + 8 * sas, ((s / sa) - 1) & 1, p.err)) {
+          !mbar_wait(b_empty_a + 8 * ra.slot, (ra.round & 1) ^ 1, p.err)) {
         *aborted = 1;
         break;
       }
       if (*aborted) break;
-      const uint32_t arow = base + L.a + sas * kATileBytes + i * 128;
-      const uint32_t swz = (uint32_t)(i & 7);
+      const uint32_t arow = base + L.a + ra.slot * kATileBytes + i * 128;
 
       if (s < n_main) {
-        const int blk = ((k0 % kCodeCols) >> 5) + h;  // block in the chunk
+        const int blk = ((k0 & (kCodeCols - 1)) >> 5) + h;  // block in chunk
         uint32_t cw[BITS];
-        load_block<BITS>(base + L.c + (cseq % sc) * code_chunk_bytes(BITS) +
-                             i * 16 * BITS + blk * 4 * BITS,
-                         cw);
-        const uint32_t pb = base + L.p + (pseq & 1) * kParamBytes;
-        const int gl0 = (k0 + 32 * h) / p.group - pc * kParamGroups;
+        load_block<BITS>(crow + rc.slot * CHUNK + blk * 4 * BITS, cw);
+        const uint32_t poff = rp.slot * kParamBytes;
+        const int gl0 = ((k0 + 32 * h) >> lg) & (kParamGroups - 1);
         __half2 zsub[GPB], dh[GPB];
 #pragma unroll
         for (int j = 0; j < GPB; ++j) {
-          const float dl = __uint_as_float(ld_shared_u32(pb + i * 64 + 4 * (gl0 + j)));
-          const uint32_t zj = ld_shared_u8(pb + kParamDeltaBytes + i * 16 + gl0 + j);
+          const int gl = gl0 + j;
+          const float dl = __uint_as_float(ld_shared_u32(
+              drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) + 4 * (gl & 3)));
+          const uint32_t zj = ld_shared_u8(zrow + poff + gl);
           dh[j] = __float2half2_rn(dl);
           zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
         }
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t o[4];
-#pragma unroll
-          for (int pp = 0; pp < 4; ++pp) {
-            const int c = 8 * c8 + 2 * pp;  // code index in the block
-            const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
-            uint32_t x;
-            if (sh + 2 * BITS <= 32)
-              x = cw[wd] >> sh;
-            else
-              x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
-            // fp16 pair (1024 + q_c, 1024 + q_c+1)
-            const uint32_t hv = (x & QMASK) |
-                                ((x << (16 - BITS)) & (QMASK << 16)) |
-                                0x64006400u;
-            const int gl = GMODE == 0 ? c / 16 : 0;
-            o[pp] = h2_bits(__hmul2(__hsub2(bits_h2(hv), zsub[gl]), dh[gl]));
-          }
-          const uint32_t chunk = (uint32_t)(4 * h + c8);
-          st_shared_v4(arow + ((chunk ^ swz) << 4), o[0], o[1], o[2], o[3]);
-        }
+        dequant_block<BITS, GMODE>(cw, zsub, dh, arow, h, swz);
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
 #pragma unroll 1
@@ -423,12 +480,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(b_full_a + 8 * sas);
+      mbar_arrive(b_full_a + 8 * ra.slot);
+      ra.next(sa);
       if (s < n_main) {
         const bool last = s + 1 >= n_main;
         const int k1 = k0 + kBK;
-        if (last || k1 / kCodeCols != cc) mbar_arrive(b_empty_c + 8 * (cseq % sc));
-        if (last || k1 / gcols != pc) mbar_arrive(b_empty_p + 8 * (pseq & 1));
+        if (last || (k1 & (kCodeCols - 1)) == 0)
+          mbar_arrive(b_empty_c + 8 * rc.slot);
+        if (last || (k1 & pmask) == 0) mbar_arrive(b_empty_p + 8 * rp.slot);
       }
     }
     __syncwarp();
@@ -492,30 +551,53 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) tmem_dealloc(tmem, tmem_cols);
 }
 
-// X~ = fp16(X * inv_s), one thread per 8 channels.
-template <typename TX>
+// Position p of a 16-channel span of the prepared activations holds channel
+// k_perm<PERM>(p) of that span. For 2-, 4- and 8-bit codes the dequantiser
+// turns one shifted code word into an fp16 pair (q_c, q_c') whose channels
+// lie 8, 4 or 2 apart; the activations are stored in the same order so the
+// tensor-core products pair the right operands. Other widths keep the
+// natural order.
+template <int PERM>
+__host__ __device__ constexpr int k_perm(int p) {
+  return PERM == 2   ? (p >> 1) + 8 * (p & 1)
+         : PERM == 4 ? 8 * (p >> 3) + ((p & 7) >> 1) + 4 * (p & 1)
+         : PERM == 8 ? 4 * (p >> 2) + ((p & 3) >> 1) + 2 * (p & 1)
+                     : p;
+}
+
+// X~ = fp16(X * inv_s), one thread per 16 channels, K-permuted for PERM.
+template <typename TX, int PERM>
 __global__ void prescale_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
                                 int64_t ldx, const float* __restrict__ inv_s,
                                 __half* __restrict__ Xs, uint32_t* err) {
-  const int64_t chunks = K / 8;
+  const int64_t spans = K / 16;
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= T * chunks) return;
-  const int64_t t = id / chunks, c = (id % chunks) * 8;
-  float v[8];
-  load8<TX>(X + t * ldx + c, v);
-  const float4 s0 = __ldg(reinterpret_cast<const float4*>(inv_s + c));
-  const float4 s1 = __ldg(reinterpret_cast<const float4*>(inv_s + c + 4));
-  const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  uint32_t o[4];
+  if (id >= T * spans) return;
+  const int64_t t = id / spans, c = (id % spans) * 16;
+  float v[16], sv[16];
+  load8<TX>(X + t * ldx + c, *reinterpret_cast<float(*)[8]>(v));
+  load8<TX>(X + t * ldx + c + 8, *reinterpret_cast<float(*)[8]>(v + 8));
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 s4 = __ldg(reinterpret_cast<const float4*>(inv_s + c) + q);
+    sv[4 * q] = s4.x;
+    sv[4 * q + 1] = s4.y;
+    sv[4 * q + 2] = s4.z;
+    sv[4 * q + 3] = s4.w;
+  }
+  uint32_t o[8];
   bool bad = false;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float a = __fmul_rn(v[2 * e], sv[2 * e]);
-    const float b = __fmul_rn(v[2 * e + 1], sv[2 * e + 1]);
-    bad |= !(fabsf(a) < 65520.f) || !(fabsf(b) < 65520.f);
-    o[e] = h2_bits(__floats2half2_rn(a, b));
+  for (int e = 0; e < 8; ++e) {
+    const int la = k_perm<PERM>(2 * e), lb = k_perm<PERM>(2 * e + 1);
+    const float fa = __fmul_rn(v[la], sv[la]);
+    const float fb = __fmul_rn(v[lb], sv[lb]);
+    bad |= !(fabsf(fa) < 65520.f) || !(fabsf(fb) < 65520.f);
+    o[e] = h2_bits(__floats2half2_rn(fa, fb));
   }
-  *reinterpret_cast<uint4*>(Xs + t * K + c) = make_uint4(o[0], o[1], o[2], o[3]);
+  uint4* dst = reinterpret_cast<uint4*>(Xs + t * K + c);
+  dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
   if (bad) flag_error(err, TTQ_DEVERR_FP16_RANGE);
 }
 
@@ -632,17 +714,23 @@ ttq_status dispatch_bits(int bits, const Maps& m, const GemmArgs& a, dim3 grid,
 
 template <typename TX>
 ttq_status launch_pre(const void* X, int64_t T, int64_t K, int64_t ldx,
-                      const float* inv_s, const void* A, int r, __half* Xs,
-                      __half* U, cudaStream_t st) {
-  const int64_t items = T * (K / 8);
+                      const float* inv_s, int bits, const void* A, int r,
+                      __half* Xs, __half* U, cudaStream_t st) {
+  const int64_t items = T * (K / 16);
   const int threads = 256;
-  prescale_kernel<TX><<<(unsigned)((items + threads - 1) / threads), threads,
-                        0, st>>>(static_cast<const TX*>(X), T, K, ldx, inv_s,
-                                 Xs, device_error_word());
+  const unsigned grid = (unsigned)((items + threads - 1) / threads);
+  const TX* x = static_cast<const TX*>(X);
+  uint32_t* err = device_error_word();
+  switch (bits) {
+    case 2: prescale_kernel<TX, 2><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
+    case 4: prescale_kernel<TX, 4><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
+    case 8: prescale_kernel<TX, 8><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
+    default: prescale_kernel<TX, 0><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
+  }
   ttq_status e = launch_status();
   if (e != TTQ_OK || r == 0) return e;
   lowrank_u_kernel<TX><<<(unsigned)T, 256, 0, st>>>(
-      static_cast<const TX*>(X), T, K, ldx, static_cast<const TX*>(A), r, U);
+      x, T, K, ldx, static_cast<const TX*>(A), r, U);
   return launch_status();
 }
 
@@ -655,15 +743,19 @@ size_t gemm_workspace_bytes(int64_t T, int64_t K, int r) {
 }
 
 ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
-                          int64_t ldx, const float* inv_s, const void* A,
-                          int r, void* Xs, void* U, cudaStream_t st) {
+                          int64_t ldx, const float* inv_s, int bits,
+                          const void* A, int r, void* Xs, void* U,
+                          cudaStream_t st) {
   __half* xs = static_cast<__half*>(Xs);
   __half* u = static_cast<__half*>(U);
   switch (xt) {
-    case TTQ_F32: return launch_pre<float>(X, T, K, ldx, inv_s, A, r, xs, u, st);
+    case TTQ_F32:
+      return launch_pre<float>(X, T, K, ldx, inv_s, bits, A, r, xs, u, st);
     case TTQ_BF16:
-      return launch_pre<__nv_bfloat16>(X, T, K, ldx, inv_s, A, r, xs, u, st);
-    case TTQ_F16: return launch_pre<__half>(X, T, K, ldx, inv_s, A, r, xs, u, st);
+      return launch_pre<__nv_bfloat16>(X, T, K, ldx, inv_s, bits, A, r, xs, u,
+                                       st);
+    case TTQ_F16:
+      return launch_pre<__half>(X, T, K, ldx, inv_s, bits, A, r, xs, u, st);
   }
   return TTQ_ERR_INVALID_ARG;
 }
@@ -674,43 +766,54 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t N, int bits, int group, const void* B,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
                                 int64_t ldy, cudaStream_t st) {
-  // Tile shape: decode splits K over a cluster; prefill picks the widest
-  // token tile that still gives at least one CTA per SM.
+  // Tile shape. Decode (T <= 32) streams the codes: a 4-deep codes ring,
+  // small activation tiles, K split over a cluster so that one wave of
+  // CTAs covers the GPU. Prefill picks the token tile with the least
+  // modelled time: waves x (fixed cost + K steps x max(MMA, dequant)),
+  // where a 64-channel step costs about 2*bn tensor cycles and ~300 cycles
+  // of dequantisation.
   const int sms = sm_count();
   const int64_t tiles_m = (N + kBM - 1) / kBM;
   const int k_steps = (int)((K + kBK - 1) / kBK);
-  int bn = 16, split = 1;
-  if (T <= 16) {
-    split = (int)std::min<int64_t>(
-        8, std::max<int64_t>(1, (2 * sms + tiles_m - 1) / tiles_m));
-    split = std::min(split, k_steps);
-  } else if (T <= 32) {
-    bn = 32;
+  const uint32_t cchunk = code_chunk_bytes(bits);
+  int bn, sx, sa, sc, split = 1;
+  if (T <= 32) {
+    bn = T <= 16 ? 16 : 32;
+    sa = 2;
+    sx = 4;
+    sc = 4;
+    while (sc > 2 && (size_t)make_layout(bits, bn, sx, sa, sc).total + 1024 >
+                         110 * 1024)
+      --sc;
   } else {
-    bn = 64;
-    const int cand[2] = {256, 128};
-    for (int c : cand)
-      if (tiles_m * ((T + c - 1) / c) >= sms) {
+    bn = 256;
+    double best = 1e30;
+    for (int c : {256, 128, 64}) {
+      const int64_t ctas = tiles_m * ((T + c - 1) / c);
+      const int64_t waves = (ctas + sms - 1) / sms;
+      const double t = (double)waves * (4000.0 + k_steps * std::max(2.0 * c, 300.0));
+      if (t < best) {
+        best = t;
         bn = c;
-        break;
       }
+    }
+    sa = 3;
+    sc = 2;
+    const size_t fixed = (size_t)sa * kATileBytes + sc * cchunk +
+                         2 * kParamBytes + 2048;
+    sx = (int)std::min<size_t>(8, (kMaxSmem - fixed) / ((size_t)bn * 128));
   }
-  int per = (k_steps + split - 1) / split;
-  split = (k_steps + per - 1) / per;  // every rank gets at least one step
-  const int64_t tiles_t = (T + bn - 1) / bn;
-
-  // Ring depths: small token tiles keep two CTAs per SM, wide ones fill
-  // the shared memory with activation stages.
-  int sa = 3, sc = 2, sx;
-  const size_t fixed = (size_t)sa * kATileBytes + sc * code_chunk_bytes(bits) +
-                       2 * kParamBytes + 2048;
-  const size_t xtile = (size_t)bn * 128;
-  sx = (int)std::min<size_t>(8, (kMaxSmem - fixed) / xtile);
-  if (bn <= 64 && fixed + 3 * xtile <= 110 * 1024)  // two CTAs per SM
-    sx = (int)std::min<size_t>(6, (110 * 1024 - fixed) / xtile);
   if (sx < 2) return TTQ_ERR_UNSUPPORTED;
   const Layout L = make_layout(bits, bn, sx, sa, sc);
   const size_t smem = L.total + 1024;
+  if (T <= 32) {
+    const int per_sm = smem <= 113 * 1024 ? 2 : 1;
+    split = (int)std::min<int64_t>(8, std::max<int64_t>(1, per_sm * sms / tiles_m));
+    split = std::min(split, k_steps);
+  }
+  const int per = (k_steps + split - 1) / split;
+  split = (k_steps + per - 1) / per;  // every rank gets at least one step
+  const int64_t tiles_t = (T + bn - 1) / bn;
   if (split > 1 && (size_t)bn * kBM * 4 > (size_t)sa * kATileBytes)
     return TTQ_ERR_UNSUPPORTED;
 
@@ -724,7 +827,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
       make_tmap(&m.d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, delta, G, N,
                 groups_ld(K, group) * 4, kParamGroups, kBM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_tmap(&m.z, CU_TENSOR_MAP_DATA_TYPE_UINT8, zero, G, N,
                 groups_ld(K, group), kParamGroups, kBM,
                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
@@ -768,7 +871,8 @@ ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
                                        align_up((size_t)T * (size_t)K * 2,
                                                 1024))
                   : nullptr;
-  ttq_status e = launch_prepare(X, xt, T, K, ldx, inv_s, A, r, Xs, U, st);
+  ttq_status e =
+      launch_prepare(X, xt, T, K, ldx, inv_s, bits, A, r, Xs, U, st);
   if (e != TTQ_OK) return e;
   return launch_gemm_prepared(Xs, U, T, K, codes, delta, zero, N, bits, group,
                               B, xt, r, Y, yt, ldy, st);

@@ -37,8 +37,9 @@ ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
                               void* workspace, cudaStream_t st);
 
 ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
-                          int64_t ldx, const float* inv_s, const void* A,
-                          int r, void* Xs, void* U, cudaStream_t st);
+                          int64_t ldx, const float* inv_s, int bits,
+                          const void* A, int r, void* Xs, void* U,
+                          cudaStream_t st);
 
 ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t K, const uint32_t* codes,

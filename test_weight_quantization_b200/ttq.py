@@ -46,7 +46,7 @@ def _load() -> ctypes.CDLL:
         "ttq_w_lowbit_gemm_workspace_size": [I64, I64, I],
         "ttq_w_lowbit_gemm": [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P,
                               I, P, I, I64, P, SZ, P],
-        "ttq_prepare_activations": [P, I, I64, I64, I64, P, P, I, P, P, P],
+        "ttq_prepare_activations": [P, I, I64, I64, I64, P, I, P, I, P, P, P],
         "ttq_w_lowbit_gemm_prepared": [P, P, I64, I64, P, P, P, I64, I, I, P,
                                        I, I, P, I, I64, P],
         "ttq_lowrank_add": [P, I, I64, I64, I64, P, P, I, I64, P, I, I64, P],
@@ -221,10 +221,11 @@ def w_lowbit_gemm(X: torch.Tensor, inv_s: torch.Tensor, codes: torch.Tensor,
     return out
 
 
-def prepare_activations(X: torch.Tensor, inv_s: torch.Tensor,
+def prepare_activations(X: torch.Tensor, inv_s: torch.Tensor, bits: int,
                         A: torch.Tensor | None = None, Xs=None, U=None):
-    """Activation side of step 4: Xs = fp16(X diag(inv_s)) [T, K] and, with
-    low-rank factors, U = fp16(X A^T) zero-padded to [T, 64]."""
+    """Activation side of step 4: Xs = fp16(X diag(inv_s)) [T, K] (channels
+    ordered for `bits`-bit codes, see ttq.h) and, with low-rank factors,
+    U = fp16(X A^T) zero-padded to [T, 64]."""
     ldx = _rows(X, "X")
     T, K = X.shape
     r = 0 if A is None else A.shape[0]
@@ -233,8 +234,8 @@ def prepare_activations(X: torch.Tensor, inv_s: torch.Tensor,
     if r and U is None:
         U = torch.empty((T, 64), dtype=torch.float16, device=X.device)
     _check(_lib.ttq_prepare_activations(
-        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(), _ptr(A), r,
-        Xs.data_ptr(), _ptr(U) if r else None, _stream()),
+        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(), bits,
+        _ptr(A), r, Xs.data_ptr(), _ptr(U) if r else None, _stream()),
         "ttq_prepare_activations")
     return Xs, (U if r else None)
 
