@@ -40,13 +40,12 @@ namespace ttq {
 namespace {
 
 constexpr int kBM = 128;           // weight rows per CTA (TMEM lanes)
-constexpr int kBK = 64;            // channels per MMA stage (128 B of fp16)
-constexpr int kCodeCols = 128;     // channels per codes chunk
+constexpr int kSK = 128;           // channels per pipeline stage
+constexpr int kSCols = kSK / 2;    // TMEM columns of one fp16 weight stage
 constexpr int kParamGroups = 16;   // groups per params chunk
-constexpr int kDequantWarps = 8;
+constexpr int kDequantWarps = 4;
 constexpr int kDq = 32 * kDequantWarps;  // dequantiser threads
 constexpr int kThreads = 64 + kDq;       // + producer warp + MMA warp
-constexpr int kATileBytes = kBM * kBK * 2;
 constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
 constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
 constexpr int kMaxSmem = 225 * 1024;
@@ -59,11 +58,13 @@ struct GemmArgs {
   void* Y;
   int yt;  // ttq_dtype of Y
   long long ldy;
-  int bn;              // tokens per tile (MMA N)
-  int sx, sa, sc;      // ring depths: activations, weight tiles, codes
+  int bn;         // tokens per tile (MMA N)
+  int S;          // pipeline depth (stages of 128 channels)
+  int tmem_cols;  // TMEM allocation: accumulator + S weight stages
+  int acc_cols;   // TMEM columns reserved for the accumulator
   int group;
-  int k_steps;         // ceil(K / 64)
-  int per;             // K steps per split rank
+  int k_stages;   // ceil(K / 128)
+  int per;        // stages per split rank
   uint32_t* err;
 };
 
@@ -72,31 +73,28 @@ __host__ __device__ inline uint32_t code_chunk_bytes(int bits) {
 }
 
 struct Layout {
-  uint32_t x, a, c, p, bars, tmem, abort_flag, total;
+  uint32_t x, c, p, part, bars, tmem, abort_flag, total, stage_x;
 };
 
-__host__ __device__ inline Layout make_layout(int bits, int bn, int sx, int sa,
-                                              int sc) {
+// Shared memory: per stage two 64-channel activation boxes and one codes
+// chunk; two params slots; the split-K partial tile (decode); barriers.
+// The fp16 weight stages live in TMEM.
+__host__ __device__ inline Layout make_layout(int bits, int bn, int S,
+                                              bool split) {
   Layout L;
+  L.stage_x = (uint32_t)(2 * bn * 128);
   L.x = 0;
-  L.a = L.x + (uint32_t)(sx * bn * 128);
-  L.c = L.a + (uint32_t)(sa * kATileBytes);
-  L.p = L.c + (uint32_t)sc * code_chunk_bytes(bits);
-  L.bars = L.p + 2u * kParamBytes;
-  const int nbars = 2 * sx + 2 * sa + 2 * sc + 4 + 1;
+  L.c = L.x + (uint32_t)S * L.stage_x;
+  L.p = L.c + (uint32_t)S * code_chunk_bytes(bits);
+  L.part = L.p + 2u * kParamBytes;
+  L.bars = L.part + (split ? (uint32_t)(bn * kBM * 4) : 0u);
+  const int nbars = 3 * S + 4 + 1;
   L.tmem = L.bars + 8u * nbars;
   L.abort_flag = L.tmem + 4;
   L.total = L.abort_flag + 4;
   return L;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a,
-                                             uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a),
-               "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
@@ -155,15 +153,15 @@ __device__ __forceinline__ float load_any(const void* p, int t, long long idx) {
   return static_cast<const float*>(p)[idx];
 }
 
-// Dequantises one 32-code block (BITS words in cw) into four 16-byte fp16
-// chunks (4h .. 4h+3) of a 128B-swizzled weight-tile row: w = (q - z) * D,
-// each pair built as fp16 (1024 + q) by OR-ing the code into the mantissa,
-// then (1024 + q) - (1024 + z), then times D (one fp16 rounding).
+// Dequantises one 32-code block (BITS words in cw) into the 16 fp16 pairs
+// o[0..15], o[p] holding block positions 2p and 2p+1: w = (q - z) * D, each
+// pair built as fp16 (1024 + q) by OR-ing the code into the mantissa, then
+// (1024 + q) - (1024 + z), then times D (one fp16 rounding).
 template <int BITS, int GMODE>
 __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
                                               const __half2* zsub,
-                                              const __half2* dh, uint32_t arow,
-                                              int h, uint32_t swz) {
+                                              const __half2* dh,
+                                              uint32_t* o) {
   constexpr uint32_t QMASK = (1u << BITS) - 1u;
   auto cvt = [&](uint32_t pair, int gl) -> uint32_t {
     return h2_bits(__hmul2(__hsub2(bits_h2(pair | 0x64006400u), zsub[gl]),
@@ -171,11 +169,10 @@ __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
   };
   if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
     // codes c and c + 16/BITS sit 16 bits apart in one word: one shift and
-    // mask yield the pair; the chunk order follows k_perm<BITS>
+    // mask yield the pair; positions follow k_perm<BITS>
     constexpr int PER_WORD = 32 / BITS;   // codes per word
     constexpr int PAIRS = PER_WORD / 2;   // pairs per word
     constexpr uint32_t PMASK = QMASK | (QMASK << 16);
-    uint32_t o[16];
 #pragma unroll
     for (int wd = 0; wd < BITS; ++wd)
 #pragma unroll
@@ -183,28 +180,18 @@ __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
         const int gl = GMODE == 0 ? (wd * PER_WORD) / 16 : 0;
         o[wd * PAIRS + j] = cvt((cw[wd] >> (BITS * j)) & PMASK, gl);
       }
-#pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8)
-      st_shared_v4(arow + (((uint32_t)(4 * h + c8) ^ swz) << 4), o[4 * c8],
-                   o[4 * c8 + 1], o[4 * c8 + 2], o[4 * c8 + 3]);
   } else {
 #pragma unroll
-    for (int c8 = 0; c8 < 4; ++c8) {
-      uint32_t o[4];
-#pragma unroll
-      for (int pp = 0; pp < 4; ++pp) {
-        const int c = 8 * c8 + 2 * pp;  // code index in the block
-        const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
-        uint32_t x;
-        if (sh + 2 * BITS <= 32)
-          x = cw[wd] >> sh;
-        else
-          x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
-        const uint32_t pair = (x & QMASK) | ((x << (16 - BITS)) & (QMASK << 16));
-        o[pp] = cvt(pair, GMODE == 0 ? c / 16 : 0);
-      }
-      st_shared_v4(arow + (((uint32_t)(4 * h + c8) ^ swz) << 4), o[0], o[1],
-                   o[2], o[3]);
+    for (int pp = 0; pp < 16; ++pp) {
+      const int c = 2 * pp;  // code index in the block
+      const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
+      uint32_t x;
+      if (sh + 2 * BITS <= 32)
+        x = cw[wd] >> sh;
+      else
+        x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
+      const uint32_t pair = (x & QMASK) | ((x << (16 - BITS)) & (QMASK << 16));
+      o[pp] = cvt(pair, GMODE == 0 ? c / 16 : 0);
     }
   }
 }
@@ -222,16 +209,23 @@ struct Ring {
   }
 };
 
+// Stage protocol (slot = stage % S):
+//   producer   waits `empty` (previous use done), then loads the codes
+//              chunk and both activation boxes, completing on `loaded`;
+//   dequant    waits `loaded`, writes the fp16 weight stage to TMEM, then
+//              arrives on `ready` (this also vouches that the activations
+//              have landed, since it observed `loaded`);
+//   MMA        waits `ready`, issues 8 MMAs, commits to `empty`, which frees
+//              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
 template <int BITS, int GMODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_c,
                        const __grid_constant__ CUtensorMap tm_d,
                        const __grid_constant__ CUtensorMap tm_z,
                        const GemmArgs p) {
-  constexpr uint32_t QMASK = (1u << BITS) - 1u;
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
 
@@ -240,15 +234,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw_base + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - raw_base);
 
-  const int sx = p.sx, sa = p.sa, sc = p.sc, bn = p.bn;
-  const Layout L = make_layout(BITS, bn, sx, sa, sc);
-  const uint32_t b_full_x = base + L.bars;
-  const uint32_t b_empty_x = b_full_x + 8 * sx;
-  const uint32_t b_full_a = b_empty_x + 8 * sx;
-  const uint32_t b_empty_a = b_full_a + 8 * sa;
-  const uint32_t b_full_c = b_empty_a + 8 * sa;
-  const uint32_t b_empty_c = b_full_c + 8 * sc;
-  const uint32_t b_full_p = b_empty_c + 8 * sc;
+  const int S = p.S, bn = p.bn;
+  const int split = (int)gridDim.z;
+  const Layout L = make_layout(BITS, bn, S, split > 1);
+  const uint32_t b_loaded = base + L.bars;
+  const uint32_t b_ready = b_loaded + 8 * S;
+  const uint32_t b_empty = b_ready + 8 * S;
+  const uint32_t b_full_p = b_empty + 8 * S;
   const uint32_t b_empty_p = b_full_p + 16;
   const uint32_t b_accum = b_empty_p + 16;
   volatile uint32_t* tmem_slot =
@@ -259,28 +251,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kBM;
   const int t0 = blockIdx.y * bn;
-  const int split = (int)gridDim.z;
   const int rank = (int)blockIdx.z;
-  const int ks_begin = min(rank * p.per, p.k_steps);
-  const int ks_end = min(ks_begin + p.per, p.k_steps);
+  const int ks_begin = min(rank * p.per, p.k_stages);
+  const int ks_end = min(ks_begin + p.per, p.k_stages);
   const int n_main = ks_end - ks_begin;
   const int n_total = n_main + ((p.r > 0 && rank == 0) ? 1 : 0);
-  const int lg = 31 - __clz(p.group);            // log2(g)
-  const int pmask = (kParamGroups << lg) - 1;   // channels per params chunk - 1
-  const uint32_t tmem_cols = bn < 32 ? 32u : (uint32_t)bn;
+  const int lg = 31 - __clz(p.group);  // log2(g)
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < sx; ++i) {
-      mbar_init(b_full_x + 8 * i, 1);
-      mbar_init(b_empty_x + 8 * i, 1);
-    }
-    for (int i = 0; i < sa; ++i) {
-      mbar_init(b_full_a + 8 * i, kDq);
-      mbar_init(b_empty_a + 8 * i, 1);
-    }
-    for (int i = 0; i < sc; ++i) {
-      mbar_init(b_full_c + 8 * i, 1);
-      mbar_init(b_empty_c + 8 * i, kDq);
+    for (int i = 0; i < S; ++i) {
+      mbar_init(b_loaded + 8 * i, 1);
+      mbar_init(b_ready + 8 * i, kDq);
+      mbar_init(b_empty + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
@@ -291,13 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(base + L.tmem, tmem_cols);
+    tmem_alloc(base + L.tmem, (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_a = tmem + (uint32_t)p.acc_cols;  // weight-stage ring
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
@@ -307,26 +290,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_d);
       tma_prefetch_desc(&tm_z);
       if (p.r > 0) tma_prefetch_desc(&tm_u);
-      Ring rx, rc, rp;
-      int nx = 0, nc = 0, np = 0;  // loads issued per ring
+      const uint32_t xbytes = (uint32_t)bn * 128u;
+      Ring rs, rp;
+      int pchunk = -1, issued = 0, np = 0;
       bool ok = true;
-      int k0 = ks_begin * kBK;
-      for (int s = 0; s < n_total && ok; ++s, k0 += kBK) {
+      for (int s = 0; s < n_total; ++s) {
+        const int k0 = (ks_begin + s) * kSK;
         if (s < n_main) {
-          if (s == 0 || (k0 & (kCodeCols - 1)) == 0) {
-            if (nc >= sc && !mbar_wait(b_empty_c + 8 * rc.slot,
-                                       (rc.round & 1) ^ 1, p.err)) {
-              ok = false;
-              break;
-            }
-            const uint32_t bar = b_full_c + 8 * rc.slot;
-            mbar_arrive_expect_tx(bar, CHUNK);
-            tma_load_2d(base + L.c + rc.slot * CHUNK, &tm_c,
-                        (k0 / kCodeCols) * 4 * BITS, m0, bar);
-            rc.next(sc);
-            ++nc;
-          }
-          if (s == 0 || (k0 & pmask) == 0) {
+          const int pc = k0 >> (lg + 4);  // params chunk: 16 groups
+          if (pc != pchunk) {
+            if (pchunk >= 0) rp.next(2);
+            pchunk = pc;
             if (np >= 2 && !mbar_wait(b_empty_p + 8 * rp.slot,
                                       (rp.round & 1) ^ 1, p.err)) {
               ok = false;
@@ -334,39 +308,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const uint32_t bar = b_full_p + 8 * rp.slot;
             const uint32_t dst = base + L.p + rp.slot * kParamBytes;
-            const int g0 = (k0 >> lg) & ~(kParamGroups - 1);
             mbar_arrive_expect_tx(bar, kParamBytes);
-            tma_load_2d(dst, &tm_d, g0, m0, bar);
-            tma_load_2d(dst + kParamDeltaBytes, &tm_z, g0, m0, bar);
-            rp.next(2);
+            tma_load_2d(dst, &tm_d, pc * kParamGroups, m0, bar);
+            tma_load_2d(dst + kParamDeltaBytes, &tm_z, pc * kParamGroups, m0,
+                        bar);
             ++np;
           }
         }
-        if (nx >= sx &&
-            !mbar_wait(b_empty_x + 8 * rx.slot, (rx.round & 1) ^ 1, p.err)) {
+        if (s >= S &&
+            !mbar_wait(b_empty + 8 * rs.slot, (rs.round & 1) ^ 1, p.err)) {
           ok = false;
           break;
         }
         if (*aborted) break;
-        const uint32_t bar = b_full_x + 8 * rx.slot;
-        mbar_arrive_expect_tx(bar, (uint32_t)bn * 128u);
-        if (s < n_main)
-          tma_load_2d(base + L.x + rx.slot * bn * 128, &tm_x, k0, t0, bar);
-        else
-          tma_load_2d(base + L.x + rx.slot * bn * 128, &tm_u, 0, t0, bar);
-        rx.next(sx);
-        ++nx;
+        const uint32_t bar = b_loaded + 8 * rs.slot;
+        const uint32_t xdst = base + L.x + rs.slot * L.stage_x;
+        if (s < n_main) {
+          mbar_arrive_expect_tx(bar, CHUNK + 2 * xbytes);
+          tma_load_2d(base + L.c + rs.slot * CHUNK, &tm_c, (k0 >> 7) * 4 * BITS,
+                      m0, bar);
+          tma_load_2d(xdst, &tm_x, k0, t0, bar);
+          tma_load_2d(xdst + xbytes, &tm_x, k0 + 64, t0, bar);
+        } else {
+          mbar_arrive_expect_tx(bar, xbytes);
+          tma_load_2d(xdst, &tm_u, 0, t0, bar);
+        }
+        rs.next(S);
+        issued = s + 1;
       }
       if (!ok) *aborted = 1;
       // never leave a bulk copy in flight into shared memory at exit: wait
       // for the last use of every slot that was loaded
-      for (int i = 0; i < sx && i < nx; ++i) {
-        const int q = nx - 1 - i;
-        mbar_wait(b_full_x + 8 * (q % sx), (uint32_t)(q / sx) & 1, p.err);
-      }
-      for (int i = 0; i < sc && i < nc; ++i) {
-        const int q = nc - 1 - i;
-        mbar_wait(b_full_c + 8 * (q % sc), (uint32_t)(q / sc) & 1, p.err);
+      for (int i = 0; i < S && i < issued; ++i) {
+        const int q = issued - 1 - i;
+        mbar_wait(b_loaded + 8 * (q % S), (uint32_t)(q / S) & 1, p.err);
       }
       for (int i = 0; i < 2 && i < np; ++i) {
         const int q = np - 1 - i;
@@ -377,119 +352,119 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------- MMA issuer -----
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kBM, bn);
-      Ring rx, ra;
+      const uint32_t xbytes = (uint32_t)bn * 128u;
+      Ring rs;
       for (int s = 0; s < n_total; ++s) {
-        if (!mbar_wait(b_full_x + 8 * rx.slot, rx.round & 1, p.err) ||
-            !mbar_wait(b_full_a + 8 * ra.slot, ra.round & 1, p.err)) {
+        if (!mbar_wait(b_ready + 8 * rs.slot, rs.round & 1, p.err)) {
           *aborted = 1;
           break;
         }
         tc_fence_after();
-        const uint64_t ad = smem_desc_sw128(base + L.a + ra.slot * kATileBytes);
-        const uint64_t bd = smem_desc_sw128(base + L.x + rx.slot * bn * 128);
+        const uint32_t ad = tmem_a + (uint32_t)(rs.slot * kSCols);
+        const uint32_t xs = base + L.x + rs.slot * L.stage_x;
+        const uint64_t bd0 = smem_desc_sw128(xs);
+        const uint64_t bd1 = smem_desc_sw128(xs + xbytes);
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          tc_mma_f16(tmem, ad + 2 * k, bd + 2 * k, idesc,
-                     (s > 0 || k > 0) ? 1u : 0u);
-        tc_commit(b_empty_x + 8 * rx.slot);
-        tc_commit(b_empty_a + 8 * ra.slot);
-        rx.next(sx);
-        ra.next(sa);
+        for (int k = 0; k < 4; ++k)
+          tc_mma_f16_ts(tmem, ad + 8 * k, bd0 + 2 * k, idesc,
+                        (s > 0 || k > 0) ? 1u : 0u);
+        if (s < n_main) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ts(tmem, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
+        }
+        tc_commit(b_empty + 8 * rs.slot);
+        rs.next(S);
       }
       tc_commit(b_accum);
     }
   } else {
     // ------------------------------------------------ dequantisers ----
-    const int q4 = warp & 3;         // TMEM lane quarter
-    const int h = (warp - 2) >> 2;   // which 32-code block of a 64-col stage
+    // One thread per weight row (= TMEM lane): a stage is four 32-code
+    // blocks, 64 fp16 pairs, written to the TMEM weight ring in two stores.
+    const int q4 = warp & 3;         // TMEM lane quarter of this warp
     const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
     const int n = m0 + i;
     const bool row_ok = n < p.N;
-    const uint32_t swz = (uint32_t)(i & 7);
     const uint32_t crow = base + L.c + i * 16 * BITS;
     // delta tile: 64-byte rows in the 64B swizzle (16-byte chunk index XOR
     // bits 1-2 of the row); zero tile: plain 16-byte rows
     const uint32_t drow = base + L.p + i * 64;
     const uint32_t dswz = (uint32_t)((i >> 1) & 3);
     const uint32_t zrow = base + L.p + kParamDeltaBytes + i * 16;
-    Ring ra, rc, rp;
-    bool first = true;
-    int k0 = ks_begin * kBK;
+    const uint32_t arow = tmem_a + ((uint32_t)(32 * q4) << 16);
+    Ring rs, rp;
+    int pchunk = -1;
+    bool ok_loop = true;
 
-    for (int s = 0; s < n_total; ++s, k0 += kBK) {
-      if (s < n_main) {
-        if (first || (k0 & (kCodeCols - 1)) == 0) {
-          if (!first) rc.next(sc);
-          if (!mbar_wait(b_full_c + 8 * rc.slot, rc.round & 1, p.err)) {
-            *aborted = 1;
-            break;
-          }
-        }
-        if (first || (k0 & pmask) == 0) {
-          if (!first) rp.next(2);
-          if (!mbar_wait(b_full_p + 8 * rp.slot, rp.round & 1, p.err)) {
-            *aborted = 1;
-            break;
-          }
-        }
-        first = false;
-      }
-      if (s >= sa &&
-          !mbar_wait(b_empty_a + 8 * ra.slot, (ra.round & 1) ^ 1, p.err)) {
-        *aborted = 1;
+    for (int s = 0; s < n_total && ok_loop; ++s) {
+      const int k0 = (ks_begin + s) * kSK;
+      if (!mbar_wait(b_loaded + 8 * rs.slot, rs.round & 1, p.err) ||
+          *aborted) {
+        ok_loop = false;
         break;
       }
-      if (*aborted) break;
-      const uint32_t arow = base + L.a + ra.slot * kATileBytes + i * 128;
-
+      const uint32_t acol = arow + (uint32_t)(rs.slot * kSCols);
       if (s < n_main) {
-        const int blk = ((k0 & (kCodeCols - 1)) >> 5) + h;  // block in chunk
-        uint32_t cw[BITS];
-        load_block<BITS>(crow + rc.slot * CHUNK + blk * 4 * BITS, cw);
-        const uint32_t poff = rp.slot * kParamBytes;
-        const int gl0 = ((k0 + 32 * h) >> lg) & (kParamGroups - 1);
-        __half2 zsub[GPB], dh[GPB];
-#pragma unroll
-        for (int j = 0; j < GPB; ++j) {
-          const int gl = gl0 + j;
-          const float dl = __uint_as_float(ld_shared_u32(
-              drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) + 4 * (gl & 3)));
-          const uint32_t zj = ld_shared_u8(zrow + poff + gl);
-          dh[j] = __float2half2_rn(dl);
-          zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
+        const int pc = k0 >> (lg + 4);
+        if (pc != pchunk) {
+          if (pchunk >= 0) rp.next(2);
+          pchunk = pc;
+          if (!mbar_wait(b_full_p + 8 * rp.slot, rp.round & 1, p.err)) {
+            ok_loop = false;
+            break;
+          }
         }
-        dequant_block<BITS, GMODE>(cw, zsub, dh, arow, h, swz);
+        const uint32_t poff = rp.slot * kParamBytes;
+        const uint32_t cbase = crow + rs.slot * CHUNK;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int blk = 2 * half + h;  // 32-code block of the stage
+            uint32_t cw[BITS];
+            load_block<BITS>(cbase + blk * 4 * BITS, cw);
+            const int gl0 = ((k0 + 32 * blk) >> lg) & (kParamGroups - 1);
+            __half2 zsub[GPB], dh[GPB];
+#pragma unroll
+            for (int j = 0; j < GPB; ++j) {
+              const int gl = gl0 + j;
+              const float dl = __uint_as_float(ld_shared_u32(
+                  drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
+                  4 * (gl & 3)));
+              const uint32_t zj = ld_shared_u8(zrow + poff + gl);
+              dh[j] = __float2half2_rn(dl);
+              zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
+            }
+            dequant_block<BITS, GMODE>(cw, zsub, dh, o + 16 * h);
+          }
+          tmem_st32(acol + 32u * half, o);
+        }
+        // release the params once their last stage is read
+        if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
+          mbar_arrive(b_empty_p + 8 * rp.slot);
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
-#pragma unroll 1
-        for (int c8 = 0; c8 < 4; ++c8) {
-          const int chunk = 4 * h + c8;
-          uint32_t o[4];
+        uint32_t o[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int rho = chunk * 8 + 2 * e;
-            float lo = 0.f, hi = 0.f;
-            if (row_ok && rho < p.r)
-              lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
-            if (row_ok && rho + 1 < p.r)
-              hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
-            o[e] = h2_bits(__floats2half2_rn(lo, hi));
-          }
-          st_shared_v4(arow + (((uint32_t)chunk ^ swz) << 4), o[0], o[1], o[2],
-                       o[3]);
+        for (int e = 0; e < 32; ++e) {
+          const int rho = 2 * e;
+          float lo = 0.f, hi = 0.f;
+          if (row_ok && rho < p.r)
+            lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
+          if (row_ok && rho + 1 < p.r)
+            hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
+          o[e] = h2_bits(__floats2half2_rn(lo, hi));
         }
+        tmem_st32(acol, o);
       }
-      fence_proxy_async_smem();
-      mbar_arrive(b_full_a + 8 * ra.slot);
-      ra.next(sa);
-      if (s < n_main) {
-        const bool last = s + 1 >= n_main;
-        const int k1 = k0 + kBK;
-        if (last || (k1 & (kCodeCols - 1)) == 0)
-          mbar_arrive(b_empty_c + 8 * rc.slot);
-        if (last || (k1 & pmask) == 0) mbar_arrive(b_empty_p + 8 * rp.slot);
-      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_ready + 8 * rs.slot);
+      rs.next(S);
     }
+    if (!ok_loop) *aborted = 1;
     __syncwarp();
 
     // ------------------------------------------------------ epilogue ----
@@ -497,10 +472,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const bool ok = acc_ok && !*aborted && n_total > 0;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
-    const int half_cols = bn >= 32 ? bn / 2 : (h == 0 ? bn : 0);
-    const int c_begin = bn >= 32 ? h * (bn / 2) : 0;
     if (split == 1) {
-      for (int j = c_begin; j < c_begin + half_cols; j += 16) {
+      for (int j = 0; j < bn; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
         if (ok && row_ok) {
@@ -512,8 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     } else {
-      float* part = reinterpret_cast<float*>(gbase + L.a);
-      for (int j = c_begin; j < c_begin + half_cols; j += 16) {
+      float* part = reinterpret_cast<float*>(gbase + L.part);
+      for (int j = 0; j < bn; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
 #pragma unroll
@@ -526,14 +499,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
     if (rank == 0 && warp >= 2) {
-      const int q4 = warp & 3, h = (warp - 2) >> 2;
-      const int i = 32 * q4 + lane;
+      const int i = 32 * (warp & 3) + lane;
       const int n = m0 + i;
-      const int half_cols = bn >= 32 ? bn / 2 : (h == 0 ? bn : 0);
-      const int c_begin = bn >= 32 ? h * (bn / 2) : 0;
-      float* part = reinterpret_cast<float*>(gbase + L.a);
+      float* part = reinterpret_cast<float*>(gbase + L.part);
       if (n < p.N && !*aborted) {
-        for (int c = c_begin; c < c_begin + half_cols; ++c) {
+        for (int c = 0; c < bn; ++c) {
           const int t = t0 + c;
           if (t >= p.T) break;
           float acc = 0.f;
@@ -548,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem, tmem_cols);
+  if (warp == 1) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
 }
 
 // Position p of a 16-channel span of the prepared activations holds channel
@@ -766,56 +736,64 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t N, int bits, int group, const void* B,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
                                 int64_t ldy, cudaStream_t st) {
-  // Tile shape. Decode (T <= 32) streams the codes: a 4-deep codes ring,
-  // small activation tiles, K split over a cluster so that one wave of
-  // CTAs covers the GPU. Prefill picks the token tile with the least
-  // modelled time: waves x (fixed cost + K steps x max(MMA, dequant)),
-  // where a 64-channel step costs about 2*bn tensor cycles and ~300 cycles
-  // of dequantisation.
+  // Tile shape. A stage is 128 channels: a codes chunk, two 64-channel
+  // activation boxes, one 64-column fp16 weight stage in TMEM.
+  // Decode (T <= 32): 256 TMEM columns per CTA (two CTAs per SM), K split
+  // over a cluster so that about one wave covers the GPU.
+  // Prefill: all 512 TMEM columns; the token tile is picked by a model of
+  // waves x (fixed cost + stages x max(MMA, dequant)), an MMA of N tokens
+  // costing about max(45, N/2) cycles (eight per stage) and a stage about
+  // 600 cycles of dequantisation.
   const int sms = sm_count();
   const int64_t tiles_m = (N + kBM - 1) / kBM;
-  const int k_steps = (int)((K + kBK - 1) / kBK);
+  const int k_stages = (int)((K + kSK - 1) / kSK);
   const uint32_t cchunk = code_chunk_bytes(bits);
-  int bn, sx, sa, sc, split = 1;
+  int bn, S, tmem_cols, acc_cols, split = 1;
+  auto fits = [&](int bn_, int S_, bool sp, size_t lim) {
+    return (size_t)make_layout(bits, bn_, S_, sp).total + 1024 <= lim;
+  };
   if (T <= 32) {
     bn = T <= 16 ? 16 : 32;
-    sa = 2;
-    sx = 4;
-    sc = 4;
-    while (sc > 2 && (size_t)make_layout(bits, bn, sx, sa, sc).total + 1024 >
-                         110 * 1024)
-      --sc;
+    acc_cols = 32;
+    tmem_cols = 256;
+    S = (tmem_cols - acc_cols) / kSCols;
+    while (S > 2 && !fits(bn, S, true, 110 * 1024)) --S;
   } else {
-    bn = 256;
+    bn = 64;
     double best = 1e30;
-    for (int c : {256, 128, 64}) {
+    for (int c : {256, 192, 128, 64}) {
+      int s_ = std::min(6, (512 - c) / kSCols);
+      while (s_ > 1 && !fits(c, s_, false, kMaxSmem)) --s_;
+      if (s_ < 2) continue;
       const int64_t ctas = tiles_m * ((T + c - 1) / c);
       const int64_t waves = (ctas + sms - 1) / sms;
-      const double t = (double)waves * (4000.0 + k_steps * std::max(2.0 * c, 300.0));
+      const double stage = std::max(8.0 * std::max(45.0, c / 2.0), 600.0);
+      // shallow pipelines expose the load latency
+      const double depth_penalty = s_ < 3 ? 1.25 : 1.0;
+      const double t = (double)waves * (4000.0 + k_stages * stage * depth_penalty);
       if (t < best) {
         best = t;
         bn = c;
       }
     }
-    sa = 3;
-    sc = 2;
-    const size_t fixed = (size_t)sa * kATileBytes + sc * cchunk +
-                         2 * kParamBytes + 2048;
-    sx = (int)std::min<size_t>(8, (kMaxSmem - fixed) / ((size_t)bn * 128));
+    acc_cols = bn;
+    tmem_cols = 512;
+    S = std::min(6, (tmem_cols - acc_cols) / kSCols);
+    while (S > 1 && !fits(bn, S, false, kMaxSmem)) --S;
   }
-  if (sx < 2) return TTQ_ERR_UNSUPPORTED;
-  const Layout L = make_layout(bits, bn, sx, sa, sc);
-  const size_t smem = L.total + 1024;
+  if (S < 2) return TTQ_ERR_UNSUPPORTED;
   if (T <= 32) {
-    const int per_sm = smem <= 113 * 1024 ? 2 : 1;
-    split = (int)std::min<int64_t>(8, std::max<int64_t>(1, per_sm * sms / tiles_m));
-    split = std::min(split, k_steps);
+    const size_t sm1 = make_layout(bits, bn, S, true).total + 1024;
+    const int per_sm = sm1 <= 113 * 1024 ? 2 : 1;
+    split = (int)std::min<int64_t>(
+        8, std::max<int64_t>(1, per_sm * sms / tiles_m));
+    split = std::min(split, k_stages);
   }
-  const int per = (k_steps + split - 1) / split;
-  split = (k_steps + per - 1) / per;  // every rank gets at least one step
+  const int per = (k_stages + split - 1) / split;
+  split = (k_stages + per - 1) / per;  // every rank gets at least one stage
+  const Layout L = make_layout(bits, bn, S, split > 1);
+  const size_t smem = L.total + 1024;
   const int64_t tiles_t = (T + bn - 1) / bn;
-  if (split > 1 && (size_t)bn * kBM * 4 > (size_t)sa * kATileBytes)
-    return TTQ_ERR_UNSUPPORTED;
 
   Maps m;
   const int64_t G = K / group;
@@ -847,11 +825,11 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.yt = (int)yt;
   a.ldy = ldy;
   a.bn = bn;
-  a.sx = sx;
-  a.sa = sa;
-  a.sc = sc;
+  a.S = S;
+  a.tmem_cols = tmem_cols;
+  a.acc_cols = acc_cols;
   a.group = group;
-  a.k_steps = k_steps;
+  a.k_stages = k_stages;
   a.per = per;
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
