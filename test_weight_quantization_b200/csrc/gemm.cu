@@ -43,9 +43,9 @@ constexpr int kBM = 128;           // weight rows per CTA (TMEM lanes)
 constexpr int kSK = 128;           // channels per pipeline stage
 constexpr int kSCols = kSK / 2;    // TMEM columns of one fp16 weight stage
 constexpr int kParamGroups = 16;   // groups per params chunk
-constexpr int kDequantWarps = 4;
-constexpr int kDq = 32 * kDequantWarps;  // dequantiser threads
-constexpr int kThreads = 64 + kDq;       // + producer warp + MMA warp
+// CTA = producer warp + MMA warp + DQW dequantiser warps (4 or 8; with 8,
+// two warps share each TMEM lane quarter and split every stage in halves)
+__host__ __device__ constexpr int cta_threads(int dqw) { return 64 + 32 * dqw; }
 constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
 constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
 constexpr int kMaxSmem = 225 * 1024;
@@ -156,17 +156,16 @@ __device__ __forceinline__ float load_any(const void* p, int t, long long idx) {
 // Dequantises one 32-code block (BITS words in cw) into the 16 fp16 pairs
 // o[0..15], o[p] holding block positions 2p and 2p+1: w = (q - z) * D, each
 // pair built as fp16 (1024 + q) by OR-ing the code into the mantissa, then
-// (1024 + q) - (1024 + z), then times D (one fp16 rounding).
+// (1024 + q) - (1024 + z), then times D (one fp16 rounding). Written as
+// four passes over all 16 pairs (extract, subtract, multiply) so that the
+// independent pairs interleave instead of running as 16 dependent chains.
 template <int BITS, int GMODE>
 __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
                                               const __half2* zsub,
                                               const __half2* dh,
                                               uint32_t* o) {
   constexpr uint32_t QMASK = (1u << BITS) - 1u;
-  auto cvt = [&](uint32_t pair, int gl) -> uint32_t {
-    return h2_bits(__hmul2(__hsub2(bits_h2(pair | 0x64006400u), zsub[gl]),
-                           dh[gl]));
-  };
+  uint32_t x[16];
   if constexpr (BITS == 2 || BITS == 4 || BITS == 8) {
     // codes c and c + 16/BITS sit 16 bits apart in one word: one shift and
     // mask yield the pair; positions follow k_perm<BITS>
@@ -176,24 +175,33 @@ __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
 #pragma unroll
     for (int wd = 0; wd < BITS; ++wd)
 #pragma unroll
-      for (int j = 0; j < PAIRS; ++j) {
-        const int gl = GMODE == 0 ? (wd * PER_WORD) / 16 : 0;
-        o[wd * PAIRS + j] = cvt((cw[wd] >> (BITS * j)) & PMASK, gl);
-      }
+      for (int j = 0; j < PAIRS; ++j)
+        x[wd * PAIRS + j] = ((cw[wd] >> (BITS * j)) & PMASK) | 0x64006400u;
   } else {
 #pragma unroll
     for (int pp = 0; pp < 16; ++pp) {
       const int c = 2 * pp;  // code index in the block
       const int bit = c * BITS, wd = bit >> 5, sh = bit & 31;
-      uint32_t x;
+      uint32_t v;
       if (sh + 2 * BITS <= 32)
-        x = cw[wd] >> sh;
+        v = cw[wd] >> sh;
       else
-        x = __funnelshift_r(cw[wd], cw[wd + 1], sh);
-      const uint32_t pair = (x & QMASK) | ((x << (16 - BITS)) & (QMASK << 16));
-      o[pp] = cvt(pair, GMODE == 0 ? c / 16 : 0);
+        v = __funnelshift_r(cw[wd], cw[wd + 1], sh);
+      x[pp] = (v & QMASK) | ((v << (16 - BITS)) & (QMASK << 16)) | 0x64006400u;
     }
   }
+  // group of pair p (g = 16 splits a block into two groups)
+  auto grp = [&](int pp) -> int {
+    if constexpr (GMODE != 0) return 0;
+    if constexpr (BITS == 2 || BITS == 4 || BITS == 8)
+      return (pp / (16 / BITS)) * (32 / BITS) / 16;  // word's first code
+    return (2 * pp) / 16;
+  };
+  __half2 t[16];
+#pragma unroll
+  for (int pp = 0; pp < 16; ++pp) t[pp] = __hsub2(bits_h2(x[pp]), zsub[grp(pp)]);
+#pragma unroll
+  for (int pp = 0; pp < 16; ++pp) o[pp] = h2_bits(__hmul2(t[pp], dh[grp(pp)]));
 }
 
 // Position in a ring of `depth` slots: the slot and how many times the
@@ -218,8 +226,8 @@ struct Ring {
 //   MMA        waits `ready`, issues 8 MMAs, commits to `empty`, which frees
 //              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
-template <int BITS, int GMODE>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int BITS, int GMODE, int DQW>
+__global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_c,
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                        const GemmArgs p) {
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
+  constexpr int kDq = 32 * DQW;            // dequantiser threads
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -383,9 +392,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     // One thread per weight row (= TMEM lane): a stage is four 32-code
     // blocks, 64 fp16 pairs, written to the TMEM weight ring in two stores.
     const int q4 = warp & 3;         // TMEM lane quarter of this warp
+    const int h = (warp - 2) >> 2;   // which half of a stage (DQW == 8)
     const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
     const int n = m0 + i;
     const bool row_ok = n < p.N;
+    const int half_lo = DQW == 8 ? h : 0, half_hi = DQW == 8 ? h + 1 : 2;
     const uint32_t crow = base + L.c + i * 16 * BITS;
     // delta tile: 64-byte rows in the 64B swizzle (16-byte chunk index XOR
     // bits 1-2 of the row); zero tile: plain 16-byte rows
@@ -418,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t poff = rp.slot * kParamBytes;
         const uint32_t cbase = crow + rs.slot * CHUNK;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int half = half_lo; half < half_hi; ++half) {
           uint32_t o[32];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -446,18 +457,20 @@ __global__ void __launch_bounds__(kThreads, 2)
           mbar_arrive(b_empty_p + 8 * rp.slot);
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
-        uint32_t o[32];
+        if (half_lo == 0) {
+          uint32_t o[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int rho = 2 * e;
-          float lo = 0.f, hi = 0.f;
-          if (row_ok && rho < p.r)
-            lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
-          if (row_ok && rho + 1 < p.r)
-            hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
-          o[e] = h2_bits(__floats2half2_rn(lo, hi));
+          for (int e = 0; e < 32; ++e) {
+            const int rho = 2 * e;
+            float lo = 0.f, hi = 0.f;
+            if (row_ok && rho < p.r)
+              lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
+            if (row_ok && rho + 1 < p.r)
+              hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
+            o[e] = h2_bits(__floats2half2_rn(lo, hi));
+          }
+          tmem_st32(acol, o);
         }
-        tmem_st32(acol, o);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -472,8 +485,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const bool ok = acc_ok && !*aborted && n_total > 0;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+    // columns of the accumulator this warp drains
+    const int c_lo = DQW == 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
+    const int c_hi = DQW == 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
+                              : bn;
     if (split == 1) {
-      for (int j = 0; j < bn; j += 16) {
+      for (int j = c_lo; j < c_hi; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
         if (ok && row_ok) {
@@ -486,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     } else {
       float* part = reinterpret_cast<float*>(gbase + L.part);
-      for (int j = 0; j < bn; j += 16) {
+      for (int j = c_lo; j < c_hi; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
 #pragma unroll
@@ -500,10 +517,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     cluster.sync();
     if (rank == 0 && warp >= 2) {
       const int i = 32 * (warp & 3) + lane;
+      const int h = (warp - 2) >> 2;
       const int n = m0 + i;
+      const int c_lo = DQW == 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
+      const int c_hi = DQW == 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
+                                : bn;
       float* part = reinterpret_cast<float*>(gbase + L.part);
       if (n < p.N && !*aborted) {
-        for (int c = 0; c < bn; ++c) {
+        for (int c = c_lo; c < c_hi; ++c) {
           const int t = t0 + c;
           if (t >= p.T) break;
           float acc = 0.f;
@@ -644,16 +665,16 @@ struct Maps {
   CUtensorMap x, u, c, d, z;
 };
 
-template <int BITS, int GMODE>
+template <int BITS, int GMODE, int DQW>
 ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
-  auto kern = lowbit_gemm_kernel<BITS, GMODE>;
+  auto kern = lowbit_gemm_kernel<BITS, GMODE, DQW>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return TTQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(cta_threads(DQW), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -667,17 +688,17 @@ ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
       cudaLaunchKernelEx(&cfg, kern, m.x, m.u, m.c, m.d, m.z, a));
 }
 
-template <int GMODE>
+template <int GMODE, int DQW>
 ttq_status dispatch_bits(int bits, const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
   switch (bits) {
-    case 2: return launch_kernel<2, GMODE>(m, a, grid, split, smem, st);
-    case 3: return launch_kernel<3, GMODE>(m, a, grid, split, smem, st);
-    case 4: return launch_kernel<4, GMODE>(m, a, grid, split, smem, st);
-    case 5: return launch_kernel<5, GMODE>(m, a, grid, split, smem, st);
-    case 6: return launch_kernel<6, GMODE>(m, a, grid, split, smem, st);
-    case 7: return launch_kernel<7, GMODE>(m, a, grid, split, smem, st);
-    case 8: return launch_kernel<8, GMODE>(m, a, grid, split, smem, st);
+    case 2: return launch_kernel<2, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 3: return launch_kernel<3, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 4: return launch_kernel<4, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 5: return launch_kernel<5, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 6: return launch_kernel<6, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 7: return launch_kernel<7, GMODE, DQW>(m, a, grid, split, smem, st);
+    case 8: return launch_kernel<8, GMODE, DQW>(m, a, grid, split, smem, st);
   }
   return TTQ_ERR_INVALID_ARG;
 }
@@ -833,8 +854,15 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.per = per;
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
-  if (group == 16) return dispatch_bits<0>(bits, m, a, grid, split, smem, st);
-  return dispatch_bits<1>(bits, m, a, grid, split, smem, st);
+  // decode packs two CTAs per SM with four dequant warps each; prefill runs
+  // one CTA per SM with eight
+  if (T <= 32) {
+    if (group == 16)
+      return dispatch_bits<0, 4>(bits, m, a, grid, split, smem, st);
+    return dispatch_bits<1, 4>(bits, m, a, grid, split, smem, st);
+  }
+  if (group == 16) return dispatch_bits<0, 8>(bits, m, a, grid, split, smem, st);
+  return dispatch_bits<1, 8>(bits, m, a, grid, split, smem, st);
 }
 
 ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
