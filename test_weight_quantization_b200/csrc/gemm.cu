@@ -59,7 +59,8 @@ struct GemmArgs {
   int yt;  // ttq_dtype of Y
   long long ldy;
   int bn;         // tokens per tile (MMA N)
-  int S;          // pipeline depth (stages of 128 channels)
+  int S;          // shared-memory ring depth (stages of 128 channels)
+  int SA;         // TMEM weight-stage ring depth (<= S)
   int tmem_cols;  // TMEM allocation: accumulator + S weight stages
   int acc_cols;   // TMEM columns reserved for the accumulator
   int group;
@@ -88,7 +89,7 @@ __host__ __device__ inline Layout make_layout(int bits, int bn, int S,
   L.p = L.c + (uint32_t)S * code_chunk_bytes(bits);
   L.part = L.p + 2u * kParamBytes;
   L.bars = L.part + (split ? (uint32_t)(bn * kBM * 4) : 0u);
-  const int nbars = 3 * S + 4 + 1;
+  const int nbars = 3 * S + S + 4 + 1;  // loaded, ready, empty, a_free
   L.tmem = L.bars + 8u * nbars;
   L.abort_flag = L.tmem + 4;
   L.total = L.abort_flag + 4;
@@ -243,13 +244,14 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
   const uint32_t base = (raw_base + 1023u) & ~1023u;
   uint8_t* const gbase = smem_raw + (base - raw_base);
 
-  const int S = p.S, bn = p.bn;
+  const int S = p.S, SA = p.SA, bn = p.bn;
   const int split = (int)gridDim.z;
   const Layout L = make_layout(BITS, bn, S, split > 1);
   const uint32_t b_loaded = base + L.bars;
   const uint32_t b_ready = b_loaded + 8 * S;
   const uint32_t b_empty = b_ready + 8 * S;
-  const uint32_t b_full_p = b_empty + 8 * S;
+  const uint32_t b_afree = b_empty + 8 * S;
+  const uint32_t b_full_p = b_afree + 8 * S;
   const uint32_t b_empty_p = b_full_p + 16;
   const uint32_t b_accum = b_empty_p + 16;
   volatile uint32_t* tmem_slot =
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
       mbar_init(b_loaded + 8 * i, 1);
       mbar_init(b_ready + 8 * i, kDq);
       mbar_init(b_empty + 8 * i, 1);
+      mbar_init(b_afree + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
@@ -362,14 +365,14 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kBM, bn);
       const uint32_t xbytes = (uint32_t)bn * 128u;
-      Ring rs;
+      Ring rs, ra;
       for (int s = 0; s < n_total; ++s) {
         if (!mbar_wait(b_ready + 8 * rs.slot, rs.round & 1, p.err)) {
           *aborted = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t ad = tmem_a + (uint32_t)(rs.slot * kSCols);
+        const uint32_t ad = tmem_a + (uint32_t)(ra.slot * kSCols);
         const uint32_t xs = base + L.x + rs.slot * L.stage_x;
         const uint64_t bd0 = smem_desc_sw128(xs);
         const uint64_t bd1 = smem_desc_sw128(xs + xbytes);
@@ -383,7 +386,9 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
             tc_mma_f16_ts(tmem, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
         }
         tc_commit(b_empty + 8 * rs.slot);
+        tc_commit(b_afree + 8 * ra.slot);
         rs.next(S);
+        ra.next(SA);
       }
       tc_commit(b_accum);
     }
@@ -404,18 +409,23 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     const uint32_t dswz = (uint32_t)((i >> 1) & 3);
     const uint32_t zrow = base + L.p + kParamDeltaBytes + i * 16;
     const uint32_t arow = tmem_a + ((uint32_t)(32 * q4) << 16);
-    Ring rs, rp;
+    Ring rs, ra, rp;
     int pchunk = -1;
     bool ok_loop = true;
 
     for (int s = 0; s < n_total && ok_loop; ++s) {
       const int k0 = (ks_begin + s) * kSK;
+      // codes and activations of this stage have landed; its TMEM weight
+      // slot is free once the MMA of stage s - SA completed
       if (!mbar_wait(b_loaded + 8 * rs.slot, rs.round & 1, p.err) ||
+          (s >= SA &&
+           !mbar_wait(b_afree + 8 * ra.slot, (ra.round & 1) ^ 1, p.err)) ||
           *aborted) {
         ok_loop = false;
         break;
       }
-      const uint32_t acol = arow + (uint32_t)(rs.slot * kSCols);
+      tc_fence_after();
+      const uint32_t acol = arow + (uint32_t)(ra.slot * kSCols);
       if (s < n_main) {
         const int pc = k0 >> (lg + 4);
         if (pc != pchunk) {
@@ -476,6 +486,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
       tc_fence_before();
       mbar_arrive(b_ready + 8 * rs.slot);
       rs.next(S);
+      ra.next(SA);
     }
     if (!ok_loop) *aborted = 1;
     __syncwarp();
@@ -769,7 +780,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   const int64_t tiles_m = (N + kBM - 1) / kBM;
   const int k_stages = (int)((K + kSK - 1) / kSK);
   const uint32_t cchunk = code_chunk_bytes(bits);
-  int bn, S, tmem_cols, acc_cols, split = 1;
+  int bn, S, SA, tmem_cols, acc_cols, split = 1;
   auto fits = [&](int bn_, int S_, bool sp, size_t lim) {
     return (size_t)make_layout(bits, bn_, S_, sp).total + 1024 <= lim;
   };
@@ -777,8 +788,11 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
     bn = T <= 16 ? 16 : 32;
     acc_cols = 32;
     tmem_cols = 256;
-    S = (tmem_cols - acc_cols) / kSCols;
-    while (S > 2 && !fits(bn, S, true, 110 * 1024)) --S;
+    SA = (tmem_cols - acc_cols) / kSCols;
+    // the shared-memory ring runs deeper than the TMEM weight ring so that
+    // loads are issued well ahead of the dequantisers
+    S = 8;
+    while (S > SA && !fits(bn, S, true, 110 * 1024)) --S;
   } else {
     bn = 64;
     double best = 1e30;
@@ -801,6 +815,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
     tmem_cols = 512;
     S = std::min(6, (tmem_cols - acc_cols) / kSCols);
     while (S > 1 && !fits(bn, S, false, kMaxSmem)) --S;
+    SA = S;
   }
   if (S < 2) return TTQ_ERR_UNSUPPORTED;
   if (T <= 32) {
@@ -847,6 +862,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.ldy = ldy;
   a.bn = bn;
   a.S = S;
+  a.SA = SA;
   a.tmem_cols = tmem_cols;
   a.acc_cols = acc_cols;
   a.group = group;
