@@ -210,6 +210,36 @@ ttq_status ttq_w_lowbit_gemm_prepared(const void* Xs, const void* U,
                                       void* Y, ttq_dtype yt, int64_t ldy,
                                       void* stream);
 
+/* ttq_w_lowbit_gemm without a workspace argument, for callers that cannot
+ * allocate device memory where they run the projection (a plugin called by
+ * an inference engine after the engine fixed its memory plan, or host code
+ * that only receives device pointers and has no allocator). The pages have
+ * no counterpart to this call; it is a deployment convenience.
+ *
+ * Same arguments and results as ttq_w_lowbit_gemm. The scratch it needs
+ * comes from an array built into the library, TTQ_NOALLOC_SCRATCH_BYTES on
+ * every GPU that loads the library, kept until the process exits. It calls
+ * no allocator.
+ *   - Inputs whose workspace (ttq_w_lowbit_gemm_workspace_size(T, K, r))
+ *     exceeds TTQ_NOALLOC_SCRATCH_BYTES return TTQ_ERR_UNSUPPORTED and
+ *     enqueue nothing; use ttq_w_lowbit_gemm for them.
+ *   - The first call on a device looks up the array's address on that
+ *     device (set-up done once per device); make that first call before
+ *     any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents,
+ *     so calls whose execution overlaps on the GPU (other streams or host
+ *     threads) race; serialise them. */
+#define TTQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+ttq_status ttq_w_lowbit_gemm_noalloc(const void* X, ttq_dtype xt, int64_t T,
+                                     int64_t K, int64_t ldx,
+                                     const float* inv_s,
+                                     const uint32_t* codes,
+                                     const float* delta, const uint8_t* zero,
+                                     int64_t N, int bits, int group,
+                                     const void* A, const void* B, int r,
+                                     void* Y, ttq_dtype yt, int64_t ldy,
+                                     void* stream);
+
 /* The low-rank term alone (TTQ review, Proposed method, bullet 5; Main
  * results, bullet 4): Y[t][n] += sum_rho (sum_j X[t][j] A[rho][j]) B[n][rho].
  * X [T, K], A [r, K], B [N, r] of dtype xt; Y [T, N] of dtype yt, pitch ldy.
