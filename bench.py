@@ -272,6 +272,25 @@ def oracle_step(wl, data, sample_tokens):
     return est, desc
 
 
+# -------------------------------------------------------- aggregation ----
+
+def slowest_rank_ms(ms: float, world: int, device) -> float:
+    """The timed region's length on the slowest rank (all-reduce MAX)."""
+    if world <= 1:
+        return ms
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def layer_tokens_per_s(world: int, n_layers: int, T: int,
+                       ms_per_step: float) -> float:
+    """Whole-job prompt tokens per second per layer: every rank runs its own
+    replica, so the job moves world * n_layers * T layer-tokens per step."""
+    return world * n_layers * T / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- main ----
 
 def dist_setup(args):
@@ -420,15 +439,10 @@ def main():
             end.record()
         torch.cuda.synchronize()
     barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = slowest_rank_ms(start.elapsed_time(end), world, device)
     clocks = clk.summary()
     ms_per_step = ms / args.steps
-    value = world * len(wl.layers) * wl.T / (ms_per_step / 1e3)
+    value = layer_tokens_per_s(world, len(wl.layers), wl.T, ms_per_step)
 
     # per-kernel times: event-instrumented replays of the same step
     with torch.cuda.stream(stream):
@@ -547,13 +561,8 @@ def end_to_end(ttq, wl, data, device, args, stream, world):
             one()
         b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": world * len(wl.layers) * wl.T / (ms / 1e3),
+    ms = slowest_rank_ms(a.elapsed_time(b) / steps, world, device)
+    return {"value": layer_tokens_per_s(world, len(wl.layers), wl.T, ms),
             "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 

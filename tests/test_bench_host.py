@@ -1,0 +1,75 @@
+"""Host logic of bench.py that needs no GPU: the multi-rank aggregation
+(world size 2 over gloo on the CPU) and the reference arm's behaviour under
+a launcher (rank 0 reports, other ranks exit without work)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, local_ms, out):
+    import torch
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = bench.slowest_rank_ms(local_ms[rank], world, torch.device("cpu"))
+        out[rank] = ms
+    finally:
+        dist.destroy_process_group()
+
+
+def test_slowest_rank_timing_over_gloo():
+    world, port = 2, _free_port()
+    local_ms = [3.0, 5.5]
+    out = mp.Manager().dict()
+    mp.spawn(_rank_main, args=(world, port, local_ms, out), nprocs=world,
+             join=True)
+    assert out[0] == out[1] == 5.5
+
+
+def test_layer_token_throughput_counts_every_replica():
+    import bench
+    # 2 ranks x 6 layers x 2048 tokens per 0.25 ms step
+    assert bench.layer_tokens_per_s(2, 6, 2048, 0.25) == pytest.approx(
+        2 * 6 * 2048 / 0.25e-3)
+    assert bench.layer_tokens_per_s(1, 6, 2048, 0.5) == pytest.approx(
+        6 * 2048 / 0.5e-3)
+
+
+def test_reference_arm_rank_nonzero_exits_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--gpus", "2", "--steps", "1",
+                        "--warmup", "0"], capture_output=True, text=True,
+                       env=env, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_reference_arm_reports_the_oracle():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--steps", "1", "--warmup",
+                        "0"], capture_output=True, text=True, env=env,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["unit"] == "tokens/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "opt125m-block"
