@@ -153,7 +153,8 @@ TTQ_EXPORT ttq_status ttq_quantize_rtn_grouped(
   if (!W || !codes || !delta || !zero || !valid_dtype(wt) || N < 1 ||
       K < 32 || K % 32 != 0 || bits < 2 || bits > 8 || !valid_group(group) ||
       K % group != 0 || ldw < K || !rows_aligned(W, wt, ldw) ||
-      (s && !aligned(s, 16)) || !aligned(codes, 4) || !aligned(delta, 4))
+      (s && !aligned(s, 16)) || !aligned(codes, 4) || !aligned(delta, 4) ||
+      N * ((K + 255) / 256) >= ((int64_t)1 << 31))
     return TTQ_ERR_INVALID_ARG;
   return launch_quantize(W, wt, N, K, ldw, s, bits, group, codes, delta, zero,
                          as_stream(stream));
@@ -197,6 +198,7 @@ TTQ_EXPORT ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt,
                                               void* U, void* stream) {
   if (!X || !inv_s || !Xs || !valid_dtype(xt) || T < 1 || K < 32 ||
       K % 32 != 0 || bits < 2 || bits > 8 || ldx < K || r < 0 || r > 64 ||
+      T * (K / 16) >= ((int64_t)1 << 31) ||
       ((r > 0) != (A && U)) ||
       (r == 0 && (A || U)) || !rows_aligned(X, xt, ldx) ||
       !aligned(inv_s, 16) || !aligned(Xs, 16) || (U && !aligned(U, 16)) ||

@@ -572,10 +572,12 @@ template <typename TX, int PERM>
 __global__ void prescale_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
                                 int64_t ldx, const float* __restrict__ inv_s,
                                 __half* __restrict__ Xs, uint32_t* err) {
-  const int64_t spans = K / 16;
-  const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (id >= T * spans) return;
-  const int64_t t = id / spans, c = (id % spans) * 16;
+  // T * K / 16 < 2^31 (checked on the host): 32-bit index math
+  const uint32_t spans = (uint32_t)(K / 16);
+  const uint32_t id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (uint32_t)T * spans) return;
+  const uint32_t tq = id / spans;
+  const int64_t t = tq, c = (int64_t)(id - tq * spans) * 16;
   float v[16], sv[16];
   load8<TX>(X + t * ldx + c, *reinterpret_cast<float(*)[8]>(v));
   load8<TX>(X + t * ldx + c + 8, *reinterpret_cast<float(*)[8]>(v + 8));

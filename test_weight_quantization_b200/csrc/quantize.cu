@@ -15,6 +15,8 @@
 // shuffles and each lane stores the one or two packed words it owns, so a
 // warp writes 8*b consecutive words. Delta and zero go out from the first
 // lane of each group.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -22,77 +24,38 @@ namespace ttq {
 namespace {
 
 constexpr int kWarpsPerCta = 8;
+constexpr int kSegsPerWarp = 2;  // 256-channel segments per warp
 
-template <typename TW, int BITS>
-__global__ void __launch_bounds__(kWarpsPerCta * 32)
-    quantize_kernel(const TW* __restrict__ W, int64_t N, int64_t K,
-                    int64_t ldw, const float* __restrict__ s, int group,
-                    uint32_t* __restrict__ codes, float* __restrict__ delta,
-                    uint8_t* __restrict__ zero) {
-  const int lane = threadIdx.x & 31;
-  const int64_t segs = (K + 255) / 256;
-  const int64_t item = (int64_t)blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  if (item >= N * segs) return;  // whole warp exits together
-  const int64_t n = item / segs;
-  const int64_t col0 = (item % segs) * 256 + lane * 8;
-  const bool active = col0 < K;  // K % 32 == 0: whole blocks/groups agree
-
-  const float qmax = (float)((1 << BITS) - 1);
-  float w[8];
-  if (active) {
-    load8<TW>(W + n * ldw + col0, w);
-    if (s != nullptr) {
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + col0));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + col0 + 4));
-      w[0] = __fmul_rn(w[0], s0.x); w[1] = __fmul_rn(w[1], s0.y);
-      w[2] = __fmul_rn(w[2], s0.z); w[3] = __fmul_rn(w[3], s0.w);
-      w[4] = __fmul_rn(w[4], s1.x); w[5] = __fmul_rn(w[5], s1.y);
-      w[6] = __fmul_rn(w[6], s1.z); w[7] = __fmul_rn(w[7], s1.w);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = 0.f;
-  }
-
-  // group range, widened to contain 0
-  float mn = 0.f, mx = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    mn = fminf(mn, w[i]);
-    mx = fmaxf(mx, w[i]);
-  }
-  const int lanes_per_group = group >> 3;
-  for (int o = 1; o < lanes_per_group; o <<= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  float d = __fdiv_rn(__fsub_rn(mx, mn), qmax);
-  if (d == 0.f) d = 1.f;
-  const float r = __frcp_rn(d);
-  const float z = fminf(fmaxf(rintf(__fmul_rn(-mn, r)), 0.f), qmax);
-
-  uint64_t chunk = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float v = fminf(fmaxf(__fadd_rn(rintf(__fmul_rn(w[i], r)), z), 0.f),
-                          qmax);
-    chunk |= (uint64_t)(uint32_t)v << (BITS * i);
-  }
-
-  // gather the four 8*BITS-bit chunks of this lane's 32-code block
-  const int qbase = lane & ~3;
+// Packs this lane's eight BITS-bit codes (chunk, codes at BITS*i) into the
+// 32-code block shared by the four lanes of its quad and stores the words
+// the lane owns (block words qpos and qpos + 4).
+template <int BITS>
+__device__ __forceinline__ void store_block(uint64_t chunk, int lane,
+                                            uint32_t* out, bool active) {
   const int qpos = lane & 3;
-  uint64_t c[4];
+  if constexpr (BITS == 4) {
+    // eight 4-bit codes are exactly block word qpos
+    if (active) out[qpos] = (uint32_t)chunk;
+  } else if constexpr (BITS == 8) {
+    if (active)
+      *reinterpret_cast<uint2*>(out + 2 * qpos) =
+          make_uint2((uint32_t)chunk, (uint32_t)(chunk >> 32));
+  } else if constexpr (BITS == 2) {
+    // two lanes (16 bits each) make one word
+    const uint32_t hi = __shfl_down_sync(0xffffffffu, (uint32_t)chunk, 1);
+    if (active && (qpos & 1) == 0)
+      out[qpos >> 1] = (uint32_t)chunk | (hi << 16);
+  } else {
+    const int qbase = lane & ~3;
+    uint64_t c[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)chunk, qbase + j);
-    const uint32_t hi =
-        __shfl_sync(0xffffffffu, (uint32_t)(chunk >> 32), qbase + j);
-    c[j] = ((uint64_t)hi << 32) | lo;
-  }
-  const int64_t ldc = codes_ld(K, BITS), ldg = groups_ld(K, group);
-  if (active) {
-    uint32_t* out = codes + n * ldc + (col0 / 32) * BITS;
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)chunk, qbase + j);
+      const uint32_t hi =
+          __shfl_sync(0xffffffffu, (uint32_t)(chunk >> 32), qbase + j);
+      c[j] = ((uint64_t)hi << 32) | lo;
+    }
+    if (!active) return;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int wi = qpos + 4 * half;  // word index inside the block
@@ -108,19 +71,119 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
       }
       out[wi] = word;
     }
-    if ((lane & (lanes_per_group - 1)) == 0) {
-      const int64_t gi = n * ldg + col0 / group;
-      delta[gi] = d;
-      zero[gi] = (uint8_t)z;
+  }
+}
+
+template <typename TW, int BITS>
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+    quantize_kernel(const TW* __restrict__ W, int64_t N, int64_t K,
+                    int64_t ldw, const float* __restrict__ s, int group,
+                    uint32_t* __restrict__ codes, float* __restrict__ delta,
+                    uint8_t* __restrict__ zero) {
+  constexpr int QMAX = (1 << BITS) - 1;
+  // rint(x) for |x| < 2^22 is exactly (x + 1.5*2^23) - 1.5*2^23 under
+  // round-to-nearest-even (the sum lands in [2^23, 2^24), where the ulp is
+  // 1, and the offset is even); the integer is the sum's low bits. Here
+  // |w*r| and |mn*r| are at most 2^b - 1 + 1/2.
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr int kMagicBits = 0x4B400000;
+  using chunk_t = typename std::conditional<(8 * BITS <= 32), uint32_t,
+                                            uint64_t>::type;
+  const int lane = threadIdx.x & 31;
+  // work items are (row, 256-channel segment) pairs, < 2^31 (checked on
+  // the host); 32-bit index math keeps the per-item cost small
+  const uint32_t segs = (uint32_t)((K + 255) / 256);
+  const uint32_t items = (uint32_t)N * segs;
+  const uint32_t item0 =
+      (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kSegsPerWarp;
+  if (item0 >= items) return;  // whole warp exits together
+  const int64_t ldc = codes_ld(K, BITS), ldg = groups_ld(K, group);
+  const int lanes_per_group = group >> 3;
+
+  // issue every segment's loads first
+  float w[kSegsPerWarp][8];
+  int64_t n_[kSegsPerWarp], col_[kSegsPerWarp];
+  bool act_[kSegsPerWarp];
+  const uint32_t row0 = item0 / segs, seg0 = item0 - row0 * segs;
+#pragma unroll
+  for (int u = 0; u < kSegsPerWarp; ++u) {
+    const uint32_t item = item0 + u;
+    const bool live = item < items;
+    uint32_t row = row0, seg = seg0 + u;
+    if (seg >= segs) {  // kSegsPerWarp <= segs is not required
+      row += seg / segs;
+      seg %= segs;
+    }
+    n_[u] = live ? row : 0;
+    col_[u] = live ? (int64_t)seg * 256 + lane * 8 : K;
+    act_[u] = live && col_[u] < K;  // K % 32 == 0: blocks/groups agree
+    if (act_[u]) {
+      load8<TW>(W + n_[u] * ldw + col_[u], w[u]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[u][i] = 0.f;
     }
   }
-  // the warp holding the row's first segment zeroes the row's padding
-  if (item % segs == 0) {
-    for (int64_t w = K * BITS / 32 + lane; w < ldc; w += 32)
-      codes[n * ldc + w] = 0u;
-    for (int64_t gi = K / group + lane; gi < ldg; gi += 32) {
-      delta[n * ldg + gi] = 0.f;
-      zero[n * ldg + gi] = 0;
+
+#pragma unroll
+  for (int u = 0; u < kSegsPerWarp; ++u) {
+    const int64_t n = n_[u], col0 = col_[u];
+    const bool active = act_[u];
+    if (active && s != nullptr) {
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + col0));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + col0 + 4));
+      w[u][0] = __fmul_rn(w[u][0], s0.x); w[u][1] = __fmul_rn(w[u][1], s0.y);
+      w[u][2] = __fmul_rn(w[u][2], s0.z); w[u][3] = __fmul_rn(w[u][3], s0.w);
+      w[u][4] = __fmul_rn(w[u][4], s1.x); w[u][5] = __fmul_rn(w[u][5], s1.y);
+      w[u][6] = __fmul_rn(w[u][6], s1.z); w[u][7] = __fmul_rn(w[u][7], s1.w);
+    }
+    // group range, widened to contain 0
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      mn = fminf(mn, w[u][i]);
+      mx = fmaxf(mx, w[u][i]);
+    }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) {  // g <= 128: at most 16 lanes
+      if (o < lanes_per_group) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+    }
+    float d = __fdiv_rn(__fsub_rn(mx, mn), (float)QMAX);
+    if (d == 0.f) d = 1.f;
+    const float r = __frcp_rn(d);
+    // z = rint(-mn * r) lies in [0, 2^b - 1] because -mn <= mx - mn; the
+    // clamp below matches the definition and never changes a value
+    const int zi = min(max(__float_as_int(__fadd_rn(__fmul_rn(-mn, r), kMagic)) -
+                               kMagicBits,
+                           0),
+                       QMAX);
+    // q = rint(w*r) + z >= rint(mn*r) + z = 0 since rint is odd and the
+    // products are monotone in w; only the upper clamp can act
+    chunk_t chunk = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int qi = __float_as_int(__fadd_rn(__fmul_rn(w[u][i], r), kMagic)) -
+                     (kMagicBits - zi);
+      chunk |= (chunk_t)(uint32_t)min(qi, QMAX) << (BITS * i);
+    }
+    store_block<BITS>((uint64_t)chunk, lane,
+                      codes + n * ldc + (col0 / 32) * BITS, active);
+    if (active && (lane & (lanes_per_group - 1)) == 0) {
+      const int64_t gi = n * ldg + col0 / group;
+      delta[gi] = d;
+      zero[gi] = (uint8_t)zi;
+    }
+    // the warp holding the row's first segment zeroes the row's padding
+    if (col0 == lane * 8 && item0 + u < items) {
+      for (int64_t w2 = K * BITS / 32 + lane; w2 < ldc; w2 += 32)
+        codes[n * ldc + w2] = 0u;
+      for (int64_t gi = K / group + lane; gi < ldg; gi += 32) {
+        delta[n * ldg + gi] = 0.f;
+        zero[n * ldg + gi] = 0;
+      }
     }
   }
 }
@@ -130,7 +193,8 @@ ttq_status launch_bits(const void* W, int64_t N, int64_t K, int64_t ldw,
                        const float* s, int bits, int group, uint32_t* codes,
                        float* delta, uint8_t* zero, cudaStream_t st) {
   const int64_t items = N * ((K + 255) / 256);
-  const dim3 grid((unsigned)((items + kWarpsPerCta - 1) / kWarpsPerCta));
+  const int64_t warps = (items + kSegsPerWarp - 1) / kSegsPerWarp;
+  const dim3 grid((unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta));
   const dim3 block(kWarpsPerCta * 32);
   const TW* w = static_cast<const TW*>(W);
 #define TTQ_Q(B)                                                              \

@@ -28,7 +28,35 @@ namespace ttq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 8;
+
+// 8 elements from the raw 16-byte vector(s) loaded for them.
+template <typename TX>
+__device__ __forceinline__ void unpack8(const uint4 (&r)[sizeof(TX) == 4 ? 2 : 1],
+                                        float (&x)[8]);
+template <>
+__device__ __forceinline__ void unpack8<float>(const uint4 (&r)[2],
+                                               float (&x)[8]) {
+  x[0] = __uint_as_float(r[0].x); x[1] = __uint_as_float(r[0].y);
+  x[2] = __uint_as_float(r[0].z); x[3] = __uint_as_float(r[0].w);
+  x[4] = __uint_as_float(r[1].x); x[5] = __uint_as_float(r[1].y);
+  x[6] = __uint_as_float(r[1].z); x[7] = __uint_as_float(r[1].w);
+}
+template <>
+__device__ __forceinline__ void unpack8<__nv_bfloat16>(const uint4 (&r)[1],
+                                                       float (&x)[8]) {
+  bf16x2_to_f32(r[0].x, x[0], x[1]);
+  bf16x2_to_f32(r[0].y, x[2], x[3]);
+  bf16x2_to_f32(r[0].z, x[4], x[5]);
+  bf16x2_to_f32(r[0].w, x[6], x[7]);
+}
+template <>
+__device__ __forceinline__ void unpack8<__half>(const uint4 (&r)[1],
+                                                float (&x)[8]) {
+  f16x2_to_f32(r[0].x, x[0], x[1]);
+  f16x2_to_f32(r[0].y, x[2], x[3]);
+  f16x2_to_f32(r[0].z, x[4], x[5]);
+  f16x2_to_f32(r[0].w, x[6], x[7]);
+}
 
 template <int PK>
 __device__ __forceinline__ float moment(float x, float p) {
@@ -64,17 +92,27 @@ __global__ void __launch_bounds__(kThreads)
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 
   if (col_ok) {
+    // keep kUnroll raw 16-byte vectors in flight per thread (two per row
+    // for fp32), converting only after all of them were issued
+    constexpr int V = sizeof(TX) == 4 ? 2 : 1;  // 16-byte vectors per row
+    constexpr int U = sizeof(TX) == 4 ? 8 : 16;  // rows in flight
     int64_t r = r_begin + row_in_pass;
-    for (; r + (int64_t)(kUnroll - 1) * rows_per_pass < r_end;
-         r += (int64_t)kUnroll * rows_per_pass) {
-      float v[kUnroll][8];
+    for (; r + (int64_t)(U - 1) * rows_per_pass < r_end;
+         r += (int64_t)U * rows_per_pass) {
+      uint4 raw[U][V];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        load8<TX>(X + (r + (int64_t)u * rows_per_pass) * ldx + col0, v[u]);
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
+        for (int v = 0; v < V; ++v)
+          raw[u][v] = ld_stream_v4(X + (r + (int64_t)u * rows_per_pass) * ldx +
+                                   col0 + v * (8 / V));
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(v[u][i], p);
+      for (int u = 0; u < U; ++u) {
+        float x[8];
+        unpack8<TX>(raw[u], x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(x[i], p);
+      }
     }
     for (; r < r_end; r += rows_per_pass) {
       float v[8];
