@@ -3,10 +3,13 @@
 on-the-fly quantization.
 
 One step is one pass of the whole path over one prompt of the workload: for
-every distinct layer input, statistics -> scales -> prepared fp16 operand;
-for every layer, group RTN of its weight -> tensor-core low-bit projection.
-The default workload is an OPT-125M-shaped block (q, k, v, o 768x768, fc1
-3072x768, fc2 768x3072; q, k, v share one input), T = 2048, b = 3, g = 32.
+every distinct layer input, statistics and scales (one launch) -> prepared
+fp16 operand; for every layer, group RTN of its weight -> tensor-core
+low-bit projection. Layers that share an input run as one projection of
+their stacked weights, and the prepared operand is built on a second stream
+while the weights are quantized. The default workload is an OPT-125M-shaped
+block (q, k, v, o 768x768, fc1 3072x768, fc2 768x3072; q, k, v share one
+input), T = 2048, b = 3, g = 32.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -53,6 +56,9 @@ def parse():
     ap.add_argument("--eager", action="store_true",
                     help="launch the step directly instead of replaying a "
                          "CUDA graph (for profilers)")
+    ap.add_argument("--separate", action="store_true",
+                    help="one call per step of the method and per layer, on "
+                         "one stream (no fused launches, for comparison)")
     return ap.parse_args()
 
 
@@ -71,19 +77,66 @@ def peaks():
 
 # ------------------------------------------------------------ workload ----
 
-class Step:
-    """Device buffers and the launch sequence of one step."""
+def layer_inputs(wl):
+    """Distinct layer inputs in the order the layers first use them."""
+    out = []
+    for L in wl.layers:
+        if L.input_name not in out:
+            out.append(L.input_name)
+    return out
 
-    def __init__(self, ttq, wl, data, device, replicas):
+
+def projection_groups(wl, separate=False):
+    """(name, input name, layers): layers that share an input and carry no
+    low-rank factors of their own run as one projection."""
+    groups = []
+    for k in layer_inputs(wl):
+        Ls = [L for L in wl.layers if L.input_name == k]
+        if separate or wl.rank or len(Ls) == 1:
+            groups += [(L.name, k, [L]) for L in Ls]
+        else:
+            groups.append(("|".join(L.name for L in Ls), k, Ls))
+    return groups
+
+
+def launch_plan(inputs, groups, separate=False):
+    """(kind, key) of every call of one step, in launch order."""
+    plan = []
+    for k in inputs:
+        plan += [("stats", k), ("scales", k)] if separate else \
+            [("stats_scales", k)]
+        plan.append(("prepare", k))
+        mine = [g for g, kk, _ in groups if kk == k]
+        plan += [("quantize", g) for g in mine]
+        plan += [("gemm", g) for g in mine]
+    return plan
+
+
+class Step:
+    """Device buffers and the launch sequence of one step.
+
+    Layers that share an input (q, k, v) run as one projection whose weight
+    is the layers' rows stacked ([2304, 768] for q|k|v): group RTN works row
+    by row and the projection column by column, so every code and output is
+    the one the separate layers would give. Per input the order is the
+    method's: statistics and scales (one launch) -> the prepared operand on
+    a second stream, beside the quantization of the weights on the first ->
+    the projections. ``separate`` restores one call per step of the method
+    and per layer on a single stream (for comparison)."""
+
+    def __init__(self, ttq, wl, data, device, replicas, separate=False):
         self.ttq, self.wl = ttq, wl
         self.T = wl.T
-        self.inputs = sorted(data["X"])
-        self.layers = list(wl.layers)
+        self.separate = separate
+        self.inputs = layer_inputs(wl)
+        self.groups = projection_groups(wl, separate)
         self.R = replicas
         self.X = [{k: v.to(device) for k, v in data["X"].items()}
                   for _ in range(replicas)]
-        self.W = [{k: v.to(device) for k, v in data["W"].items()}
-                  for _ in range(replicas)]
+        self.W = []
+        for _ in range(replicas):
+            self.W.append({g: torch.cat([data["W"][L.name] for L in Ls]).to(
+                device).contiguous() for g, _, Ls in self.groups})
         self.A = {k: v.to(device) for k, v in data["A"].items()}
         self.B = {k: v.to(device) for k, v in data["B"].items()}
         f32 = dict(dtype=torch.float32, device=device)
@@ -91,6 +144,7 @@ class Step:
                      for k in self.inputs}
         self.s = {k: torch.empty_like(v) for k, v in self.sums.items()}
         self.inv = {k: torch.empty_like(v) for k, v in self.sums.items()}
+        self.counter = ttq.new_counter(device)
         self.Xs = {k: torch.empty(self.X[0][k].shape, dtype=torch.float16,
                                   device=device) for k in self.inputs}
         r = wl.rank
@@ -98,58 +152,88 @@ class Step:
                                  device=device) for k in self.inputs} if r \
             else {}
         b, g = wl.bits, wl.group
-        self.codes, self.delta, self.zero, self.Y = {}, {}, {}, {}
-        for L in self.layers:
-            self.codes[L.name] = torch.empty((L.N, ttq.codes_ld(L.K, b)),
-                                             dtype=torch.int32, device=device)
-            gl = ttq.groups_ld(L.K, g)
-            self.delta[L.name] = torch.empty((L.N, gl), **f32)
-            self.zero[L.name] = torch.empty((L.N, gl), dtype=torch.uint8,
-                                            device=device)
-            self.Y[L.name] = torch.empty((self.T, L.N), dtype=wl.dtype,
-                                         device=device)
+        self.codes, self.delta, self.zero, self.Y, self.N = {}, {}, {}, {}, {}
+        for name, _, Ls in self.groups:
+            N, K = sum(L.N for L in Ls), Ls[0].K
+            self.N[name] = N
+            self.codes[name] = torch.empty((N, ttq.codes_ld(K, b)),
+                                           dtype=torch.int32, device=device)
+            gl = ttq.groups_ld(K, g)
+            self.delta[name] = torch.empty((N, gl), **f32)
+            self.zero[name] = torch.empty((N, gl), dtype=torch.uint8,
+                                          device=device)
+            self.Y[name] = torch.empty((self.T, N), dtype=wl.dtype,
+                                       device=device)
+        self.side = None if separate else torch.cuda.Stream(device)
+        self.plan = launch_plan(self.inputs, self.groups, separate)
 
     def input_bytes(self):
         return sum(v.numel() * v.element_size() for v in self.X[0].values()) + \
             sum(v.numel() * v.element_size() for v in self.W[0].values())
 
-    def calls(self, rep):
-        """(kind, callable) in launch order for replica ``rep``."""
+    def kernel_launches(self):
+        """Kernels one step launches (the prepare of a low-rank input runs a
+        second kernel for X A^T)."""
+        return len(self.plan) + (len(self.inputs) if self.wl.rank else 0)
+
+    def _fn(self, rep, kind, key):
         t, wl = self.ttq, self.wl
         X, W = self.X[rep], self.W[rep]
-        out = []
-        for k in self.inputs:
+        if kind == "stats":
+            return lambda: t.act_stats(X[key], wl.p, out=self.sums[key])
+        if kind == "scales":
+            return lambda: t.awq_scales(self.sums[key], self.T, wl.alpha,
+                                        wl.lam, wl.p, self.s[key],
+                                        self.inv[key])
+        if kind == "stats_scales":
+            return lambda: t.act_stats_scales(
+                X[key], self.counter, wl.alpha, wl.lam, wl.p, self.sums[key],
+                self.s[key], self.inv[key])
+        if kind == "prepare":
             A = None
             if wl.rank:
                 # the low-rank factors belong to a layer; layers that share
                 # an input in these workloads never both carry factors
-                owners = [L.name for L in self.layers if L.input_name == k]
-                A = self.A[owners[0]]
-            out.append(("stats", lambda k=k: t.act_stats(X[k], wl.p,
-                                                         out=self.sums[k])))
-            out.append(("scales", lambda k=k: t.awq_scales(
-                self.sums[k], self.T, wl.alpha, wl.lam, wl.p, self.s[k],
-                self.inv[k])))
-            out.append(("prepare", lambda k=k, A=A: t.prepare_activations(
-                X[k], self.inv[k], wl.bits, A, self.Xs[k], self.U.get(k))))
-        for L in self.layers:
-            k, n = L.input_name, L.name
-            out.append(("quantize", lambda k=k, n=n: t.quantize_rtn_grouped(
-                W[n], self.s[k], wl.bits, wl.group, self.codes[n],
-                self.delta[n], self.zero[n])))
-            out.append(("gemm", lambda k=k, n=n, L=L: t.w_lowbit_gemm_prepared(
-                self.Xs[k], self.U.get(k), self.codes[n], self.delta[n],
-                self.zero[n], L.N, wl.bits, wl.group,
-                self.B.get(n) if wl.rank else None, out=self.Y[n])))
-        return out
+                owner = next(g for g, k, _ in self.groups if k == key)
+                A = self.A[owner]
+            return lambda: t.prepare_activations(
+                X[key], self.inv[key], wl.bits, A, self.Xs[key],
+                self.U.get(key))
+        k = next(kk for g, kk, _ in self.groups if g == key)
+        if kind == "quantize":
+            return lambda: t.quantize_rtn_grouped(
+                W[key], self.s[k], wl.bits, wl.group, self.codes[key],
+                self.delta[key], self.zero[key])
+        return lambda: t.w_lowbit_gemm_prepared(
+            self.Xs[k], self.U.get(k), self.codes[key], self.delta[key],
+            self.zero[key], self.N[key], wl.bits, wl.group,
+            self.B.get(key) if wl.rank else None, out=self.Y[key])
 
     def run(self, rep, events=None):
-        for i, (kind, fn) in enumerate(self.calls(rep)):
-            if events is not None:
-                events[i][0].record()
-            fn()
-            if events is not None:
-                events[i][1].record()
+        main = torch.cuda.current_stream()
+        joins = {}
+        for i, (kind, key) in enumerate(self.plan):
+            fn = self._fn(rep, kind, key)
+            on_side = kind == "prepare" and self.side is not None
+            if kind == "gemm" and key in joins:
+                main.wait_event(joins.pop(key))
+            if on_side:
+                fork = torch.cuda.Event()
+                fork.record(main)
+                self.side.wait_event(fork)
+            st = self.side if on_side else main
+            with torch.cuda.stream(st):
+                if events is not None:
+                    events[i][0].record()
+                fn()
+                if events is not None:
+                    events[i][1].record()
+            if on_side:
+                done = torch.cuda.Event()
+                done.record(self.side)
+                for g, kk, _ in self.groups:
+                    if kk == key:
+                        joins[g] = done
 
 
 def algorithmic_work(wl):
@@ -159,6 +243,7 @@ def algorithmic_work(wl):
     xb = 2 if wl.dtype != torch.float32 else 4
     seen, w = set(), {"stats": 0, "scales": 0, "prepare": 0, "quantize": 0,
                       "gemm": 0, "gemm_flops": 0}
+    # (the fused statistics + scales launch moves both steps' bytes)
     for L in wl.layers:
         if L.input_name not in seen:
             seen.add(L.input_name)
@@ -170,6 +255,7 @@ def algorithmic_work(wl):
         w["gemm"] += T * L.K * 2 + L.N * L.K * b // 8 + 5 * L.N * L.K // g + \
             T * L.N * xb
         w["gemm_flops"] += 2 * T * L.N * L.K + 2 * T * wl.rank * (L.K + L.N)
+    w["stats_scales"] = w["stats"] + w["scales"]
     return w
 
 
@@ -376,10 +462,10 @@ def main():
     device = torch.device("cuda", local)
     data = make_inputs(wl)
 
-    probe = Step(ttq, wl, data, device, 1)
+    probe = Step(ttq, wl, data, device, 1, args.separate)
     rep = max(2, math.ceil(2.5 * L2_BYTES / probe.input_bytes()))
     del probe
-    step = Step(ttq, wl, data, device, rep)
+    step = Step(ttq, wl, data, device, rep, args.separate)
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
 
@@ -389,11 +475,10 @@ def main():
             step.run(r)
     stream.synchronize()
     ttq.device_error(clear=True)
-    calls = step.calls(0)
-    kinds = [k for k, _ in calls]
+    kinds = [k for k, _ in step.plan]
     # external events record timestamps when replayed inside a graph
     ev = [[[torch.cuda.Event(enable_timing=True, external=not args.eager)
-            for _ in range(2)] for _ in calls] for _ in range(rep)]
+            for _ in range(2)] for _ in kinds] for _ in range(rep)]
 
     class Eager:
         def __init__(self, r, events=None):
@@ -507,14 +592,21 @@ def main():
                 "group": wl.group,
                 "layers": ", ".join(f"{L.name} {L.N}x{L.K}"
                                     for L in wl.layers),
+                "projections": ", ".join(
+                    f"{g} {step.N[g]}x{Ls[0].K}" for g, _, Ls in step.groups),
                 "operands": "fp16 x fp16 -> fp32 (tensor cores); quantizer "
                             "fp32; statistics fp32",
                 "l2": f"inputs rotate over {rep} replicas "
                       f"({rep * step.input_bytes() / 2**20:.0f} MiB > L2)",
                 "parallelism": f"replicas x{world}",
-                "launch": "eager" if args.eager else "CUDA graph per replica"},
+                "launch": ("eager" if args.eager else
+                           "CUDA graph per replica") + (
+                    "; one stream, one call per step and layer"
+                    if args.separate else
+                    "; statistics+scales fused; prepare on a second stream "
+                    "beside the quantizer")},
             "roofline": roof, "kernels": kernels,
-            "gpu_launches": len(kinds) * args.steps,
+            "gpu_launches": step.kernel_launches() * args.steps,
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -530,10 +622,10 @@ def end_to_end(ttq, wl, data, device, args, stream, world):
     (eager calls, one per step of the method) and copies every output back.
     The layer weights are the model's resident parameters and stay on the
     device."""
-    step = Step(ttq, wl, data, device, 1)
+    step = Step(ttq, wl, data, device, 1, args.separate)
     hx = {k: v.pin_memory() for k, v in data["X"].items()}
-    hy = {L.name: torch.empty((wl.T, L.N), dtype=wl.dtype).pin_memory()
-          for L in wl.layers}
+    hy = {g: torch.empty((wl.T, step.N[g]), dtype=wl.dtype).pin_memory()
+          for g, _, _ in step.groups}
     h2d = sum(v.numel() * v.element_size() for v in hx.values())
     d2h = sum(v.numel() * v.element_size() for v in hy.values())
 

@@ -128,6 +128,28 @@ ttq_status ttq_awq_scales(const float* sum, int64_t T_total, int64_t K,
                           const ttq_params* prm, float* s, float* inv_s,
                           void* stream);
 
+/* Steps 1 and 2 in one launch: ttq_act_stats on X followed by
+ * ttq_awq_scales on the resulting sums, with the same arithmetic (TTQ
+ * review, Proposed method, bullets 2-4). The CTAs that finish the
+ * statistics last compute the scales, so nothing waits and no second launch
+ * is needed.
+ *   X, T, K, ldx, accumulate, sum_out   as for ttq_act_stats (p = prm->p).
+ *   T_total  token count behind sum_out (T, or the running total when
+ *            accumulate == 1); the scales divide by it.
+ *   prm      alpha, lambda and p as for ttq_awq_scales.
+ *   s, inv_s [K] float32 outputs as for ttq_awq_scales.
+ *   counter  one uint32 of device memory that is zero before the first call;
+ *            every call leaves it zero again. Calls that may run at the same
+ *            time (different streams) need different counters.
+ * sum_out is bit-identical to ttq_act_stats; s and inv_s agree with
+ * ttq_awq_scales to the last few bits of the fp64 mean (the mean is summed
+ * in a different fixed order). */
+ttq_status ttq_act_stats_scales(const void* X, ttq_dtype xt, int64_t T,
+                                int64_t K, int64_t ldx, int accumulate,
+                                int64_t T_total, const ttq_params* prm,
+                                float* sum_out, float* s, float* inv_s,
+                                uint32_t* counter, void* stream);
+
 /* Step 3, group-wise RTN of the scaled weights (TTQ review, Proposed
  * method, bullet 1). For row n and group G, in fp32 with IEEE round-to-
  * nearest-even for every operation and no fused multiply-add:
@@ -262,7 +284,7 @@ const char* ttq_status_string(ttq_status status);
  * is non-zero. Returns the TTQ_DEVERR_* bits, or -1 if the copy failed. */
 int ttq_device_error(int clear);
 
-/* ABI version of this header. */
+/* ABI version of this header (3: ttq_act_stats_scales added). */
 int ttq_abi_version(void);
 
 #ifdef __cplusplus

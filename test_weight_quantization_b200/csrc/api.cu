@@ -84,7 +84,7 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 2; }
+TTQ_EXPORT int ttq_abi_version(void) { return 3; }
 
 TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
   if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
@@ -144,6 +144,23 @@ TTQ_EXPORT ttq_status ttq_awq_scales(const float* sum, int64_t T_total,
     return TTQ_ERR_INVALID_ARG;
   return launch_awq_scales(sum, T_total, K, prm->alpha, prm->lambda, prm->p,
                            s, inv_s, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_act_stats_scales(
+    const void* X, ttq_dtype xt, int64_t T, int64_t K, int64_t ldx,
+    int accumulate, int64_t T_total, const ttq_params* prm, float* sum_out,
+    float* s, float* inv_s, uint32_t* counter, void* stream) {
+  if (!X || !sum_out || !s || !inv_s || !prm || !counter || !valid_dtype(xt) ||
+      T < 1 || K < 8 || K % 8 != 0 || ldx < K || !rows_aligned(X, xt, ldx) ||
+      !aligned(sum_out, 4) || !aligned(s, 4) || !aligned(inv_s, 4) ||
+      !aligned(counter, 4) || (accumulate != 0 && accumulate != 1) ||
+      T_total < T || !(prm->alpha >= 0.f) || !isfinite(prm->alpha) ||
+      !(prm->lambda >= 0.f && prm->lambda <= 1.f) || !(prm->p > 0.f) ||
+      !isfinite(prm->p))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_act_stats_scales(X, xt, T, K, ldx, accumulate, T_total,
+                                 prm->alpha, prm->lambda, prm->p, sum_out, s,
+                                 inv_s, counter, as_stream(stream));
 }
 
 TTQ_EXPORT ttq_status ttq_quantize_rtn_grouped(

@@ -46,11 +46,63 @@ inline ttq_status cuda_status(cudaError_t e) {
 
 inline ttq_status launch_status() { return cuda_status(cudaGetLastError()); }
 
+// Every kernel of the library is launched with programmatic stream
+// serialisation: its grid may be scheduled while the kernel before it on the
+// stream is still running, so that launch and prologue overlap that
+// kernel's tail. Each kernel calls griddep_wait() before it touches global
+// memory, which restores stream order for all data. cluster_z / cluster_y
+// > 1 add a thread-block cluster of that shape.
+struct LaunchShape {
+  dim3 grid;
+  dim3 block;
+  size_t smem = 0;
+  unsigned cluster_y = 1, cluster_z = 1;
+};
+
+template <typename... KArgs, typename... Args>
+inline ttq_status launch(const LaunchShape& ls, cudaStream_t st,
+                         void (*kern)(KArgs...), Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = ls.grid;
+  cfg.blockDim = ls.block;
+  cfg.dynamicSmemBytes = ls.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (ls.cluster_y > 1 || ls.cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = ls.cluster_y;
+    attr[n].val.clusterDim.z = ls.cluster_z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+}
+
 // -------------------------------------------------------------- device ---
 
 // A wait that does not finish within this many SM clocks (~1-2 s) gives up,
 // records TTQ_DEVERR_TIMEOUT and lets the kernel wind down.
 constexpr long long kWaitLimitClocks = 3000000000LL;
+
+// Programmatic dependent launch, device side: wait until the kernel before
+// this one on the stream has completed and its writes are visible, then
+// allow the kernel after this one to be scheduled.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_enter() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -120,6 +172,39 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---- TMA ----
+// Shared -> global tensor store of one box (coordinates of its first
+// element; the inner coordinate times the element size is a multiple of 16
+// bytes and no coordinate is negative), tracked by the bulk async-group.
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src,
+                                             int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], "
+      "[%1];" ::"l"(reinterpret_cast<uint64_t>(tmap)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until every committed bulk store of this thread has finished
+// reading its shared-memory source (the global writes complete on their
+// own before the grid is done).
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Barrier over `count` threads (a multiple of 32) on hardware barrier ID
+// (1..15; 0 is __syncthreads).
+template <int ID>
+__device__ __forceinline__ void named_bar_sync(int count) {
+  asm volatile("bar.sync %0, %1;" ::"n"(ID), "r"(count) : "memory");
+}
+__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(
                    reinterpret_cast<uint64_t>(tmap))
@@ -249,6 +334,59 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 }
 
 // Loads 16 consecutive fp32 columns of this warp's 32 TMEM lanes.
+// 32 consecutive columns of this warp's 32 lanes, load and wait in one
+// statement so no use of the registers can be scheduled before the wait.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
+      "[%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 16 lanes x 32 columns in the accumulator-fragment order of the 16x256b
+// shape: for each 8-column chunk k, thread t holds (lane t/4, columns 2(t%4)
+// and 2(t%4)+1) in r[4k], r[4k+1] and (lane t/4 + 8, same columns) in
+// r[4k+2], r[4k+3]. Load and wait in one statement.
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr,
+                                                   uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Four 8x8 16-bit matrices, transposed on the way to shared memory: thread
+// t supplies the row address of row t%8 of matrix t/8 and, in a_i, the
+// fragment element pair (row t/4, columns 2(t%4), 2(t%4)+1) of matrix i.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t a0,
+                                                  uint32_t a1, uint32_t a2,
+                                                  uint32_t a3) {
+  asm volatile(
+      "stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};"
+      ::"r"(addr), "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(

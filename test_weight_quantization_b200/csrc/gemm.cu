@@ -66,6 +66,10 @@ struct GemmArgs {
   int group;
   int k_stages;   // ceil(K / 128)
   int per;        // stages per split rank
+  int y_mode;     // 0: per-row stores (rows not 16-byte aligned);
+                  // 1: staged tile [tokens][128] stored through tm_y;
+                  // 2: 16-bit Y staged by stmatrix in 128-byte swizzled
+                  //    boxes of 64 rows, two stores per group
   uint32_t* err;
 };
 
@@ -131,6 +135,9 @@ __device__ __forceinline__ void load_block(uint32_t addr, uint32_t (&w)[BITS]) {
 }
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) {
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 h) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) {
@@ -234,6 +241,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
                        const __grid_constant__ CUtensorMap tm_c,
                        const __grid_constant__ CUtensorMap tm_d,
                        const __grid_constant__ CUtensorMap tm_z,
+                       const __grid_constant__ CUtensorMap tm_y,
                        const GemmArgs p) {
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
@@ -284,6 +292,9 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     *aborted = 0;
     fence_barrier_init();
   }
+  // everything below reads what earlier kernels wrote (or owns TMEM that a
+  // still-running kernel on this SM may hold)
+  griddep_enter();
   if (warp == 1) {
     tmem_alloc(base + L.tmem, (uint32_t)p.tmem_cols);
     tmem_relinquish();
@@ -500,7 +511,8 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     const int c_lo = DQW == 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
     const int c_hi = DQW == 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
                               : bn;
-    if (split == 1) {
+    if (split == 1 && p.y_mode == 0) {
+      // Y rows not 16-byte aligned: each thread stores its row directly
       for (int j = c_lo; j < c_hi; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
@@ -511,6 +523,111 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
             if (t < p.T) store_y(p.Y, p.yt, (long long)t * p.ldy + n, v[c]);
           }
         }
+      }
+    } else if (split == 1 && p.y_mode == 2) {
+      // 16-bit Y. Each warp reads its 32 rows in two halves of 16 lanes in
+      // the 16x256b fragment order, packs column pairs, and writes 8x8
+      // blocks transposed into [tokens][64 rows] boxes (128-byte rows,
+      // 16-byte chunk index XOR token % 8, the tensor map's 128-byte
+      // swizzle), so every store instruction moves 512 bytes without bank
+      // conflicts. The activation ring is idle once every MMA completed.
+      const int box_t = c_hi - c_lo;
+      const uint32_t gtile =
+          base + L.x + (uint32_t)h * 2u * (uint32_t)box_t * 128u;
+      const bool bf = p.yt == TTQ_BF16;
+      const int mi = lane >> 3, mr = lane & 7;  // matrix and row addressed
+#pragma unroll
+      for (int lh = 0; lh < 2; ++lh) {
+        const int nb = 32 * q4 + 16 * lh;  // first row of this lane half
+        const uint32_t box = gtile + (uint32_t)(nb >> 6) * (uint32_t)box_t * 128u;
+        const int chunk = ((nb & 63) >> 3) + (mi & 1);
+        for (int j = 0; j < box_t; j += 32) {
+          uint32_t rr[16];
+          tmem_ld_16x256b_x4(
+              t_lane + ((uint32_t)(16 * lh) << 16) + (uint32_t)(c_lo + j), rr);
+          uint32_t pk[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float a0 = __uint_as_float(rr[4 * k]);
+            const float a1 = __uint_as_float(rr[4 * k + 1]);
+            const float b0 = __uint_as_float(rr[4 * k + 2]);
+            const float b1 = __uint_as_float(rr[4 * k + 3]);
+            if (bf) {
+              pk[2 * k] = bf2_bits(__floats2bfloat162_rn(a0, a1));
+              pk[2 * k + 1] = bf2_bits(__floats2bfloat162_rn(b0, b1));
+            } else {
+              pk[2 * k] = h2_bits(__floats2half2_rn(a0, a1));
+              pk[2 * k + 1] = h2_bits(__floats2half2_rn(b0, b1));
+            }
+          }
+          if (ok) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const int row = j + 8 * (2 * q + (mi >> 1)) + mr;
+              const uint32_t addr = box + (uint32_t)row * 128u +
+                                    ((uint32_t)(chunk ^ (row & 7)) << 4);
+              stmatrix_x4_trans(addr, pk[4 * q], pk[4 * q + 1],
+                                pk[4 * q + 2], pk[4 * q + 3]);
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      if (h == 0)
+        named_bar_sync<1>(128);
+      else
+        named_bar_sync<2>(128);
+      if (ok && box_t > 0 && t0 + c_lo < p.T && q4 == 0 && lane == 0) {
+        tma_store_2d(&tm_y, gtile, m0, t0 + c_lo);
+        if (m0 + 64 < p.N)
+          tma_store_2d(&tm_y, gtile + (uint32_t)box_t * 128u, m0 + 64,
+                       t0 + c_lo);
+        bulk_commit_group();
+        bulk_wait_read();
+      }
+    } else if (split == 1) {
+      // The accumulator tile goes TMEM -> registers -> shared memory as a
+      // [tokens][128 rows] tile of Y's dtype (the activation ring is idle
+      // once every MMA completed), then the four warps that drained a
+      // column range hand it to the tensor memory accelerator as one box;
+      // rows beyond N and tokens beyond T are clipped by the store.
+      const uint32_t esz = p.yt == TTQ_F32 ? 4u : 2u;
+      const uint32_t ytile = base + L.x;
+      auto put = [&](int col, float v) {
+        const uint32_t a = ytile + ((uint32_t)col * kBM + (uint32_t)i) * esz;
+        if (p.yt == TTQ_F32)
+          st_shared_f32(a, v);
+        else if (p.yt == TTQ_BF16)
+          st_shared_u16(a, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+        else
+          st_shared_u16(a, __half_as_ushort(__float2half_rn(v)));
+      };
+      int j = c_lo;
+      for (; j + 32 <= c_hi; j += 32) {
+        float v[32];
+        tmem_ld32(t_lane + (uint32_t)j, v);
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) put(j + c, v[c]);
+        }
+      }
+      if (j < c_hi) {  // a 16-column remainder (decode tiles)
+        float v[16];
+        tmem_ld16(t_lane + (uint32_t)j, v);
+        if (ok) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) put(j + c, v[c]);
+        }
+      }
+      fence_proxy_async_smem();
+      if (h == 0)
+        named_bar_sync<1>(128);
+      else
+        named_bar_sync<2>(128);
+      if (ok && c_hi > c_lo && t0 + c_lo < p.T && q4 == 0 && lane == 0) {
+        tma_store_2d(&tm_y, ytile + (uint32_t)c_lo * kBM * esz, m0, t0 + c_lo);
+        bulk_commit_group();
+        bulk_wait_read();
       }
     } else {
       float* part = reinterpret_cast<float*>(gbase + L.part);
@@ -572,6 +689,7 @@ template <typename TX, int PERM>
 __global__ void prescale_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
                                 int64_t ldx, const float* __restrict__ inv_s,
                                 __half* __restrict__ Xs, uint32_t* err) {
+  griddep_enter();
   // T * K / 16 < 2^31 (checked on the host): 32-bit index math
   const uint32_t spans = (uint32_t)(K / 16);
   const uint32_t id = blockIdx.x * blockDim.x + threadIdx.x;
@@ -611,6 +729,7 @@ __global__ void __launch_bounds__(256)
     lowrank_u_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
                      int64_t ldx, const TX* __restrict__ A, int r,
                      __half* __restrict__ U) {
+  griddep_enter();
   const int64_t t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int rho = warp; rho < 64; rho += 8) {
@@ -675,7 +794,7 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr,
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Maps {
-  CUtensorMap x, u, c, d, z;
+  CUtensorMap x, u, c, d, z, y;
 };
 
 template <int BITS, int GMODE, int DQW>
@@ -685,20 +804,12 @@ ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return TTQ_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(cta_threads(DQW), 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = (unsigned)split;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(
-      cudaLaunchKernelEx(&cfg, kern, m.x, m.u, m.c, m.d, m.z, a));
+  LaunchShape ls;
+  ls.grid = grid;
+  ls.block = dim3(cta_threads(DQW), 1, 1);
+  ls.smem = smem;
+  ls.cluster_z = (unsigned)split;
+  return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, m.y, a);
 }
 
 template <int GMODE, int DQW>
@@ -725,17 +836,22 @@ ttq_status launch_pre(const void* X, int64_t T, int64_t K, int64_t ldx,
   const unsigned grid = (unsigned)((items + threads - 1) / threads);
   const TX* x = static_cast<const TX*>(X);
   uint32_t* err = device_error_word();
+  LaunchShape ls;
+  ls.grid = dim3(grid);
+  ls.block = dim3(threads);
+  ttq_status e;
   switch (bits) {
-    case 2: prescale_kernel<TX, 2><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
-    case 4: prescale_kernel<TX, 4><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
-    case 8: prescale_kernel<TX, 8><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
-    default: prescale_kernel<TX, 0><<<grid, threads, 0, st>>>(x, T, K, ldx, inv_s, Xs, err); break;
+    case 2: e = launch(ls, st, prescale_kernel<TX, 2>, x, T, K, ldx, inv_s, Xs, err); break;
+    case 4: e = launch(ls, st, prescale_kernel<TX, 4>, x, T, K, ldx, inv_s, Xs, err); break;
+    case 8: e = launch(ls, st, prescale_kernel<TX, 8>, x, T, K, ldx, inv_s, Xs, err); break;
+    default: e = launch(ls, st, prescale_kernel<TX, 0>, x, T, K, ldx, inv_s, Xs, err); break;
   }
-  ttq_status e = launch_status();
   if (e != TTQ_OK || r == 0) return e;
-  lowrank_u_kernel<TX><<<(unsigned)T, 256, 0, st>>>(
-      x, T, K, ldx, static_cast<const TX*>(A), r, U);
-  return launch_status();
+  LaunchShape lu;
+  lu.grid = dim3((unsigned)T);
+  lu.block = dim3(256);
+  return launch(lu, st, lowrank_u_kernel<TX>, x, T, K, ldx,
+                static_cast<const TX*>(A), r, U);
 }
 
 }  // namespace
@@ -783,6 +899,8 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   const int k_stages = (int)((K + kSK - 1) / kSK);
   const uint32_t cchunk = code_chunk_bytes(bits);
   int bn, S, SA, tmem_cols, acc_cols, split = 1;
+  // dual: two CTAs per SM, four dequantiser warps and 256 TMEM columns each
+  bool dual = T <= 32;
   auto fits = [&](int bn_, int S_, bool sp, size_t lim) {
     return (size_t)make_layout(bits, bn_, S_, sp).total + 1024 <= lim;
   };
@@ -795,7 +913,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
     // loads are issued well ahead of the dequantisers
     S = 8;
     while (S > SA && !fits(bn, S, true, 110 * 1024)) --S;
-  } else {
+  } else if (!dual) {
     bn = 64;
     double best = 1e30;
     for (int c : {256, 192, 128, 64}) {
@@ -851,6 +969,31 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                            128, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B));
   if (!ok) return TTQ_ERR_CUDA;
   if (r == 0) m.u = m.x;  // never read without a low-rank stage
+  // Y is stored by the tensor memory accelerator in boxes of 128 rows x the
+  // tokens one group of four dequantiser warps drains (half the tile with
+  // eight dequantisers); the split-K form reduces through the cluster
+  // instead and never reads this map
+  const int dqw = dual ? 4 : 8;
+  const int box_t = dqw == 8 ? bn / 2 : bn;
+  int y_mode = 0;
+  if (split == 1 && ((uint64_t)ldy * dtype_bytes(yt)) % 16 == 0 &&
+      reinterpret_cast<uintptr_t>(Y) % 16 == 0)
+    y_mode = (yt != TTQ_F32 && box_t % 32 == 0) ? 2 : 1;
+  if (y_mode > 0) {
+    const CUtensorMapDataType ydt =
+        yt == TTQ_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+        : yt == TTQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const bool ok_y =
+        y_mode == 2
+            ? make_tmap(&m.y, ydt, Y, N, T, (uint64_t)ldy * dtype_bytes(yt),
+                        64, box_t, CU_TENSOR_MAP_SWIZZLE_128B)
+            : make_tmap(&m.y, ydt, Y, N, T, (uint64_t)ldy * dtype_bytes(yt),
+                        kBM, box_t, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok_y) return TTQ_ERR_CUDA;
+  } else {
+    m.y = m.x;
+  }
 
   GemmArgs a;
   a.Blr = B;
@@ -870,11 +1013,12 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.group = group;
   a.k_stages = k_stages;
   a.per = per;
+  a.y_mode = y_mode;
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
   // decode packs two CTAs per SM with four dequant warps each; prefill runs
   // one CTA per SM with eight
-  if (T <= 32) {
+  if (dual) {
     if (group == 16)
       return dispatch_bits<0, 4>(bits, m, a, grid, split, smem, st);
     return dispatch_bits<1, 4>(bits, m, a, grid, split, smem, st);

@@ -13,6 +13,13 @@ ttq_status launch_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                             int64_t ldx, float p, int accumulate,
                             float* sum_out, cudaStream_t st);
 
+ttq_status launch_act_stats_scales(const void* X, ttq_dtype xt, int64_t T,
+                                   int64_t K, int64_t ldx, int accumulate,
+                                   int64_t T_total, double alpha,
+                                   double lambda, double p, float* sum_out,
+                                   float* s, float* inv_s,
+                                   unsigned int* counter, cudaStream_t st);
+
 ttq_status launch_awq_scales(const float* sum, int64_t T_total, int64_t K,
                              double alpha, double lambda, double p, float* s,
                              float* inv_s, cudaStream_t st);

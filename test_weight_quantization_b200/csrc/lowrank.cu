@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(kThreads)
                        const TX* __restrict__ B, int r, int64_t N,
                        TY* __restrict__ Y, int64_t ldy) {
   __shared__ float U[kTok][64];
+  griddep_enter();
   const int64_t t0 = (int64_t)blockIdx.x * kTok;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int item = warp; item < kTok * r; item += kThreads / 32) {
@@ -64,11 +65,12 @@ template <typename TX, typename TY>
 ttq_status launch_typed(const void* X, int64_t T, int64_t K, int64_t ldx,
                         const void* A, const void* B, int r, int64_t N,
                         void* Y, int64_t ldy, cudaStream_t st) {
-  const unsigned grid = (unsigned)((T + kTok - 1) / kTok);
-  lowrank_add_kernel<TX, TY><<<grid, kThreads, 0, st>>>(
-      static_cast<const TX*>(X), T, K, ldx, static_cast<const TX*>(A),
-      static_cast<const TX*>(B), r, N, static_cast<TY*>(Y), ldy);
-  return launch_status();
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)((T + kTok - 1) / kTok));
+  ls.block = dim3(kThreads);
+  return launch(ls, st, lowrank_add_kernel<TX, TY>, static_cast<const TX*>(X),
+                T, K, ldx, static_cast<const TX*>(A),
+                static_cast<const TX*>(B), r, N, static_cast<TY*>(Y), ldy);
 }
 
 template <typename TX>

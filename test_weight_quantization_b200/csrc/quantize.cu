@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32)
   constexpr int kMagicBits = 0x4B400000;
   using chunk_t = typename std::conditional<(8 * BITS <= 32), uint32_t,
                                             uint64_t>::type;
+  griddep_enter();
   const int lane = threadIdx.x & 31;
   // work items are (row, 256-channel segment) pairs, < 2^31 (checked on
   // the host); 32-bit index math keeps the per-item cost small
@@ -194,27 +195,26 @@ ttq_status launch_bits(const void* W, int64_t N, int64_t K, int64_t ldw,
                        float* delta, uint8_t* zero, cudaStream_t st) {
   const int64_t items = N * ((K + 255) / 256);
   const int64_t warps = (items + kSegsPerWarp - 1) / kSegsPerWarp;
-  const dim3 grid((unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta));
-  const dim3 block(kWarpsPerCta * 32);
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta));
+  ls.block = dim3(kWarpsPerCta * 32);
   const TW* w = static_cast<const TW*>(W);
-#define TTQ_Q(B)                                                              \
-  case B:                                                                     \
-    quantize_kernel<TW, B><<<grid, block, 0, st>>>(w, N, K, ldw, s, group,    \
-                                                   codes, delta, zero);       \
-    break;
+#define TTQ_Q(B)                                                            \
+  case B:                                                                   \
+    return launch(ls, st, quantize_kernel<TW, B>, w, N, K, ldw, s, group,   \
+                  codes, delta, zero);
   switch (bits) {
     TTQ_Q(2) TTQ_Q(3) TTQ_Q(4) TTQ_Q(5) TTQ_Q(6) TTQ_Q(7) TTQ_Q(8)
-    default:
-      return TTQ_ERR_INVALID_ARG;
   }
 #undef TTQ_Q
-  return launch_status();
+  return TTQ_ERR_INVALID_ARG;
 }
 
 // q_out[n][j] = code of channel j; one thread per 32-code block.
 __global__ void unpack_kernel(const uint32_t* __restrict__ codes, int64_t N,
                               int64_t K, int bits,
                               uint8_t* __restrict__ q_out) {
+  griddep_enter();
   const int64_t blocks = K / 32;
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= N * blocks) return;
@@ -253,10 +253,10 @@ ttq_status launch_quantize(const void* W, ttq_dtype wt, int64_t N, int64_t K,
 ttq_status launch_unpack(const uint32_t* codes, int64_t N, int64_t K, int bits,
                          uint8_t* q_out, cudaStream_t st) {
   const int64_t total = N * (K / 32);
-  const int threads = 256;
-  unpack_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0,
-                  st>>>(codes, N, K, bits, q_out);
-  return launch_status();
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)((total + 255) / 256));
+  ls.block = dim3(256);
+  return launch(ls, st, unpack_kernel, codes, N, K, bits, q_out);
 }
 
 }  // namespace ttq

@@ -1,11 +1,8 @@
 // scales.cu — step 2 of TTQ: AWQ scales from the shrunk diagonal covariance.
 //
-// TTQ review, "Proposed method", bullets 2-4: AWQ with a closed form on the
-// diagonal input covariance, shrunk by lambda, hyperparameters fixed. With
-// m_j = sum_j / T:
-//   c_j = (1 - lambda) m_j + lambda mean_k(m_k),   s_j = c_j^(alpha/p).
+// TTQ review, "Proposed method", bullets 2-4 (arithmetic in awq_scale.cuh).
 // O(K) work in one CTA; the mean reduced in a fixed order.
-#include "common.cuh"
+#include "awq_scale.cuh"
 #include "kernels.h"
 
 namespace ttq {
@@ -13,46 +10,17 @@ namespace {
 
 constexpr int kThreads = 1024;
 
-// One CTA: the mean in fp64 (fixed order), then per channel the shrunk
-// statistic c_j in fp64 and s_j = c_j^(alpha/p). The power runs in fp32 on
-// c_j rounded to fp32 (relative error below 1e-6, far inside the 1e-5
-// agreement with the fp64 definition) because fp64 pow is slow.
 __global__ void __launch_bounds__(kThreads)
     awq_scales_kernel(const float* __restrict__ sum, int64_t T_total,
                       int64_t K, double alpha, double lambda, double p,
                       float* __restrict__ s, float* __restrict__ inv_s) {
   __shared__ double warp_sums[kThreads / 32];
-  __shared__ double mbar_s;
+  griddep_enter();
   const double invT = 1.0 / (double)T_total;
-  double local = 0.0;
+  const double mbar = awq_channel_mean<kThreads>(sum, K, invT, warp_sums);
   for (int64_t j = threadIdx.x; j < K; j += kThreads)
-    local += (double)sum[j] * invT;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1)
-    local += __shfl_xor_sync(0xffffffffu, local, o);
-  if ((threadIdx.x & 31) == 0) warp_sums[threadIdx.x >> 5] = local;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double total = 0.0;
-    for (int w = 0; w < kThreads / 32; ++w) total += warp_sums[w];
-    mbar_s = total / (double)K;
-  }
-  __syncthreads();
-  const double mbar = mbar_s;
-  const float expo = (float)(alpha / p);
-  for (int64_t j = threadIdx.x; j < K; j += kThreads) {
-    const double m = (double)sum[j] * invT;
-    const double c = (1.0 - lambda) * m + lambda * mbar;
-    float sj = 1.f, ij = 1.f;
-    if (alpha != 0.0 && c > 0.0 && isfinite(c)) {
-      const float cf = (float)c;
-      sj = (cf > 1e-30f && cf < 1e30f) ? powf(cf, expo)
-                                       : (float)pow(c, alpha / p);
-      ij = 1.f / sj;
-    }
-    s[j] = sj;
-    inv_s[j] = ij;
-  }
+    awq_scale_one(__ldcg(sum + j), invT, mbar, alpha, lambda, p, s[j],
+                  inv_s[j]);
 }
 
 }  // namespace
@@ -60,9 +28,11 @@ __global__ void __launch_bounds__(kThreads)
 ttq_status launch_awq_scales(const float* sum, int64_t T_total, int64_t K,
                              double alpha, double lambda, double p, float* s,
                              float* inv_s, cudaStream_t st) {
-  awq_scales_kernel<<<1, kThreads, 0, st>>>(sum, T_total, K, alpha, lambda, p,
-                                            s, inv_s);
-  return launch_status();
+  LaunchShape ls;
+  ls.grid = dim3(1);
+  ls.block = dim3(kThreads);
+  return launch(ls, st, awq_scales_kernel, sum, T_total, K, alpha, lambda, p,
+                s, inv_s);
 }
 
 }  // namespace ttq

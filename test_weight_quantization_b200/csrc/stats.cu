@@ -14,11 +14,16 @@
 //   - rows split across a thread-block cluster of up to 8 CTAs; partial sums
 //     are reduced through distributed shared memory by cluster rank 0 in a
 //     fixed order, so the result is deterministic and no global scratch is
-//     needed.
+//     needed;
+//   - optionally (ttq_act_stats_scales) step 2 runs in the same launch: the
+//     cluster that finishes its column tile last, told by a counter in
+//     global memory, computes the scales of all K channels. Nothing waits on
+//     another CTA, so the fused form adds no spin and no co-residency need.
 #include <cooperative_groups.h>
 
 #include <algorithm>
 
+#include "awq_scale.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -65,13 +70,25 @@ __device__ __forceinline__ float moment(float x, float p) {
   return powf(fabsf(x), p);
 }
 
+// Step 2 fused behind the statistics; s == nullptr leaves it out.
+struct ScalesTail {
+  float* s;
+  float* inv_s;
+  unsigned int* counter;  // zero on entry; the last cluster resets it
+  int64_t T_total;
+  double alpha, lambda, p;
+};
+
 // grid = (column tiles, cluster size); cluster = (1, C, 1).
 template <typename TX, int PK>
 __global__ void __launch_bounds__(kThreads)
     act_stats_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
                      int64_t ldx, float p, int accumulate, int cw,
-                     float* __restrict__ sum_out) {
-  extern __shared__ float smem[];  // [rows_per_pass][cw] then part[cw]
+                     float* __restrict__ sum_out, ScalesTail tail) {
+  // [rows_per_pass][cw] then part[cw]
+  extern __shared__ __align__(16) float smem[];
+  __shared__ int last_flag;
+  griddep_enter();
   cg::cluster_group cluster = cg::this_cluster();
   const int tpr = cw / 8;                 // threads per row segment
   const int rows_per_pass = kThreads / tpr;
@@ -145,13 +162,46 @@ __global__ void __launch_bounds__(kThreads)
       sum_out[col] = accumulate ? sum_out[col] + s : s;
     }
   }
-  cluster.sync();  // keep every CTA's shared memory alive until read
+  if (tail.s == nullptr) {
+    cluster.sync();  // keep every CTA's shared memory alive until read
+    return;
+  }
+
+  // Fused step 2. Rank 0 publishes its tile (fence, then one arrival per
+  // cluster); the arrival that completes the count marks its cluster last
+  // and tells every CTA of the cluster through its shared memory.
+  if (rank == 0) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      const unsigned prev = atomicAdd(tail.counter, 1u);
+      const int last = prev == gridDim.x - 1;
+      if (last) {
+        __threadfence();
+        *tail.counter = 0u;  // every arrival of this launch is in
+      }
+      for (int q = 0; q < C; ++q) *cluster.map_shared_rank(&last_flag, q) = last;
+    }
+  }
+  cluster.sync();  // after this no CTA reads another's shared memory
+  if (!last_flag) return;
+  __threadfence();
+  // every CTA of the last cluster forms the same mean, then the scales of
+  // its share of the channels
+  double* warp_sums = reinterpret_cast<double*>(smem);
+  const double invT = 1.0 / (double)tail.T_total;
+  const double mbar =
+      awq_channel_mean<kThreads>(sum_out, K, invT, warp_sums);
+  for (int64_t j = (int64_t)rank * kThreads + tid; j < K;
+       j += (int64_t)C * kThreads)
+    awq_scale_one(__ldcg(sum_out + j), invT, mbar, tail.alpha, tail.lambda,
+                  tail.p, tail.s[j], tail.inv_s[j]);
 }
 
 template <typename TX, int PK>
 ttq_status launch_typed(const void* X, int64_t T, int64_t K, int64_t ldx,
                         float p, int accumulate, float* sum_out,
-                        cudaStream_t st) {
+                        const ScalesTail& tail, cudaStream_t st) {
   const int cw = K >= 1024 ? 128 : 64;
   const int64_t col_tiles = (K + cw - 1) / cw;
   const int target = 2 * sm_count();
@@ -162,31 +212,41 @@ ttq_status launch_typed(const void* X, int64_t T, int64_t K, int64_t ldx,
   const int rows_per_pass = kThreads / (cw / 8);
   const size_t smem = sizeof(float) * ((size_t)rows_per_pass * cw + cw);
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)col_tiles, (unsigned)C, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = C;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, act_stats_kernel<TX, PK>,
-                                        static_cast<const TX*>(X), T, K, ldx,
-                                        p, accumulate, cw, sum_out));
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)col_tiles, (unsigned)C, 1);
+  ls.block = dim3(kThreads, 1, 1);
+  ls.smem = smem;
+  ls.cluster_y = (unsigned)C;
+  return launch(ls, st, act_stats_kernel<TX, PK>, static_cast<const TX*>(X),
+                T, K, ldx, p, accumulate, cw, sum_out, tail);
 }
 
 template <typename TX>
 ttq_status launch_p(const void* X, int64_t T, int64_t K, int64_t ldx, float p,
-                    int accumulate, float* sum_out, cudaStream_t st) {
+                    int accumulate, float* sum_out, const ScalesTail& tail,
+                    cudaStream_t st) {
   if (p == 2.0f)
-    return launch_typed<TX, 2>(X, T, K, ldx, p, accumulate, sum_out, st);
+    return launch_typed<TX, 2>(X, T, K, ldx, p, accumulate, sum_out, tail,
+                               st);
   if (p == 1.0f)
-    return launch_typed<TX, 1>(X, T, K, ldx, p, accumulate, sum_out, st);
-  return launch_typed<TX, 0>(X, T, K, ldx, p, accumulate, sum_out, st);
+    return launch_typed<TX, 1>(X, T, K, ldx, p, accumulate, sum_out, tail,
+                               st);
+  return launch_typed<TX, 0>(X, T, K, ldx, p, accumulate, sum_out, tail, st);
+}
+
+ttq_status launch_x(const void* X, ttq_dtype xt, int64_t T, int64_t K,
+                    int64_t ldx, float p, int accumulate, float* sum_out,
+                    const ScalesTail& tail, cudaStream_t st) {
+  switch (xt) {
+    case TTQ_F32:
+      return launch_p<float>(X, T, K, ldx, p, accumulate, sum_out, tail, st);
+    case TTQ_BF16:
+      return launch_p<__nv_bfloat16>(X, T, K, ldx, p, accumulate, sum_out,
+                                     tail, st);
+    case TTQ_F16:
+      return launch_p<__half>(X, T, K, ldx, p, accumulate, sum_out, tail, st);
+  }
+  return TTQ_ERR_INVALID_ARG;
 }
 
 }  // namespace
@@ -194,15 +254,18 @@ ttq_status launch_p(const void* X, int64_t T, int64_t K, int64_t ldx, float p,
 ttq_status launch_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                             int64_t ldx, float p, int accumulate,
                             float* sum_out, cudaStream_t st) {
-  switch (xt) {
-    case TTQ_F32:
-      return launch_p<float>(X, T, K, ldx, p, accumulate, sum_out, st);
-    case TTQ_BF16:
-      return launch_p<__nv_bfloat16>(X, T, K, ldx, p, accumulate, sum_out, st);
-    case TTQ_F16:
-      return launch_p<__half>(X, T, K, ldx, p, accumulate, sum_out, st);
-  }
-  return TTQ_ERR_INVALID_ARG;
+  const ScalesTail none = {nullptr, nullptr, nullptr, 0, 0.0, 0.0, 0.0};
+  return launch_x(X, xt, T, K, ldx, p, accumulate, sum_out, none, st);
+}
+
+ttq_status launch_act_stats_scales(const void* X, ttq_dtype xt, int64_t T,
+                                   int64_t K, int64_t ldx, int accumulate,
+                                   int64_t T_total, double alpha,
+                                   double lambda, double p, float* sum_out,
+                                   float* s, float* inv_s,
+                                   unsigned int* counter, cudaStream_t st) {
+  const ScalesTail tail = {s, inv_s, counter, T_total, alpha, lambda, p};
+  return launch_x(X, xt, T, K, ldx, (float)p, accumulate, sum_out, tail, st);
 }
 
 }  // namespace ttq

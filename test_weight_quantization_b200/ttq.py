@@ -42,6 +42,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "ttq_act_stats": [P, I, I64, I64, I64, F, I, P, P],
         "ttq_awq_scales": [P, I64, I64, P, P, P, P],
+        "ttq_act_stats_scales": [P, I, I64, I64, I64, I, I64, P, P, P, P, P,
+                                 P],
         "ttq_quantize_rtn_grouped": [P, I, I64, I64, I64, P, I, I, P, P, P, P],
         "ttq_w_lowbit_gemm_workspace_size": [I64, I64, I],
         "ttq_w_lowbit_gemm": [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P,
@@ -71,7 +73,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 
 # Names the C ABI exports (include/ttq.h).
-EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_quantize_rtn_grouped",
+EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_act_stats_scales",
+           "ttq_quantize_rtn_grouped",
            "ttq_w_lowbit_gemm_workspace_size", "ttq_w_lowbit_gemm",
            "ttq_prepare_activations", "ttq_w_lowbit_gemm_prepared",
            "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
@@ -167,6 +170,33 @@ def awq_scales(sums: torch.Tensor, T_total: int, alpha: float = 0.5,
                                ctypes.addressof(prm), s.data_ptr(),
                                inv_s.data_ptr(), _stream()), "ttq_awq_scales")
     return s, inv_s
+
+
+def new_counter(device=None) -> torch.Tensor:
+    """A zeroed device word for act_stats_scales (one per concurrent
+    stream; each call leaves it zero again)."""
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def act_stats_scales(X: torch.Tensor, counter: torch.Tensor,
+                     alpha: float = 0.5, lam: float = 0.1, p: float = 2.0,
+                     sums=None, s=None, inv_s=None, accumulate: bool = False,
+                     T_total: int | None = None):
+    """Steps 1 and 2 in one launch: (sums, s, inv_s), each fp32 [K]."""
+    ldx = _rows(X, "X")
+    _dev(counter, "counter")
+    T, K = X.shape
+    f32 = dict(dtype=torch.float32, device=X.device)
+    sums = torch.empty(K, **f32) if sums is None else sums
+    s = torch.empty(K, **f32) if s is None else s
+    inv_s = torch.empty(K, **f32) if inv_s is None else inv_s
+    prm = _Params(0, 0, alpha, lam, p)
+    _check(_lib.ttq_act_stats_scales(
+        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, 1 if accumulate else 0,
+        int(T if T_total is None else T_total), ctypes.addressof(prm),
+        sums.data_ptr(), s.data_ptr(), inv_s.data_ptr(), counter.data_ptr(),
+        _stream()), "ttq_act_stats_scales")
+    return sums, s, inv_s
 
 
 def quantize_rtn_grouped(W: torch.Tensor, s: torch.Tensor | None, bits: int,

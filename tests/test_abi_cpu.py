@@ -45,7 +45,7 @@ def test_status_strings_and_version(lib):
     assert lib.ttq_status_string(0) == b"TTQ_OK"
     assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
     assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
-    assert lib.ttq_abi_version() == 2
+    assert lib.ttq_abi_version() == 3
 
 
 def test_workspace_size(lib):
@@ -65,6 +65,21 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert lib.ttq_act_stats(fake, 1, 8, 60, 64, 2.0, 0, fake, None) == 1  # K%8
     assert lib.ttq_act_stats(fake, 1, 8, 64, 64, -1.0, 0, fake, None) == 1
     assert lib.ttq_act_stats(fake, 7, 8, 64, 64, 2.0, 0, fake, None) == 1
+    f = lib.ttq_act_stats_scales
+    f.argtypes = [P, I, I64, I64, I64, I, I64, P, P, P, P, P, P]
+
+    class Prm(ctypes.Structure):
+        _fields_ = [("bits", I), ("group", I), ("alpha", F), ("lambda_", F),
+                    ("p", F)]
+    prm = Prm(0, 0, 0.5, 0.1, 2.0)
+    pp = ctypes.addressof(prm)
+    assert f(fake, 1, 8, 64, 64, 0, 8, pp, fake, fake, fake, None, None) == 1
+    assert f(fake, 1, 8, 64, 64, 0, 7, pp, fake, fake, fake, fake, None) == 1
+    assert f(fake, 1, 8, 64, 64, 2, 8, pp, fake, fake, fake, fake, None) == 1
+    assert f(fake, 1, 8, 64, 64, 0, 8, None, fake, fake, fake, fake, None) == 1
+    bad = Prm(0, 0, 0.5, 1.5, 2.0)
+    assert f(fake, 1, 8, 64, 64, 0, 8, ctypes.addressof(bad), fake, fake, fake,
+             fake, None) == 1
     lib.ttq_quantize_rtn_grouped.argtypes = [P, I, I64, I64, I64, P, I, I, P,
                                              P, P, P]
     q = lib.ttq_quantize_rtn_grouped

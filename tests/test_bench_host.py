@@ -51,6 +51,44 @@ def test_layer_token_throughput_counts_every_replica():
         6 * 2048 / 0.5e-3)
 
 
+def test_projection_groups_stack_layers_that_share_an_input():
+    import bench
+    from test_weight_quantization_b200.inputs import WORKLOADS
+    wl = WORKLOADS["opt125m-block"]
+    g = bench.projection_groups(wl)
+    assert [(n, k, sum(L.N for L in Ls)) for n, k, Ls in g] == [
+        ("q|k|v", "attn_in", 2304), ("o", "attn_out", 768),
+        ("fc1", "mlp_in", 3072), ("fc2", "mlp_mid", 768)]
+    # every layer appears exactly once
+    assert sorted(L.name for _, _, Ls in g for L in Ls) == sorted(
+        L.name for L in wl.layers)
+    assert len(bench.projection_groups(wl, separate=True)) == 6
+    # low-rank layers keep their own factors: never stacked
+    gem = WORKLOADS["gemma1b-mlp"]
+    assert all(len(Ls) == 1 for _, _, Ls in bench.projection_groups(gem))
+
+
+def test_launch_plan_follows_the_method_per_input():
+    import bench
+    from test_weight_quantization_b200.inputs import WORKLOADS
+    wl = WORKLOADS["opt125m-block"]
+    inputs = bench.layer_inputs(wl)
+    assert inputs == ["attn_in", "attn_out", "mlp_in", "mlp_mid"]
+    plan = bench.launch_plan(inputs, bench.projection_groups(wl))
+    assert len(plan) == 16
+    assert plan[:4] == [("stats_scales", "attn_in"), ("prepare", "attn_in"),
+                        ("quantize", "q|k|v"), ("gemm", "q|k|v")]
+    sep = bench.launch_plan(inputs, bench.projection_groups(wl, True), True)
+    assert len(sep) == 4 * 3 + 6 * 2
+    # each projection comes after its input's scales and prepare
+    for p in (plan, sep):
+        for i, (kind, key) in enumerate(p):
+            if kind == "gemm":
+                k = next(kk for g, kk, _ in bench.projection_groups(
+                    wl, p is sep) if g == key)
+                assert ("prepare", k) in p[:i]
+
+
 def test_reference_arm_rank_nonzero_exits_without_work():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),

@@ -134,3 +134,39 @@ def test_decode_sweep_full_size(ttq):
                 assert_gemm_close(np32(Y)[tok], ref,
                                   f"decode b={bits} g={group} T={T} "
                                   f"{layer.name}", Y.dtype)
+
+
+def test_stacked_projection_matches_layers(ttq):
+    """q, k, v of the OPT block as one projection of their stacked weights
+    (as the benchmark runs them): codes equal the per-layer codes row for
+    row, outputs equal the per-layer outputs column block for column block,
+    and the fused statistics + scales launch feeds both."""
+    from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs
+    wl = WORKLOADS["opt125m-block"]
+    data = make_inputs(wl)
+    X = data["X"]["attn_in"].cuda()
+    Ls = [L for L in wl.layers if L.input_name == "attn_in"]
+    Ws = [data["W"][L.name].cuda() for L in Ls]
+    ctr = ttq.new_counter()
+    sums, s, inv = ttq.act_stats_scales(X, ctr, wl.alpha, wl.lam, wl.p)
+    Xs, _ = ttq.prepare_activations(X, inv, wl.bits)
+    cs, ds, zs = ttq.quantize_rtn_grouped(torch.cat(Ws), s, wl.bits, wl.group)
+    Ys = ttq.w_lowbit_gemm_prepared(Xs, None, cs, ds, zs, cs.shape[0], wl.bits,
+                                    wl.group, out_dtype=wl.dtype)
+    row = 0
+    for L, W in zip(Ls, Ws):
+        c, d, z = ttq.quantize_rtn_grouped(W, s, wl.bits, wl.group)
+        assert torch.equal(c, cs[row:row + L.N])
+        assert torch.equal(d, ds[row:row + L.N])
+        assert torch.equal(z, zs[row:row + L.N])
+        Y = ttq.w_lowbit_gemm_prepared(Xs, None, c, d, z, L.N, wl.bits,
+                                       wl.group, out_dtype=wl.dtype)
+        # same operands, same K order: the tensor-core sums agree exactly
+        assert torch.equal(Y, Ys[:, row:row + L.N])
+        row += L.N
+    tok = sample_rows(wl.T, 8, 5)
+    cd, dd, zd = dense(cs, ds, zs, X.shape[1], wl.bits, wl.group)
+    ref = oracle.lowbit_gemm(np32(X.cpu()[:wl.T]), np32(inv), cd, dd, zd,
+                             cs.shape[0], wl.bits, wl.group, rows=tok)
+    assert_gemm_close(np32(Ys)[tok], ref, "stacked q|k|v", Ys.dtype)
+    assert int(ctr.item()) == 0

@@ -89,6 +89,58 @@ def test_scales_zero_statistic(ttq):
     assert torch.all(s == 1) and torch.all(inv == 1)
 
 
+# ------------------------------------------------ fused stats + scales ----
+
+@pytest.mark.parametrize("dt", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("T,K", [(1, 8), (37, 264), (2048, 768),
+                                 (300, 3072), (64, 14336)])
+@pytest.mark.parametrize("alpha,lam,p", [(0.5, 0.1, 2.0), (0.0, 0.1, 2.0),
+                                         (0.4, 0.0, 1.0), (0.6, 0.3, 3.0)])
+def test_stats_scales_fused(ttq, dt, T, K, alpha, lam, p):
+    """One launch gives the sums of act_stats bit for bit and the oracle's
+    scales; the counter comes back to zero."""
+    X = acts(T, K, 3 * T + K, DT[dt]).cuda()
+    ctr = ttq.new_counter()
+    sums, s, inv = ttq.act_stats_scales(X, ctr, alpha, lam, p)
+    assert torch.equal(sums, ttq.act_stats(X, p))
+    rs, rinv = oracle.awq_scales(np32(sums).astype(np.float64), T, alpha, lam,
+                                 p)
+    assert_rel_close(np32(s), rs, what="fused s")
+    assert_rel_close(np32(inv), rinv, what="fused inv_s")
+    s2, inv2 = ttq.awq_scales(sums, T, alpha, lam, p)
+    assert torch.allclose(s, s2, rtol=1e-6, atol=0)
+    assert int(ctr.item()) == 0
+
+
+def test_stats_scales_fused_repeated_and_accumulate(ttq):
+    """Back-to-back calls reuse one counter; the chunked form divides by the
+    running token count."""
+    X = acts(900, 1152, 11, torch.bfloat16).cuda()
+    ctr = ttq.new_counter()
+    first = [t.clone() for t in ttq.act_stats_scales(X, ctr)]
+    for _ in range(5):
+        again = ttq.act_stats_scales(X, ctr)
+        for a, b in zip(first, again):
+            assert torch.equal(a, b)
+    sums, s, inv = ttq.act_stats_scales(X[:400], ctr)
+    sums, s, inv = ttq.act_stats_scales(X[400:], ctr, sums=sums, s=s,
+                                        inv_s=inv, accumulate=True,
+                                        T_total=900)
+    assert_rel_close(np32(sums), oracle.act_sums(np32(X.cpu())),
+                     what="chunked sums")
+    rs, rinv = oracle.awq_scales(np32(sums).astype(np.float64), 900, 0.5, 0.1,
+                                 2.0)
+    assert_rel_close(np32(s), rs, what="chunked s")
+    assert int(ctr.item()) == 0
+
+
+def test_stats_scales_fused_zero_input(ttq):
+    X = torch.zeros(64, 256, dtype=torch.bfloat16, device="cuda")
+    ctr = ttq.new_counter()
+    sums, s, inv = ttq.act_stats_scales(X, ctr, 0.5, 0.0, 2.0)
+    assert torch.all(sums == 0) and torch.all(s == 1) and torch.all(inv == 1)
+
+
 # ---------------------------------------------------------- quantize ----
 
 def dense(c, d, z, K, bits, group):
@@ -185,6 +237,30 @@ def test_gemm_shapes(ttq, T, bits, group):
     Y, inv, c, d, z = run_path(ttq, X, W, bits, group)
     ref = oracle_y(X, inv, c, d, z, N, bits, group)
     assert_gemm_close(np32(Y), ref, f"T={T} b={bits} g={group}", Y.dtype)
+
+
+@pytest.mark.parametrize("N,pitch", [(264, 264), (264, 320), (300, 300),
+                                     (136, 136)])
+@pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
+def test_gemm_output_tile_store(ttq, N, pitch, out):
+    """Both ways the projection writes Y: 16-byte aligned rows go through
+    a shared-memory tile and a tensor store (ragged N and T clipped), other
+    pitches through per-row stores. Columns beyond N stay untouched."""
+    T, K, bits, group = 300, 384, 4, 32
+    X = acts(T, K, 31, torch.bfloat16)
+    W = weights(N, K, 32, torch.bfloat16)
+    Xg, Wg = X.cuda(), W.cuda()
+    sums = ttq.act_stats(Xg)
+    s, inv = ttq.awq_scales(sums, T)
+    c, d, z = ttq.quantize_rtn_grouped(Wg, s, bits, group)
+    big = torch.full((T, pitch), 7.0, dtype=DT[out], device="cuda")
+    Y = big[:, :N]
+    ttq.w_lowbit_gemm(Xg, inv, c, d, z, N, bits, group, out=Y)
+    torch.cuda.synchronize()
+    ref = oracle_y(X, inv, c, d, z, N, bits, group)
+    assert_gemm_close(np32(Y), ref, f"N={N} pitch={pitch} {out}", Y.dtype)
+    if pitch > N:
+        assert torch.all(big[:, N:] == 7.0)
 
 
 @pytest.mark.parametrize("bits", [6, 7, 8])
