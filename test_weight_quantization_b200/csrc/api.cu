@@ -170,8 +170,8 @@ TTQ_EXPORT ttq_status ttq_quantize_rtn_grouped(
   if (!W || !codes || !delta || !zero || !valid_dtype(wt) || N < 1 ||
       K < 32 || K % 32 != 0 || bits < 2 || bits > 8 || !valid_group(group) ||
       K % group != 0 || ldw < K || !rows_aligned(W, wt, ldw) ||
-      (s && !aligned(s, 16)) || !aligned(codes, 4) || !aligned(delta, 4) ||
-      N * ((K + 255) / 256) >= ((int64_t)1 << 31))
+      (s && !aligned(s, 16)) || !aligned(codes, 16) || !aligned(delta, 16) ||
+      !aligned(zero, 16) || N * (K / 32) >= ((int64_t)1 << 31))
     return TTQ_ERR_INVALID_ARG;
   return launch_quantize(W, wt, N, K, ldw, s, bits, group, codes, delta, zero,
                          as_stream(stream));

@@ -292,9 +292,11 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     *aborted = 0;
     fence_barrier_init();
   }
-  // everything below reads what earlier kernels wrote (or owns TMEM that a
-  // still-running kernel on this SM may hold)
-  griddep_enter();
+  // The set-up above and the TMEM allocation touch no global memory, so
+  // they overlap the previous kernel on the stream. (An allocation can
+  // only wait for TMEM of a CTA that is already running on this SM, which
+  // releases it when it ends.) Everything after the wait may read what
+  // earlier kernels wrote.
   if (warp == 1) {
     tmem_alloc(base + L.tmem, (uint32_t)p.tmem_cols);
     tmem_relinquish();
@@ -302,6 +304,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_enter();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tmem_a = tmem + (uint32_t)p.acc_cols;  // weight-stage ring
 

@@ -8,13 +8,15 @@
 //   D = (mx - mn)/(2^b - 1) (1 if 0);  r = 1/D;
 //   z = clamp(rint(-mn*r));  q = clamp(rint(w*r) + z).
 //
-// Design (HBM-bound): one warp per 256-channel segment of a row; a lane owns
-// 8 consecutive channels loaded as one 16-byte vector. A group spans g/8
-// lanes and its min/max is a butterfly shuffle inside that lane segment.
-// Four lanes hold one 32-code block; they exchange their 8*b-bit chunks by
-// shuffles and each lane stores the one or two packed words it owns, so a
-// warp writes 8*b consecutive words. Delta and zero go out from the first
-// lane of each group.
+// Design (HBM-bound, kept below the instruction budget): one lane per
+// 32-code block, i.e. 32 consecutive channels of one weight row, loaded as
+// 64 contiguous bytes (bf16/fp16) and packed by the lane itself into its
+// `bits` words, which it stores directly. Consecutive lanes take consecutive
+// blocks of the [N, K/32] block grid, so a warp reads and writes contiguous
+// spans. A group of g >= 32 channels spans g/32 neighbouring lanes and its
+// range is a 1- or 2-level shuffle; with g = 16 a lane holds two groups.
+// The IEEE divide and reciprocal of a group run once per 32 elements.
+#include <algorithm>
 #include <type_traits>
 
 #include "common.cuh"
@@ -24,167 +26,384 @@ namespace ttq {
 namespace {
 
 constexpr int kWarpsPerCta = 8;
-constexpr int kSegsPerWarp = 2;  // 256-channel segments per warp
+// scales staged in shared memory up to this size (two CTAs per SM)
+constexpr int64_t kMaxStagedScaleBytes = 96 * 1024;
 
-// Packs this lane's eight BITS-bit codes (chunk, codes at BITS*i) into the
-// 32-code block shared by the four lanes of its quad and stores the words
-// the lane owns (block words qpos and qpos + 4).
+// Raw bytes of one block's 32 weights: 4 x 16 bytes for 16-bit types,
+// 8 x 16 bytes for fp32.
+template <typename TW>
+struct RawBlock {
+  static constexpr int V = sizeof(TW) * 32 / 16;
+  uint4 v[V];
+};
+
+template <typename TW>
+__device__ __forceinline__ void load_raw(const TW* p, RawBlock<TW>& r) {
+#pragma unroll
+  for (int i = 0; i < RawBlock<TW>::V; ++i)
+    r.v[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+}
+
+template <typename TW>
+__device__ __forceinline__ void unpack_raw(const RawBlock<TW>& r,
+                                           float (&w)[32]);
+template <>
+__device__ __forceinline__ void unpack_raw<float>(const RawBlock<float>& r,
+                                                  float (&w)[32]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    w[4 * i] = __uint_as_float(r.v[i].x);
+    w[4 * i + 1] = __uint_as_float(r.v[i].y);
+    w[4 * i + 2] = __uint_as_float(r.v[i].z);
+    w[4 * i + 3] = __uint_as_float(r.v[i].w);
+  }
+}
+template <>
+__device__ __forceinline__ void unpack_raw<__nv_bfloat16>(
+    const RawBlock<__nv_bfloat16>& r, float (&w)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    bf16x2_to_f32(r.v[i].x, w[8 * i], w[8 * i + 1]);
+    bf16x2_to_f32(r.v[i].y, w[8 * i + 2], w[8 * i + 3]);
+    bf16x2_to_f32(r.v[i].z, w[8 * i + 4], w[8 * i + 5]);
+    bf16x2_to_f32(r.v[i].w, w[8 * i + 6], w[8 * i + 7]);
+  }
+}
+template <>
+__device__ __forceinline__ void unpack_raw<__half>(const RawBlock<__half>& r,
+                                                   float (&w)[32]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f16x2_to_f32(r.v[i].x, w[8 * i], w[8 * i + 1]);
+    f16x2_to_f32(r.v[i].y, w[8 * i + 2], w[8 * i + 3]);
+    f16x2_to_f32(r.v[i].z, w[8 * i + 4], w[8 * i + 5]);
+    f16x2_to_f32(r.v[i].w, w[8 * i + 6], w[8 * i + 7]);
+  }
+}
+
+// The block's BITS words at `out` (4 * BITS bytes, aligned to the largest
+// power of two dividing 4 * BITS times the block index).
 template <int BITS>
-__device__ __forceinline__ void store_block(uint64_t chunk, int lane,
-                                            uint32_t* out, bool active) {
-  const int qpos = lane & 3;
-  if constexpr (BITS == 4) {
-    // eight 4-bit codes are exactly block word qpos
-    if (active) out[qpos] = (uint32_t)chunk;
-  } else if constexpr (BITS == 8) {
-    if (active)
-      *reinterpret_cast<uint2*>(out + 2 * qpos) =
-          make_uint2((uint32_t)chunk, (uint32_t)(chunk >> 32));
-  } else if constexpr (BITS == 2) {
-    // two lanes (16 bits each) make one word
-    const uint32_t hi = __shfl_down_sync(0xffffffffu, (uint32_t)chunk, 1);
-    if (active && (qpos & 1) == 0)
-      out[qpos >> 1] = (uint32_t)chunk | (hi << 16);
+__device__ __forceinline__ void store_words(uint32_t* out,
+                                            const uint32_t (&cw)[BITS]) {
+  if constexpr (BITS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS; i += 4)
+      *reinterpret_cast<uint4*>(out + i) =
+          make_uint4(cw[i], cw[i + 1], cw[i + 2], cw[i + 3]);
+  } else if constexpr (BITS % 2 == 0) {
+#pragma unroll
+    for (int i = 0; i < BITS; i += 2)
+      *reinterpret_cast<uint2*>(out + i) = make_uint2(cw[i], cw[i + 1]);
   } else {
-    const int qbase = lane & ~3;
-    uint64_t c[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)chunk, qbase + j);
-      const uint32_t hi =
-          __shfl_sync(0xffffffffu, (uint32_t)(chunk >> 32), qbase + j);
-      c[j] = ((uint64_t)hi << 32) | lo;
-    }
-    if (!active) return;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int wi = qpos + 4 * half;  // word index inside the block
-      if (wi >= BITS) continue;
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int lo_bit = 8 * BITS * j;  // chunk j spans [lo_bit, +8*BITS)
-        const int shift = lo_bit - 32 * wi;
-        if (lo_bit + 8 * BITS <= 32 * wi || lo_bit >= 32 * wi + 32) continue;
-        word |= shift >= 0 ? (uint32_t)(c[j] << shift)
-                           : (uint32_t)(c[j] >> (-shift));
+    for (int i = 0; i < BITS; ++i) out[i] = cw[i];
+  }
+}
+
+// Row and block of the warp-relative item `lane` of a warp whose first
+// item is item0: one division per warp, then at most 32/bpr + 1 steps.
+__device__ __forceinline__ void locate(uint32_t item0, uint32_t bpr, int lane,
+                                       uint32_t& n, uint32_t& k) {
+  n = item0 / bpr;
+  k = item0 - n * bpr + (uint32_t)lane;
+  while (k >= bpr) {
+    k -= bpr;
+    ++n;
+  }
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Shared-memory layout of the staged scales: block b's 32 scales at float
+// offset 36 b (16 bytes of padding), so the eight lanes of a quarter-warp
+// (eight consecutive blocks) read eight disjoint bank quadruples.
+constexpr int kScalePitch = 36;
+
+struct QuantCtx {
+  const float* s;     // global scales (null: s = 1)
+  const float* s_sm;  // staged scales, or null
+  int64_t K, ldc, ldg;
+  int group, lpg;
+  uint32_t* codes;
+  float* delta;
+  uint8_t* zero;
+};
+
+// The packing is additive: bits(M + v) = bits(M) + v for |v| < 2^22, so a
+// code q placed at bit sh of a word contributes (bits(M + q - z) << sh)
+// and the word is corrected once by the constant sum of (bits(M) << sh)
+// minus z times the sum of (1 << sh); all mod 2^32 and exact because the
+// codes' fields are disjoint. A code that straddles two words is formed
+// explicitly and split.
+template <int BITS>
+struct PackConst {
+  uint32_t cm[BITS];     // sum of bits(M) << sh over whole codes
+  uint32_t sz[2][BITS];  // sum of 1 << sh over whole codes of group half
+  __host__ __device__ constexpr PackConst() : cm(), sz() {
+    for (int e = 0; e < 32; ++e) {
+      const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
+      if (sh + BITS <= 32) {
+        cm[wd] += 0x4B400000u << sh;
+        sz[e / 16][wd] += 1u << sh;
       }
-      out[wi] = word;
+    }
+  }
+};
+
+// STAGED: the scales come from shared memory (staged per CTA, ones when s
+// is null); otherwise from global memory (null: no scaling).
+template <int BITS, bool G16, bool STAGED>
+__device__ __forceinline__ void quantize_item(const QuantCtx& c,
+                                              float (&w)[32], uint32_t n,
+                                              uint32_t k, bool live) {
+  constexpr int QMAX = (1 << BITS) - 1;
+  constexpr int NG = G16 ? 2 : 1;  // groups held by one lane
+  constexpr int E = 32 / NG;       // elements per held group
+  // rint(x) for |x| < 2^22 is exactly (x + 1.5*2^23) - 1.5*2^23 under
+  // round-to-nearest-even (the sum lands in [2^23, 2^24), where the ulp is
+  // 1, and the offset is even).
+  constexpr float kMagic = 12582912.0f;  // M = 1.5 * 2^23
+  constexpr uint32_t kMagicBits = 0x4B400000u;
+  constexpr float kTop = kMagic + (float)QMAX;
+  constexpr PackConst<BITS> pc;
+
+  const int64_t col0 = (int64_t)k * 32;
+  if (!live) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = 0.f;
+  } else if (STAGED || c.s != nullptr) {
+    const float* sb = c.s_sm + k * kScalePitch;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 sv =
+          STAGED ? *reinterpret_cast<const float4*>(sb + 4 * i)
+                 : __ldg(reinterpret_cast<const float4*>(c.s + col0) + i);
+      w[4 * i] = __fmul_rn(w[4 * i], sv.x);
+      w[4 * i + 1] = __fmul_rn(w[4 * i + 1], sv.y);
+      w[4 * i + 2] = __fmul_rn(w[4 * i + 2], sv.z);
+      w[4 * i + 3] = __fmul_rn(w[4 * i + 3], sv.w);
+    }
+  }
+  // groups never straddle warp-items (32 is a multiple of group/32 and a
+  // row holds whole groups), so a lane past the end never shares one with
+  // a live lane
+
+  float d[NG], r[NG], zf[NG], topz[NG];
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    // group range, widened to contain 0 (min and max are exact, so the
+    // order of the comparisons does not matter)
+    float mn = 0.f, mx = 0.f;
+#pragma unroll
+    for (int e = gi * E; e < (gi + 1) * E; e += 2) {
+      mn = min3f(mn, w[e], w[e + 1]);
+      mx = max3f(mx, w[e], w[e + 1]);
+    }
+    if constexpr (!G16) {
+#pragma unroll
+      for (int o = 1; o < 4; o <<= 1) {  // g <= 128: at most 4 lanes
+        if (o < c.lpg) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+      }
+    }
+    float dd = __fdiv_rn(__fsub_rn(mx, mn), (float)QMAX);
+    if (dd == 0.f) dd = 1.f;
+    d[gi] = dd;
+    r[gi] = __frcp_rn(dd);
+    // clamp(rint(-mn * r), 0, 2^b - 1); rint(-mn * r) lies in that range
+    // already because -mn <= mx - mn, the clamp matches the definition
+    zf[gi] = fminf(fmaxf(__fadd_rn(__fmul_rn(-mn, r[gi]), kMagic), kMagic),
+                   kTop) - kMagic;
+    // q = min(rint(w*r) + z, 2^b - 1) <=> M + q - z = min(M + rint(w*r),
+    // M + 2^b - 1 - z); q >= 0 since rint(w*r) >= rint(mn*r) = -z
+    topz[gi] = kTop - zf[gi];
+  }
+
+  // code e at bits [e*BITS, e*BITS + BITS) of the block's little-endian
+  // stream
+  uint32_t cw[BITS];
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) cw[i] = 0u;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int gi = e / E;
+    const float t =
+        fminf(__fadd_rn(__fmul_rn(w[e], r[gi]), kMagic), topz[gi]);
+    const uint32_t tb = __float_as_uint(t);  // bits(M) + q - z
+    const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
+    if (sh + BITS <= 32) {
+      cw[wd] += tb << sh;
+    } else {
+      const uint32_t q = tb - kMagicBits + (uint32_t)zf[gi];
+      cw[wd] += q << sh;
+      cw[wd + 1] += q >> (32 - sh);
+    }
+  }
+  const uint32_t z0 = (uint32_t)zf[0], z1 = (uint32_t)zf[NG - 1];
+#pragma unroll
+  for (int i = 0; i < BITS; ++i)
+    cw[i] = cw[i] - pc.cm[i] + z0 * pc.sz[0][i] + z1 * pc.sz[1][i];
+  if (!live) return;
+
+  uint32_t* crow = c.codes + (int64_t)n * c.ldc;
+  store_words<BITS>(crow + (int64_t)k * BITS, cw);
+  if (G16) {
+    const int64_t gi = (int64_t)n * c.ldg + 2 * (int64_t)k;
+    *reinterpret_cast<float2*>(c.delta + gi) = make_float2(d[0], d[NG - 1]);
+    *reinterpret_cast<uint16_t*>(c.zero + gi) = (uint16_t)(z0 | (z1 << 8));
+  } else if ((k & (uint32_t)(c.lpg - 1)) == 0) {
+    const int64_t gi = (int64_t)n * c.ldg + col0 / c.group;
+    c.delta[gi] = d[0];
+    c.zero[gi] = (uint8_t)z0;
+  }
+  // the lane holding the row's first block zeroes the row's padding
+  if (k == 0) {
+    for (int64_t w2 = c.K * BITS / 32; w2 < c.ldc; ++w2) crow[w2] = 0u;
+    for (int64_t gi = c.K / c.group; gi < c.ldg; ++gi) {
+      c.delta[(int64_t)n * c.ldg + gi] = 0.f;
+      c.zero[(int64_t)n * c.ldg + gi] = 0;
     }
   }
 }
 
-template <typename TW, int BITS>
-__global__ void __launch_bounds__(kWarpsPerCta * 32)
+// Position of one lane in the [N, K/32] block grid, advanced by a fixed
+// number of blocks at a time (no division after the first).
+struct BlockPos {
+  uint32_t n, k;
+  __device__ __forceinline__ void advance(uint32_t dn, uint32_t dk,
+                                          uint32_t bpr) {
+    n += dn;
+    k += dk;
+    if (k >= bpr) {
+      k -= bpr;
+      ++n;
+    }
+  }
+};
+
+// G16: group = 16 (two groups per lane); otherwise group >= 32 spans
+// group/32 lanes. A persistent grid: every warp walks warp-items (32
+// consecutive blocks of the [N, K/32] block grid) with a stride of the
+// grid's warp count and keeps the raw weights of its next two warp-items
+// in flight (one for fp32) while it quantizes the current one, so the
+// loads overlap the arithmetic (about 64 KB in flight per SM).
+template <typename TW, int BITS, bool G16, bool STAGED>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, 2)
     quantize_kernel(const TW* __restrict__ W, int64_t N, int64_t K,
                     int64_t ldw, const float* __restrict__ s, int group,
                     uint32_t* __restrict__ codes, float* __restrict__ delta,
                     uint8_t* __restrict__ zero) {
-  constexpr int QMAX = (1 << BITS) - 1;
-  // rint(x) for |x| < 2^22 is exactly (x + 1.5*2^23) - 1.5*2^23 under
-  // round-to-nearest-even (the sum lands in [2^23, 2^24), where the ulp is
-  // 1, and the offset is even); the integer is the sum's low bits. Here
-  // |w*r| and |mn*r| are at most 2^b - 1 + 1/2.
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr int kMagicBits = 0x4B400000;
-  using chunk_t = typename std::conditional<(8 * BITS <= 32), uint32_t,
-                                            uint64_t>::type;
+  extern __shared__ __align__(16) float s_sm[];
   griddep_enter();
-  const int lane = threadIdx.x & 31;
-  // work items are (row, 256-channel segment) pairs, < 2^31 (checked on
-  // the host); 32-bit index math keeps the per-item cost small
-  const uint32_t segs = (uint32_t)((K + 255) / 256);
-  const uint32_t items = (uint32_t)N * segs;
-  const uint32_t item0 =
-      (blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5)) * kSegsPerWarp;
-  if (item0 >= items) return;  // whole warp exits together
-  const int64_t ldc = codes_ld(K, BITS), ldg = groups_ld(K, group);
-  const int lanes_per_group = group >> 3;
-
-  // issue every segment's loads first
-  float w[kSegsPerWarp][8];
-  int64_t n_[kSegsPerWarp], col_[kSegsPerWarp];
-  bool act_[kSegsPerWarp];
-  const uint32_t row0 = item0 / segs, seg0 = item0 - row0 * segs;
-#pragma unroll
-  for (int u = 0; u < kSegsPerWarp; ++u) {
-    const uint32_t item = item0 + u;
-    const bool live = item < items;
-    uint32_t row = row0, seg = seg0 + u;
-    if (seg >= segs) {  // kSegsPerWarp <= segs is not required
-      row += seg / segs;
-      seg %= segs;
+  QuantCtx c;
+  c.s = s;
+  c.s_sm = s_sm;
+  c.K = K;
+  c.ldc = codes_ld(K, BITS);
+  c.ldg = groups_ld(K, group);
+  c.group = group;
+  c.lpg = G16 ? 1 : group >> 5;
+  c.codes = codes;
+  c.delta = delta;
+  c.zero = zero;
+  if constexpr (STAGED) {
+    const int64_t chunks = K / 4;
+    for (int64_t q = threadIdx.x; q < chunks; q += blockDim.x) {
+      const float4 v = s ? __ldg(reinterpret_cast<const float4*>(s) + q)
+                         : make_float4(1.f, 1.f, 1.f, 1.f);
+      *reinterpret_cast<float4*>(s_sm + (q >> 3) * kScalePitch + 4 * (q & 7)) =
+          v;
     }
-    n_[u] = live ? row : 0;
-    col_[u] = live ? (int64_t)seg * 256 + lane * 8 : K;
-    act_[u] = live && col_[u] < K;  // K % 32 == 0: blocks/groups agree
-    if (act_[u]) {
-      load8<TW>(W + n_[u] * ldw + col_[u], w[u]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) w[u][i] = 0.f;
+    __syncthreads();
+  }
+  const int lane = threadIdx.x & 31;
+  // warp-items are < 2^26 (the host checks N * K / 32 < 2^31)
+  const uint32_t bpr = (uint32_t)(K / 32);
+  const uint32_t total = (uint32_t)N * bpr;
+  const uint32_t n_items = (total + 31u) / 32u;
+  const uint32_t stride = gridDim.x * kWarpsPerCta;
+  uint32_t wi = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (wi >= n_items) return;  // whole warp exits together
+  // one stride of warp-items is 32 * stride blocks
+  const uint32_t dn = (32u * stride) / bpr, dk = (32u * stride) % bpr;
+
+  // locate this lane's first block (one division per warp)
+  BlockPos p0;
+  {
+    const uint32_t item0 = wi * 32u;
+    p0.n = item0 / bpr;
+    p0.k = item0 - p0.n * bpr + (uint32_t)lane;
+    while (p0.k >= bpr) {
+      p0.k -= bpr;
+      ++p0.n;
     }
   }
-
-#pragma unroll
-  for (int u = 0; u < kSegsPerWarp; ++u) {
-    const int64_t n = n_[u], col0 = col_[u];
-    const bool active = act_[u];
-    if (active && s != nullptr) {
-      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + col0));
-      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + col0 + 4));
-      w[u][0] = __fmul_rn(w[u][0], s0.x); w[u][1] = __fmul_rn(w[u][1], s0.y);
-      w[u][2] = __fmul_rn(w[u][2], s0.z); w[u][3] = __fmul_rn(w[u][3], s0.w);
-      w[u][4] = __fmul_rn(w[u][4], s1.x); w[u][5] = __fmul_rn(w[u][5], s1.y);
-      w[u][6] = __fmul_rn(w[u][6], s1.z); w[u][7] = __fmul_rn(w[u][7], s1.w);
-    }
-    // group range, widened to contain 0
-    float mn = 0.f, mx = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      mn = fminf(mn, w[u][i]);
-      mx = fmaxf(mx, w[u][i]);
-    }
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {  // g <= 128: at most 16 lanes
-      if (o < lanes_per_group) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  auto is_live = [&](uint32_t item) {
+    return item * 32u + (uint32_t)lane < total;
+  };
+  auto load = [&](const BlockPos& q, bool live, RawBlock<TW>& raw) {
+    if (live) load_raw<TW>(W + (int64_t)q.n * ldw + (int64_t)q.k * 32, raw);
+  };
+  float w[32];
+  if constexpr (sizeof(TW) == 2) {
+    // two slots used alternately; a slot is unpacked, then refilled with
+    // the warp-item two strides ahead before the arithmetic starts
+    RawBlock<TW> raw0, raw1;
+    BlockPos p1 = p0;
+    p1.advance(dn, dk, bpr);
+    bool l0 = is_live(wi), l1 = wi + stride < n_items && is_live(wi + stride);
+    load(p0, l0, raw0);
+    load(p1, l1, raw1);
+    for (;;) {
+      {
+        unpack_raw<TW>(raw0, w);
+        const BlockPos cp = p0;
+        const bool cl = l0;
+        p0 = p1;
+        p0.advance(dn, dk, bpr);
+        l0 = wi + 2 * stride < n_items && is_live(wi + 2 * stride);
+        load(p0, l0, raw0);
+        quantize_item<BITS, G16, STAGED>(c, w, cp.n, cp.k, cl);
       }
-    }
-    float d = __fdiv_rn(__fsub_rn(mx, mn), (float)QMAX);
-    if (d == 0.f) d = 1.f;
-    const float r = __frcp_rn(d);
-    // z = rint(-mn * r) lies in [0, 2^b - 1] because -mn <= mx - mn; the
-    // clamp below matches the definition and never changes a value
-    const int zi = min(max(__float_as_int(__fadd_rn(__fmul_rn(-mn, r), kMagic)) -
-                               kMagicBits,
-                           0),
-                       QMAX);
-    // q = rint(w*r) + z >= rint(mn*r) + z = 0 since rint is odd and the
-    // products are monotone in w; only the upper clamp can act
-    chunk_t chunk = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int qi = __float_as_int(__fadd_rn(__fmul_rn(w[u][i], r), kMagic)) -
-                     (kMagicBits - zi);
-      chunk |= (chunk_t)(uint32_t)min(qi, QMAX) << (BITS * i);
-    }
-    store_block<BITS>((uint64_t)chunk, lane,
-                      codes + n * ldc + (col0 / 32) * BITS, active);
-    if (active && (lane & (lanes_per_group - 1)) == 0) {
-      const int64_t gi = n * ldg + col0 / group;
-      delta[gi] = d;
-      zero[gi] = (uint8_t)zi;
-    }
-    // the warp holding the row's first segment zeroes the row's padding
-    if (col0 == lane * 8 && item0 + u < items) {
-      for (int64_t w2 = K * BITS / 32 + lane; w2 < ldc; w2 += 32)
-        codes[n * ldc + w2] = 0u;
-      for (int64_t gi = K / group + lane; gi < ldg; gi += 32) {
-        delta[n * ldg + gi] = 0.f;
-        zero[n * ldg + gi] = 0;
+      wi += stride;
+      if (wi >= n_items) break;
+      {
+        unpack_raw<TW>(raw1, w);
+        const BlockPos cp = p1;
+        const bool cl = l1;
+        p1 = p0;
+        p1.advance(dn, dk, bpr);
+        l1 = wi + 2 * stride < n_items && is_live(wi + 2 * stride);
+        load(p1, l1, raw1);
+        quantize_item<BITS, G16, STAGED>(c, w, cp.n, cp.k, cl);
       }
+      wi += stride;
+      if (wi >= n_items) break;
+    }
+  } else {
+    RawBlock<TW> raw0;
+    bool l0 = is_live(wi);
+    load(p0, l0, raw0);
+    for (; wi < n_items; wi += stride) {
+      unpack_raw<TW>(raw0, w);
+      const BlockPos cp = p0;
+      const bool cl = l0;
+      p0.advance(dn, dk, bpr);
+      l0 = wi + stride < n_items && is_live(wi + stride);
+      load(p0, l0, raw0);
+      quantize_item<BITS, G16, STAGED>(c, w, cp.n, cp.k, cl);
     }
   }
 }
@@ -193,16 +412,33 @@ template <typename TW>
 ttq_status launch_bits(const void* W, int64_t N, int64_t K, int64_t ldw,
                        const float* s, int bits, int group, uint32_t* codes,
                        float* delta, uint8_t* zero, cudaStream_t st) {
-  const int64_t items = N * ((K + 255) / 256);
-  const int64_t warps = (items + kSegsPerWarp - 1) / kSegsPerWarp;
+  const int64_t items = N * (K / 32);
+  const int64_t warps = (items + 31) / 32;
+  // persistent: as many CTAs as stay resident (2 per SM)
+  const int64_t resident = (int64_t)sm_count() * 2;
+  const int64_t ctas = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
   LaunchShape ls;
-  ls.grid = dim3((unsigned)((warps + kWarpsPerCta - 1) / kWarpsPerCta));
+  ls.grid = dim3((unsigned)std::min(ctas, resident));
   ls.block = dim3(kWarpsPerCta * 32);
+  // the scales go to shared memory when two CTAs per SM still fit
+  const size_t s_bytes = (size_t)(K / 32) * kScalePitch * 4;
+  const bool staged = (int64_t)s_bytes <= kMaxStagedScaleBytes;
+  ls.smem = staged ? s_bytes : 0;
   const TW* w = static_cast<const TW*>(W);
-#define TTQ_Q(B)                                                            \
-  case B:                                                                   \
-    return launch(ls, st, quantize_kernel<TW, B>, w, N, K, ldw, s, group,   \
-                  codes, delta, zero);
+  auto go = [&](auto kern) -> ttq_status {
+    if (ls.smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)ls.smem) != cudaSuccess)
+      return TTQ_ERR_CUDA;
+    return launch(ls, st, kern, w, N, K, ldw, s, group, codes, delta, zero);
+  };
+#define TTQ_Q(B)                                                          \
+  case B:                                                                 \
+    return group == 16                                                    \
+               ? (staged ? go(quantize_kernel<TW, B, true, true>)         \
+                         : go(quantize_kernel<TW, B, true, false>))       \
+               : (staged ? go(quantize_kernel<TW, B, false, true>)        \
+                         : go(quantize_kernel<TW, B, false, false>));
   switch (bits) {
     TTQ_Q(2) TTQ_Q(3) TTQ_Q(4) TTQ_Q(5) TTQ_Q(6) TTQ_Q(7) TTQ_Q(8)
   }

@@ -9,8 +9,9 @@
 //   - a thread owns 8 consecutive channels and loads them as one 16-byte
 //     vector (two for fp32); CW/8 threads cover a row segment of CW channels
 //     and the 256-thread CTA covers 256/(CW/8) rows per pass;
-//   - each CTA walks a contiguous range of rows with 8 independent loads in
-//     flight per thread, accumulating in fp32 registers;
+//   - each CTA walks a contiguous range of rows with 16 independent loads
+//     in flight per thread (8 for fp32), the last partial group predicated,
+//     accumulating in fp32 registers;
 //   - rows split across a thread-block cluster of up to 8 CTAs; partial sums
 //     are reduced through distributed shared memory by cluster rank 0 in a
 //     fixed order, so the result is deterministic and no global scratch is
@@ -131,11 +132,25 @@ __global__ void __launch_bounds__(kThreads)
         for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(x[i], p);
       }
     }
-    for (; r < r_end; r += rows_per_pass) {
-      float v[8];
-      load8<TX>(X + r * ldx + col0, v);
+    // fewer than U passes remain: one predicated block keeps them all in
+    // flight (a row past the end reads as zero and adds exactly 0)
+    if (r < r_end) {
+      uint4 raw[U][V];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(v[i], p);
+      for (int u = 0; u < U; ++u) {
+        const int64_t rr = r + (int64_t)u * rows_per_pass;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+          raw[u][v] = rr < r_end ? ld_stream_v4(X + rr * ldx + col0 + v * (8 / V))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float x[8];
+        unpack8<TX>(raw[u], x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += moment<PK>(x[i], p);
+      }
     }
   }
 
