@@ -45,7 +45,10 @@ constexpr int kSCols = kSK / 2;    // TMEM columns of one fp16 weight stage
 constexpr int kParamGroups = 16;   // groups per params chunk
 // CTA = producer warp + MMA warp + DQW dequantiser warps (4 or 8; with 8,
 // two warps share each TMEM lane quarter and split every stage in halves)
-__host__ __device__ constexpr int cta_threads(int dqw) { return 64 + 32 * dqw; }
+constexpr int kDqWarp0 = 2;  // first dequantiser warp
+__host__ __device__ constexpr int cta_threads(int dqw) {
+  return 32 * (kDqWarp0 + dqw);
+}
 constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
 constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
 constexpr int kMaxSmem = 225 * 1024;
@@ -410,8 +413,8 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
     // ------------------------------------------------ dequantisers ----
     // One thread per weight row (= TMEM lane): a stage is four 32-code
     // blocks, 64 fp16 pairs, written to the TMEM weight ring in two stores.
-    const int q4 = warp & 3;         // TMEM lane quarter of this warp
-    const int h = (warp - 2) >> 2;   // which half of a stage (DQW == 8)
+    const int q4 = warp & 3;                // TMEM lane quarter of this warp
+    const int h = (warp - kDqWarp0) >> 2;   // which half of a stage (DQW 8)
     const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
     const int n = m0 + i;
     const bool row_ok = n < p.N;
@@ -644,25 +647,42 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
   }
 
   if (split > 1) {
+    // Split-K: every rank's partial tile [bn][128] sits in its shared
+    // memory. All ranks reduce disjoint 4-row pieces of the tile: each
+    // thread issues the `split` 16-byte loads of a piece at once, then
+    // sums them in rank order, so the result does not depend on timing.
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
-    if (rank == 0 && warp >= 2) {
-      const int i = 32 * (warp & 3) + lane;
-      const int h = (warp - 2) >> 2;
-      const int n = m0 + i;
-      const int c_lo = DQW == 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
-      const int c_hi = DQW == 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
-                                : bn;
-      float* part = reinterpret_cast<float*>(gbase + L.part);
-      if (n < p.N && !*aborted) {
-        for (int c = c_lo; c < c_hi; ++c) {
-          const int t = t0 + c;
-          if (t >= p.T) break;
-          float acc = 0.f;
-          for (int q = 0; q < split; ++q)
-            acc += cluster.map_shared_rank(part, q)[c * kBM + i];
-          store_y(p.Y, p.yt, (long long)t * p.ldy + n, acc);
-        }
+    if (warp >= kDqWarp0 && !*aborted) {
+      constexpr int kDqThreads = 32 * DQW;
+      const int tid = rank * kDqThreads + (threadIdx.x - 32 * kDqWarp0);
+      const int nthr = split * kDqThreads;
+      const int pieces = bn * (kBM / 4);
+      const float* part = reinterpret_cast<const float*>(gbase + L.part);
+      for (int pc = tid; pc < pieces; pc += nthr) {
+        const int c = pc / (kBM / 4), i4 = (pc % (kBM / 4)) * 4;
+        const int t = t0 + c;
+        if (t >= p.T) continue;
+        float4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q < split)
+            v[q] = *reinterpret_cast<const float4*>(
+                cluster.map_shared_rank(part, q) + c * kBM + i4);
+        float4 acc = v[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q)
+          if (q < split) {
+            acc.x += v[q].x;
+            acc.y += v[q].y;
+            acc.z += v[q].z;
+            acc.w += v[q].w;
+          }
+        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (m0 + i4 + e < p.N)
+            store_y(p.Y, p.yt, (long long)t * p.ldy + m0 + i4 + e, a4[e]);
       }
     }
     cluster.sync();
