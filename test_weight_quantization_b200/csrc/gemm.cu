@@ -33,6 +33,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "kperm.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -238,7 +239,7 @@ struct Ring {
 //              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
 template <int BITS, int GMODE, int DQW>
-__global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
+__global__ void __launch_bounds__(cta_threads(DQW), 2)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_c,
@@ -693,20 +694,6 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW == 4 ? 2 : 1)
   if (warp == 1) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
 }
 
-// Position p of a 16-channel span of the prepared activations holds channel
-// k_perm<PERM>(p) of that span. For 2-, 4- and 8-bit codes the dequantiser
-// turns one shifted code word into an fp16 pair (q_c, q_c') whose channels
-// lie 8, 4 or 2 apart; the activations are stored in the same order so the
-// tensor-core products pair the right operands. Other widths keep the
-// natural order.
-template <int PERM>
-__host__ __device__ constexpr int k_perm(int p) {
-  return PERM == 2   ? (p >> 1) + 8 * (p & 1)
-         : PERM == 4 ? 8 * (p >> 3) + ((p & 7) >> 1) + 4 * (p & 1)
-         : PERM == 8 ? 4 * (p >> 2) + ((p & 3) >> 1) + 2 * (p & 1)
-                     : p;
-}
-
 // X~ = fp16(X * inv_s), one thread per 16 channels, K-permuted for PERM.
 template <typename TX, int PERM>
 __global__ void prescale_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
@@ -909,6 +896,10 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t N, int bits, int group, const void* B,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
                                 int64_t ldy, cudaStream_t st) {
+  // one or two tokens: the CUDA-core matrix-vector product (gemv.cu)
+  if (gemv_applies(T, K))
+    return launch_gemv(Xs, U, T, K, codes, delta, zero, N, bits, group, B, bt,
+                       r, Y, yt, ldy, st);
   // Tile shape. A stage is 128 channels: a codes chunk, two 64-channel
   // activation boxes, one 64-column fp16 weight stage in TMEM.
   // Decode (T <= 32): 256 TMEM columns per CTA (two CTAs per SM), K split
@@ -997,7 +988,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   // eight dequantisers); the split-K form reduces through the cluster
   // instead and never reads this map
   const int dqw = dual ? 4 : 8;
-  const int box_t = dqw == 8 ? bn / 2 : bn;
+  const int box_t = (dqw == 8 && bn >= 32) ? bn / 2 : bn;
   int y_mode = 0;
   if (split == 1 && ((uint64_t)ldy * dtype_bytes(yt)) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(Y) % 16 == 0)
@@ -1041,6 +1032,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
   // decode packs two CTAs per SM with four dequant warps each; prefill runs
   // one CTA per SM with eight
+
   if (dual) {
     if (group == 16)
       return dispatch_bits<0, 4>(bits, m, a, grid, split, smem, st);

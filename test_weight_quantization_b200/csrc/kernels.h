@@ -48,6 +48,15 @@ ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                           const void* A, int r, void* Xs, void* U,
                           cudaStream_t st);
 
+// The decode projection on CUDA cores (T <= 2), used by
+// launch_gemm_prepared when it applies.
+bool gemv_applies(int64_t T, int64_t K);
+ttq_status launch_gemv(const void* Xs, const void* U, int64_t T, int64_t K,
+                       const uint32_t* codes, const float* delta,
+                       const uint8_t* zero, int64_t N, int bits, int group,
+                       const void* B, ttq_dtype bt, int r, void* Y,
+                       ttq_dtype yt, int64_t ldy, cudaStream_t st);
+
 ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t K, const uint32_t* codes,
                                 const float* delta, const uint8_t* zero,

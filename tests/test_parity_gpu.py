@@ -263,6 +263,37 @@ def test_gemm_output_tile_store(ttq, N, pitch, out):
         assert torch.all(big[:, N:] == 7.0)
 
 
+@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("group", [16, 32, 128])
+def test_decode_gemv(ttq, T, bits, group):
+    """One or two tokens take the CUDA-core matrix-vector path; every code
+    width and group size against the oracle (K spans 10 row passes of a
+    warp's lanes and a ragged one)."""
+    N, K = 300, 1408
+    X = acts(T, K, 40 + T + bits, torch.bfloat16)
+    W = weights(N, K, 41 + bits, torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, bits, group)
+    ref = oracle_y(X, inv, c, d, z, N, bits, group)
+    assert_gemm_close(np32(Y), ref, f"gemv T={T} b={bits} g={group}", Y.dtype)
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("T", [1, 2])
+def test_decode_gemv_lowrank_and_dtypes(ttq, out, T):
+    N, K, r, bits, group = 200, 512, 16, 4, 64
+    X = acts(T, K, 50 + T, torch.bfloat16)
+    W = weights(N, K, 51, torch.bfloat16)
+    rng = np.random.default_rng(52)
+    A = torch.from_numpy(rng.standard_normal((r, K)).astype(np.float32) * .05
+                         ).to(torch.bfloat16)
+    B = torch.from_numpy(rng.standard_normal((N, r)).astype(np.float32) * .05
+                         ).to(torch.bfloat16)
+    Y, inv, c, d, z = run_path(ttq, X, W, bits, group, A, B, out_dtype=DT[out])
+    ref = oracle_y(X, inv, c, d, z, N, bits, group, A, B)
+    assert_gemm_close(np32(Y), ref, f"gemv lowrank T={T} {out}", Y.dtype)
+
+
 @pytest.mark.parametrize("bits", [6, 7, 8])
 def test_gemm_wide_codes(ttq, bits):
     X = acts(64, 256, 13, torch.bfloat16)
