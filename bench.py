@@ -436,8 +436,9 @@ def kernel_source_hash():
 
 
 def traffic_from_profiles(kind, workload):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, or
-    None when absent or taken on a different kernel source."""
+    """DRAM bytes per launch (read + write, averaged over one step's
+    launches) of a kernel from a committed ncu summary, or None when absent
+    or taken on a different kernel source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -446,7 +447,7 @@ def traffic_from_profiles(kind, workload):
     e = d.get(f"{kind}/{workload}")
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
-    return e.get("dram_bytes_per_step")
+    return e["dram_bytes_per_step"] / max(1, e.get("launches_per_step", 1))
 
 
 def main():
@@ -568,6 +569,11 @@ def main():
                 "peak_kind": f"{pk['source']} HBM copy"}
     roof["kernel"] = dom
     roof["traffic"] = traffic_from_profiles(dom, wl.name)
+    roof["traffic_unit"] = "DRAM bytes per launch (ncu, cold serialised)"
+    # algorithmic work of one launch, averaged over the step's launches
+    n_dom = kinds.count(dom)
+    roof["algorithmic_per_launch"] = (
+        work["gemm_flops"] if dom == "gemm" else work[dom]) / max(1, n_dom)
 
     # end to end through the binding: host buffers in, host buffers out
     e2e = None

@@ -41,8 +41,9 @@ __device__ double awq_channel_mean(const float* sum, int64_t K, double invT,
 
 // s_j and 1/s_j of one channel. c_j is formed in fp64; the power runs in
 // fp32 on c_j rounded to fp32 (relative error below 1e-6, far inside the
-// 1e-5 agreement with the fp64 definition), with fp64 pow outside the range
-// where fp32 keeps full precision.
+// 1e-5 agreement with the fp64 definition): square or fourth roots for the
+// exponents 1/2 and 1/4 (alpha = 0.5 with p = 1 or 2), powf otherwise, and
+// fp64 pow outside the range where fp32 keeps full precision.
 __device__ __forceinline__ void awq_scale_one(float sum_j, double invT,
                                               double mbar, double alpha,
                                               double lambda, double p,
@@ -52,8 +53,15 @@ __device__ __forceinline__ void awq_scale_one(float sum_j, double invT,
   float sj = 1.f, ij = 1.f;
   if (alpha != 0.0 && c > 0.0 && isfinite(c)) {
     const float cf = (float)c;
-    sj = (cf > 1e-30f && cf < 1e30f) ? powf(cf, (float)(alpha / p))
-                                     : (float)pow(c, alpha / p);
+    const double e = alpha / p;
+    if (!(cf > 1e-30f && cf < 1e30f))
+      sj = (float)pow(c, e);
+    else if (e == 0.5)  // square and fourth roots: within 2 ulp, cheaper
+      sj = sqrtf(cf);
+    else if (e == 0.25)
+      sj = sqrtf(sqrtf(cf));
+    else
+      sj = powf(cf, (float)e);
     ij = 1.f / sj;
   }
   s = sj;

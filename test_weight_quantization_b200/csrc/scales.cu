@@ -18,9 +18,20 @@ __global__ void __launch_bounds__(kThreads)
   griddep_enter();
   const double invT = 1.0 / (double)T_total;
   const double mbar = awq_channel_mean<kThreads>(sum, K, invT, warp_sums);
-  for (int64_t j = threadIdx.x; j < K; j += kThreads)
-    awq_scale_one(__ldcg(sum + j), invT, mbar, alpha, lambda, p, s[j],
-                  inv_s[j]);
+  // four independent channels per iteration to overlap their latencies
+  for (int64_t j0 = threadIdx.x; j0 < K; j0 += 4 * kThreads) {
+    float sj[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + u * kThreads;
+      sj[u] = j < K ? __ldcg(sum + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + u * kThreads;
+      if (j < K) awq_scale_one(sj[u], invT, mbar, alpha, lambda, p, s[j], inv_s[j]);
+    }
+  }
 }
 
 }  // namespace

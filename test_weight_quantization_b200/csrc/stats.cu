@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kThreads)
   // [rows_per_pass][cw] then part[cw]
   extern __shared__ __align__(16) float smem[];
   __shared__ int last_flag;
+  __shared__ double tile_part[kThreads / 32];
   griddep_enter();
   cg::cluster_group cluster = cg::this_cluster();
   const int tpr = cw / 8;                 // threads per row segment
@@ -168,13 +169,16 @@ __global__ void __launch_bounds__(kThreads)
   cluster.sync();
 
   // Cluster reduction by rank 0, ranks in order.
+  double tile = 0.0;  // this thread's column (cw <= kThreads)
   if (rank == 0) {
     for (int c = tid; c < cw; c += kThreads) {
       const int64_t col = (int64_t)blockIdx.x * cw + c;
       if (col >= K) continue;
       float s = 0.f;
       for (int q = 0; q < C; ++q) s += cluster.map_shared_rank(part, q)[c];
-      sum_out[col] = accumulate ? sum_out[col] + s : s;
+      s = accumulate ? sum_out[col] + s : s;
+      sum_out[col] = s;
+      tile += (double)s;
     }
   }
   if (tail.s == nullptr) {
@@ -182,10 +186,24 @@ __global__ void __launch_bounds__(kThreads)
     return;
   }
 
-  // Fused step 2. Rank 0 publishes its tile (fence, then one arrival per
-  // cluster); the arrival that completes the count marks its cluster last
-  // and tells every CTA of the cluster through its shared memory.
+  // Fused step 2. Rank 0 adds its tile's sums (fixed tree) and leaves the
+  // fp64 total in words 2b, 2b+1 of s (b = column tile; s is written only
+  // after every tile total was read), then publishes (fence, one arrival
+  // per cluster); the arrival that completes the count marks its cluster
+  // last and tells every CTA of the cluster through its shared memory.
   if (rank == 0) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+      tile += __shfl_xor_sync(0xffffffffu, tile, o);
+    if ((tid & 31) == 0) tile_part[tid >> 5] = tile;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < kThreads / 32; ++w) t += tile_part[w];
+      const unsigned long long bits = (unsigned long long)__double_as_longlong(t);
+      tail.s[2 * blockIdx.x] = __uint_as_float((uint32_t)bits);
+      tail.s[2 * blockIdx.x + 1] = __uint_as_float((uint32_t)(bits >> 32));
+    }
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -201,16 +219,40 @@ __global__ void __launch_bounds__(kThreads)
   cluster.sync();  // after this no CTA reads another's shared memory
   if (!last_flag) return;
   __threadfence();
-  // every CTA of the last cluster forms the same mean, then the scales of
-  // its share of the channels
-  double* warp_sums = reinterpret_cast<double*>(smem);
+  // every CTA of the last cluster adds the tile totals in tile order (the
+  // same value in every CTA and whichever cluster is last) ...
   const double invT = 1.0 / (double)tail.T_total;
-  const double mbar =
-      awq_channel_mean<kThreads>(sum_out, K, invT, warp_sums);
-  for (int64_t j = (int64_t)rank * kThreads + tid; j < K;
-       j += (int64_t)C * kThreads)
-    awq_scale_one(__ldcg(sum_out + j), invT, mbar, tail.alpha, tail.lambda,
-                  tail.p, tail.s[j], tail.inv_s[j]);
+  if (tid < 32) {
+    double t = 0.0;
+    for (int b = tid; b < (int)gridDim.x; b += 32) {
+      const uint32_t lo = __float_as_uint(__ldcg(tail.s + 2 * b));
+      const uint32_t hi = __float_as_uint(__ldcg(tail.s + 2 * b + 1));
+      t += __longlong_as_double(
+          (long long)(((unsigned long long)hi << 32) | lo));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (tid == 0) tile_part[0] = t;
+  }
+  cluster.sync();  // every tile total read before s is overwritten
+  const double mbar = tile_part[0] * invT / (double)K;
+  // ... then the scales of its share of the channels, four at a time
+  const int64_t stride = (int64_t)C * kThreads;
+  for (int64_t j0 = (int64_t)rank * kThreads + tid; j0 < K; j0 += 4 * stride) {
+    float sj[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + u * stride;
+      sj[u] = j < K ? __ldcg(sum_out + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = j0 + u * stride;
+      if (j < K)
+        awq_scale_one(sj[u], invT, mbar, tail.alpha, tail.lambda, tail.p,
+                      tail.s[j], tail.inv_s[j]);
+    }
+  }
 }
 
 template <typename TX, int PK>
