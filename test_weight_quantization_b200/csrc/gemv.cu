@@ -9,14 +9,17 @@
 //   - a warp owns one weight row at a time and its lanes take the row's
 //     32-code blocks (lane l: blocks l, l + 32, ...), the codes and group
 //     parameters of several blocks in flight per lane;
-//   - a code q of b bits becomes the exact float 1 + q / 2^b by placing it
-//     in the top mantissa bits of 1.0 (a shift and one logic operation),
-//     so each weight costs one FMA per token:
-//       sum_{j in blk} x_j (q_j - z) D
-//         = D 2^b sum_j x_j (1 + q_j / 2^b) - D (2^b + z) sum_j x_j;
+//   - a code q of b bits that sits at bit p < 24 - b of its word (or of the
+//     word shifted right by 9, or, straddling two words, funnel-shifted to
+//     bit 0) is read in place: OR-ing its field into the mantissa of 1.0
+//     gives 1 + q 2^(p-23), and subtracting 1 is exact. The activation of
+//     that channel is staged pre-multiplied by 2^(23-p), so one logic op,
+//     one FADD and one FMA per token make x_j q_j exactly (integer work is
+//     the scarce pipe here):
+//       sum_{j in blk} x_j (q_j - z) D = D sum_j x_j q_j - D z sum_j x_j;
 //   - the activations (fp16, as prepared for the tensor path) are staged
 //     once per CTA as fp32 in shared memory in natural channel order, with
-//     the sums of every 16-channel span;
+//     the sums of every 16-channel span (of the unscaled values);
 //   - the row's lanes reduce by shuffles in a fixed order (deterministic).
 #include <algorithm>
 
@@ -31,19 +34,36 @@ constexpr int kGvThreads = 1024;   // one CTA per SM
 constexpr int kBlkPitch = 36;      // floats per staged 32-channel block
 constexpr int kMaxGvTokens = 2;
 
-// Code i of a 32-code block (bit stream over BITS words) as 1 + q / 2^BITS.
+// Where code I of a 32-code block is read: kind 0 in place in its word,
+// kind 1 in the word shifted right by 9, kind 2 funnel-shifted to bit 0
+// (it straddles two words); pos is the field's bit in the source.
 template <int BITS, int I>
-__device__ __forceinline__ float code_float(const uint32_t (&cw)[BITS]) {
-  constexpr int bit = I * BITS, wd = bit >> 5, sh = bit & 31;
-  constexpr int top = 23 - BITS;  // q lands in mantissa bits [top, 23)
-  constexpr uint32_t mask = ((1u << BITS) - 1u) << top;
-  uint32_t v;
-  if constexpr (sh + BITS <= 32) {
-    v = sh <= top ? cw[wd] << (top - sh) : cw[wd] >> (sh - top);
-  } else {
-    v = __funnelshift_r(cw[wd], cw[wd + 1], sh) << top;
-  }
-  return __uint_as_float((v & mask) | 0x3F800000u);
+struct CodeAt {
+  static constexpr int bit = I * BITS, wd = bit >> 5, sh = bit & 31;
+  static constexpr int kind = sh + BITS <= 23 ? 0 : sh + BITS <= 32 ? 1 : 2;
+  static constexpr int pos = kind == 0 ? sh : kind == 1 ? sh - 9 : 0;
+};
+
+__host__ __device__ constexpr int code_pos(int bits, int i) {
+  return ((i * bits) & 31) + bits <= 23
+             ? ((i * bits) & 31)
+             : ((i * bits) & 31) + bits <= 32 ? ((i * bits) & 31) - 9 : 0;
+}
+
+// q * 2^(pos - 23) for code I (exact).
+template <int BITS, int I>
+__device__ __forceinline__ float code_val(const uint32_t (&cw)[BITS],
+                                          const uint32_t (&cw9)[BITS]) {
+  using C = CodeAt<BITS, I>;
+  constexpr uint32_t mask = ((1u << BITS) - 1u) << C::pos;
+  uint32_t src;
+  if constexpr (C::kind == 0)
+    src = cw[C::wd];
+  else if constexpr (C::kind == 1)
+    src = cw9[C::wd];
+  else
+    src = __funnelshift_r(cw[C::wd], cw[C::wd + 1], C::sh);
+  return __fsub_rn(__uint_as_float((src & mask) | 0x3F800000u), 1.f);
 }
 
 template <int BITS>
@@ -71,10 +91,11 @@ __device__ __forceinline__ void load_codes(const uint32_t* p,
   }
 }
 
-// sum over codes [LO, HI) of the block of x_j (1 + q_j / 2^BITS) for the
-// NT tokens whose staged blocks start at xb[t].
+// sum over codes [I, HI) of the block of x'_j q_j 2^(pos_j - 23) = x_j q_j
+// for the NT tokens whose staged (pre-scaled) blocks start at xb[t].
 template <int BITS, int NT, int I, int HI>
 __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
+                                          const uint32_t (&cw9)[BITS],
                                           const float* const (&xb)[NT],
                                           float (&acc)[NT]) {
   if constexpr (I < HI) {
@@ -82,10 +103,10 @@ __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
 #pragma unroll
     for (int t = 0; t < NT; ++t)
       xv[t] = *reinterpret_cast<const float4*>(xb[t] + I);
-    const float f0 = code_float<BITS, I>(cw);
-    const float f1 = code_float<BITS, I + 1>(cw);
-    const float f2 = code_float<BITS, I + 2>(cw);
-    const float f3 = code_float<BITS, I + 3>(cw);
+    const float f0 = code_val<BITS, I>(cw, cw9);
+    const float f1 = code_val<BITS, I + 1>(cw, cw9);
+    const float f2 = code_val<BITS, I + 2>(cw, cw9);
+    const float f3 = code_val<BITS, I + 3>(cw, cw9);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       acc[t] = fmaf(f0, xv[t].x, acc[t]);
@@ -93,7 +114,7 @@ __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
       acc[t] = fmaf(f2, xv[t].z, acc[t]);
       acc[t] = fmaf(f3, xv[t].w, acc[t]);
     }
-    dot_range<BITS, NT, I + 4, HI>(cw, xb, acc);
+    dot_range<BITS, NT, I + 4, HI>(cw, cw9, xb, acc);
   }
 }
 
@@ -113,7 +134,6 @@ __global__ void __launch_bounds__(kGvThreads, 1)
                 int64_t ldy) {
   // blocks in flight per lane (about 16 code words)
   constexpr int U_BLK = BITS <= 2 ? 8 : BITS <= 4 ? 4 : 2;
-  constexpr float kScale = (float)(1 << BITS);
   extern __shared__ __align__(16) float xs_sm[];  // [NT][K/32][kBlkPitch]
   const int bpr = (int)(K / 32);
   float* span_sum = xs_sm + (size_t)NT * bpr * kBlkPitch;  // [NT][K/16]
@@ -130,18 +150,19 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     float v[16];
 #pragma unroll
     for (int e = 0; e < 8; ++e) f16x2_to_f32(w[e], v[2 * e], v[2 * e + 1]);
+    // the span's sum (natural values, any order: a sum of 16 inputs)
+    float sum = 0.f;
+#pragma unroll
+    for (int pp = 0; pp < 16; ++pp) sum += v[pp];
+    span_sum[t * 2 * bpr + span] = sum;
     float* dst = xs_sm + ((size_t)t * bpr + (span >> 1)) * kBlkPitch +
                  (span & 1) * 16;
 #pragma unroll
-    for (int pp = 0; pp < 16; ++pp) dst[k_perm<PERM>(pp)] = v[pp];
-  }
-  __syncthreads();
-  for (int q = threadIdx.x; q < NT * 2 * bpr; q += kGvThreads) {
-    const float* b = xs_sm + (size_t)(q >> 1) * kBlkPitch + (q & 1) * 16;
-    float s = 0.f;
-#pragma unroll
-    for (int c = 0; c < 16; ++c) s += b[c];
-    span_sum[q] = s;
+    for (int pp = 0; pp < 16; ++pp) {
+      const int ch = k_perm<PERM>(pp);              // channel in the span
+      const int i = (int)(span & 1) * 16 + ch;      // code index in the block
+      dst[ch] = ldexpf(v[pp], 23 - code_pos(BITS, i));
+    }
   }
   __syncthreads();
 
@@ -149,6 +170,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   const int64_t ldc = codes_ld(K, BITS), ldg = groups_ld(K, group);
   const int warps = gridDim.x * (kGvThreads / 32);
   const int cpr = (bpr + 32 * U_BLK - 1) / (32 * U_BLK);  // chunks per row
+  const int blk_shift = 31 - __clz(group) - 5;  // block -> group: >> (lg g - 5)
 
   struct Item {
     uint32_t cw[U_BLK][BITS];
@@ -170,7 +192,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           it.d1[u] = d2.y;
           it.zz[u] = __ldg(reinterpret_cast<const uint16_t*>(zrow) + bk);
         } else {
-          const int gi = (bk * 32) / group;
+          const int gi = bk >> blk_shift;  // g >= 32: whole blocks per group
           it.d0[u] = __ldg(drow + gi);
           it.d1[u] = 0.f;
           it.zz[u] = __ldg(zrow + gi);
@@ -187,38 +209,37 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int u = 0; u < U_BLK; ++u) {
       const int bk = ch * 32 * U_BLK + lane + 32 * u;
       if (bk < bpr) {
+        uint32_t cw9[BITS];
+#pragma unroll
+        for (int w = 0; w < BITS; ++w) cw9[w] = it.cw[u][w] >> 9;
         const float* xb[NT];
 #pragma unroll
-        for (int t = 0; t < NT; ++t)
-          xb[t] = xs_sm + ((size_t)t * bpr + bk) * kBlkPitch;
+        for (int t = 0; t < NT; ++t) xb[t] = xs_sm + (t * bpr + bk) * kBlkPitch;
         const float* ss = span_sum + 2 * bk;
         if constexpr (G16) {
           // two groups of 16 in the block
           float a0[NT], a1[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) a0[t] = a1[t] = 0.f;
-          dot_range<BITS, NT, 0, 16>(it.cw[u], xb, a0);
-          dot_range<BITS, NT, 16, 32>(it.cw[u], xb, a1);
+          dot_range<BITS, NT, 0, 16>(it.cw[u], cw9, xb, a0);
+          dot_range<BITS, NT, 16, 32>(it.cw[u], cw9, xb, a1);
           const float z0 = (float)(it.zz[u] & 0xFFu);
           const float z1 = (float)(it.zz[u] >> 8);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            y[t] = fmaf(it.d0[u] * kScale, a0[t], y[t]);
-            y[t] = fmaf(-it.d0[u] * (kScale + z0), ss[t * 2 * bpr], y[t]);
-            y[t] = fmaf(it.d1[u] * kScale, a1[t], y[t]);
-            y[t] = fmaf(-it.d1[u] * (kScale + z1), ss[t * 2 * bpr + 1], y[t]);
+            y[t] = fmaf(it.d0[u], fmaf(-z0, ss[t * 2 * bpr], a0[t]), y[t]);
+            y[t] = fmaf(it.d1[u], fmaf(-z1, ss[t * 2 * bpr + 1], a1[t]), y[t]);
           }
         } else {
           float a[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) a[t] = 0.f;
-          dot_range<BITS, NT, 0, 32>(it.cw[u], xb, a);
+          dot_range<BITS, NT, 0, 32>(it.cw[u], cw9, xb, a);
           const float z = (float)it.zz[u];
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
             const float sb = ss[t * 2 * bpr] + ss[t * 2 * bpr + 1];
-            y[t] = fmaf(it.d0[u] * kScale, a[t], y[t]);
-            y[t] = fmaf(-it.d0[u] * (kScale + z), sb, y[t]);
+            y[t] = fmaf(it.d0[u], fmaf(-z, sb, a[t]), y[t]);
           }
         }
       }

@@ -133,7 +133,7 @@ struct QuantCtx {
   const float* s;     // global scales (null: s = 1)
   const float* s_sm;  // staged scales, or null
   int64_t K, ldc, ldg;
-  int group, lpg;
+  int group, lpg, lg;  // lg = log2(group)
   uint32_t* codes;
   float* delta;
   uint8_t* zero;
@@ -264,7 +264,7 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
     *reinterpret_cast<float2*>(c.delta + gi) = make_float2(d[0], d[NG - 1]);
     *reinterpret_cast<uint16_t*>(c.zero + gi) = (uint16_t)(z0 | (z1 << 8));
   } else if ((k & (uint32_t)(c.lpg - 1)) == 0) {
-    const int64_t gi = (int64_t)n * c.ldg + col0 / c.group;
+    const int64_t gi = (int64_t)n * c.ldg + (col0 >> c.lg);
     c.delta[gi] = d[0];
     c.zero[gi] = (uint8_t)z0;
   }
@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2)
   c.ldg = groups_ld(K, group);
   c.group = group;
   c.lpg = G16 ? 1 : group >> 5;
+  c.lg = 31 - __clz(group);
   c.codes = codes;
   c.delta = delta;
   c.zero = zero;
