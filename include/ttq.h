@@ -187,7 +187,11 @@ size_t ttq_w_lowbit_gemm_workspace_size(int64_t T, int64_t K, int r);
  * The tensor cores take fp16 operands: X / s is rounded once to fp16 and
  * each weight (q - z) * D once to fp16; products accumulate in fp32.
  * |X / s| must stay below 65504 (else TTQ_DEVERR_FP16_RANGE is raised).
- * T <= 16 runs the decode (skinny) configuration, larger T the prefill one.
+ * Which kernel runs depends on T: T <= 2 a CUDA-core matrix-vector product
+ * (the weight (q - z) D is applied in fp32, the activations are the fp16
+ * X / s), T <= 32 the tensor-core decode configuration (K split across a
+ * cluster), larger T the prefill one. The results agree to the tolerances
+ * of the parity tests, not bit for bit across these regimes.
  * Requires K % 32 == 0, K % group == 0, 0 <= r <= 64. */
 ttq_status ttq_w_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
                              int64_t K, int64_t ldx, const float* inv_s,
@@ -218,8 +222,8 @@ ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt, int64_t T,
                                    int bits, const void* A, int r, void* Xs,
                                    void* U, void* stream);
 
-/* ttq_w_lowbit_gemm_prepared: the tensor-core projection on prepared
- * operands, one kernel launch:
+/* ttq_w_lowbit_gemm_prepared: the projection on prepared operands, one
+ * kernel launch (T <= 2: CUDA cores, otherwise tensor cores, as above):
  *   Y[t][n] = sum_j Xs[t][j] (q[n][j] - z) D + sum_rho U[t][rho] B[n][rho].
  * Xs, U as written by ttq_prepare_activations for the same bits; B [N, r]
  * of dtype bt. */

@@ -276,7 +276,8 @@ def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
                            B: torch.Tensor | None = None,
                            out: torch.Tensor | None = None,
                            out_dtype=torch.bfloat16) -> torch.Tensor:
-    """Tensor-core projection on prepared operands (one kernel launch)."""
+    """The projection on prepared operands (one kernel launch; one or two
+    tokens run on CUDA cores, more on tensor cores)."""
     _dev(Xs, "Xs")
     T, K = Xs.shape
     r = 0 if B is None else B.shape[1]
