@@ -295,6 +295,12 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
     mbar_init(b_accum, 1);
     *aborted = 0;
     fence_barrier_init();
+    // the tensor maps are kernel parameters: no need to wait for them
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(&tm_d);
+    tma_prefetch_desc(&tm_z);
+    if (p.r > 0) tma_prefetch_desc(&tm_u);
   }
   // The set-up above and the TMEM allocation touch no global memory, so
   // they overlap the previous kernel on the stream. (An allocation can
@@ -315,11 +321,6 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer ----
     if (lane == 0) {
-      tma_prefetch_desc(&tm_x);
-      tma_prefetch_desc(&tm_c);
-      tma_prefetch_desc(&tm_d);
-      tma_prefetch_desc(&tm_z);
-      if (p.r > 0) tma_prefetch_desc(&tm_u);
       const uint32_t xbytes = (uint32_t)bn * 128u;
       Ring rs, rp;
       int pchunk = -1, issued = 0, np = 0;

@@ -188,9 +188,10 @@ __global__ void __launch_bounds__(kThreads)
 
   // Fused step 2. Rank 0 adds its tile's sums (fixed tree) and leaves the
   // fp64 total in words 2b, 2b+1 of s (b = column tile; s is written only
-  // after every tile total was read), then publishes (fence, one arrival
-  // per cluster); the arrival that completes the count marks its cluster
-  // last and tells every CTA of the cluster through its shared memory.
+  // after every tile total was read), then publishes with one
+  // acquire-release arrival per cluster; the arrival that completes the
+  // count marks its cluster last and tells every CTA of the cluster through
+  // its shared memory.
   if (rank == 0) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
@@ -203,22 +204,21 @@ __global__ void __launch_bounds__(kThreads)
       const unsigned long long bits = (unsigned long long)__double_as_longlong(t);
       tail.s[2 * blockIdx.x] = __uint_as_float((uint32_t)bits);
       tail.s[2 * blockIdx.x + 1] = __uint_as_float((uint32_t)(bits >> 32));
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const unsigned prev = atomicAdd(tail.counter, 1u);
+      // acquire-release at GPU scope: the CTA's writes (ordered before this
+      // thread by the barrier above) are released with the arrival, and the
+      // last arrival acquires every other cluster's
+      unsigned prev;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                   : "=r"(prev)
+                   : "l"(tail.counter)
+                   : "memory");
       const int last = prev == gridDim.x - 1;
-      if (last) {
-        __threadfence();
-        *tail.counter = 0u;  // every arrival of this launch is in
-      }
+      if (last) *tail.counter = 0u;  // every arrival of this launch is in
       for (int q = 0; q < C; ++q) *cluster.map_shared_rank(&last_flag, q) = last;
     }
   }
   cluster.sync();  // after this no CTA reads another's shared memory
   if (!last_flag) return;
-  __threadfence();
   // every CTA of the last cluster adds the tile totals in tile order (the
   // same value in every CTA and whichever cluster is last) ...
   const double invT = 1.0 / (double)tail.T_total;
