@@ -426,10 +426,20 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
-def kernel_source_hash():
+# The sources a kernel's counters depend on (its file and the headers it
+# includes from the package).
+KERNEL_SOURCES = {
+    "gemm": ("gemm.cu", "common.cuh", "kperm.cuh"),
+    "stats_scales": ("stats.cu", "awq_scale.cuh", "common.cuh"),
+    "quantize": ("quantize.cu", "common.cuh"),
+    "prepare": ("gemm.cu", "common.cuh", "kperm.cuh"),
+}
+
+
+def kernel_source_hash(kind="gemm"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "test_weight_quantization_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kind]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:12]
@@ -445,7 +455,8 @@ def traffic_from_profiles(kind, workload):
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{kind}/{workload}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if (not e or kind not in KERNEL_SOURCES or
+            e.get("source_hash") != kernel_source_hash(kind)):
         return None
     return e["dram_bytes_per_step"] / max(1, e.get("launches_per_step", 1))
 

@@ -140,7 +140,10 @@ ttq_status ttq_awq_scales(const float* sum, int64_t T_total, int64_t K,
  *   s, inv_s [K] float32 outputs as for ttq_awq_scales.
  *   counter  one uint32 of device memory that is zero before the first call;
  *            every call leaves it zero again. Calls that may run at the same
- *            time (different streams) need different counters.
+ *            time (different streams) need different counters. After a
+ *            call that failed on the device, zero it again.
+ * sum_out, s, inv_s and counter must not overlap (s holds partial results
+ * during the launch); overlapping arguments return TTQ_ERR_INVALID_ARG.
  * sum_out is bit-identical to ttq_act_stats; s and inv_s agree with
  * ttq_awq_scales to the last few bits of the fp64 mean (the mean is summed
  * in a different fixed order). */

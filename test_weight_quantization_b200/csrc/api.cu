@@ -46,6 +46,13 @@ bool rows_aligned(const void* p, ttq_dtype t, int64_t ld) {
 
 bool valid_group(int g) { return g == 16 || g == 32 || g == 64 || g == 128; }
 
+// Whether byte ranges [a, a + na) and [b, b + nb) overlap.
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a);
+  const uintptr_t y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 }  // namespace
@@ -157,6 +164,13 @@ TTQ_EXPORT ttq_status ttq_act_stats_scales(
       T_total < T || !(prm->alpha >= 0.f) || !isfinite(prm->alpha) ||
       !(prm->lambda >= 0.f && prm->lambda <= 1.f) || !(prm->p > 0.f) ||
       !isfinite(prm->p))
+    return TTQ_ERR_INVALID_ARG;
+  // the launch keeps partial results in s until the scales are written:
+  // the sums, the two scale arrays and the counter must not overlap
+  const size_t kb = (size_t)K * sizeof(float);
+  if (overlaps(sum_out, kb, s, kb) || overlaps(sum_out, kb, inv_s, kb) ||
+      overlaps(s, kb, inv_s, kb) || overlaps(counter, 4, sum_out, kb) ||
+      overlaps(counter, 4, s, kb) || overlaps(counter, 4, inv_s, kb))
     return TTQ_ERR_INVALID_ARG;
   return launch_act_stats_scales(X, xt, T, K, ldx, accumulate, T_total,
                                  prm->alpha, prm->lambda, prm->p, sum_out, s,

@@ -77,6 +77,17 @@ def test_bad_arguments_are_rejected_before_launch(lib):
     assert f(fake, 1, 8, 64, 64, 0, 7, pp, fake, fake, fake, fake, None) == 1
     assert f(fake, 1, 8, 64, 64, 2, 8, pp, fake, fake, fake, fake, None) == 1
     assert f(fake, 1, 8, 64, 64, 0, 8, None, fake, fake, fake, fake, None) == 1
+    # overlapping outputs are refused (s holds partials during the launch)
+    base = 0x200000
+    same = ctypes.c_void_p(base)
+    assert f(fake, 1, 8, 64, 64, 0, 8, pp, same, same, ctypes.c_void_p(base + 4096),
+             ctypes.c_void_p(base + 8192), None) == 1
+    assert f(fake, 1, 8, 64, 64, 0, 8, pp, ctypes.c_void_p(base),
+             ctypes.c_void_p(base + 128), ctypes.c_void_p(base + 4096),
+             ctypes.c_void_p(base + 8192), None) == 1  # s starts inside sums
+    assert f(fake, 1, 8, 64, 64, 0, 8, pp, ctypes.c_void_p(base),
+             ctypes.c_void_p(base + 4096), ctypes.c_void_p(base + 8192),
+             ctypes.c_void_p(base + 4096 + 16), None) == 1  # counter in s
     bad = Prm(0, 0, 0.5, 1.5, 2.0)
     assert f(fake, 1, 8, 64, 64, 0, 8, ctypes.addressof(bad), fake, fake, fake,
              fake, None) == 1
