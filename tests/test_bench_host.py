@@ -111,3 +111,20 @@ def test_reference_arm_reports_the_oracle():
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "opt125m-block"
+
+
+def test_measure_table_shapes_meet_the_call_constraints():
+    """Every shape the measurement CLI times is a valid call of the ABI
+    (K a multiple of 32 and of g, b in 2..8, g in {16, 32, 64, 128})."""
+    from test_weight_quantization_b200 import measure
+    for kind, args in measure.TABLE:
+        assert kind in measure.FNS
+        if kind == "quantize":
+            N, K, b, g = args
+        elif kind == "gemm":
+            T, N, K, b, g = args
+            assert T >= 1
+        else:
+            continue
+        assert K % 32 == 0 and K % g == 0 and 2 <= b <= 8
+        assert g in (16, 32, 64, 128)
