@@ -140,3 +140,34 @@ def test_packed_pitches(lib):
     assert lib.ttq_groups_ld(4096, 128) == 32
     assert lib.ttq_groups_ld(48, 16) == 16
     assert lib.ttq_codes_ld(100, 3) == 0 and lib.ttq_groups_ld(96, 24) == 0
+
+
+def test_empty_inputs_are_refused_before_launch(lib):
+    """T = 0, N = 0 or K = 0 is an invalid argument for every call (the
+    header requires T, N >= 1 and K a positive multiple of 32 or 8); nothing
+    is launched, so fake pointers are never touched."""
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fake = ctypes.c_void_p(0x100000)
+    st = lib.ttq_act_stats
+    st.argtypes = [P, I, I64, I64, I64, F, I, P, P]
+    assert st(fake, 1, 0, 64, 64, 2.0, 0, fake, None) == 1
+    assert st(fake, 1, 8, 0, 64, 2.0, 0, fake, None) == 1
+    q = lib.ttq_quantize_rtn_grouped
+    q.argtypes = [P, I, I64, I64, I64, P, I, I, P, P, P, P]
+    assert q(fake, 1, 0, 64, 64, None, 4, 32, fake, fake, fake, None) == 1
+    assert q(fake, 1, 4, 0, 64, None, 4, 32, fake, fake, fake, None) == 1
+    pr = lib.ttq_prepare_activations
+    pr.argtypes = [P, I, I64, I64, I64, P, I, P, I, P, P, P]
+    assert pr(fake, 1, 0, 64, 64, fake, 4, None, 0, fake, None, None) == 1
+    gp = lib.ttq_w_lowbit_gemm_prepared
+    gp.argtypes = [P, P, I64, I64, P, P, P, I64, I, I, P, I, I, P, I, I64, P]
+    assert gp(fake, None, 0, 64, fake, fake, fake, 32, 4, 32, None, 1, 0,
+              fake, 1, 32, None) == 1
+    assert gp(fake, None, 4, 64, fake, fake, fake, 0, 4, 32, None, 1, 0,
+              fake, 1, 32, None) == 1
+    lr = lib.ttq_lowrank_add
+    lr.argtypes = [P, I, I64, I64, I64, P, P, I, I64, P, I, I64, P]
+    assert lr(fake, 1, 0, 64, 64, fake, fake, 16, 32, fake, 1, 32, None) == 1
+    un = lib.ttq_unpack_codes
+    un.argtypes = [P, I64, I64, I, P, P]
+    assert un(fake, 0, 64, 4, fake, None) == 1
