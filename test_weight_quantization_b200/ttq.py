@@ -318,11 +318,14 @@ def unpack_codes(codes: torch.Tensor, K: int, bits: int) -> torch.Tensor:
 
 
 class TTQLinear:
-    """One linear layer run the TTQ way: per prompt, statistics -> scales ->
-    quantize -> low-bit projection (+ optional static low-rank term).
+    """One linear layer run the TTQ way: per prompt, statistics and scales
+    (one launch) -> quantize -> low-bit projection (+ optional static
+    low-rank term).
 
     ``W`` is the stored weight ([N, K], or the residual W - B A when ``A`` and
-    ``B`` are given). Buffers are allocated once per (T) and reused.
+    ``B`` are given). Buffers are allocated once per (T) and reused; the
+    layer's arrival counter makes concurrent use of one layer object on
+    several streams unsafe (use one object per stream).
     """
 
     def __init__(self, W: torch.Tensor, params: TTQParams, A=None, B=None):
@@ -332,6 +335,7 @@ class TTQLinear:
         self.sums = torch.empty(K, dtype=torch.float32, device=dev)
         self.s = torch.empty(K, dtype=torch.float32, device=dev)
         self.inv_s = torch.empty(K, dtype=torch.float32, device=dev)
+        self.counter = new_counter(dev)
         self.codes = torch.empty((N, codes_ld(K, params.bits)),
                                  dtype=torch.int32, device=dev)
         gl = groups_ld(K, params.group)
@@ -342,9 +346,8 @@ class TTQLinear:
     def calibrate(self, X: torch.Tensor) -> None:
         """Online statistics and quantization from this prompt's input."""
         p = self.prm
-        act_stats(X, p.p, out=self.sums)
-        awq_scales(self.sums, X.shape[0], p.alpha, p.lam, p.p, self.s,
-                   self.inv_s)
+        act_stats_scales(X, self.counter, p.alpha, p.lam, p.p, self.sums,
+                         self.s, self.inv_s)
         quantize_rtn_grouped(self.W, self.s, p.bits, p.group, self.codes,
                              self.delta, self.zero)
 

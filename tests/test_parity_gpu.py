@@ -392,5 +392,12 @@ def test_layer_object_matches_calls(ttq):
     W = weights(96, 256, 30, torch.bfloat16).cuda()
     layer = ttq.TTQLinear(W, ttq.TTQParams(bits=3, group=32))
     y = layer(X)
-    Y, *_ = run_path(ttq, X.cpu(), W.cpu(), 3, 32)
+    # the same calls by hand: fused statistics + scales, quantize, project
+    _, s, inv = ttq.act_stats_scales(X, ttq.new_counter())
+    c, d, z = ttq.quantize_rtn_grouped(W, s, 3, 32)
+    Y = ttq.w_lowbit_gemm(X, inv, c, d, z, W.shape[0], 3, 32)
     assert torch.equal(y, Y)
+    assert torch.equal(y, layer(X))  # the layer's counter is reusable
+    # and the result agrees with the oracle
+    ref = oracle_y(X.cpu(), inv, c, d, z, W.shape[0], 3, 32)
+    assert_gemm_close(np32(y), ref, "layer object", y.dtype)
