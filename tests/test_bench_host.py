@@ -128,3 +128,27 @@ def test_measure_table_shapes_meet_the_call_constraints():
             continue
         assert K % 32 == 0 and K % g == 0 and 2 <= b <= 8
         assert g in (16, 32, 64, 128)
+
+
+def test_algorithmic_work_closed_forms():
+    """The roofline numerator: flops 2 T N K per layer (plus the low-rank
+    slab), bytes read and written once, each distinct input counted once."""
+    import bench
+    from test_weight_quantization_b200.inputs import WORKLOADS
+    wl = WORKLOADS["opt125m-block"]
+    w = bench.algorithmic_work(wl)
+    T = 2048
+    nk = 4 * 768 * 768 + 3072 * 768 + 768 * 3072
+    assert w["gemm_flops"] == 2 * T * nk
+    # q, k, v share one input: four distinct inputs of K = 768, 768, 768, 3072
+    kin = 768 + 768 + 768 + 3072
+    assert w["stats"] == T * kin * 2 + kin * 4
+    assert w["prepare"] == T * kin * 4 + kin * 4
+    assert w["stats_scales"] == w["stats"] + w["scales"]
+    # quantize: bf16 W in, b/8 bytes of codes and 5/g bytes of params out
+    assert w["quantize"] == sum(L.N * L.K * 2 + L.K * 4 + L.N * L.K * 3 // 8 +
+                                5 * L.N * L.K // 32 for L in wl.layers)
+    gem = WORKLOADS["gemma1b-mlp"]
+    wg = bench.algorithmic_work(gem)
+    assert wg["gemm_flops"] == sum(2 * 1024 * L.N * L.K + 2 * 1024 * 16 *
+                                   (L.K + L.N) for L in gem.layers)
