@@ -319,6 +319,48 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2)
   c.codes = codes;
   c.delta = delta;
   c.zero = zero;
+  const int lane = threadIdx.x & 31;
+  // warp-items are < 2^26 (the host checks N * K / 32 < 2^31)
+  const uint32_t bpr = (uint32_t)(K / 32);
+  const uint32_t total = (uint32_t)N * bpr;
+  const uint32_t n_items = (total + 31u) / 32u;
+  const uint32_t stride = gridDim.x * kWarpsPerCta;
+  uint32_t wi = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const bool has_work = wi < n_items;
+  // one stride of warp-items is 32 * stride blocks
+  const uint32_t dn = (32u * stride) / bpr, dk = (32u * stride) % bpr;
+  auto is_live = [&](uint32_t item) {
+    return item * 32u + (uint32_t)lane < total;
+  };
+  auto load = [&](const BlockPos& q, bool live, RawBlock<TW>& raw) {
+    if (live) load_raw<TW>(W + (int64_t)q.n * ldw + (int64_t)q.k * 32, raw);
+  };
+
+  // locate this lane's first block (one division per warp) and start the
+  // first loads before the scales are staged: they do not depend on them.
+  // Slot 0 holds the warp-item in hand, slot 1 the next one (16-bit
+  // weights only; fp32 rows are twice the bytes and keep one slot).
+  constexpr bool kTwoSlots = sizeof(TW) == 2;
+  BlockPos p0 = {0u, 0u}, p1 = {0u, 0u};
+  bool l0 = false, l1 = false;
+  RawBlock<TW> raw0, raw1;
+  if (has_work) {
+    const uint32_t item0 = wi * 32u;
+    p0.n = item0 / bpr;
+    p0.k = item0 - p0.n * bpr + (uint32_t)lane;
+    while (p0.k >= bpr) {
+      p0.k -= bpr;
+      ++p0.n;
+    }
+    l0 = is_live(wi);
+    load(p0, l0, raw0);
+    if constexpr (kTwoSlots) {
+      p1 = p0;
+      p1.advance(dn, dk, bpr);
+      l1 = wi + stride < n_items && is_live(wi + stride);
+      load(p1, l1, raw1);
+    }
+  }
   if constexpr (STAGED) {
     const int64_t chunks = K / 4;
     for (int64_t q = threadIdx.x; q < chunks; q += blockDim.x) {
@@ -329,44 +371,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2)
     }
     __syncthreads();
   }
-  const int lane = threadIdx.x & 31;
-  // warp-items are < 2^26 (the host checks N * K / 32 < 2^31)
-  const uint32_t bpr = (uint32_t)(K / 32);
-  const uint32_t total = (uint32_t)N * bpr;
-  const uint32_t n_items = (total + 31u) / 32u;
-  const uint32_t stride = gridDim.x * kWarpsPerCta;
-  uint32_t wi = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  if (wi >= n_items) return;  // whole warp exits together
-  // one stride of warp-items is 32 * stride blocks
-  const uint32_t dn = (32u * stride) / bpr, dk = (32u * stride) % bpr;
+  if (!has_work) return;  // whole warp
 
-  // locate this lane's first block (one division per warp)
-  BlockPos p0;
-  {
-    const uint32_t item0 = wi * 32u;
-    p0.n = item0 / bpr;
-    p0.k = item0 - p0.n * bpr + (uint32_t)lane;
-    while (p0.k >= bpr) {
-      p0.k -= bpr;
-      ++p0.n;
-    }
-  }
-  auto is_live = [&](uint32_t item) {
-    return item * 32u + (uint32_t)lane < total;
-  };
-  auto load = [&](const BlockPos& q, bool live, RawBlock<TW>& raw) {
-    if (live) load_raw<TW>(W + (int64_t)q.n * ldw + (int64_t)q.k * 32, raw);
-  };
   float w[32];
-  if constexpr (sizeof(TW) == 2) {
-    // two slots used alternately; a slot is unpacked, then refilled with
-    // the warp-item two strides ahead before the arithmetic starts
-    RawBlock<TW> raw0, raw1;
-    BlockPos p1 = p0;
-    p1.advance(dn, dk, bpr);
-    bool l0 = is_live(wi), l1 = wi + stride < n_items && is_live(wi + stride);
-    load(p0, l0, raw0);
-    load(p1, l1, raw1);
+  if constexpr (kTwoSlots) {
+    // the two slots used alternately; a slot is unpacked, then refilled
+    // with the warp-item two strides ahead before the arithmetic starts
     for (;;) {
       {
         unpack_raw<TW>(raw0, w);
@@ -394,9 +404,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, 2)
       if (wi >= n_items) break;
     }
   } else {
-    RawBlock<TW> raw0;
-    bool l0 = is_live(wi);
-    load(p0, l0, raw0);
     for (; wi < n_items; wi += stride) {
       unpack_raw<TW>(raw0, w);
       const BlockPos cp = p0;
