@@ -436,12 +436,20 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without comments and whitespace (what compiles)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return re.sub(r"\s+", "", text)
+
+
 def kernel_source_hash(kind="gemm"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "test_weight_quantization_b200", "csrc")
     for name in KERNEL_SOURCES[kind]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:12]
 
 

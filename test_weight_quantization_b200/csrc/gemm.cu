@@ -7,25 +7,30 @@
 //
 // Orientation: the weight rows are the MMA's M dimension (128 TMEM lanes)
 // and the tokens its N dimension (16..256 TMEM columns), so one dequantised
-// 128 x 64 weight tile feeds up to 256 tokens. Operands are fp16: the
+// 128 x 128 weight stage feeds up to 256 tokens. Operands are fp16: the
 // activations are scaled by 1/s and rounded once to fp16 by a pre-pass
 // (prescale_kernel), each weight (q - z) * D is rounded once to fp16 in the
 // dequantiser; products accumulate in fp32 in TMEM.
 //
-// CTA = 10 warps, four shared-memory rings filled by the tensor memory
-// accelerator (TMA) and drained in K order:
-//   X~ ring      64-channel fp16 activation tiles (128B swizzle)      warp 0
-//   codes ring   128 rows x 128 channels of packed codes                warp 0
-//   params ring  128 rows x 16 groups of delta (fp32) and zero (u8)     warp 0
-//   A ring       64-channel fp16 weight tiles (128B swizzle)       warps 2-9
-// warp 1 owns TMEM and issues tcgen05.mma from one thread; warps 2-9 are
-// the dequantisers (two threads per weight row, one 32-code block each:
-// fp16 pairs built with the 1024+q exponent trick) and then the epilogue
-// (TMEM -> Y). Decode (T <= 16) splits K over a cluster of up to 8 CTAs
-// whose partial tiles rank 0 sums through distributed shared memory in a
-// fixed order. The rank-r low-rank term is one extra K stage,
-// [X~ | U] [W_hat | B]^T with U = X A^T (fp16, from lowrank_u_kernel).
-// Every wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds down).
+// CTA = producer warp + MMA warp + 8 dequantiser warps (prefill, one CTA
+// per SM) or 4 (decode, two CTAs per SM). Shared-memory rings filled by the
+// tensor memory accelerator (TMA) and drained in K order by stage:
+//   X~ ring      two 64-channel fp16 activation boxes (128B swizzle)
+//   codes ring   128 rows x 128 channels of packed codes
+//   params ring  128 rows x 16 groups of delta (fp32) and zero (u8)
+// The dequantisers write each fp16 weight stage straight to a TMEM ring
+// (tcgen05.st; a thread = a weight row = a TMEM lane) and the MMA warp's
+// elected thread consumes it with the A-from-TMEM form of tcgen05.mma
+// (fp16 pairs are built with the 1024+q exponent trick). Epilogue: the
+// accumulator leaves TMEM in 16x256b fragment order, is packed to 16-bit
+// pairs and written transposed by stmatrix into 128-byte-swizzled boxes of
+// the idle activation ring, and a TMA tensor store writes Y. Decode
+// (3 <= T <= 32; one or two tokens use gemv.cu) splits K over a cluster of
+// up to 8 CTAs whose partial tiles every rank reduces in part through
+// distributed shared memory, in rank order. The rank-r low-rank term is one
+// extra K stage, [X~ | U] [W_hat | B]^T with U = X A^T (fp16, from
+// lowrank_u_kernel). Every wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA
+// winds down).
 #include <cooperative_groups.h>
 
 #include <algorithm>
