@@ -2,7 +2,8 @@
 //
 // Every entry point validates its arguments on the host before enqueuing
 // anything, then calls an internal launcher. Nothing here allocates device
-// memory; the only library state is the sticky device error word below.
+// memory; the library's device state is the sticky error word below and the
+// built-in scratch array of noalloc.cu (host side: cached SM counts).
 #include <math.h>
 
 #include <atomic>

@@ -1,8 +1,9 @@
 // common.cuh — device helpers shared by the libttq kernels (sm_100a).
 //
-// Hand-written PTX wrappers for mbarriers, TMA, cp.async and tcgen05, the
-// bounded waits every spin uses, and vectorised dtype loads. Nothing here is
-// specific to one kernel.
+// Hand-written PTX wrappers for mbarriers, TMA loads and stores, stmatrix,
+// programmatic dependent launch and tcgen05, the bounded waits every spin
+// uses, the launch helper every kernel goes through, and vectorised dtype
+// loads. Nothing here is specific to one kernel.
 #pragma once
 
 #include <cuda.h>
