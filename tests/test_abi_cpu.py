@@ -171,3 +171,30 @@ def test_empty_inputs_are_refused_before_launch(lib):
     un = lib.ttq_unpack_codes
     un.argtypes = [P, I64, I64, I, P, P]
     assert un(fake, 0, 64, 4, fake, None) == 1
+
+
+def test_binding_refuses_host_tensors_and_bad_layouts():
+    """The Python binding checks its tensors before calling the library:
+    host tensors and rows that are not contiguous raise TTQError."""
+    import torch
+    from test_weight_quantization_b200 import ttq
+    X = torch.zeros(4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ttq.TTQError):
+        ttq.act_stats(X)
+    with pytest.raises(ttq.TTQError):
+        ttq.quantize_rtn_grouped(X, None, 4, 32)
+    with pytest.raises(ttq.TTQError):
+        ttq.act_stats_scales(X, torch.zeros(1, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("K", [32, 96, 768, 4096, 11008])
+@pytest.mark.parametrize("bits", [2, 3, 4, 5, 8])
+def test_row_pitches_match_the_documented_formulas(lib, K, bits):
+    """ttq_codes_ld: K*bits/32 words rounded up to 4; ttq_groups_ld: K/g
+    entries rounded up to 16 (16-byte rows for TMA)."""
+    from test_weight_quantization_b200 import ttq
+    words = K * bits // 32
+    assert ttq.codes_ld(K, bits) == (words + 3) // 4 * 4
+    for g in (16, 32, 64, 128):
+        if K % g == 0:
+            assert ttq.groups_ld(K, g) == (K // g + 15) // 16 * 16
