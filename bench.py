@@ -322,39 +322,82 @@ class ClockSampler:
 
 # ------------------------------------------------------------- oracle -----
 
-def oracle_step(wl, data, sample_tokens):
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _ranges(n, parts):
+    """[lo, hi) pieces of range(n), at most ``parts`` of near-equal size."""
+    parts = max(1, min(parts, n))
+    b = [n * i // parts for i in range(parts + 1)]
+    return [(b[i], b[i + 1]) for i in range(parts)]
+
+
+def oracle_step(wl, data, sample_tokens, threads=1, outputs=None):
     """The CPU oracle on a bounded sample of one step: statistics, scales and
     quantization at full size, the projection on the first ``sample_tokens``
-    tokens, scaled linearly to T. Returns (seconds per step, description)."""
+    tokens, scaled linearly to T. Returns (seconds per step, description).
+
+    With ``threads`` > 1 the unchanged oracle functions run concurrently on
+    disjoint slices: the statistics over token ranges (the partial sums are
+    added), the quantizer and the projection over output rows. The C calls
+    release the GIL. ``outputs``, when a dict, receives every layer's
+    (codes, delta, zero, Y sample) for checking."""
     import numpy as np
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     T = wl.T
     Ts = min(sample_tokens, T)
     Xn = {k: v.float().numpy() for k, v in data["X"].items()}
-    t0 = time.perf_counter()
-    s, inv = {}, {}
-    for k, X in Xn.items():
-        sums = oracle.act_sums(X, wl.p)
-        s[k], inv[k] = oracle.awq_scales(sums, T, wl.alpha, wl.lam, wl.p)
-    t_full = time.perf_counter() - t0
-    t_gemm = 0.0
-    for L in wl.layers:
-        W = data["W"][L.name].float().numpy()
-        t1 = time.perf_counter()
-        c, d, z = oracle.quantize(W, s[L.input_name].astype(np.float32),
-                                  wl.bits, wl.group)
-        t_full += time.perf_counter() - t1
-        A = B = None
-        if wl.rank:
-            A = data["A"][L.name].float().numpy()
-            B = data["B"][L.name].float().numpy()
-        t2 = time.perf_counter()
-        oracle.lowbit_gemm(Xn[L.input_name][:Ts], inv[L.input_name], c, d, z,
-                           L.N, wl.bits, wl.group, A, B)
-        t_gemm += time.perf_counter() - t2
+    pool = ThreadPoolExecutor(threads) if threads > 1 else None
+
+    def each(fn, n):
+        pieces = _ranges(n, threads)
+        if pool is None:
+            return [fn(a, b) for a, b in pieces]
+        return list(pool.map(lambda ab: fn(*ab), pieces))
+
+    try:
+        t0 = time.perf_counter()
+        s, inv = {}, {}
+        for k, X in Xn.items():
+            sums = sum(each(lambda a, b: oracle.act_sums(X[a:b], wl.p), T))
+            s[k], inv[k] = oracle.awq_scales(sums, T, wl.alpha, wl.lam, wl.p)
+        t_full = time.perf_counter() - t0
+        t_gemm = 0.0
+        for L in wl.layers:
+            W = data["W"][L.name].float().numpy()
+            s32 = s[L.input_name].astype(np.float32)
+            t1 = time.perf_counter()
+            parts = each(lambda a, b: oracle.quantize(W[a:b], s32, wl.bits,
+                                                      wl.group), L.N)
+            c, d, z = (np.concatenate(x) for x in zip(*parts))
+            t_full += time.perf_counter() - t1
+            A = B = None
+            if wl.rank:
+                A = data["A"][L.name].float().numpy()
+                B = data["B"][L.name].float().numpy()
+            Xs = Xn[L.input_name][:Ts]
+            t2 = time.perf_counter()
+            ys = each(lambda a, b: oracle.lowbit_gemm(
+                Xs, inv[L.input_name], c[a:b], d[a:b], z[a:b], b - a, wl.bits,
+                wl.group, A, None if B is None else B[a:b]), L.N)
+            t_gemm += time.perf_counter() - t2
+            if outputs is not None:
+                outputs[L.name] = (c, d, z, np.concatenate(ys, axis=1))
+    finally:
+        if pool is not None:
+            pool.shutdown()
     est = t_full + t_gemm * (T / Ts)
+    how = ("1 thread" if threads == 1 else
+           f"{threads} threads on disjoint token ranges (statistics) and "
+           f"output rows (quantizer, projection)")
     desc = (f"stats, scales and quantize at full size; projection on {Ts} of "
-            f"{T} tokens scaled x{T / Ts:g}; 1 thread")
+            f"{T} tokens scaled x{T / Ts:g}; {how}")
     return est, desc
 
 
@@ -599,11 +642,17 @@ def main():
     if not args.no_e2e:
         e2e = end_to_end(ttq, wl, data, device, args, stream, world)
 
-    cpu = None
+    cpu = cpu_all = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS)
         cpu = {"value": len(wl.layers) * wl.T / est, "unit": "tokens/s",
                "cores": 1, "kind": "oracle", "sample": desc}
+        cores = host_cores()
+        if cores > 1:
+            est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS, cores)
+            cpu_all = {"value": len(wl.layers) * wl.T / est,
+                       "unit": "tokens/s", "cores": cores,
+                       "kind": "oracle, threaded", "sample": desc}
 
     if rank == 0:
         line = {
@@ -632,7 +681,8 @@ def main():
                     "beside the quantizer")},
             "roofline": roof, "kernels": kernels,
             "gpu_launches": step.kernel_launches() * args.steps,
-            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "cpu_baseline": cpu, "cpu_baseline_all_cores": cpu_all,
+            "e2e": e2e, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

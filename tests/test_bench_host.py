@@ -152,3 +152,39 @@ def test_algorithmic_work_closed_forms():
     wg = bench.algorithmic_work(gem)
     assert wg["gemm_flops"] == sum(2 * 1024 * L.N * L.K + 2 * 1024 * 16 *
                                    (L.K + L.N) for L in gem.layers)
+
+
+def test_threaded_oracle_baseline_computes_the_same_step():
+    """The all-cores CPU baseline runs the unchanged oracle on disjoint
+    slices; its codes, scales and projection equal the one-thread run (the
+    partial channel sums only change the fp64 summation order)."""
+    import dataclasses
+    import numpy as np
+    import bench
+    from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs
+    for name in ("opt125m-block", "gemma1b-mlp"):
+        base = WORKLOADS[name]
+        wl = dataclasses.replace(base, T=96, layers=base.layers[:2])
+        data = make_inputs(wl)
+        one, many = {}, {}
+        bench.oracle_step(wl, data, 8, threads=1, outputs=one)
+        est, desc = bench.oracle_step(wl, data, 8, threads=5, outputs=many)
+        assert est > 0 and "5 threads" in desc
+        assert one.keys() == many.keys() == {L.name for L in wl.layers}
+        for k in one:
+            for a, b in zip(one[k][:3], many[k][:3]):
+                assert np.array_equal(a, b)
+            np.testing.assert_allclose(many[k][3], one[k][3], rtol=1e-12,
+                                       atol=1e-12)
+            assert one[k][3].shape == (8, next(L.N for L in wl.layers
+                                                if L.name == k))
+
+
+def test_host_cores_and_ranges_cover_the_work():
+    import bench
+    assert bench.host_cores() >= 1
+    for n, parts in ((10, 3), (7, 7), (5, 9), (768, 224), (1, 1)):
+        r = bench._ranges(n, parts)
+        assert r[0][0] == 0 and r[-1][1] == n and len(r) == min(n, parts)
+        assert all(a < b for a, b in r)
+        assert all(r[i][1] == r[i + 1][0] for i in range(len(r) - 1))
