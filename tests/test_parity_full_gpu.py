@@ -63,6 +63,14 @@ def check_layer(ttq, wl, name, X, W, A, B, bits, group, T_tok, qrows,
     np.testing.assert_array_equal(gd, rd, err_msg=f"{name} delta")
     np.testing.assert_array_equal(gz, rz, err_msg=f"{name} zero")
     np.testing.assert_array_equal(gc, rc, err_msg=f"{name} codes")
+    # the oracle's own scales (fp64, stored as fp32) differ from the GPU's by
+    # an fp32 ulp or two on some channels; codes may move only where that
+    # shifts w*s/D across a rounding boundary, a few per million
+    oc, _, _ = oracle.quantize(Wn, rs.astype(np.float32), bits, group)
+    moved = int(np.count_nonzero(oracle.unpack_codes(oc, K, bits) !=
+                                 oracle.unpack_codes(rc, K, bits)))
+    print(f"{name}: {moved} of {Wn.size} codes differ with the oracle's s")
+    assert moved <= max(16, 1e-4 * Wn.size), f"{name}: {moved} codes moved"
     # projection of the first T_tok tokens, as the benchmark launches it
     Xt = Xg[:T_tok]
     Ag = None if A is None else A.cuda()
