@@ -291,7 +291,20 @@ const char* ttq_status_string(ttq_status status);
  * is non-zero. Returns the TTQ_DEVERR_* bits, or -1 if the copy failed. */
 int ttq_device_error(int clear);
 
-/* ABI version of this header (3: ttq_act_stats_scales added). */
+/* Self-test of the failure path shared by every kernel's waits: one
+ * device thread initialises an mbarrier and waits for its first phase with
+ * the same bounded wait the kernels use. With arrive != 0 the thread
+ * arrives first and the wait completes (*out = 1). With arrive == 0
+ * nothing ever arrives: after about 1.5 s of SM clocks the wait gives up,
+ * raises TTQ_DEVERR_TIMEOUT in the sticky error word and the kernel returns
+ * normally (*out = 0), leaving the context usable. out: one device uint32,
+ * 4-byte aligned, written asynchronously on `stream`. Returns
+ * TTQ_ERR_INVALID_ARG for a NULL or misaligned out, TTQ_ERR_CUDA if the
+ * launch fails. Not part of the method; for tests of error handling. */
+ttq_status ttq_selftest_bounded_wait(int arrive, uint32_t* out, void* stream);
+
+/* ABI version of this header (3: ttq_act_stats_scales added; 4:
+ * ttq_selftest_bounded_wait added). */
 int ttq_abi_version(void);
 
 #ifdef __cplusplus

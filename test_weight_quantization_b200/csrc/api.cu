@@ -92,7 +92,7 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 3; }
+TTQ_EXPORT int ttq_abi_version(void) { return 4; }
 
 TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
   if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
@@ -280,4 +280,10 @@ TTQ_EXPORT ttq_status ttq_unpack_codes(const uint32_t* codes, int64_t N,
       bits > 8 || !aligned(codes, 4))
     return TTQ_ERR_INVALID_ARG;
   return launch_unpack(codes, N, K, bits, q_out, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_selftest_bounded_wait(int arrive, uint32_t* out,
+                                                void* stream) {
+  if (!out || !aligned(out, sizeof(uint32_t))) return TTQ_ERR_INVALID_ARG;
+  return launch_bounded_wait_check(arrive ? 1 : 0, out, as_stream(stream));
 }

@@ -64,6 +64,11 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
                                 int64_t ldy, cudaStream_t st);
 
+// One thread runs the library's bounded mbarrier wait; *out = 1 if the
+// phase completed, 0 if the wait gave up (selftest.cu).
+ttq_status launch_bounded_wait_check(int arrive, uint32_t* out,
+                                     cudaStream_t st);
+
 ttq_status launch_lowrank_add(const void* X, ttq_dtype xt, int64_t T,
                               int64_t K, int64_t ldx, const void* A,
                               const void* B, int r, int64_t N, void* Y,

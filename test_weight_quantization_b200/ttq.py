@@ -58,6 +58,7 @@ def _load() -> ctypes.CDLL:
         "ttq_abi_version": [],
         "ttq_codes_ld": [I64, I],
         "ttq_groups_ld": [I64, I],
+        "ttq_selftest_bounded_wait": [I, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -79,7 +80,7 @@ EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_act_stats_scales",
            "ttq_prepare_activations", "ttq_w_lowbit_gemm_prepared",
            "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
            "ttq_device_error", "ttq_abi_version", "ttq_codes_ld",
-           "ttq_groups_ld")
+           "ttq_groups_ld", "ttq_selftest_bounded_wait")
 
 
 class _Params(ctypes.Structure):
@@ -141,6 +142,21 @@ def groups_ld(K: int, group: int) -> int:
 def device_error(clear: bool = True) -> int:
     """Sticky device error bits (synchronising read)."""
     return int(_lib.ttq_device_error(1 if clear else 0))
+
+
+def selftest_bounded_wait(arrive: bool) -> tuple[bool, int]:
+    """Runs the kernels' bounded wait on a barrier that completes (arrive)
+    or never does. Returns (whether the wait completed, the device error
+    bits, which are cleared). Synchronises the device."""
+    out = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    _check(_lib.ttq_selftest_bounded_wait(1 if arrive else 0, out.data_ptr(),
+                                          _stream()),
+           "ttq_selftest_bounded_wait")
+    torch.cuda.synchronize()
+    done = int(out.item())
+    if done not in (0, 1):
+        raise TTQError(f"ttq_selftest_bounded_wait wrote {done}")
+    return done == 1, device_error(clear=True)
 
 
 def act_stats(X: torch.Tensor, p: float = 2.0, out: torch.Tensor | None = None,

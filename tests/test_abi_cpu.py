@@ -45,7 +45,7 @@ def test_status_strings_and_version(lib):
     assert lib.ttq_status_string(0) == b"TTQ_OK"
     assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
     assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
-    assert lib.ttq_abi_version() == 3
+    assert lib.ttq_abi_version() == 4
 
 
 def test_workspace_size(lib):
@@ -60,6 +60,10 @@ def test_workspace_size(lib):
 def test_bad_arguments_are_rejected_before_launch(lib):
     P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
     fake = ctypes.c_void_p(0x100000)  # never dereferenced: checks fail first
+    lib.ttq_selftest_bounded_wait.argtypes = [I, P, P]
+    assert lib.ttq_selftest_bounded_wait(0, None, None) == 1
+    assert lib.ttq_selftest_bounded_wait(1, ctypes.c_void_p(0x100002),
+                                         None) == 1  # misaligned
     lib.ttq_act_stats.argtypes = [P, I, I64, I64, I64, F, I, P, P]
     assert lib.ttq_act_stats(None, 1, 8, 64, 64, 2.0, 0, fake, None) == 1
     assert lib.ttq_act_stats(fake, 1, 8, 60, 64, 2.0, 0, fake, None) == 1  # K%8

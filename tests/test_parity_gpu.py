@@ -401,3 +401,25 @@ def test_layer_object_matches_calls(ttq):
     # and the result agrees with the oracle
     ref = oracle_y(X.cpu(), inv, c, d, z, W.shape[0], 3, 32)
     assert_gemm_close(np32(y), ref, "layer object", y.dtype)
+
+
+def test_bounded_wait_gives_up_and_leaves_the_context_usable(ttq):
+    """The failure path of every in-kernel wait: a barrier that nothing
+    arrives at makes the wait give up after its clock limit, raise
+    TTQ_DEVERR_TIMEOUT and return; later launches still run correctly."""
+    import time
+    ttq.device_error(clear=True)
+    done, err = ttq.selftest_bounded_wait(True)
+    assert done and err == 0
+    t0 = time.perf_counter()
+    done, err = ttq.selftest_bounded_wait(False)
+    waited = time.perf_counter() - t0
+    assert not done and err & ttq.DEVERR_TIMEOUT
+    assert 0.3 < waited < 30.0
+    # the context is intact: a quantization after the timeout is bit-exact
+    W = weights(64, 256, 5, torch.bfloat16)
+    c, d, z, rc, rd, rz = quantize_both(ttq, W, None, 4, 32)
+    np.testing.assert_array_equal(c, rc)
+    np.testing.assert_array_equal(d, rd)
+    np.testing.assert_array_equal(z, rz)
+    assert ttq.device_error(clear=True) == 0
