@@ -12,6 +12,7 @@ Inference On The Fly" (TTQ review, section "Proposed method", bullets 1-7).
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from dataclasses import dataclass
 
@@ -109,8 +110,21 @@ def _stream() -> int:
 
 
 def _dev(t: torch.Tensor, name: str) -> None:
+    """A CUDA tensor on the current device (the one the call launches on)."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TTQError(f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise TTQError(f"{name} is on {t.device}; the call launches on "
+                       f"cuda:{cur}")
+
+
+def _code(t: torch.Tensor, name: str) -> int:
+    """The ttq_dtype of a floating tensor."""
+    if t.dtype not in _DTYPE:
+        raise TTQError(f"{name} must be float32, bfloat16 or float16, not "
+                       f"{t.dtype}")
+    return _DTYPE[t.dtype]
 
 
 def _rows(t: torch.Tensor, name: str) -> int:
@@ -121,6 +135,65 @@ def _rows(t: torch.Tensor, name: str) -> int:
     return t.stride(0)
 
 
+_CODE_DTYPES = (torch.int32, torch.uint32)
+
+
+def _buf(t: torch.Tensor, name: str, dtypes, rows: int,
+         cols: int | None = None) -> None:
+    """A dense device buffer: at least ``rows`` entries ([rows] vector), or
+    at least ``rows`` rows of exactly ``cols`` entries."""
+    _dev(t, name)
+    dtypes = dtypes if isinstance(dtypes, tuple) else (dtypes,)
+    if t.dtype not in dtypes:
+        raise TTQError(f"{name} must be {' or '.join(map(str, dtypes))}, "
+                       f"not {t.dtype}")
+    if cols is None:
+        ok = t.dim() == 1 and t.numel() >= rows
+        want = f"[{rows}]"
+    else:
+        ok = t.dim() == 2 and t.shape[0] >= rows and t.shape[1] == cols
+        want = f"[{rows}, {cols}]"
+    if not ok or not t.is_contiguous():
+        raise TTQError(f"{name} must be a dense buffer of shape {want}, got "
+                       f"{tuple(t.shape)} with strides {t.stride()}")
+
+
+def _packed(codes, delta, zero, N: int, K: int, bits: int, group: int):
+    """Codes, delta and zero of an [N, K] weight in the packed layout."""
+    cl, gl = codes_ld(K, bits), groups_ld(K, group)
+    if cl <= 0 or gl <= 0:
+        raise TTQError(f"no packed layout for K={K}, bits={bits}, "
+                       f"group={group}")
+    _buf(codes, "codes", _CODE_DTYPES, N, cl)
+    _buf(delta, "delta", torch.float32, N, gl)
+    _buf(zero, "zero", torch.uint8, N, gl)
+
+
+def _out(Y: torch.Tensor, name: str, T: int, N: int) -> int:
+    """An output [T, N] with contiguous rows; returns its row pitch."""
+    ld = _rows(Y, name)
+    _code(Y, name)
+    if tuple(Y.shape) != (T, N):
+        raise TTQError(f"{name} must have shape ({T}, {N}), got "
+                       f"{tuple(Y.shape)}")
+    return ld
+
+
+def _factors(A, B, N: int, K: int, dtype) -> int:
+    """The low-rank factors A [r, K] and B [N, r] (both or neither);
+    returns r."""
+    if (A is None) != (B is None):
+        raise TTQError("A and B come together")
+    if A is None:
+        return 0
+    r = A.shape[0] if A.dim() == 2 else -1
+    _buf(A, "A", dtype, r, K)
+    _buf(B, "B", dtype, N, r)
+    if B.shape[0] != N:
+        raise TTQError(f"B must have {N} rows, got {B.shape[0]}")
+    return r
+
+
 def _ptr(t):
     return None if t is None else t.data_ptr()
 
@@ -129,11 +202,13 @@ def abi_version() -> int:
     return int(_lib.ttq_abi_version())
 
 
+@functools.lru_cache(maxsize=4096)
 def codes_ld(K: int, bits: int) -> int:
     """Row pitch (uint32 words) of the packed codes."""
     return int(_lib.ttq_codes_ld(K, bits))
 
 
+@functools.lru_cache(maxsize=4096)
 def groups_ld(K: int, group: int) -> int:
     """Row pitch (entries) of delta and zero."""
     return int(_lib.ttq_groups_ld(K, group))
@@ -166,8 +241,8 @@ def act_stats(X: torch.Tensor, p: float = 2.0, out: torch.Tensor | None = None,
     T, K = X.shape
     if out is None:
         out = torch.empty(K, dtype=torch.float32, device=X.device)
-    _dev(out, "out")
-    _check(_lib.ttq_act_stats(X.data_ptr(), _DTYPE[X.dtype], T, K, ldx,
+    _buf(out, "out", torch.float32, K)
+    _check(_lib.ttq_act_stats(X.data_ptr(), _code(X, "X"), T, K, ldx,
                               float(p), 1 if accumulate else 0,
                               out.data_ptr(), _stream()), "ttq_act_stats")
     return out
@@ -176,11 +251,13 @@ def act_stats(X: torch.Tensor, p: float = 2.0, out: torch.Tensor | None = None,
 def awq_scales(sums: torch.Tensor, T_total: int, alpha: float = 0.5,
                lam: float = 0.1, p: float = 2.0, s=None, inv_s=None):
     """Step 2: (s, inv_s) fp32 [K] from the channel sums."""
-    _dev(sums, "sums")
+    _buf(sums, "sums", torch.float32, 0)
     K = sums.shape[0]
     s = torch.empty(K, dtype=torch.float32, device=sums.device) if s is None \
         else s
     inv_s = torch.empty_like(s) if inv_s is None else inv_s
+    _buf(s, "s", torch.float32, K)
+    _buf(inv_s, "inv_s", torch.float32, K)
     prm = _Params(0, 0, alpha, lam, p)
     _check(_lib.ttq_awq_scales(sums.data_ptr(), int(T_total), K,
                                ctypes.addressof(prm), s.data_ptr(),
@@ -200,15 +277,17 @@ def act_stats_scales(X: torch.Tensor, counter: torch.Tensor,
                      T_total: int | None = None):
     """Steps 1 and 2 in one launch: (sums, s, inv_s), each fp32 [K]."""
     ldx = _rows(X, "X")
-    _dev(counter, "counter")
+    _buf(counter, "counter", _CODE_DTYPES, 1)
     T, K = X.shape
     f32 = dict(dtype=torch.float32, device=X.device)
     sums = torch.empty(K, **f32) if sums is None else sums
     s = torch.empty(K, **f32) if s is None else s
     inv_s = torch.empty(K, **f32) if inv_s is None else inv_s
+    for t, name in ((sums, "sums"), (s, "s"), (inv_s, "inv_s")):
+        _buf(t, name, torch.float32, K)
     prm = _Params(0, 0, alpha, lam, p)
     _check(_lib.ttq_act_stats_scales(
-        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, 1 if accumulate else 0,
+        X.data_ptr(), _code(X, "X"), T, K, ldx, 1 if accumulate else 0,
         int(T if T_total is None else T_total), ctypes.addressof(prm),
         sums.data_ptr(), s.data_ptr(), inv_s.data_ptr(), counter.data_ptr(),
         _stream()), "ttq_act_stats_scales")
@@ -231,8 +310,11 @@ def quantize_rtn_grouped(W: torch.Tensor, s: torch.Tensor | None, bits: int,
     if zero is None:
         zero = torch.empty((N, groups_ld(K, group)), dtype=torch.uint8,
                            device=dev)
+    if s is not None:
+        _buf(s, "s", torch.float32, K)
+    _packed(codes, delta, zero, N, K, bits, group)
     _check(_lib.ttq_quantize_rtn_grouped(
-        W.data_ptr(), _DTYPE[W.dtype], N, K, ldw, _ptr(s), bits, group,
+        W.data_ptr(), _code(W, "W"), N, K, ldw, _ptr(s), bits, group,
         codes.data_ptr(), delta.data_ptr(), zero.data_ptr(), _stream()),
         "ttq_quantize_rtn_grouped")
     return codes, delta, zero
@@ -251,17 +333,22 @@ def w_lowbit_gemm(X: torch.Tensor, inv_s: torch.Tensor, codes: torch.Tensor,
     """Step 4: Y = (X diag(inv_s)) W_hat^T [+ (X A^T) B^T], [T, N]."""
     ldx = _rows(X, "X")
     T, K = X.shape
-    r = 0 if A is None else A.shape[0]
+    r = _factors(A, B, N, K, X.dtype)
+    _buf(inv_s, "inv_s", torch.float32, K)
+    _packed(codes, delta, zero, N, K, bits, group)
     if out is None:
         out = torch.empty((T, N), dtype=out_dtype or X.dtype, device=X.device)
-    ldy = _rows(out, "out")
+    ldy = _out(out, "out", T, N)
     need = workspace_size(T, K, r)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _dev(workspace, "workspace")
+    if not workspace.is_contiguous():
+        raise TTQError("workspace must be contiguous")
     _check(_lib.ttq_w_lowbit_gemm(
-        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(),
+        X.data_ptr(), _code(X, "X"), T, K, ldx, inv_s.data_ptr(),
         codes.data_ptr(), delta.data_ptr(), zero.data_ptr(), N, bits, group,
-        _ptr(A), _ptr(B), r, out.data_ptr(), _DTYPE[out.dtype], ldy,
+        _ptr(A), _ptr(B), r, out.data_ptr(), _code(out, "out"), ldy,
         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
         _stream()), "ttq_w_lowbit_gemm")
     return out
@@ -274,13 +361,20 @@ def prepare_activations(X: torch.Tensor, inv_s: torch.Tensor, bits: int,
     U = fp16(X A^T) zero-padded to [T, 64]."""
     ldx = _rows(X, "X")
     T, K = X.shape
-    r = 0 if A is None else A.shape[0]
+    r = 0
+    if A is not None:
+        r = A.shape[0] if A.dim() == 2 else -1
+        _buf(A, "A", X.dtype, r, K)
+    _buf(inv_s, "inv_s", torch.float32, K)
     if Xs is None:
         Xs = torch.empty((T, K), dtype=torch.float16, device=X.device)
+    _buf(Xs, "Xs", torch.float16, T, K)
     if r and U is None:
         U = torch.empty((T, 64), dtype=torch.float16, device=X.device)
+    if r:
+        _buf(U, "U", torch.float16, T, 64)
     _check(_lib.ttq_prepare_activations(
-        X.data_ptr(), _DTYPE[X.dtype], T, K, ldx, inv_s.data_ptr(), bits,
+        X.data_ptr(), _code(X, "X"), T, K, ldx, inv_s.data_ptr(), bits,
         _ptr(A), r, Xs.data_ptr(), _ptr(U) if r else None, _stream()),
         "ttq_prepare_activations")
     return Xs, (U if r else None)
@@ -295,15 +389,28 @@ def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
     """The projection on prepared operands (one kernel launch; one or two
     tokens run on CUDA cores, more on tensor cores)."""
     _dev(Xs, "Xs")
+    if Xs.dim() != 2:
+        raise TTQError("Xs must be 2D")
     T, K = Xs.shape
-    r = 0 if B is None else B.shape[1]
+    _buf(Xs, "Xs", torch.float16, T, K)
+    r = 0
+    if B is not None:
+        r = B.shape[1] if B.dim() == 2 else -1
+        _buf(B, "B", B.dtype, N, r)
+        _code(B, "B")
+        if B.shape[0] != N:
+            raise TTQError(f"B must have {N} rows, got {B.shape[0]}")
+        if U is None:
+            raise TTQError("a low-rank projection needs U")
+        _buf(U, "U", torch.float16, T, 64)
+    _packed(codes, delta, zero, N, K, bits, group)
     if out is None:
         out = torch.empty((T, N), dtype=out_dtype, device=Xs.device)
-    ldy = _rows(out, "out")
+    ldy = _out(out, "out", T, N)
     _check(_lib.ttq_w_lowbit_gemm_prepared(
         Xs.data_ptr(), _ptr(U) if r else None, T, K, codes.data_ptr(),
         delta.data_ptr(), zero.data_ptr(), N, bits, group, _ptr(B),
-        _DTYPE[B.dtype] if r else 0, r, out.data_ptr(), _DTYPE[out.dtype],
+        _code(B, "B") if r else 0, r, out.data_ptr(), _code(out, "out"),
         ldy, _stream()), "ttq_w_lowbit_gemm_prepared")
     return out
 
@@ -312,13 +419,14 @@ def lowrank_add(X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                 Y: torch.Tensor) -> torch.Tensor:
     """Y += (X A^T) B^T in place."""
     ldx = _rows(X, "X")
-    ldy = _rows(Y, "Y")
     T, K = X.shape
-    r = A.shape[0]
+    _dev(B, "B")
     N = B.shape[0]
-    _check(_lib.ttq_lowrank_add(X.data_ptr(), _DTYPE[X.dtype], T, K, ldx,
+    r = _factors(A, B, N, K, X.dtype)
+    ldy = _out(Y, "Y", T, N)
+    _check(_lib.ttq_lowrank_add(X.data_ptr(), _code(X, "X"), T, K, ldx,
                                 A.data_ptr(), B.data_ptr(), r, N, Y.data_ptr(),
-                                _DTYPE[Y.dtype], ldy, _stream()),
+                                _code(Y, "Y"), ldy, _stream()),
            "ttq_lowrank_add")
     return Y
 
@@ -327,6 +435,7 @@ def unpack_codes(codes: torch.Tensor, K: int, bits: int) -> torch.Tensor:
     """One uint8 per weight, [N, K]."""
     _dev(codes, "codes")
     N = codes.shape[0]
+    _buf(codes, "codes", _CODE_DTYPES, N, codes_ld(K, bits))
     q = torch.empty((N, K), dtype=torch.uint8, device=codes.device)
     _check(_lib.ttq_unpack_codes(codes.data_ptr(), N, K, bits, q.data_ptr(),
                                  _stream()), "ttq_unpack_codes")
