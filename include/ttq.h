@@ -38,8 +38,16 @@
  *     returns TTQ_ERR_CUDA. The library never aborts the process.
  *   - Faults found on the device (a bounded wait that gave up, an fp16 range
  *     overflow) set a sticky device error word; ttq_device_error() reads it.
- *   - All device pointers must be 16-byte aligned; ldx, ldw, ldy must make
- *     every row start 16-byte aligned.
+ *   - Alignment. X, W, Xs, U and A, and the s, inv_s, codes, delta and
+ *     zero that the quantizer and the projection read, must start on a
+ *     16-byte boundary, and ldx, ldw must keep every row of X and W 16-byte
+ *     aligned (the kernels read them with 16-byte or tensor-memory-
+ *     accelerator loads); the pitches of ttq_codes_ld and ttq_groups_ld
+ *     keep the rows of codes, delta and zero aligned. Y, B, the sums, the
+ *     s and inv_s written by the statistics calls, and the counter need
+ *     only their element's alignment; rows of Y that are not 16-byte
+ *     aligned are written by a per-row path. A pointer that breaks these
+ *     rules returns TTQ_ERR_INVALID_ARG.
  */
 #ifndef TTQ_H_
 #define TTQ_H_

@@ -210,7 +210,7 @@ TTQ_EXPORT ttq_status ttq_w_lowbit_gemm(
       K % group != 0 || r < 0 || r > 64 || ((r > 0) != (A && B)) ||
       (r == 0 && (A || B)) || ldx < K || ldy < N ||
       !rows_aligned(X, xt, ldx) || !aligned(inv_s, 16) ||
-      !aligned(codes, 4) || !aligned(delta, 4) ||
+      !aligned(codes, 16) || !aligned(delta, 16) || !aligned(zero, 16) ||
       !aligned(Y, dtype_bytes(yt)) || !aligned(workspace, 256) ||
       (r > 0 && (!rows_aligned(A, xt, K) || !aligned(B, dtype_bytes(xt)))) ||
       T >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) ||
@@ -250,8 +250,8 @@ TTQ_EXPORT ttq_status ttq_w_lowbit_gemm_prepared(
       !valid_group(group) || K % group != 0 || r < 0 || r > 64 ||
       ((r > 0) != (U && B)) || (r == 0 && (U || B)) ||
       (r > 0 && !valid_dtype(bt)) || ldy < N || !aligned(Xs, 16) ||
-      (U && !aligned(U, 16)) || !aligned(codes, 4) || !aligned(delta, 4) ||
-      !aligned(Y, dtype_bytes(yt)) ||
+      (U && !aligned(U, 16)) || !aligned(codes, 16) || !aligned(delta, 16) ||
+      !aligned(zero, 16) || !aligned(Y, dtype_bytes(yt)) ||
       (r > 0 && !aligned(B, dtype_bytes(bt))) || T >= ((int64_t)1 << 31) ||
       K >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31))
     return TTQ_ERR_INVALID_ARG;

@@ -78,8 +78,9 @@ TTQ_EXPORT ttq_status ttq_w_lowbit_gemm_noalloc(
       bits > 8 || !group_ok || K % group != 0 || r < 0 || r > 64 ||
       ((r > 0) != (A && B)) || (r == 0 && (A || B)) || ldx < K || ldy < N ||
       !is_aligned(X, 16) || (ldx * dtype_bytes(xt)) % 16 != 0 ||
-      !is_aligned(inv_s, 16) || !is_aligned(codes, 4) ||
-      !is_aligned(delta, 4) || !is_aligned(Y, dtype_bytes(yt)) ||
+      !is_aligned(inv_s, 16) || !is_aligned(codes, 16) ||
+      !is_aligned(delta, 16) || !is_aligned(zero, 16) ||
+      !is_aligned(Y, dtype_bytes(yt)) ||
       (r > 0 && (!is_aligned(A, 16) || (K * dtype_bytes(xt)) % 16 != 0 ||
                  !is_aligned(B, dtype_bytes(xt)))) ||
       T >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) ||

@@ -202,3 +202,42 @@ def test_row_pitches_match_the_documented_formulas(lib, K, bits):
     for g in (16, 32, 64, 128):
         if K % g == 0:
             assert ttq.groups_ld(K, g) == (K // g + 15) // 16 * 16
+
+
+def _no_cuda_device():
+    import torch
+    return not torch.cuda.is_available()
+
+
+@pytest.mark.skipif(not _no_cuda_device(),
+                    reason="its control calls would launch on fake pointers")
+def test_packed_operands_must_be_16_byte_aligned(lib):
+    """The projection reads codes, delta and zero with 16-byte and
+    tensor-memory-accelerator loads: a pointer off a 16-byte boundary is an
+    invalid argument for every projection entry point. Each refused call
+    differs from an accepted one only in that pointer (the accepted control
+    cannot launch here: this host has no CUDA device)."""
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    ok = 0x100000
+    g = lib.ttq_w_lowbit_gemm
+    g.argtypes = [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P, I, P, I,
+                  I64, P, ctypes.c_size_t, P]
+    gp = lib.ttq_w_lowbit_gemm_prepared
+    gp.argtypes = [P, P, I64, I64, P, P, P, I64, I, I, P, I, I, P, I, I64, P]
+    na = lib.ttq_w_lowbit_gemm_noalloc
+    na.argtypes = [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P, I, P, I,
+                   I64, P]
+
+    def calls(c, d, z):
+        return (
+            g(ok, 1, 16, 64, 64, ok, c, d, z, 32, 4, 32, None, None, 0, ok, 1,
+              32, ok, 1 << 20, None),
+            gp(ok, None, 4, 64, c, d, z, 32, 4, 32, None, 1, 0, ok, 1, 32,
+               None),
+            na(ok, 1, 16, 64, 64, ok, c, d, z, 32, 4, 32, None, None, 0, ok,
+               1, 32, None))
+    assert all(st != 1 for st in calls(ok, ok, ok))
+    for off in (4, 8):
+        for c, d, z in ((ok + off, ok, ok), (ok, ok + off, ok),
+                        (ok, ok, ok + off)):
+            assert calls(c, d, z) == (1, 1, 1), (off, c, d, z)
