@@ -109,6 +109,8 @@ def test_reference_arm_reports_the_oracle():
     assert line["impl"] == "reference"
     assert line["unit"] == "tokens/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+    import bench
+    assert line["cpu_baseline"]["cores"] == bench.host_cores()
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["config"]["workload"] == "opt125m-block"
 
