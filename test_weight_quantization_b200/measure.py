@@ -8,12 +8,13 @@
 
 Each call is captured REPS times in a CUDA graph and timed with CUDA events
 around a replay, after three warm-up calls. Inputs are seeded and
-synthetic (N(0, 1) activations, N(0, 0.02^2) weights, bf16). Operands that
-exceed L2 are read from HBM; for the decode projection the weights rotate
-over enough copies to exceed L2. Rates are algorithmic (every input read
-once, every output written once) and the fraction is taken against
-MEASURED_PEAKS.json (HBM copy GB/s, or sustained bf16 TFLOP/s for the
-prefill projection). Prints one line per measurement.
+synthetic (N(0, 1) activations, N(0, 0.02^2) weights, bf16). For the
+memory-bound kernels (statistics, prepare, quantize, decode projection)
+consecutive calls read different copies of the input, enough of them to
+span 2.5x the L2 cache, so every call reads HBM. Rates are algorithmic
+(every input read once, every output written once) and the fraction is
+taken against MEASURED_PEAKS.json (HBM copy GB/s, or sustained bf16
+TFLOP/s for the prefill projection). Prints one line per measurement.
 """
 from __future__ import annotations
 
@@ -64,6 +65,11 @@ def graph_us(fns):
     return a.elapsed_time(b) / n * 1e3
 
 
+def rotation(nbytes):
+    """Copies of an operand of ``nbytes`` that together span 2.5x L2."""
+    return max(1, min(64, -(-int(2.5 * L2_BYTES) // max(1, int(nbytes)))))
+
+
 def _gen(seed):
     return torch.Generator(device="cuda").manual_seed(seed)
 
@@ -91,33 +97,38 @@ def report(name, us, byts=None, flops=None):
 
 
 def stats(T, K):
-    X = acts(T, K)
+    Xr = [acts(T, K)]
+    Xr += [Xr[0].clone() for _ in range(rotation(T * K * 2) - 1)]
     ctr = ttq.new_counter()
     sums = torch.empty(K, device="cuda")
     s = torch.empty_like(sums)
     inv = torch.empty_like(sums)
-    us = graph_us([lambda: ttq.act_stats(X, 2.0, out=sums)])
+    us = graph_us([lambda X=X: ttq.act_stats(X, 2.0, out=sums) for X in Xr])
     report(f"stats          T={T:5d} K={K:6d}", us, T * K * 2 + K * 4)
-    us = graph_us([lambda: ttq.act_stats_scales(X, ctr, 0.5, 0.1, 2.0, sums,
-                                                s, inv)])
+    us = graph_us([lambda X=X: ttq.act_stats_scales(X, ctr, 0.5, 0.1, 2.0,
+                                                    sums, s, inv)
+                   for X in Xr])
     report(f"stats+scales   T={T:5d} K={K:6d}", us, T * K * 2 + K * 12)
 
 
 def prepare(T, K, bits):
-    X = acts(T, K)
+    Xr = [acts(T, K)]
+    Xr += [Xr[0].clone() for _ in range(rotation(T * K * 4) - 1)]
     inv = torch.ones(K, device="cuda")
     Xs = torch.empty(T, K, dtype=torch.float16, device="cuda")
-    us = graph_us([lambda: ttq.prepare_activations(X, inv, bits, None, Xs)])
+    us = graph_us([lambda X=X: ttq.prepare_activations(X, inv, bits, None, Xs)
+                   for X in Xr])
     report(f"prepare        T={T:5d} K={K:6d} b={bits}", us, T * K * 4 + K * 4)
 
 
 def quantize(N, K, bits, group):
-    W = weights(N, K)
-    s = torch.ones(K, device="cuda")
-    c, d, z = ttq.quantize_rtn_grouped(W, s, bits, group)
-    us = graph_us([lambda: ttq.quantize_rtn_grouped(W, s, bits, group, c, d,
-                                                    z)])
+    Wr = [weights(N, K)]
     byts = N * K * 2 + K * 4 + N * K * bits // 8 + 5 * N * K // group
+    Wr += [Wr[0].clone() for _ in range(rotation(byts) - 1)]
+    s = torch.ones(K, device="cuda")
+    c, d, z = ttq.quantize_rtn_grouped(Wr[0], s, bits, group)
+    us = graph_us([lambda W=W: ttq.quantize_rtn_grouped(W, s, bits, group, c,
+                                                        d, z) for W in Wr])
     report(f"quantize       N={N:6d} K={K:6d} b={bits} g={group:3d}", us, byts)
 
 
@@ -133,7 +144,7 @@ def gemm(T, N, K, bits, group):
     copies = [(c, d, z)]
     if T <= 16:
         # decode: rotate the packed weights so that every call reads HBM
-        n = max(2, int(2.5 * L2_BYTES // wbytes) + 1)
+        n = max(2, rotation(wbytes))
         copies += [(c.clone(), d.clone(), z.clone()) for _ in range(n - 1)]
     fns = [lambda cc=cc, dd=dd, zz=zz: ttq.w_lowbit_gemm_prepared(
         Xs, None, cc, dd, zz, N, bits, group, out=Y) for cc, dd, zz in copies]
