@@ -241,3 +241,35 @@ def test_packed_operands_must_be_16_byte_aligned(lib):
         for c, d, z in ((ok + off, ok, ok), (ok, ok + off, ok),
                         (ok, ok, ok + off)):
             assert calls(c, d, z) == (1, 1, 1), (off, c, d, z)
+
+
+@pytest.mark.skipif(not _no_cuda_device(),
+                    reason="an accepted call would launch on fake pointers")
+def test_sizes_beyond_the_index_range_are_refused(lib):
+    """The largest sizes each entry point accepts: 32-bit block and row
+    counts. One past them is an invalid argument, refused before launch
+    (these pointers are never dereferenced)."""
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    ok = 0x100000
+    big = 1 << 31
+    q = lib.ttq_quantize_rtn_grouped
+    q.argtypes = [P, I, I64, I64, I64, P, I, I, P, P, P, P]
+    # N * (K / 32) blocks must stay below 2^31
+    assert q(ok, 1, big // 2, 64, 64, None, 4, 32, ok, ok, ok, None) == 1
+    g = lib.ttq_w_lowbit_gemm
+    g.argtypes = [P, I, I64, I64, I64, P, P, P, P, I64, I, I, P, P, I, P, I,
+                  I64, P, ctypes.c_size_t, P]
+    assert g(ok, 1, big, 64, 64, ok, ok, ok, ok, 32, 4, 32, None, None, 0, ok,
+             1, 32, ok, 1 << 62, None) == 1                       # T
+    assert g(ok, 1, 16, 64, 64, ok, ok, ok, ok, big, 4, 32, None, None, 0, ok,
+             1, big, ok, 1 << 20, None) == 1                      # N
+    gp = lib.ttq_w_lowbit_gemm_prepared
+    gp.argtypes = [P, P, I64, I64, P, P, P, I64, I, I, P, I, I, P, I, I64, P]
+    assert gp(ok, None, big, 64, ok, ok, ok, 32, 4, 32, None, 1, 0, ok, 1, 32,
+              None) == 1
+    assert gp(ok, None, 4, 64, ok, ok, ok, big, 4, 32, None, 1, 0, ok, 1, big,
+              None) == 1
+    pr = lib.ttq_prepare_activations
+    pr.argtypes = [P, I, I64, I64, I64, P, I, P, I, P, P, P]
+    # T * (K / 16) spans must stay below 2^31
+    assert pr(ok, 1, big // 4, 64, 64, ok, 4, None, 0, ok, None, None) == 1
