@@ -401,6 +401,37 @@ def oracle_step(wl, data, sample_tokens, threads=1, outputs=None):
     return est, desc
 
 
+def parity_summary(step, outputs):
+    """The timed step's codes and sampled outputs against the oracle's (the
+    oracle with its own statistics and scales, on the tokens of its sample).
+    Every replica holds the same inputs, so the buffers of the last replay
+    are the step's result."""
+    import numpy as np
+    import oracle
+    wl = step.wl
+    moved = total = 0
+    worst = 0.0
+    tokens = 0
+    for g, _, Ls in step.groups:
+        codes = step.codes[g].cpu().numpy().view(np.uint32)
+        Y = step.Y[g].float().cpu().numpy()
+        row = 0
+        for L in Ls:
+            oc, _, _, oy = outputs[L.name]
+            gq = oracle.unpack_codes(codes[row:row + L.N, :oc.shape[1]], L.K,
+                                     wl.bits)
+            moved += int(np.count_nonzero(gq != oracle.unpack_codes(
+                oc, L.K, wl.bits)))
+            total += gq.size
+            tokens = oy.shape[0]
+            ys = Y[:tokens, row:row + L.N].astype(np.float64)
+            worst = max(worst, float(np.linalg.norm(ys - oy) /
+                                     max(np.linalg.norm(oy), 1e-300)))
+            row += L.N
+    return {"codes_differing": moved, "codes": total,
+            "y_tokens": tokens, "y_rel_fro_max": worst}
+
+
 # -------------------------------------------------------- aggregation ----
 
 def slowest_rank_ms(ms: float, world: int, device) -> float:
@@ -643,13 +674,19 @@ def main():
     if not args.no_e2e:
         e2e = end_to_end(ttq, wl, data, device, args, stream, world)
 
-    cpu = cpu_one = None
+    cpu = cpu_one = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # the unchanged oracle on every host core, and on one core
         cores = host_cores()
-        est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS, cores)
+        outputs = {}
+        est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS, cores,
+                                outputs)
         cpu = {"value": len(wl.layers) * wl.T / est, "unit": "tokens/s",
                "cores": cores, "kind": "oracle", "sample": desc}
+        try:
+            parity = parity_summary(step, outputs)
+        except Exception as e:  # a report: never a reason to lose the line
+            parity = {"error": repr(e)[:200]}
         if cores > 1:
             est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS)
             cpu_one = {"value": len(wl.layers) * wl.T / est,
@@ -684,7 +721,7 @@ def main():
             "roofline": roof, "kernels": kernels,
             "gpu_launches": step.kernel_launches() * args.steps,
             "cpu_baseline": cpu, "cpu_baseline_one_core": cpu_one,
-            "e2e": e2e, "clocks": clocks,
+            "parity": parity, "e2e": e2e, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

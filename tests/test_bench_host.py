@@ -190,3 +190,44 @@ def test_host_cores_and_ranges_cover_the_work():
         assert r[0][0] == 0 and r[-1][1] == n and len(r) == min(n, parts)
         assert all(a < b for a, b in r)
         assert all(r[i][1] == r[i + 1][0] for i in range(len(r) - 1))
+
+
+def test_parity_summary_reads_the_step_buffers():
+    """The bench line's parity report: the step's (stacked) codes and
+    sampled outputs against the oracle's. Buffers equal to the oracle's give
+    zero moved codes and zero error; one changed code and one changed
+    output are seen."""
+    import dataclasses
+    import numpy as np
+    import torch
+    import bench
+    from test_weight_quantization_b200 import ttq
+    from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs
+    base = WORKLOADS["opt125m-block"]
+    wl = dataclasses.replace(base, T=64, layers=base.layers[:4])
+    data = make_inputs(wl)
+    outputs = {}
+    bench.oracle_step(wl, data, 8, 1, outputs)
+
+    class FakeStep:
+        pass
+    st = FakeStep()
+    st.wl, st.groups = wl, bench.projection_groups(wl)
+    st.codes, st.Y = {}, {}
+    for g, _, Ls in st.groups:
+        K = Ls[0].K
+        c = np.concatenate([outputs[L.name][0] for L in Ls])
+        padded = np.zeros((c.shape[0], ttq.codes_ld(K, wl.bits)), np.uint32)
+        padded[:, :c.shape[1]] = c
+        st.codes[g] = torch.from_numpy(padded.view(np.int32))
+        y = np.concatenate([outputs[L.name][3] for L in Ls], axis=1)
+        st.Y[g] = torch.from_numpy(y.astype(np.float32))
+    assert [g for g, _, _ in st.groups] == ["q|k|v", "o"]
+    rep = bench.parity_summary(st, outputs)
+    assert rep["codes_differing"] == 0
+    assert rep["codes"] == sum(L.N * L.K for L in wl.layers)
+    assert rep["y_tokens"] == 8 and rep["y_rel_fro_max"] < 1e-6
+    st.codes["q|k|v"][800, 0] ^= 1          # code 0 of row 32 of k
+    st.Y["o"][3, 5] += 1.0
+    rep = bench.parity_summary(st, outputs)
+    assert rep["codes_differing"] == 1 and rep["y_rel_fro_max"] > 1e-3
