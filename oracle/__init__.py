@@ -19,7 +19,10 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ttq_oracle.c")
-_LIB = os.path.join(_HERE, "libttq_oracle.so")
+# TTQ_ORACLE_LIB names a prebuilt variant of this library instead (the tests
+# that plant a mistake in a copy of the source and check that a pin fails).
+_VARIANT = os.environ.get("TTQ_ORACLE_LIB")
+_LIB = _VARIANT or os.path.join(_HERE, "libttq_oracle.so")
 
 # -ffp-contract=off and no -ffast-math: the quantizer's fp32 arithmetic must be
 # exactly the IEEE operations written in the source.
@@ -29,6 +32,8 @@ CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
 
 def build(force: bool = False) -> str:
     """Compiles the oracle with gcc if the library is missing or stale."""
+    if _VARIANT:
+        return _LIB
     if (force or not os.path.exists(_LIB)
             or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)):
         tmp = _LIB + ".tmp%d" % os.getpid()
