@@ -49,6 +49,20 @@ MISTAKES = [
     ("low_rank_factor_transposed",
      "acc += u[rho] * (double)B[n * r + rho];",
      "acc += u[rho] * (double)B[rho * N + n];"),
+    ("low_rank_term_on_scaled_x",
+     "acc += (double)x[j] * (double)A[(int64_t)rho * K + j];",
+     "acc += xs[j] * (double)A[(int64_t)rho * K + j];"),
+    ("dequantized_weight_without_delta",
+     "What_s[n * K + j] = (q - z) * (double)delta[n * G + j / group];",
+     "What_s[n * K + j] = (q - z);"),
+    ("loss_error_sign",
+     "e[j] = (double)W[n * K + j] - W_eff[n * K + j];",
+     "e[j] = (double)W[n * K + j] + W_eff[n * K + j];"),
+    ("loss_not_divided_by_T",
+     "return total / (double)T;", "return total;"),
+    ("near_ties_never_counted",
+     "if (frac <= (double)nextafterf(fabsf(v), INFINITY) - fabs((double)v))",
+     "if (frac < 0.0)"),
 ]
 
 
