@@ -21,6 +21,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -41,12 +42,15 @@ from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs  # noqa
 METRIC = "prompt tokens/s per layer incl. on-the-fly quant"
 L2_BYTES = 126 * 1024 * 1024
 ORACLE_SAMPLE_TOKENS = 128
+REFERENCE_SECONDS = 60.0
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    # 5000 steps of ~0.13 ms keep the GPU busy for ~0.6 s, long enough for
+    # several clock samples inside the timed region
+    ap.add_argument("--steps", type=int, default=5000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="opt125m-block",
@@ -262,7 +266,10 @@ def algorithmic_work(wl):
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+    """nvidia-smi samples every 100 ms; the summary keeps the samples taken
+    between mark_start() and mark_end() (all of them, flagged, if none
+    fell inside)."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
               "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,"
@@ -272,6 +279,13 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
 
     def __enter__(self):
         try:
@@ -298,26 +312,46 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not self.path or not os.path.exists(self.path):
             return None
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-                except ValueError:
-                    continue
+            lines = f.readlines()
         os.unlink(self.path)
+        return self.summarize(lines, self.t0, self.t1)
+
+    @staticmethod
+    def summarize(lines, t0=None, t1=None):
+        """Median SM clock, max clock and active throttle reasons of the CSV
+        rows (timestamp first) that fall in [t0, t1]."""
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0],
+                                                "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]),
+                             parts[6:10]))
+            except ValueError:
+                continue
         if not rows:
             return None
+        inside = rows
+        if t0 is not None and t1 is not None:
+            slack = datetime.timedelta(milliseconds=50)
+            inside = [r for r in rows if r[0] is not None and
+                      t0 - slack <= r[0] <= t1 + slack]
+        in_region = bool(inside)
+        use = inside if inside else rows
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+        reasons = sorted({names[i] for *_, r in use for i, v in enumerate(r)
                           if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows),
-                "sm_max_mhz": max(r[1] for r in rows), "samples": len(rows),
-                "reasons": reasons}
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in use), "samples": len(use),
+                "in_timed_region": in_region, "reasons": reasons}
 
 
 # ------------------------------------------------------------- oracle -----
@@ -468,17 +502,20 @@ def dist_setup(args):
 
 def run_reference(args, wl):
     """The oracle as it stands, on the host cores, each step a bounded
-    sample of the workload."""
+    sample of the workload. A step takes a fraction of a second here, so the
+    run stops after REFERENCE_SECONDS (at least three steps) even when more
+    steps were asked for; the line gives the steps it timed."""
     torch.set_num_threads(1)
     data = make_inputs(wl)
     sample = 16
     cores = host_cores()
-    for _ in range(args.warmup):
+    for _ in range(min(args.warmup, 3)):
         oracle_step(wl, data, sample, cores)
     times = []
     desc = ""
     t0 = time.perf_counter()
-    for _ in range(args.steps):
+    while len(times) < args.steps and (
+            len(times) < 3 or time.perf_counter() - t0 < REFERENCE_SECONDS):
         est, desc = oracle_step(wl, data, sample, cores)
         times.append(est)
     wall = time.perf_counter() - t0
@@ -486,8 +523,9 @@ def run_reference(args, wl):
     value = len(wl.layers) * wl.T / per_step
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
-        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": len(times),
+        "steps_requested": args.steps, "warmup": min(args.warmup, 3),
+        "ms_per_step": per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "T": wl.T, "bits": wl.bits,
@@ -612,12 +650,14 @@ def main():
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        clk.mark_start()
         with torch.cuda.stream(stream):
             start.record()
             for i in range(args.steps):
                 graphs[i % rep].replay()
             end.record()
         torch.cuda.synchronize()
+        clk.mark_end()
     barrier()
     ms = slowest_rank_ms(start.elapsed_time(end), world, device)
     clocks = clk.summary()

@@ -231,3 +231,29 @@ def test_parity_summary_reads_the_step_buffers():
     st.Y["o"][3, 5] += 1.0
     rep = bench.parity_summary(st, outputs)
     assert rep["codes_differing"] == 1 and rep["y_rel_fro_max"] > 1e-3
+
+
+def test_clock_summary_keeps_the_samples_of_the_timed_region():
+    """nvidia-smi rows (timestamp first): the summary keeps the rows taken
+    between the marks, and falls back to all rows, flagged, if none are."""
+    import datetime
+    import bench
+    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
+
+    def row(ms, mhz, cap="Not Active"):
+        ts = (base + datetime.timedelta(milliseconds=ms)).strftime(
+            "%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return (f"{ts}, 0, {mhz}, 1965, 700.5, 0x0, Not Active, Not Active, "
+                f"Not Active, {cap}\n")
+    lines = [row(0, 1200), row(100, 1965), row(200, 1965, "Active"),
+             row(300, 1950), row(400, 1000)]
+    t0 = base + datetime.timedelta(milliseconds=90)
+    t1 = base + datetime.timedelta(milliseconds=310)
+    s = bench.ClockSampler.summarize(lines, t0, t1)
+    assert s["samples"] == 3 and s["in_timed_region"]
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    late = base + datetime.timedelta(seconds=9)
+    s = bench.ClockSampler.summarize(lines, late, late)
+    assert s["samples"] == 5 and not s["in_timed_region"]
+    assert bench.ClockSampler.summarize(["garbage\n"]) is None
