@@ -60,6 +60,8 @@ def _load():
         lib.oracle_quantize.argtypes = [P, I64, I64, I64, P, I, I, P, P, P]
         lib.oracle_count_near_ties.argtypes = [P, I64, I64, I64, P, I, I]
         lib.oracle_count_near_ties.restype = I64
+        lib.oracle_near_tie_mask.argtypes = [P, I64, I64, I64, P, I, I, P, P]
+        lib.oracle_near_tie_mask.restype = I64
         lib.oracle_dequantize.argtypes = [P, P, P, I64, I64, I, I, P]
         lib.oracle_lowbit_gemm.argtypes = [P, I64, I64, I64, P, I64, P, P, P,
                                            P, I64, I, I, P, P, I, P]
@@ -116,12 +118,33 @@ def quantize(W, s, bits: int, group: int):
 
 
 def count_near_ties(W, s, bits: int, group: int) -> int:
-    """Weights whose pre-round value is within 1 fp32 ulp of a .5 boundary."""
+    """Weights whose pre-round quotient w/D is within one fp32 step of a
+    half-integer (see near_tie_mask)."""
     W = _f32(W)
     N, K = W.shape
     s32 = None if s is None else _f32(s)
     return int(_load().oracle_count_near_ties(_ptr(W), N, K, K, _ptr(s32),
                                               bits, group))
+
+
+def near_tie_mask(W, s, bits: int, group: int):
+    """Where two valid fp32 evaluations of the quantizer may disagree.
+
+    Returns (mask uint8 [N, K], weight_ties, group_ties): bit 0 of mask is
+    set where the weight's own quotient w/D lies within one fp32 step of a
+    half-integer, bit 1 where its group's zero-point quotient -mn/D does (any
+    code of the group may move with it); the counts are of such weights and
+    of such groups.
+    """
+    W = _f32(W)
+    N, K = W.shape
+    s32 = None if s is None else _f32(s)
+    mask = np.zeros((N, K), np.uint8)
+    groups = ctypes.c_int64(0)
+    weights = _load().oracle_near_tie_mask(_ptr(W), N, K, K, _ptr(s32), bits,
+                                           group, _ptr(mask),
+                                           ctypes.byref(groups))
+    return mask, int(weights), int(groups.value)
 
 
 def pack_codes(q, bits: int) -> np.ndarray:

@@ -15,9 +15,16 @@
  *       c_j = (1 - lambda) m_j + lambda mean_k(m_k);
  *   (c) the AWQ scale is the statistic's root raised to alpha:
  *       s_j = c_j^(alpha/p), with s_j = 1 when alpha == 0 or c_j <= 0;
- *   (d) RTN is asymmetric min-max over the range widened to contain 0, with
- *       one reciprocal 1/D per group and round-half-to-even;
+ *   (d) RTN is asymmetric min-max over the range widened to contain 0:
+ *       D = (mx - mn)/(2^b - 1), z = rint(-mn/D), q = rint(w/D) + z, each
+ *       quotient an IEEE fp32 division and rint round-half-to-even;
  *   (e) the all-zero group has D = 1, z = 0.
+ *   (f) two valid fp32 evaluations of w/D (a division, or a product with a
+ *       rounded reciprocal) can round to different codes only where the
+ *       quotient lies within one fp32 step of a half-integer; such
+ *       "near-ties" are found and counted here, per weight and, for the
+ *       zero point, per group (a zero-point near-tie can move every code of
+ *       its group).
  *
  * Precision: statistics, scales, GEMM and loss in fp64; the quantizer in
  * fp32 with IEEE operations only (compile with -ffp-contract=off, never
@@ -141,10 +148,9 @@ static void rtn_group(const float* w, int g, int bits, uint8_t* q,
   }
   float d = (mx - mn) / qmax;
   if (d == 0.0f) d = 1.0f;
-  float r = 1.0f / d;
-  float z = clampf(rintf(-mn * r), 0.0f, qmax);
+  float z = clampf(rintf(-mn / d), 0.0f, qmax);
   for (int i = 0; i < g; ++i) {
-    float v = rintf(w[i] * r) + z;
+    float v = rintf(w[i] / d) + z;
     q[i] = (uint8_t)clampf(v, 0.0f, qmax);
   }
   *delta = d;
@@ -175,35 +181,58 @@ void oracle_quantize(const float* W, int64_t N, int64_t K, int64_t ldw,
   free(w);
 }
 
-/* Counts scaled weights whose pre-round value w*r lies within one fp32 ulp
- * of a half-integer, where two valid fp32 evaluation orders may round to
- * different codes. Same arithmetic as oracle_quantize. */
-int64_t oracle_count_near_ties(const float* W, int64_t N, int64_t K,
-                               int64_t ldw, const float* s, int bits,
-                               int group) {
-  int64_t G = K / group, count = 0;
+/* 1 when the fp32 value v is a half-integer k + 1/2 or one of the two fp32
+ * neighbours of the half-integer nearest to it. */
+static int near_half(float v) {
+  float h = floorf(v) + 0.5f; /* the nearest half-integer (exact, |v| < 2^22) */
+  return v == h || nextafterf(v, INFINITY) == h ||
+         nextafterf(v, -INFINITY) == h;
+}
+
+/* Marks the near-ties of oracle_quantize's rounding, with the same
+ * arithmetic. Bit 0 of mask[n*K + j] is set where the pre-round quotient
+ * w_j/D lies within one fp32 step of a half-integer; bit 1 where the zero
+ * point's quotient -mn/D of j's group does (every code of that group may
+ * move with it). Returns the number of weight near-ties; *group_ties
+ * receives the number of groups with a zero-point near-tie. mask may be
+ * NULL. */
+int64_t oracle_near_tie_mask(const float* W, int64_t N, int64_t K,
+                             int64_t ldw, const float* s, int bits, int group,
+                             uint8_t* mask, int64_t* group_ties) {
+  int64_t G = K / group, weights = 0, groups = 0;
   const float qmax = (float)((1 << bits) - 1);
+  float* w = (float*)malloc(sizeof(float) * (size_t)group);
   for (int64_t n = 0; n < N; ++n)
     for (int64_t gi = 0; gi < G; ++gi) {
       float mn = 0.0f, mx = 0.0f;
       for (int i = 0; i < group; ++i) {
         int64_t j = gi * group + i;
-        float v = W[n * ldw + j] * (s ? s[j] : 1.0f);
-        if (v < mn) mn = v;
-        if (v > mx) mx = v;
+        w[i] = W[n * ldw + j] * (s ? s[j] : 1.0f);
+        if (w[i] < mn) mn = w[i];
+        if (w[i] > mx) mx = w[i];
       }
       float d = (mx - mn) / qmax;
       if (d == 0.0f) d = 1.0f;
-      float r = 1.0f / d;
+      int zero_tie = near_half(-mn / d);
+      groups += zero_tie;
       for (int i = 0; i < group; ++i) {
-        int64_t j = gi * group + i;
-        float v = (W[n * ldw + j] * (s ? s[j] : 1.0f)) * r;
-        double frac = fabs((double)v - floor((double)v) - 0.5);
-        if (frac <= (double)nextafterf(fabsf(v), INFINITY) - fabs((double)v))
-          ++count;
+        int weight_tie = near_half(w[i] / d);
+        weights += weight_tie;
+        if (mask)
+          mask[n * K + gi * group + i] =
+              (uint8_t)(weight_tie | (zero_tie << 1));
       }
     }
-  return count;
+  free(w);
+  if (group_ties) *group_ties = groups;
+  return weights;
+}
+
+/* Number of weight near-ties (see oracle_near_tie_mask). */
+int64_t oracle_count_near_ties(const float* W, int64_t N, int64_t K,
+                               int64_t ldw, const float* s, int bits,
+                               int group) {
+  return oracle_near_tie_mask(W, N, K, ldw, s, bits, group, NULL, NULL);
 }
 
 /* Scaled-domain dequantized weight What_s[n][j] = (q - z) * D in fp64. */

@@ -3,10 +3,14 @@
 // TTQ review, "Proposed method", bullet 1: weights are quantized on the fly
 // with group-wise round-to-nearest. Per group of g input channels of one
 // weight row, in fp32 with explicit round-to-nearest-even operations (no
-// contraction into FMA), exactly as ttq.h states:
+// contraction into FMA), as ttq.h states:
 //   w = W*s;  mn = min(0, min w);  mx = max(0, max w);
-//   D = (mx - mn)/(2^b - 1) (1 if 0);  r = 1/D;
-//   z = clamp(rint(-mn*r));  q = clamp(rint(w*r) + z).
+//   D = (mx - mn)/(2^b - 1) (1 if 0);
+//   z = clamp(rint(-mn/D));  q = clamp(rint(w*r) + z),  r = RN(1/D).
+// The zero point takes the IEEE quotient, once per group. The codes take
+// the product with the rounded reciprocal: it lies within one fp32 step of
+// the IEEE quotient w/D, so a code can differ from rint(w/D) + z only where
+// that quotient is within one step of a half-integer (a near-tie).
 //
 // Design (HBM-bound, kept below the instruction budget): one lane per
 // 32-code block, i.e. 32 consecutive channels of one weight row, loaded as
@@ -15,7 +19,7 @@
 // blocks of the [N, K/32] block grid, so a warp reads and writes contiguous
 // spans. A group of g >= 32 channels spans g/32 neighbouring lanes and its
 // range is a 1- or 2-level shuffle; with g = 16 a lane holds two groups.
-// The IEEE divide and reciprocal of a group run once per 32 elements.
+// The IEEE divides and the reciprocal of a group run once per 32 elements.
 #include <algorithm>
 #include <type_traits>
 
@@ -222,9 +226,9 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
     if (dd == 0.f) dd = 1.f;
     d[gi] = dd;
     r[gi] = __frcp_rn(dd);
-    // clamp(rint(-mn * r), 0, 2^b - 1); rint(-mn * r) lies in that range
+    // clamp(rint(-mn / D), 0, 2^b - 1); rint(-mn / D) lies in that range
     // already because -mn <= mx - mn, the clamp matches the definition
-    zf[gi] = fminf(fmaxf(__fadd_rn(__fmul_rn(-mn, r[gi]), kMagic), kMagic),
+    zf[gi] = fminf(fmaxf(__fadd_rn(__fdiv_rn(-mn, dd), kMagic), kMagic),
                    kTop) - kMagic;
     // q = min(rint(w*r) + z, 2^b - 1) <=> M + q - z = min(M + rint(w*r),
     // M + 2^b - 1 - z); q >= 0 since rint(w*r) >= rint(mn*r) = -z

@@ -33,9 +33,15 @@ MISTAKES = [
      "float mn = 0.0f, mx = 0.0f; /* the range always contains 0 */",
      "float mn = w[0], mx = w[0];"),
     ("no_zero_point",
-     "float z = clampf(rintf(-mn * r), 0.0f, qmax);", "float z = 0.0f;"),
+     "float z = clampf(rintf(-mn / d), 0.0f, qmax);", "float z = 0.0f;"),
     ("round_half_away_from_zero",
-     "float v = rintf(w[i] * r) + z;", "float v = roundf(w[i] * r) + z;"),
+     "float v = rintf(w[i] / d) + z;", "float v = roundf(w[i] / d) + z;"),
+    ("quotient_by_rounded_reciprocal",
+     "float v = rintf(w[i] / d) + z;",
+     "float v = rintf(w[i] * (1.0f / d)) + z;"),
+    ("zero_point_by_rounded_reciprocal",
+     "float z = clampf(rintf(-mn / d), 0.0f, qmax);",
+     "float z = clampf(rintf(-mn * (1.0f / d)), 0.0f, qmax);"),
     ("clamp_one_code_short",
      "q[i] = (uint8_t)clampf(v, 0.0f, qmax);",
      "q[i] = (uint8_t)clampf(v, 0.0f, qmax - 1.0f);"),
@@ -61,8 +67,14 @@ MISTAKES = [
     ("loss_not_divided_by_T",
      "return total / (double)T;", "return total;"),
     ("near_ties_never_counted",
-     "if (frac <= (double)nextafterf(fabsf(v), INFINITY) - fabs((double)v))",
-     "if (frac < 0.0)"),
+     "int weight_tie = near_half(w[i] / d);", "int weight_tie = 0;"),
+    ("near_ties_counted_two_steps_out",
+     "return v == h || nextafterf(v, INFINITY) == h ||",
+     "return v == h || nextafterf(nextafterf(v, INFINITY), INFINITY) == h ||"
+     " nextafterf(nextafterf(v, -INFINITY), -INFINITY) == h ||"
+     " nextafterf(v, INFINITY) == h ||"),
+    ("zero_point_near_ties_ignored",
+     "int zero_tie = near_half(-mn / d);", "int zero_tie = 0;"),
 ]
 
 

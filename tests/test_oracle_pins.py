@@ -9,6 +9,7 @@ bullets 1-5.
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -390,3 +391,156 @@ def test_near_tie_counter_sees_exact_ties():
     W = np.zeros((1, 32), np.float32)
     W[0, :4] = [-1.0, 2.0, 0.5, 1.5]      # D = 1: 0.5 and 1.5 are ties
     assert oracle.count_near_ties(W, None, 2, 16) >= 2
+
+
+# ------------------------------------------- RTN by its exact definition ---
+# Group RTN divides: q = rint(w/D) + z and z = rint(-mn/D), each quotient
+# one IEEE fp32 division (correctly rounded) and rint round-half-to-even.
+# The references below evaluate that definition in exact rational
+# arithmetic, rounding to fp32 by hand, so they share no floating-point
+# operation with the oracle.
+
+def _rn32(x: Fraction) -> float:
+    """x rounded to the nearest fp32 value, ties to even."""
+    if x == 0:
+        return 0.0
+    a = abs(x)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    step = Fraction(2) ** (max(e, -126) - 23)
+    m = a / step
+    f = m.numerator // m.denominator
+    rem = m - f
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and f % 2 == 1):
+        f += 1
+    return math.copysign(float(f * step), float(x))
+
+
+def _exact_rtn_group(w, bits):
+    """(codes, D, z) of one group of fp32 scaled weights, exactly."""
+    qmax = (1 << bits) - 1
+    mn = min(0.0, float(w.min()))
+    mx = max(0.0, float(w.max()))
+    d = _rn32(Fraction(_rn32(Fraction(mx) - Fraction(mn))) / qmax)
+    if d == 0.0:
+        d = 1.0
+    z = min(max(round(_rn32(Fraction(-mn) / Fraction(d))), 0), qmax)
+    q = [min(max(round(_rn32(Fraction(float(v)) / Fraction(d))) + z, 0), qmax)
+         for v in w]
+    return q, d, z
+
+
+def _reciprocal_disagreements(seed, bits, count):
+    """Groups where rint(x * (1/D)) and rint(x / D) differ, found by a
+    seeded search over random (min, max, weight) triples in numpy fp32:
+    rows of 32 weights [mn, mx, w, 0, ...] whose first group's zero point
+    or third weight rounds differently under the two."""
+    rng = np.random.default_rng(seed)
+    M = 1 << 22
+    qmax = np.float32((1 << bits) - 1)
+    mn = -np.abs(rng.standard_normal(M)).astype(np.float32)
+    mx = np.abs(rng.standard_normal(M)).astype(np.float32)
+    w = (rng.uniform(-1, 1, M).astype(np.float32) *
+         np.maximum(-mn, mx)).astype(np.float32)
+    w = np.clip(w, mn, mx)
+    d = (mx - mn) / qmax
+    r = np.float32(1) / d
+    zero_idx = np.nonzero(np.rint(-mn / d) != np.rint(-mn * r))[0][:count]
+    weight_idx = np.nonzero(np.rint(w / d) != np.rint(w * r))[0][:count]
+    rows = []
+    for i in np.concatenate([zero_idx, weight_idx]):
+        row = np.zeros(32, np.float32)   # a second, all-zero group
+        row[:3] = [mn[i], mx[i], w[i]]
+        rows.append(row)
+    return np.array(rows, np.float32), len(zero_idx), len(weight_idx)
+
+
+@pytest.mark.parametrize("bits,seed", [(8, 40), (7, 41)])
+def test_quantize_is_rtn_by_division_not_by_reciprocal(bits, seed):
+    """On groups where a rounded reciprocal would change the zero point or a
+    code, the oracle gives the exact rounding of the quotients. (Such groups
+    are rarer at fewer bits, where the quotients are smaller.)"""
+    W, n_zero, n_weight = _reciprocal_disagreements(seed, bits, 12)
+    assert n_zero >= 3 and n_weight >= 3, (n_zero, n_weight)
+    codes, delta, zero = oracle.quantize(W, None, bits, 16)
+    q = oracle.unpack_codes(codes, 32, bits)
+    for n in range(W.shape[0]):
+        eq, ed, ez = _exact_rtn_group(W[n, :16], bits)
+        assert float(delta[n, 0]) == ed, n
+        assert int(zero[n, 0]) == ez, n
+        assert list(q[n, :16]) == eq, n
+
+
+def test_quantize_matches_exact_definition_on_random_groups():
+    rng = np.random.default_rng(12)
+    for bits, group in ((2, 16), (3, 32), (5, 64), (8, 128)):
+        W = (rng.standard_normal((3, 256)) * 0.02).astype(np.float32)
+        s = np.exp(rng.standard_normal(256) * 0.6).astype(np.float32)
+        codes, delta, zero = oracle.quantize(W, s, bits, group)
+        q = oracle.unpack_codes(codes, 256, bits)
+        Ws = W * s[None, :]
+        for n in range(3):
+            for gi in range(256 // group):
+                sl = slice(gi * group, (gi + 1) * group)
+                eq, ed, ez = _exact_rtn_group(Ws[n, sl], bits)
+                assert float(delta[n, gi]) == ed
+                assert int(zero[n, gi]) == ez
+                assert list(q[n, sl]) == eq
+
+
+def _steps_from(v, k):
+    """The fp32 value k representable steps from v (k may be negative)."""
+    out = np.float32(v)
+    for _ in range(abs(k)):
+        out = np.nextafter(out, np.float32(np.inf if k > 0 else -np.inf),
+                           dtype=np.float32)
+    return out
+
+
+def test_near_tie_mask_is_one_step_wide():
+    """D = 1 exactly (b = 4, range [0, 15]), so each quotient is the weight
+    itself: the tie and its two neighbours count, two and three steps away
+    do not."""
+    W = np.zeros((1, 16), np.float32)
+    W[0, 0] = 15.0
+    offsets = [0, 1, -1, 2, -2, 3]
+    for i, k in enumerate(offsets):
+        W[0, 1 + i] = _steps_from(2.5, k)
+    W[0, 7] = 3.0
+    _, delta, _ = oracle.quantize(W, None, 4, 16)
+    assert delta[0, 0] == 1.0
+    mask, weights, groups = oracle.near_tie_mask(W, None, 4, 16)
+    assert list(mask[0, 1:7]) == [1, 1, 1, 0, 0, 0]
+    assert mask[0, 0] == 0 and mask[0, 7] == 0
+    assert weights == 3 and groups == 0
+    assert oracle.count_near_ties(W, None, 4, 16) == 3
+
+
+def test_near_tie_mask_counts_zero_point_groups():
+    """Three groups with D = 1 (b = 4) whose zero-point quotient -mn/D is
+    2.5 exactly, one step above it, and three steps above it: the first two
+    are zero-point near-ties and every weight of theirs is marked."""
+    mns = [np.float32(-2.5), -_steps_from(2.5, 1), -_steps_from(2.5, 3)]
+    mxs = [np.float32(12.5), np.float32(12.5),
+           np.float32(12.5) - np.float32(2.0 ** -20)]
+    W = np.zeros((3, 16), np.float32)
+    W[:, 3:] = 1.0
+    for n in range(3):
+        W[n, 0], W[n, 1] = mns[n], mxs[n]
+    _, delta, zero = oracle.quantize(W, None, 4, 16)
+    assert np.all(delta == 1.0)
+    # the construction: quotients 2.5, one step and three steps above it
+    assert [int(np.round((-W[n, 0] - np.float32(2.5)) /
+                         np.float32(2.0 ** -22))) for n in range(3)] == \
+        [0, 1, 3]
+    mask, weights, groups = oracle.near_tie_mask(W, None, 4, 16)
+    assert groups == 2
+    assert np.all(mask[:2] != 0)          # whole groups excused
+    # mn and mx are themselves weights within a step of -2.5 and 12.5
+    assert list(mask[0, :2]) == [3, 3] and list(mask[1, :2]) == [3, 3]
+    assert np.all(mask[:2, 2:] == 2)
+    assert mask[2, 1] == 1 and mask[2, 0] == 0 and np.all(mask[2, 2:] == 0)
+    assert weights == 5

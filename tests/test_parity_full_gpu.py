@@ -12,7 +12,8 @@ import pytest
 import torch
 
 import oracle
-from parity_util import assert_gemm_close, assert_rel_close, np32
+from parity_util import (assert_codes_match, assert_gemm_close,
+                         assert_rel_close, np32)
 
 pytestmark = pytest.mark.gpu
 
@@ -60,9 +61,8 @@ def check_layer(ttq, wl, name, X, W, A, B, bits, group, T_tok, qrows,
     Wn = np32(W) if rows is None else np32(W)[rows]
     rc, rd, rz = oracle.quantize(Wn, np32(s), bits, group)
     gc, gd, gz = dense(c, d, z, K, bits, group, rows)
-    np.testing.assert_array_equal(gd, rd, err_msg=f"{name} delta")
-    np.testing.assert_array_equal(gz, rz, err_msg=f"{name} zero")
-    np.testing.assert_array_equal(gc, rc, err_msg=f"{name} codes")
+    assert_codes_match(gc, gd, gz, rc, rd, rz, Wn, np32(s), bits, group,
+                       f"{name} codes")
     # the oracle's own scales (fp64, stored as fp32) differ from the GPU's by
     # an fp32 ulp or two on some channels; codes may move only where that
     # shifts w*s/D across a rounding boundary, a few per million
@@ -122,12 +122,12 @@ def test_decode_sweep_full_size(ttq):
                 s, inv = ttq.awq_scales(sums, X.shape[0])
                 c, d, z = ttq.quantize_rtn_grouped(W.cuda(), s, bits, group)
                 rows = sample_rows(layer.N, 24, bits * 100 + group)
-                rc, rd, rz = oracle.quantize(np32(W)[rows], np32(s), bits,
-                                             group)
+                Wn = np32(W)[rows]
+                rc, rd, rz = oracle.quantize(Wn, np32(s), bits, group)
                 gc, gd, gz = dense(c, d, z, layer.K, bits, group, rows)
-                np.testing.assert_array_equal(gc, rc)
-                np.testing.assert_array_equal(gd, rd)
-                np.testing.assert_array_equal(gz, rz)
+                assert_codes_match(gc, gd, gz, rc, rd, rz, Wn, np32(s), bits,
+                                   group, f"decode b={bits} g={group} "
+                                   f"{layer.name}")
                 cd, dd, zd = dense(c, d, z, layer.K, bits, group)
                 # one decode width per (b, g, layer) keeps the oracle short;
                 # across the sweep every width meets every layer
