@@ -7,29 +7,28 @@ every distinct layer input, statistics and scales (one launch) -> prepared
 fp16 operand; for every layer, group RTN of its weight -> tensor-core
 low-bit projection. Layers that share an input run as one projection of
 their stacked weights, and the prepared operand is built on a second stream
-while the weights are quantized. The default workload is an OPT-125M-shaped
-block (q, k, v, o 768x768, fc1 3072x768, fc2 768x3072; q, k, v share one
-input), T = 2048, b = 3, g = 32.
+while the weights are quantized. The default workload is the largest one
+that fits one GPU: Llama-7B-shaped prefill layers (attn 4096x4096, up
+11008x4096, down 4096x11008), T = 4096, b = 4, g = 128.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
 
 With N > 1 (launched by torchrun) every rank runs an independent replica
 (the path has no exchange step), the timed region is bracketed by a barrier
 and a device synchronisation, and the slowest rank's time counts.
-Rank 0 prints one JSON line.
+Rank 0 prints one JSON line. ``--impl reference`` times the CPU oracle
+instead (rank 0 only), each step the whole path on a bounded prompt sample.
 """
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import torch
@@ -41,20 +40,29 @@ from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs  # noqa
 
 METRIC = "prompt tokens/s per layer incl. on-the-fly quant"
 L2_BYTES = 126 * 1024 * 1024
+# prompt tokens of the oracle's sample step (the whole path on a prompt of
+# this many tokens of the workload's inputs)
 ORACLE_SAMPLE_TOKENS = 128
-REFERENCE_SECONDS = 60.0
+# the oracle's CPU baseline repeats its sample step for at least this long
+CPU_BASELINE_SECONDS = 10.0
+# the reference arm shrinks its sample so that warm-up and steps together
+# take about this long
+REFERENCE_BUDGET_SECONDS = 150.0
+# a timed region at least this long is compared with the sustained tensor
+# peak, a shorter one with the burst peak
+SUSTAINED_REGION_SECONDS = 1.0
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # 5000 steps of ~0.13 ms keep the GPU busy for ~0.6 s, long enough for
-    # several clock samples inside the timed region
-    ap.add_argument("--steps", type=int, default=5000)
+    # about 1 ms per Llama-sized step: 1000 steps take about a second
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="opt125m-block",
-                    choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="llama7b-prefill",
+                    choices=sorted(w for w in WORKLOADS
+                                   if w != "decode-sweep"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--eager", action="store_true",
@@ -266,92 +274,106 @@ def algorithmic_work(wl):
 # -------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    """nvidia-smi samples every 100 ms; the summary keeps the samples taken
-    between mark_start() and mark_end() (all of them, flagged, if none
-    fell inside)."""
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,"
-              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the active clock-event (throttle) reasons of
+    one GPU through NVML every ``period`` seconds on a background thread
+    (read-only queries). The summary keeps the samples taken between
+    mark_start() and mark_end(); if none fell inside, all samples, flagged.
+    """
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, cuda_index, period=0.002):
+        self.cuda_index = cuda_index
+        self.period = period
+        self.samples = []      # (monotonic seconds, sm MHz, reason bits)
+        self.max_mhz = None
         self.t0 = self.t1 = None
+        self._stop = None
+        self._thread = None
+        self._nvml = None
 
-    def mark_start(self):
-        self.t0 = datetime.datetime.now()
-
-    def mark_end(self):
-        self.t1 = datetime.datetime.now()
+    def _handle(self, nvml):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.cuda_index).uuid)
+            return nvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def __enter__(self):
+        import threading
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu),
-                 f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-f", self.path],
-                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nvml
+            nvml.nvmlInit()
+            h = self._handle(nvml)
+            self.max_mhz = float(nvml.nvmlDeviceGetMaxClockInfo(
+                h, nvml.NVML_CLOCK_SM))
+        except Exception:
+            return self
+        self._nvml = nvml
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    mhz = nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM)
+                    bits = nvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    break
+                self.samples.append((time.monotonic(), float(mhz), int(bits)))
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        time.sleep(0.05)
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        if self._nvml is not None:
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def summary(self):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
+        if self.max_mhz is None:
             return None
-        with open(self.path) as f:
-            lines = f.readlines()
-        os.unlink(self.path)
-        return self.summarize(lines, self.t0, self.t1)
+        return self.summarize(self.samples, self.max_mhz, self.t0, self.t1)
 
-    @staticmethod
-    def summarize(lines, t0=None, t1=None):
-        """Median SM clock, max clock and active throttle reasons of the CSV
-        rows (timestamp first) that fall in [t0, t1]."""
-        rows = []
-        for line in lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 10:
-                continue
-            try:
-                ts = datetime.datetime.strptime(parts[0],
-                                                "%Y/%m/%d %H:%M:%S.%f")
-            except ValueError:
-                ts = None
-            try:
-                rows.append((ts, float(parts[2]), float(parts[3]),
-                             parts[6:10]))
-            except ValueError:
-                continue
-        if not rows:
+    @classmethod
+    def summarize(cls, samples, max_mhz, t0=None, t1=None):
+        """Median SM clock, the maximum clock and the active reasons of the
+        samples (time, MHz, reason bits) that fall in [t0, t1]."""
+        if not samples:
             return None
-        inside = rows
+        inside = samples
         if t0 is not None and t1 is not None:
-            slack = datetime.timedelta(milliseconds=50)
-            inside = [r for r in rows if r[0] is not None and
-                      t0 - slack <= r[0] <= t1 + slack]
-        in_region = bool(inside)
-        use = inside if inside else rows
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        reasons = sorted({names[i] for *_, r in use for i, v in enumerate(r)
-                          if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[1] for r in use),
-                "sm_max_mhz": max(r[2] for r in use), "samples": len(use),
-                "in_timed_region": in_region, "reasons": reasons}
+            inside = [x for x in samples if t0 <= x[0] <= t1]
+        use = inside if inside else samples
+        reasons = sorted({name for _, _, bits in use
+                          for name, bit in cls.REASONS if bits & bit})
+        return {"sm_mhz": statistics.median(x[1] for x in use),
+                "sm_max_mhz": max_mhz, "samples": len(use),
+                "in_timed_region": bool(inside), "reasons": reasons,
+                "source": "NVML, every %g ms" % (cls_period_ms(use))}
+
+
+def cls_period_ms(samples):
+    """Median spacing of the samples, in ms (0 for fewer than two)."""
+    if len(samples) < 2:
+        return 0.0
+    gaps = [b[0] - a[0] for a, b in zip(samples, samples[1:])]
+    return round(statistics.median(gaps) * 1e3, 2)
 
 
 # ------------------------------------------------------------- oracle -----
@@ -371,22 +393,22 @@ def _ranges(n, parts):
     return [(b[i], b[i + 1]) for i in range(parts)]
 
 
-def oracle_step(wl, data, sample_tokens, threads=1, outputs=None):
-    """The CPU oracle on a bounded sample of one step: statistics, scales and
-    quantization at full size, the projection on the first ``sample_tokens``
-    tokens, scaled linearly to T. Returns (seconds per step, description).
+def oracle_step(wl, data, tokens, threads=1, outputs=None):
+    """The CPU oracle on a bounded sample of one step: the whole path for a
+    prompt made of the first ``tokens`` tokens of every layer input
+    (statistics and scales over those tokens, group RTN of the full
+    weights, projection of those tokens). Returns (seconds, description).
 
     With ``threads`` > 1 the unchanged oracle functions run concurrently on
     disjoint slices: the statistics over token ranges (the partial sums are
     added), the quantizer and the projection over output rows. The C calls
     release the GIL. ``outputs``, when a dict, receives every layer's
-    (codes, delta, zero, Y sample) for checking."""
+    (codes, delta, zero, Y) for checking."""
     import numpy as np
     import oracle
     from concurrent.futures import ThreadPoolExecutor
-    T = wl.T
-    Ts = min(sample_tokens, T)
-    Xn = {k: v.float().numpy() for k, v in data["X"].items()}
+    Ts = min(tokens, wl.T)
+    Xn = {k: v[:Ts].float().numpy() for k, v in data["X"].items()}
     pool = ThreadPoolExecutor(threads) if threads > 1 else None
 
     def each(fn, n):
@@ -399,71 +421,137 @@ def oracle_step(wl, data, sample_tokens, threads=1, outputs=None):
         t0 = time.perf_counter()
         s, inv = {}, {}
         for k, X in Xn.items():
-            sums = sum(each(lambda a, b: oracle.act_sums(X[a:b], wl.p), T))
-            s[k], inv[k] = oracle.awq_scales(sums, T, wl.alpha, wl.lam, wl.p)
-        t_full = time.perf_counter() - t0
-        t_gemm = 0.0
+            sums = sum(each(lambda a, b: oracle.act_sums(X[a:b], wl.p), Ts))
+            s[k], inv[k] = oracle.awq_scales(sums, Ts, wl.alpha, wl.lam, wl.p)
         for L in wl.layers:
             W = data["W"][L.name].float().numpy()
             s32 = s[L.input_name].astype(np.float32)
-            t1 = time.perf_counter()
             parts = each(lambda a, b: oracle.quantize(W[a:b], s32, wl.bits,
                                                       wl.group), L.N)
             c, d, z = (np.concatenate(x) for x in zip(*parts))
-            t_full += time.perf_counter() - t1
             A = B = None
             if wl.rank:
                 A = data["A"][L.name].float().numpy()
                 B = data["B"][L.name].float().numpy()
-            Xs = Xn[L.input_name][:Ts]
-            t2 = time.perf_counter()
+            X = Xn[L.input_name]
             ys = each(lambda a, b: oracle.lowbit_gemm(
-                Xs, inv[L.input_name], c[a:b], d[a:b], z[a:b], b - a, wl.bits,
+                X, inv[L.input_name], c[a:b], d[a:b], z[a:b], b - a, wl.bits,
                 wl.group, A, None if B is None else B[a:b]), L.N)
-            t_gemm += time.perf_counter() - t2
             if outputs is not None:
                 outputs[L.name] = (c, d, z, np.concatenate(ys, axis=1))
+        seconds = time.perf_counter() - t0
     finally:
         if pool is not None:
             pool.shutdown()
-    est = t_full + t_gemm * (T / Ts)
     how = ("1 thread" if threads == 1 else
            f"{threads} threads on disjoint token ranges (statistics) and "
            f"output rows (quantizer, projection)")
-    desc = (f"stats, scales and quantize at full size; projection on {Ts} of "
-            f"{T} tokens scaled x{T / Ts:g}; {how}")
-    return est, desc
+    desc = (f"the whole path (statistics, scales, group RTN of the full "
+            f"weights, projection) on a prompt of the first {Ts} of the "
+            f"{wl.T} tokens; {how}")
+    return seconds, desc
 
 
-def parity_summary(step, outputs):
-    """The timed step's codes and sampled outputs against the oracle's (the
-    oracle with its own statistics and scales, on the tokens of its sample).
-    Every replica holds the same inputs, so the buffers of the last replay
-    are the step's result."""
+def cpu_baseline(wl, data, threads, min_seconds=CPU_BASELINE_SECONDS,
+                 tokens=ORACLE_SAMPLE_TOKENS):
+    """The oracle's sample step repeated for at least ``min_seconds`` (and
+    at least twice); tokens/s per layer over the steps it ran."""
+    times, desc = [], ""
+    while len(times) < 2 or sum(times) < min_seconds:
+        sec, desc = oracle_step(wl, data, tokens, threads)
+        times.append(sec)
+    Ts = min(tokens, wl.T)
+    return {"value": len(wl.layers) * Ts * len(times) / sum(times),
+            "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{desc}; {len(times)} steps, "
+                      f"{sum(times):.1f} s"}
+
+
+def parity_summary(step, threads=1, qrows=64, ytokens=8, seed=5):
+    """The timed step's results against the oracle, on the step's own
+    inputs and upstream outputs: the statistics of every input in full;
+    the scales from the GPU's sums; for every projection the codes of
+    ``qrows`` sampled weight rows (quantized by the oracle with the GPU's
+    scales; bit-exact apart from the near-ties the oracle marks) and every
+    output channel of ``ytokens`` sampled tokens (the oracle's projection
+    of the GPU's codes). Every replica holds the same inputs, so the buffers
+    of the last replay are the step's result."""
     import numpy as np
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     wl = step.wl
-    moved = total = 0
-    worst = 0.0
-    tokens = 0
-    for g, _, Ls in step.groups:
-        codes = step.codes[g].cpu().numpy().view(np.uint32)
-        Y = step.Y[g].float().cpu().numpy()
-        row = 0
-        for L in Ls:
-            oc, _, _, oy = outputs[L.name]
-            gq = oracle.unpack_codes(codes[row:row + L.N, :oc.shape[1]], L.K,
-                                     wl.bits)
-            moved += int(np.count_nonzero(gq != oracle.unpack_codes(
-                oc, L.K, wl.bits)))
-            total += gq.size
-            tokens = oy.shape[0]
-            ys = Y[:tokens, row:row + L.N].astype(np.float64)
-            worst = max(worst, float(np.linalg.norm(ys - oy) /
-                                     max(np.linalg.norm(oy), 1e-300)))
-            row += L.N
-    return {"codes_differing": moved, "codes": total,
-            "y_tokens": tokens, "y_rel_fro_max": worst}
+    rng = np.random.default_rng(seed)
+    rep = {"stats_rel_max": 0.0, "scales_rel_max": 0.0, "codes": 0,
+           "codes_differing": 0, "codes_differing_off_near_ties": 0,
+           "weight_near_ties": 0, "zero_point_near_tie_groups": 0,
+           "delta_differing": 0, "y_tokens": 0, "y_rel_fro_max": 0.0}
+
+    def rel(a, b):
+        b = np.asarray(b, np.float64)
+        return float(np.max(np.abs(np.asarray(a, np.float64) - b) /
+                            np.maximum(np.abs(b), 1e-30)))
+
+    pool = ThreadPoolExecutor(threads) if threads > 1 else None
+    try:
+        for k in step.inputs:
+            X = step.X[0][k].float().cpu().numpy()
+            sums = step.sums[k].cpu().numpy()
+            rep["stats_rel_max"] = max(rep["stats_rel_max"], rel(
+                sums, oracle.act_sums(X, wl.p)))
+            rs, _ = oracle.awq_scales(sums.astype(np.float64), wl.T,
+                                      wl.alpha, wl.lam, wl.p)
+            rep["scales_rel_max"] = max(rep["scales_rel_max"], rel(
+                step.s[k].cpu().numpy(), rs))
+        for g, k, Ls in step.groups:
+            K = Ls[0].K
+            N = step.N[g]
+            W = step.W[0][g].float().cpu().numpy()
+            s32 = step.s[k].cpu().numpy()
+            inv32 = step.inv[k].cpu().numpy()
+            words, G = K * wl.bits // 32, K // wl.group
+            codes = step.codes[g].cpu().numpy().view(np.uint32)[:, :words]
+            delta = step.delta[g].cpu().numpy()[:, :G]
+            zero = step.zero[g].cpu().numpy()[:, :G]
+            rows = np.sort(rng.choice(N, size=min(qrows, N), replace=False))
+            rc, rd, rz = oracle.quantize(W[rows], s32, wl.bits, wl.group)
+            mask, wt, gt = oracle.near_tie_mask(W[rows], s32, wl.bits,
+                                                wl.group)
+            diff = oracle.unpack_codes(codes[rows], K, wl.bits) != \
+                oracle.unpack_codes(rc, K, wl.bits)
+            rep["codes"] += diff.size
+            rep["codes_differing"] += int(diff.sum())
+            rep["codes_differing_off_near_ties"] += int(
+                (diff & (mask == 0)).sum())
+            rep["weight_near_ties"] += wt
+            rep["zero_point_near_tie_groups"] += gt
+            rep["delta_differing"] += int((delta[rows] != rd).sum())
+            inner = np.arange(1, wl.T - 1)
+            tok = np.unique(np.concatenate([[0, wl.T - 1], rng.choice(
+                inner, size=min(max(0, ytokens - 2), inner.size),
+                replace=False)])).astype(np.int64)
+            X = step.X[0][k].float().cpu().numpy()[tok]
+            A = B = None
+            if wl.rank:
+                A = step.A[g].float().cpu().numpy()
+                B = step.B[g].float().cpu().numpy()
+
+            def part(ab):
+                a, b = ab
+                return oracle.lowbit_gemm(
+                    X, inv32, codes[a:b], delta[a:b], zero[a:b], b - a,
+                    wl.bits, wl.group, A, None if B is None else B[a:b])
+            pieces = _ranges(N, threads)
+            ys = list(pool.map(part, pieces)) if pool else \
+                [part(ab) for ab in pieces]
+            ref = np.concatenate(ys, axis=1)
+            Y = step.Y[g].float().cpu().numpy()[tok].astype(np.float64)
+            rep["y_tokens"] = len(tok)
+            rep["y_rel_fro_max"] = max(rep["y_rel_fro_max"], float(
+                np.linalg.norm(Y - ref) / max(np.linalg.norm(ref), 1e-300)))
+    finally:
+        if pool is not None:
+            pool.shutdown()
+    return rep
 
 
 # -------------------------------------------------------- aggregation ----
@@ -501,42 +589,78 @@ def dist_setup(args):
 
 
 def run_reference(args, wl):
-    """The oracle as it stands, on the host cores, each step a bounded
-    sample of the workload. A step takes a fraction of a second here, so the
-    run stops after REFERENCE_SECONDS (at least three steps) even when more
-    steps were asked for; the line gives the steps it timed."""
+    """The oracle as it stands, on every host core, each step the whole path
+    on a bounded prompt sample (ORACLE_SAMPLE_TOKENS tokens, the sample of
+    the GPU arm's cpu_baseline). When warm-up and steps together would take
+    longer than REFERENCE_BUDGET_SECONDS the sample shrinks in proportion,
+    judged from one untimed calibration step. ms_per_step is the measured
+    wall time per timed step; value is the tokens those steps processed per
+    second per layer."""
     torch.set_num_threads(1)
     data = make_inputs(wl)
-    sample = 16
     cores = host_cores()
-    for _ in range(min(args.warmup, 3)):
-        oracle_step(wl, data, sample, cores)
-    times = []
-    desc = ""
+    tokens = min(ORACLE_SAMPLE_TOKENS, wl.T)
+    t_cal, _ = oracle_step(wl, data, tokens, cores)
+    total = (args.steps + args.warmup) * t_cal
+    if total > REFERENCE_BUDGET_SECONDS:
+        tokens = max(1, int(tokens * REFERENCE_BUDGET_SECONDS / total))
+    for _ in range(args.warmup):
+        oracle_step(wl, data, tokens, cores)
+    times, desc = [], ""
     t0 = time.perf_counter()
-    while len(times) < args.steps and (
-            len(times) < 3 or time.perf_counter() - t0 < REFERENCE_SECONDS):
-        est, desc = oracle_step(wl, data, sample, cores)
-        times.append(est)
+    for _ in range(args.steps):
+        sec, desc = oracle_step(wl, data, tokens, cores)
+        times.append(sec)
     wall = time.perf_counter() - t0
-    per_step = sum(times) / len(times)
-    value = len(wl.layers) * wl.T / per_step
+    per_step = wall / max(1, len(times))
+    value = len(wl.layers) * tokens / per_step
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": len(times),
-        "steps_requested": args.steps, "warmup": min(args.warmup, 3),
-        "ms_per_step": per_step * 1e3,
+        "warmup": args.warmup, "ms_per_step": per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "T": wl.T, "bits": wl.bits,
-                   "group": wl.group, "layers": len(wl.layers)},
+        "config": workload_config(wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
-        "wall_s": wall,
+        "sample_tokens": tokens, "wall_s": wall,
     }
     print(json.dumps(line), flush=True)
+
+
+def input_bytes(wl):
+    """Bytes of one replica's inputs: every distinct layer input and every
+    weight, at the workload's storage type."""
+    xb = 4 if wl.dtype == torch.float32 else 2
+    ks = {L.input_name: L.K for L in wl.layers}
+    return (sum(wl.T * K * xb for K in ks.values()) +
+            sum(L.N * L.K * xb for L in wl.layers) +
+            sum(wl.rank * (L.N + L.K) * xb for L in wl.layers))
+
+
+def replicas_for(wl):
+    """Input replicas the timed loop rotates over: together at least 2.5x
+    the L2 cache, so every step reads its inputs from HBM."""
+    return max(2, math.ceil(2.5 * L2_BYTES / input_bytes(wl)))
+
+
+def workload_config(wl, n_gpus):
+    """The ``config`` of the JSON line (both arms print the same)."""
+    rep = replicas_for(wl)
+    return {
+        "workload": wl.name, "T": wl.T, "bits": wl.bits, "group": wl.group,
+        "alpha": wl.alpha, "lambda": wl.lam, "p": wl.p, "rank": wl.rank,
+        "layers": ", ".join(f"{L.name} {L.N}x{L.K}" for L in wl.layers),
+        "projections": ", ".join(f"{g} {sum(L.N for L in Ls)}x{Ls[0].K}"
+                                 for g, _, Ls in projection_groups(wl)),
+        "operands": "fp16 x fp16 -> fp32 (tensor cores); quantizer fp32; "
+                    "statistics fp32",
+        "l2": f"inputs rotate over {rep} replicas "
+              f"({rep * input_bytes(wl) / 2**20:.0f} MiB > L2)",
+        "parallelism": f"independent replicas x{n_gpus}",
+    }
 
 
 # The sources a kernel's counters depend on (its file and the headers it
@@ -595,9 +719,7 @@ def main():
     device = torch.device("cuda", local)
     data = make_inputs(wl)
 
-    probe = Step(ttq, wl, data, device, 1, args.separate)
-    rep = max(2, math.ceil(2.5 * L2_BYTES / probe.input_bytes()))
-    del probe
+    rep = replicas_for(wl)
     step = Step(ttq, wl, data, device, rep, args.separate)
     stream = torch.cuda.Stream(device)
     torch.cuda.synchronize()
@@ -688,50 +810,30 @@ def main():
         e["gbs"] = work[kind] / (msk / 1e3) / 1e9
         kernels[kind] = e
     dom = max(per_kind, key=per_kind.get)
-    if dom == "gemm":
-        peak = pk["bf16_tflops_sustained"]
-        achieved = kernels["gemm"]["tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_kind": f"{pk['source']} bf16 sustained (fp16 dense rate "
-                             "= bf16 nominal)"}
-    else:
-        peak = pk["hbm_gbs"]
-        achieved = kernels[dom]["gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak,
-                "unit": "GB/s", "frac": achieved / peak,
-                "peak_kind": f"{pk['source']} HBM copy"}
-    roof["kernel"] = dom
+    region_s = ms / 1e3
+    roof = roofline(dom, kernels, pk, region_s)
     roof["traffic"] = traffic_from_profiles(dom, wl.name)
     roof["traffic_unit"] = "DRAM bytes per launch (ncu, cold serialised)"
     # algorithmic work of one launch, averaged over the step's launches
     n_dom = kinds.count(dom)
     roof["algorithmic_per_launch"] = (
         work["gemm_flops"] if dom == "gemm" else work[dom]) / max(1, n_dom)
+    roof["timed_region_s"] = region_s
 
     # end to end through the binding: host buffers in, host buffers out
     e2e = None
     if not args.no_e2e:
-        e2e = end_to_end(ttq, wl, data, device, args, stream, world)
+        e2e = end_to_end(ttq, wl, data, device, args, world)
 
-    cpu = cpu_one = parity = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # the unchanged oracle on every host core, and on one core
         cores = host_cores()
-        outputs = {}
-        est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS, cores,
-                                outputs)
-        cpu = {"value": len(wl.layers) * wl.T / est, "unit": "tokens/s",
-               "cores": cores, "kind": "oracle", "sample": desc}
         try:
-            parity = parity_summary(step, outputs)
+            parity = parity_summary(step, cores)
         except Exception as e:  # a report: never a reason to lose the line
             parity = {"error": repr(e)[:200]}
-        if cores > 1:
-            est, desc = oracle_step(wl, data, ORACLE_SAMPLE_TOKENS)
-            cpu_one = {"value": len(wl.layers) * wl.T / est,
-                       "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                       "sample": desc}
+        # the unchanged oracle on every host core
+        cpu = cpu_baseline(wl, data, cores)
 
     if rank == 0:
         line = {
@@ -739,29 +841,17 @@ def main():
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-            "data": "synthetic",
-            "config": {
-                "workload": wl.name, "T": wl.T, "bits": wl.bits,
-                "group": wl.group,
-                "layers": ", ".join(f"{L.name} {L.N}x{L.K}"
-                                    for L in wl.layers),
-                "projections": ", ".join(
-                    f"{g} {step.N[g]}x{Ls[0].K}" for g, _, Ls in step.groups),
-                "operands": "fp16 x fp16 -> fp32 (tensor cores); quantizer "
-                            "fp32; statistics fp32",
-                "l2": f"inputs rotate over {rep} replicas "
-                      f"({rep * step.input_bytes() / 2**20:.0f} MiB > L2)",
-                "parallelism": f"replicas x{world}",
-                "launch": ("eager" if args.eager else
-                           "CUDA graph per replica") + (
-                    "; one stream, one call per step and layer"
-                    if args.separate else
-                    "; statistics+scales fused; prepare on a second stream "
-                    "beside the quantizer")},
+            "data": "synthetic", "config": workload_config(wl, world),
+            "launch": ("eager" if args.eager else
+                       "CUDA graph per replica") + (
+                "; one stream, one call per step and layer"
+                if args.separate else
+                "; statistics+scales fused; prepare on a second stream "
+                "beside the quantizer"),
             "roofline": roof, "kernels": kernels,
             "gpu_launches": step.kernel_launches() * args.steps,
-            "cpu_baseline": cpu, "cpu_baseline_one_core": cpu_one,
-            "parity": parity, "e2e": e2e, "clocks": clocks,
+            "cpu_baseline": cpu, "parity": parity, "e2e": e2e,
+            "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -770,47 +860,99 @@ def main():
         dist.destroy_process_group()
 
 
-def end_to_end(ttq, wl, data, device, args, stream, world):
+def roofline(dom, kernels, pk, region_s):
+    """The roofline object of the dominant kernel. A tensor-core kernel is
+    compared with the measured bf16 burst peak when the timed region is
+    shorter than SUSTAINED_REGION_SECONDS and with the sustained peak
+    otherwise (fp16 has the same dense rate as bf16)."""
+    if dom == "gemm":
+        sustained = region_s >= SUSTAINED_REGION_SECONDS
+        peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+        achieved = kernels["gemm"]["tflops"]
+        return {"bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "kernel": dom,
+                "peak_kind": f"{pk['source']} bf16 "
+                             f"{'sustained' if sustained else 'burst'} "
+                             f"(timed region {region_s:.3g} s; fp16 dense "
+                             f"rate = bf16)"}
+    peak = pk["hbm_gbs"]
+    achieved = kernels[dom]["gbs"]
+    return {"bound": "hbm", "achieved": achieved, "peak": peak,
+            "unit": "GB/s", "frac": achieved / peak, "kernel": dom,
+            "peak_kind": f"{pk['source']} HBM copy"}
+
+
+def end_to_end(ttq, wl, data, device, args, world):
     """Same metric through the Python binding with host buffers: each step
     copies its prompt activations from pinned host memory, runs the path
-    (eager calls, one per step of the method) and copies every output back.
-    The layer weights are the model's resident parameters and stay on the
-    device."""
-    step = Step(ttq, wl, data, device, 1, args.separate)
+    (eager calls, one per step of the method) and copies every output back
+    to pinned host memory. The layer weights are the model's resident
+    parameters and stay on the device. Steps are pipelined over two buffer
+    sets: the copy-in of step i+1 and the copy-out of step i-1 run on their
+    own streams while step i computes. Every byte of every step still
+    crosses PCIe inside the timed region."""
+    sets = [Step(ttq, wl, data, device, 1, args.separate) for _ in range(2)]
     hx = {k: v.pin_memory() for k, v in data["X"].items()}
-    hy = {g: torch.empty((wl.T, step.N[g]), dtype=wl.dtype).pin_memory()
-          for g, _, _ in step.groups}
+    hy = [{g: torch.empty((wl.T, sets[0].N[g]), dtype=wl.dtype).pin_memory()
+           for g, _, _ in sets[0].groups} for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in hx.values())
-    d2h = sum(v.numel() * v.element_size() for v in hy.values())
+    d2h = sum(v.numel() * v.element_size() for v in hy[0].values())
+    comp = torch.cuda.Stream(device)
+    cin = torch.cuda.Stream(device)
+    cout = torch.cuda.Stream(device)
+    free_in = [None, None]    # compute of the set's last step done
+    free_out = [None, None]   # copy-out of the set's last step done
 
-    def one():
-        for k, v in hx.items():
-            step.X[0][k].copy_(v, non_blocking=True)
-        step.run(0)
-        for n, v in hy.items():
-            v.copy_(step.Y[n], non_blocking=True)
+    def one(i):
+        b = i % 2
+        st = sets[b]
+        with torch.cuda.stream(cin):
+            if free_in[b] is not None:
+                cin.wait_event(free_in[b])
+            for k, v in hx.items():
+                st.X[0][k].copy_(v, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(cin)
+        with torch.cuda.stream(comp):
+            comp.wait_event(loaded)
+            if free_out[b] is not None:
+                comp.wait_event(free_out[b])
+            st.run(0)
+            done = torch.cuda.Event()
+            done.record(comp)
+        free_in[b] = done
+        with torch.cuda.stream(cout):
+            cout.wait_event(done)
+            for n, v in hy[b].items():
+                v.copy_(st.Y[n], non_blocking=True)
+            out = torch.cuda.Event()
+            out.record(cout)
+        free_out[b] = out
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            one()
-    stream.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    steps = max(5, args.steps // 2)
+    for i in range(max(3, args.warmup)):
+        one(i)
+    torch.cuda.synchronize()
+    steps = max(5, min(args.steps, 200))
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
-        a.record()
-        for _ in range(steps):
-            one()
-        b.record()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(cin)
+    for i in range(steps):
+        one(i)
+    # the region ends when the last copy-out has landed
+    torch.cuda.current_stream().wait_stream(cout)
+    torch.cuda.current_stream().wait_stream(comp)
+    b.record(torch.cuda.current_stream())
     torch.cuda.synchronize()
     ms = slowest_rank_ms(a.elapsed_time(b) / steps, world, device)
     return {"value": layer_tokens_per_s(world, len(wl.layers), wl.T, ms),
-            "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "copy-in, compute and copy-out on three streams "
+                         "over two buffer sets"}
 
 
 if __name__ == "__main__":

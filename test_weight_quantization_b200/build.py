@@ -77,6 +77,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
         objs = list(ex.map(lambda s: _compile(s, headers, NVCC_FLAGS, verbose),
                            sources))
+    # objects of older sources or flags are never used again
+    for o in glob.glob(os.path.join(BUILD, "*.o")):
+        if o not in objs:
+            os.remove(o)
     link_key = _digest(objs, ["link"])
     stamp = LIB + ".stamp"
     if (force or not os.path.exists(LIB) or not os.path.exists(stamp)

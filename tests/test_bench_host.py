@@ -99,20 +99,64 @@ def test_reference_arm_rank_nonzero_exits_without_work():
 
 
 def test_reference_arm_reports_the_oracle():
+    """The reference arm times exactly the steps and warm-up asked for,
+    reports the measured time per step, and prints the GPU arm's config."""
     env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),
-                        "--impl", "reference", "--steps", "1", "--warmup",
-                        "0"], capture_output=True, text=True, env=env,
-                       timeout=600)
+                        "--impl", "reference", "--steps", "2", "--warmup",
+                        "1", "--workload", "single-768"], capture_output=True,
+                       text=True, env=env, timeout=600)
     assert r.returncode == 0, r.stderr
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference"
     assert line["unit"] == "tokens/s" and line["value"] > 0
-    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["steps"] == 2 and line["warmup"] == 1
     import bench
+    from test_weight_quantization_b200.inputs import WORKLOADS
+    assert line["config"] == bench.workload_config(WORKLOADS["single-768"], 1)
+    # value is the sample's tokens over the measured time per step
+    assert line["value"] == pytest.approx(
+        1 * line["sample_tokens"] / (line["ms_per_step"] * 1e-3), rel=1e-9)
+    assert line["ms_per_step"] * line["steps"] <= line["wall_s"] * 1e3 * (
+        1 + 1e-9)
+    assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["cores"] == bench.host_cores()
     assert line["e2e"]["h2d_bytes_per_step"] == 0
-    assert line["config"]["workload"] == "opt125m-block"
+
+
+def test_roofline_peak_follows_the_timed_region():
+    """A timed region under a second is compared with the burst tensor peak,
+    a longer one with the sustained peak; frac is achieved / peak."""
+    import bench
+    pk = {"hbm_gbs": 6545.0, "bf16_tflops": 1627.8,
+          "bf16_tflops_sustained": 1395.0, "source": "measured"}
+    k = {"gemm": {"tflops": 1000.0, "gbs": 10.0}, "quantize": {"gbs": 5000}}
+    short = bench.roofline("gemm", k, pk, 0.02)
+    assert short["peak"] == 1627.8 and "burst" in short["peak_kind"]
+    assert short["frac"] == pytest.approx(1000.0 / 1627.8)
+    long = bench.roofline("gemm", k, pk, 3.0)
+    assert long["peak"] == 1395.0 and "sustained" in long["peak_kind"]
+    mem = bench.roofline("quantize", k, pk, 3.0)
+    assert mem["bound"] == "hbm" and mem["frac"] == pytest.approx(5000 / 6545)
+
+
+def test_default_workload_is_the_largest_single_gpu_configuration():
+    import bench
+    sys_argv = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        args = bench.parse()
+    finally:
+        sys.argv = sys_argv
+    assert args.workload == "llama7b-prefill"
+    from test_weight_quantization_b200.inputs import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    # 3 layers of 4096 tokens; inputs of 154 MiB and weights of 212 MiB per
+    # replica, two replicas > 2.5 x L2
+    assert bench.input_bytes(wl) == 2 * 4096 * (4096 + 4096 + 11008) + \
+        2 * (4096 * 4096 + 2 * 11008 * 4096)
+    assert bench.replicas_for(wl) * bench.input_bytes(wl) >= \
+        2.5 * bench.L2_BYTES
 
 
 def test_measure_table_shapes_meet_the_call_constraints():
@@ -193,67 +237,81 @@ def test_host_cores_and_ranges_cover_the_work():
 
 
 def test_parity_summary_reads_the_step_buffers():
-    """The bench line's parity report: the step's (stacked) codes and
-    sampled outputs against the oracle's. Buffers equal to the oracle's give
-    zero moved codes and zero error; one changed code and one changed
-    output are seen."""
+    """The bench line's parity report on a stand-in step whose buffers hold
+    the oracle's own results: zero differences; one changed code and one
+    changed output are seen."""
     import dataclasses
     import numpy as np
     import torch
     import bench
+    import oracle
     from test_weight_quantization_b200 import ttq
     from test_weight_quantization_b200.inputs import WORKLOADS, make_inputs
     base = WORKLOADS["opt125m-block"]
     wl = dataclasses.replace(base, T=64, layers=base.layers[:4])
     data = make_inputs(wl)
-    outputs = {}
-    bench.oracle_step(wl, data, 8, 1, outputs)
 
     class FakeStep:
         pass
     st = FakeStep()
     st.wl, st.groups = wl, bench.projection_groups(wl)
-    st.codes, st.Y = {}, {}
-    for g, _, Ls in st.groups:
+    st.inputs = bench.layer_inputs(wl)
+    st.X = [dict(data["X"])]
+    st.sums, st.s, st.inv = {}, {}, {}
+    for k in st.inputs:
+        X = data["X"][k].float().numpy()
+        sums = oracle.act_sums(X).astype(np.float32)
+        s, inv = oracle.awq_scales(sums.astype(np.float64), wl.T, wl.alpha,
+                                   wl.lam, wl.p)
+        st.sums[k] = torch.from_numpy(sums)
+        st.s[k] = torch.from_numpy(s.astype(np.float32))
+        st.inv[k] = torch.from_numpy(inv.astype(np.float32))
+    st.W, st.N, st.codes, st.delta, st.zero, st.Y = [{}], {}, {}, {}, {}, {}
+    for g, k, Ls in st.groups:
         K = Ls[0].K
-        c = np.concatenate([outputs[L.name][0] for L in Ls])
-        padded = np.zeros((c.shape[0], ttq.codes_ld(K, wl.bits)), np.uint32)
-        padded[:, :c.shape[1]] = c
-        st.codes[g] = torch.from_numpy(padded.view(np.int32))
-        y = np.concatenate([outputs[L.name][3] for L in Ls], axis=1)
+        W = torch.cat([data["W"][L.name] for L in Ls])
+        st.W[0][g], st.N[g] = W, W.shape[0]
+        c, d, z = oracle.quantize(W.float().numpy(), st.s[k].numpy(),
+                                  wl.bits, wl.group)
+        cp = np.zeros((c.shape[0], ttq.codes_ld(K, wl.bits)), np.uint32)
+        cp[:, :c.shape[1]] = c
+        gl = ttq.groups_ld(K, wl.group)
+        dp = np.zeros((c.shape[0], gl), np.float32)
+        zp = np.zeros((c.shape[0], gl), np.uint8)
+        dp[:, :d.shape[1]], zp[:, :z.shape[1]] = d, z
+        st.codes[g] = torch.from_numpy(cp.view(np.int32))
+        st.delta[g], st.zero[g] = torch.from_numpy(dp), torch.from_numpy(zp)
+        y = oracle.lowbit_gemm(data["X"][k].float().numpy(),
+                               st.inv[k].numpy(), c, d, z, W.shape[0],
+                               wl.bits, wl.group)
         st.Y[g] = torch.from_numpy(y.astype(np.float32))
     assert [g for g, _, _ in st.groups] == ["q|k|v", "o"]
-    rep = bench.parity_summary(st, outputs)
-    assert rep["codes_differing"] == 0
+    rep = bench.parity_summary(st, threads=3, qrows=2304, ytokens=64)
+    assert rep["codes_differing"] == 0 and rep["delta_differing"] == 0
     assert rep["codes"] == sum(L.N * L.K for L in wl.layers)
-    assert rep["y_tokens"] == 8 and rep["y_rel_fro_max"] < 1e-6
+    assert rep["stats_rel_max"] < 1e-6 and rep["scales_rel_max"] < 1e-6
+    assert rep["y_tokens"] == 64 and rep["y_rel_fro_max"] < 1e-6
     st.codes["q|k|v"][800, 0] ^= 1          # code 0 of row 32 of k
     st.Y["o"][3, 5] += 1.0
-    rep = bench.parity_summary(st, outputs)
-    assert rep["codes_differing"] == 1 and rep["y_rel_fro_max"] > 1e-3
+    rep = bench.parity_summary(st, threads=3, qrows=2304, ytokens=64)
+    assert rep["codes_differing"] == 1
+    assert rep["codes_differing_off_near_ties"] == 1
+    assert rep["y_rel_fro_max"] > 1e-3
 
 
 def test_clock_summary_keeps_the_samples_of_the_timed_region():
-    """nvidia-smi rows (timestamp first): the summary keeps the rows taken
-    between the marks, and falls back to all rows, flagged, if none are."""
-    import datetime
+    """NVML samples (time, SM MHz, reason bits): the summary keeps the
+    samples taken between the marks and names the active reasons; with none
+    inside it falls back to all samples, flagged."""
     import bench
-    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
-
-    def row(ms, mhz, cap="Not Active"):
-        ts = (base + datetime.timedelta(milliseconds=ms)).strftime(
-            "%Y/%m/%d %H:%M:%S.%f")[:-3]
-        return (f"{ts}, 0, {mhz}, 1965, 700.5, 0x0, Not Active, Not Active, "
-                f"Not Active, {cap}\n")
-    lines = [row(0, 1200), row(100, 1965), row(200, 1965, "Active"),
-             row(300, 1950), row(400, 1000)]
-    t0 = base + datetime.timedelta(milliseconds=90)
-    t1 = base + datetime.timedelta(milliseconds=310)
-    s = bench.ClockSampler.summarize(lines, t0, t1)
+    samples = [(0.0, 1200.0, 0), (0.1, 1965.0, 0), (0.2, 1965.0, 0x4),
+               (0.3, 1950.0, 0), (0.4, 1000.0, 0x8 | 0x40)]
+    s = bench.ClockSampler.summarize(samples, 1965.0, 0.09, 0.31)
     assert s["samples"] == 3 and s["in_timed_region"]
-    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"]
-    late = base + datetime.timedelta(seconds=9)
-    s = bench.ClockSampler.summarize(lines, late, late)
+    s = bench.ClockSampler.summarize(samples, 1965.0, 9.0, 9.0)
     assert s["samples"] == 5 and not s["in_timed_region"]
-    assert bench.ClockSampler.summarize(["garbage\n"]) is None
+    assert s["reasons"] == ["hw_slowdown", "hw_thermal_slowdown",
+                            "sw_power_cap"]
+    assert bench.ClockSampler.summarize([], 1965.0) is None

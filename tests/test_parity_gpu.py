@@ -288,6 +288,19 @@ def test_gemm_output_tile_store(ttq, N, pitch, out):
         assert torch.all(big[:, N:] == 7.0)
 
 
+def test_one_and_two_tokens_with_very_long_rows(ttq):
+    """K = 22528: one token still takes the CUDA-core product; for two
+    tokens its staged activations would exceed the shared-memory budget, so
+    the tensor-core decode configuration runs instead."""
+    N, K = 192, 22528
+    X = acts(2, K, 41, torch.bfloat16)
+    W = weights(N, K, 42, torch.bfloat16)
+    for T in (1, 2):
+        Y, inv, c, d, z = run_path(ttq, X[:T], W, 4, 128)
+        assert_gemm_close(np32(Y), oracle_y(X[:T], inv, c, d, z, N, 4, 128),
+                          f"long rows T={T}", Y.dtype)
+
+
 @pytest.mark.parametrize("T", [1, 2])
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("group", [16, 32, 128])

@@ -52,6 +52,8 @@ def noalloc(ttq, X, inv, c, d, z, N, bits, group, Y, A=None, B=None):
     (64, 640, 768, 4, 32, 0),     # prefill tile shape, several K stages
     (4, 300, 512, 3, 16, 0),      # decode configuration, ragged rows
     (200, 272, 384, 4, 64, 16),   # with the low-rank stage
+    (1, 300, 512, 4, 32, 0),      # one token: the CUDA-core product
+    (2, 272, 384, 3, 32, 16),     # two tokens with the low-rank term
 ])
 def test_noalloc_matches_workspace_entry_point(ttq, T, N, K, bits, group, r):
     g = torch.Generator().manual_seed(T + N + K)
@@ -80,14 +82,28 @@ def test_noalloc_matches_workspace_entry_point(ttq, T, N, K, bits, group, r):
 
 
 def test_noalloc_refuses_inputs_beyond_its_scratch(ttq):
-    T, K, N = 4096, 4096, 128  # needs 32 MiB of scratch
-    assert ttq.workspace_size(T, K) > SCRATCH_BYTES
-    X = torch.zeros(T, K, dtype=torch.bfloat16, device="cuda")
+    """The limit is exact: 2048 tokens of 4096 channels fill the scratch
+    (2048 * 4096 * 2 bytes) and run; one token more, or the same tokens with
+    a low-rank term, is refused with nothing launched."""
+    K, N = 4096, 128
+    assert ttq.workspace_size(2048, K) == SCRATCH_BYTES
+    assert ttq.workspace_size(2049, K) > SCRATCH_BYTES
+    assert ttq.workspace_size(2048, K, 16) > SCRATCH_BYTES
+    X = torch.zeros(2049, K, dtype=torch.bfloat16, device="cuda")
     inv = torch.ones(K, device="cuda")
     c = torch.zeros(N, ttq.codes_ld(K, 4), dtype=torch.int32, device="cuda")
     d = torch.zeros(N, ttq.groups_ld(K, 128), device="cuda")
     z = torch.zeros(N, ttq.groups_ld(K, 128), dtype=torch.uint8, device="cuda")
-    Y = torch.zeros(T, N, dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros(16, K, dtype=torch.bfloat16, device="cuda")
+    B = torch.zeros(N, 16, dtype=torch.bfloat16, device="cuda")
+    Y = torch.full((2049, N), 7.0, dtype=torch.bfloat16, device="cuda")
     assert noalloc(ttq, X, inv, c, d, z, N, 4, 128, Y) == 2  # UNSUPPORTED
+    assert noalloc(ttq, X[:2048], inv, c, d, z, N, 4, 128, Y[:2048], A,
+                   B) == 2
     torch.cuda.synchronize()
-    assert not Y.any()
+    assert torch.all(Y == 7.0)
+    # the exact fit runs (zero weights give a zero projection)
+    assert noalloc(ttq, X[:2048], inv, c, d, z, N, 4, 128, Y[:2048]) == 0
+    torch.cuda.synchronize()
+    assert ttq.device_error(clear=True) == 0
+    assert not Y[:2048].any() and torch.all(Y[2048:] == 7.0)
