@@ -136,6 +136,28 @@ ttq_status ttq_awq_scales(const float* sum, int64_t T_total, int64_t K,
                           const ttq_params* prm, float* s, float* inv_s,
                           void* stream);
 
+/* Step 2 for a layer whose input channels are split over several GPUs
+ * (row-parallel tensor parallelism; the pages describe one GPU, the split
+ * is ours). The channel mean mbar of the shrinkage (TTQ review, Proposed
+ * method, bullet 3) runs over ALL input channels, so it needs one scalar
+ * from every shard:
+ *   ttq_channel_moment_total: *total = sum_j sum[j] / T_total over this
+ *     shard's K channels, in fp64 and a fixed order (device double, 8-byte
+ *     aligned).
+ *   The caller adds the shards' totals (one all-reduce of one double).
+ *   ttq_awq_scales_sharded: the scales of this shard's K channels as in
+ *     ttq_awq_scales, but with mbar = *total / K_total, where *total (device
+ *     double) is the added total and K_total the layer's channel count.
+ * Invalid pointers, sizes or K_total < K return TTQ_ERR_INVALID_ARG. With
+ * one shard (K_total = K) the scales equal ttq_awq_scales' to the rounding
+ * of the fp64 mean. */
+ttq_status ttq_channel_moment_total(const float* sum, int64_t T_total,
+                                    int64_t K, double* total, void* stream);
+ttq_status ttq_awq_scales_sharded(const float* sum, int64_t T_total, int64_t K,
+                                  int64_t K_total, const ttq_params* prm,
+                                  const double* total, float* s, float* inv_s,
+                                  void* stream);
+
 /* Steps 1 and 2 in one launch: ttq_act_stats on X followed by
  * ttq_awq_scales on the resulting sums, with the same arithmetic (TTQ
  * review, Proposed method, bullets 2-4). The CTAs that finish the
@@ -172,11 +194,12 @@ ttq_status ttq_act_stats_scales(const void* X, ttq_dtype xt, int64_t T,
  * where rint rounds half to even. Outputs codes (layout above), delta = D,
  * zero = z; padding is zeroed.
  *   W      [N, K] of dtype wt, row pitch ldw.
- * D and z are exactly these values. For the codes the kernel forms w_j / D
- * as w_j * RN(1/D), one rounded reciprocal per group; that product lies
- * within one fp32 step of the IEEE quotient, so a code can differ from the
- * formula only where w_j / D is within one fp32 step of a half-integer (a
- * near-tie, about one weight in 10^5 to 10^6 at 8 bits, fewer at fewer).
+ * D and z are exactly these values. For the codes the kernel rounds the
+ * exact product w_j * RN(1/D) to an integer (one rounded reciprocal per
+ * group); that product lies within 2^-24 |w_j / D| of the quotient, so a
+ * code can differ from the formula only where the IEEE quotient w_j / D is
+ * within one fp32 step of a half-integer (a near-tie, about one weight in
+ * 10^5 to 10^6 at 8 bits, fewer at fewer).
  * Requires 2 <= bits <= 8, group in {16,32,64,128}, K % 32 == 0,
  * K % group == 0. Deterministic. */
 ttq_status ttq_quantize_rtn_grouped(const void* W, ttq_dtype wt, int64_t N,
@@ -203,10 +226,11 @@ size_t ttq_w_lowbit_gemm_workspace_size(int64_t T, int64_t K, int r);
  * The tensor cores take fp16 operands: X / s is rounded once to fp16 and
  * each weight (q - z) * D once to fp16; products accumulate in fp32.
  * |X / s| must stay below 65504 (else TTQ_DEVERR_FP16_RANGE is raised).
- * Which kernel runs depends on T: T <= 2 a CUDA-core matrix-vector product
+ * Which kernel runs depends on T: T <= 4 a CUDA-core matrix-vector product
  * (the weight (q - z) D is applied in fp32, the activations are the fp16
- * X / s), T <= 32 the tensor-core decode configuration (K split across a
- * cluster), larger T the prefill one. The results agree to the tolerances
+ * X / s) when its staged activations (about 4.75 T K bytes) fit its shared
+ * memory, otherwise and up to T = 32 the tensor-core decode configuration
+ * (K split across a cluster), larger T the prefill one. The results agree to the tolerances
  * of the parity tests, not bit for bit across these regimes.
  * Requires K % 32 == 0, K % group == 0, 0 <= r <= 64. */
 ttq_status ttq_w_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,
@@ -239,7 +263,7 @@ ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt, int64_t T,
                                    void* U, void* stream);
 
 /* ttq_w_lowbit_gemm_prepared: the projection on prepared operands, one
- * kernel launch (T <= 2: CUDA cores, otherwise tensor cores, as above):
+ * kernel launch (T <= 4: CUDA cores, otherwise tensor cores, as above):
  *   Y[t][n] = sum_j Xs[t][j] (q[n][j] - z) D + sum_rho U[t][rho] B[n][rho].
  * Xs, U as written by ttq_prepare_activations for the same bits; B [N, r]
  * of dtype bt. */
@@ -317,7 +341,8 @@ int ttq_device_error(int clear);
 ttq_status ttq_selftest_bounded_wait(int arrive, uint32_t* out, void* stream);
 
 /* ABI version of this header (3: ttq_act_stats_scales added; 4:
- * ttq_selftest_bounded_wait added). */
+ * ttq_selftest_bounded_wait added; 5: ttq_channel_moment_total and
+ * ttq_awq_scales_sharded added). */
 int ttq_abi_version(void);
 
 #ifdef __cplusplus

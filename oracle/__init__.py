@@ -55,6 +55,8 @@ def _load():
         D = ctypes.c_double
         lib.oracle_act_sums.argtypes = [P, I64, I64, I64, D, P]
         lib.oracle_awq_scales.argtypes = [P, I64, I64, D, D, D, P, P]
+        lib.oracle_awq_scales_given_mean.argtypes = [P, I64, I64, D, D, D, D,
+                                                     P, P]
         lib.oracle_pack_codes.argtypes = [P, I64, I64, I, P]
         lib.oracle_unpack_codes.argtypes = [P, I64, I64, I, P]
         lib.oracle_quantize.argtypes = [P, I64, I64, I64, P, I, I, P, P, P]
@@ -96,6 +98,20 @@ def awq_scales(sums, T_total: int, alpha: float, lam: float, p: float):
     inv = np.empty(K, np.float64)
     _load().oracle_awq_scales(_ptr(sums), int(T_total), K, float(alpha),
                               float(lam), float(p), _ptr(s), _ptr(inv))
+    return s, inv
+
+
+def awq_scales_given_mean(sums, T_total: int, mbar: float, alpha: float,
+                          lam: float, p: float):
+    """(s, inv_s) in fp64 of a shard of channels whose shrinkage mean mbar
+    is taken over all channels (step 2)."""
+    sums = np.ascontiguousarray(np.asarray(sums, dtype=np.float64))
+    K = sums.shape[0]
+    s = np.empty(K, np.float64)
+    inv = np.empty(K, np.float64)
+    _load().oracle_awq_scales_given_mean(_ptr(sums), int(T_total), K,
+                                         float(mbar), float(alpha), float(lam),
+                                         float(p), _ptr(s), _ptr(inv))
     return s, inv
 
 

@@ -89,6 +89,26 @@ void oracle_awq_scales(const double* sum, int64_t T_total, int64_t K,
   free(m);
 }
 
+/* Step 2 with the mean of the shrinkage given: for a layer whose input
+ * channels are split into shards, mbar is the mean over ALL channels while
+ * m_j and the scales are this shard's (the same formulas as above). */
+void oracle_awq_scales_given_mean(const double* sum, int64_t T_total,
+                                  int64_t K, double mbar, double alpha,
+                                  double lambda, double p, double* s,
+                                  double* inv_s) {
+  for (int64_t j = 0; j < K; ++j) {
+    double m = sum[j] / (double)T_total;
+    double c = (1.0 - lambda) * m + lambda * mbar;
+    double sj;
+    if (alpha == 0.0 || !(c > 0.0) || !isfinite(c))
+      sj = 1.0;
+    else
+      sj = pow(c, alpha / p);
+    s[j] = sj;
+    inv_s[j] = 1.0 / sj;
+  }
+}
+
 /* ---- Packing (storage format of the codes; ours, the pages fix none) ----
  * Block k of a row holds channels 32k..32k+31 in `bits` words; channel
  * 32k + c sits at bits [c*bits, c*bits + bits) of the block. */

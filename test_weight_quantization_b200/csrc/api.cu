@@ -92,7 +92,7 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 4; }
+TTQ_EXPORT int ttq_abi_version(void) { return 5; }
 
 TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
   if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
@@ -152,6 +152,31 @@ TTQ_EXPORT ttq_status ttq_awq_scales(const float* sum, int64_t T_total,
     return TTQ_ERR_INVALID_ARG;
   return launch_awq_scales(sum, T_total, K, prm->alpha, prm->lambda, prm->p,
                            s, inv_s, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_channel_moment_total(const float* sum,
+                                               int64_t T_total, int64_t K,
+                                               double* total, void* stream) {
+  if (!sum || !total || T_total < 1 || K < 1 || !aligned(sum, 4) ||
+      !aligned(total, 8))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_channel_total(sum, T_total, K, total, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_awq_scales_sharded(const float* sum, int64_t T_total,
+                                             int64_t K, int64_t K_total,
+                                             const ttq_params* prm,
+                                             const double* total, float* s,
+                                             float* inv_s, void* stream) {
+  if (!sum || !total || !s || !inv_s || !prm || T_total < 1 || K < 1 ||
+      K_total < K || !(prm->alpha >= 0.f) || !isfinite(prm->alpha) ||
+      !(prm->lambda >= 0.f && prm->lambda <= 1.f) || !(prm->p > 0.f) ||
+      !isfinite(prm->p) || !aligned(sum, 4) || !aligned(total, 8) ||
+      !aligned(s, 4) || !aligned(inv_s, 4))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_awq_scales_sharded(sum, T_total, K, K_total, total,
+                                   prm->alpha, prm->lambda, prm->p, s, inv_s,
+                                   as_stream(stream));
 }
 
 TTQ_EXPORT ttq_status ttq_act_stats_scales(

@@ -10,13 +10,13 @@
 
 namespace ttq {
 
-// mean_k(sum_k / T) in fp64 by the NT threads of one CTA, in a fixed order
+// sum_k (sum_k / T) in fp64 by the NT threads of one CTA, in a fixed order
 // (thread-strided partials, a butterfly inside each warp, warps in order),
 // so every CTA that runs it gets the same value. warp_sums holds NT/32
 // doubles of shared memory; sum is read through L2 (other CTAs wrote it).
 template <int NT>
-__device__ double awq_channel_mean(const float* sum, int64_t K, double invT,
-                                   double* warp_sums) {
+__device__ double awq_channel_total(const float* sum, int64_t K, double invT,
+                                    double* warp_sums) {
   double local = 0.0;
   int64_t j = threadIdx.x;
   for (; j + 3 * NT < K; j += 4 * NT) {
@@ -36,7 +36,14 @@ __device__ double awq_channel_mean(const float* sum, int64_t K, double invT,
   double total = 0.0;
   for (int w = 0; w < NT / 32; ++w) total += warp_sums[w];
   __syncthreads();  // warp_sums may be reused by the caller
-  return total / (double)K;
+  return total;
+}
+
+// mean_k(sum_k / T): the total above divided by K.
+template <int NT>
+__device__ double awq_channel_mean(const float* sum, int64_t K, double invT,
+                                   double* warp_sums) {
+  return awq_channel_total<NT>(sum, K, invT, warp_sums) / (double)K;
 }
 
 // s_j and 1/s_j of one channel. c_j is formed in fp64; the power runs in

@@ -12,7 +12,7 @@
 // (prescale_kernel), each weight (q - z) * D is rounded once to fp16 in the
 // dequantiser; products accumulate in fp32 in TMEM.
 //
-// CTA = producer warp + MMA warp + 8 dequantiser warps (prefill, one CTA
+// CTA = producer warp + MMA warp + 16 dequantiser warps (prefill, one CTA
 // per SM) or 4 (decode, two CTAs per SM). Shared-memory rings filled by the
 // tensor memory accelerator (TMA) and drained in K order by stage:
 //   X~ ring      two 64-channel fp16 activation boxes (128B swizzle)
@@ -25,9 +25,9 @@
 // accumulator leaves TMEM in 16x256b fragment order, is packed to 16-bit
 // pairs and written transposed by stmatrix into 128-byte-swizzled boxes of
 // the idle activation ring, and a TMA tensor store writes Y. Decode
-// (3 <= T <= 32; one or two tokens use gemv.cu) splits K over a cluster of
-// up to 8 CTAs whose partial tiles every rank reduces in part through
-// distributed shared memory, in rank order. The rank-r low-rank term is one
+// (T <= 32 where gemv.cu, which takes up to four tokens, does not apply)
+// splits K over a cluster of up to 8 CTAs whose partial tiles every rank
+// reduces in part through distributed shared memory, in rank order. The rank-r low-rank term is one
 // extra K stage, [X~ | U] [W_hat | B]^T with U = X A^T (fp16, from
 // lowrank_u_kernel). Every wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA
 // winds down).
@@ -49,11 +49,22 @@ constexpr int kBM = 128;           // weight rows per CTA (TMEM lanes)
 constexpr int kSK = 128;           // channels per pipeline stage
 constexpr int kSCols = kSK / 2;    // TMEM columns of one fp16 weight stage
 constexpr int kParamGroups = 16;   // groups per params chunk
-// CTA = producer warp + MMA warp + DQW dequantiser warps (4 or 8; with 8,
-// two warps share each TMEM lane quarter and split every stage in halves)
-constexpr int kDqWarp0 = 2;  // first dequantiser warp
-__host__ __device__ constexpr int cta_threads(int dqw) {
-  return 32 * (kDqWarp0 + dqw);
+// CTA = producer warp + MMA warp + DQW dequantiser warps (4, 8 or 16; with
+// 8 or 16, two or four warps share each TMEM lane quarter and split every
+// stage into parts of 64 or 32 channels)
+// Warps: 0 the TMA producer, 1 .. NACC the MMA issuers (NACC accumulators,
+// one per issuer), then the dequantisers.
+__host__ __device__ constexpr int dq_warp0(int nacc) { return 1 + nacc; }
+// dequantiser warps of the prefill form (four per SM sub-partition, so that
+// one warp's dependent chain of shared-memory loads, unpacking and TMEM
+// stores overlaps the others')
+constexpr int kPrefillDequantWarps = 16;
+// MMA issuers of the decode form at 16 tokens (half as many at 32): one
+// thread issues an M = 128, N = 16 MMA only every ~140 cycles whatever the
+// accumulator, while issuers in different warps overlap
+constexpr int kDecodeIssuers = 4;
+__host__ __device__ constexpr int cta_threads(int dqw, int nacc) {
+  return 32 * (dq_warp0(nacc) + dqw);
 }
 constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
 constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
@@ -243,8 +254,8 @@ struct Ring {
 //   MMA        waits `ready`, issues 8 MMAs, commits to `empty`, which frees
 //              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
-template <int BITS, int GMODE, int DQW>
-__global__ void __launch_bounds__(cta_threads(DQW), 2)
+template <int BITS, int GMODE, int DQW, int NACC>
+__global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_c,
@@ -255,6 +266,8 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
   constexpr int kDq = 32 * DQW;            // dequantiser threads
+  constexpr int kDqWarp0 = dq_warp0(NACC);
+  static_assert(NACC == 1 || DQW == 4, "several accumulators: decode form");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -290,14 +303,14 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
     for (int i = 0; i < S; ++i) {
       mbar_init(b_loaded + 8 * i, 1);
       mbar_init(b_ready + 8 * i, kDq);
-      mbar_init(b_empty + 8 * i, 1);
-      mbar_init(b_afree + 8 * i, 1);
+      mbar_init(b_empty + 8 * i, NACC);
+      mbar_init(b_afree + 8 * i, NACC);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
       mbar_init(b_empty_p + 8 * i, kDq);
     }
-    mbar_init(b_accum, 1);
+    mbar_init(b_accum, NACC);
     *aborted = 0;
     fence_barrier_init();
     // the tensor maps are kernel parameters: no need to wait for them
@@ -384,12 +397,20 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
         mbar_wait(b_full_p + 8 * (q & 1), (uint32_t)(q >> 1) & 1, p.err);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------- MMA issuer -----
+  } else if (warp <= NACC) {
+    // ------------------------------------------------ MMA issuers -----
+    // A stage is eight K steps of 16 channels. With NACC issuers, issuer j
+    // (one elected thread of warp 1 + j) issues K steps j*8/NACC .. into
+    // its own accumulator at column j*bn, so the issuers' MMAs overlap; the
+    // accumulators are added in order before the epilogue.
     if (lane == 0) {
+      constexpr int KPI = 8 / NACC;  // K steps per issuer and stage
+      const int j = warp - 1;
+      const uint32_t acc = tmem + (uint32_t)(j * bn);
       const uint32_t idesc = idesc_f16_f32(kBM, bn);
       const uint32_t xbytes = (uint32_t)bn * 128u;
       Ring rs, ra;
+      bool first = true;
       for (int s = 0; s < n_total; ++s) {
         if (!mbar_wait(b_ready + 8 * rs.slot, rs.round & 1, p.err)) {
           *aborted = 1;
@@ -400,14 +421,17 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
         const uint32_t xs = base + L.x + rs.slot * L.stage_x;
         const uint64_t bd0 = smem_desc_sw128(xs);
         const uint64_t bd1 = smem_desc_sw128(xs + xbytes);
+        // the low-rank stage has only the four K steps of its first box
+        const int steps = s < n_main ? 8 : 4;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          tc_mma_f16_ts(tmem, ad + 8 * k, bd0 + 2 * k, idesc,
-                        (s > 0 || k > 0) ? 1u : 0u);
-        if (s < n_main) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma_f16_ts(tmem, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
+        for (int u = 0; u < KPI; ++u) {
+          const int kidx = j * KPI + u;
+          if (kidx < steps) {
+            const uint64_t bd =
+                kidx < 4 ? bd0 + 2 * kidx : bd1 + 2 * (kidx - 4);
+            tc_mma_f16_ts(acc, ad + 8 * kidx, bd, idesc, first ? 0u : 1u);
+            first = false;
+          }
         }
         tc_commit(b_empty + 8 * rs.slot);
         tc_commit(b_afree + 8 * ra.slot);
@@ -419,13 +443,15 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
   } else {
     // ------------------------------------------------ dequantisers ----
     // One thread per weight row (= TMEM lane): a stage is four 32-code
-    // blocks, 64 fp16 pairs, written to the TMEM weight ring in two stores.
+    // blocks, 64 fp16 pairs, written to the TMEM weight ring; the DQW / 4
+    // warps of a lane quarter take equal parts of it.
+    constexpr int kParts = DQW / 4;
     const int q4 = warp & 3;                // TMEM lane quarter of this warp
-    const int h = (warp - kDqWarp0) >> 2;   // which half of a stage (DQW 8)
+    const int h = (warp - kDqWarp0) >> 2;   // which part of a stage
     const int i = 32 * q4 + lane;    // weight row in the tile = TMEM lane
     const int n = m0 + i;
     const bool row_ok = n < p.N;
-    const int half_lo = DQW == 8 ? h : 0, half_hi = DQW == 8 ? h + 1 : 2;
+    const int half_lo = kParts == 2 ? h : 0, half_hi = kParts == 2 ? h + 1 : 2;
     const uint32_t crow = base + L.c + i * 16 * BITS;
     // delta tile: 64-byte rows in the 64B swizzle (16-byte chunk index XOR
     // bits 1-2 of the row); zero tile: plain 16-byte rows
@@ -462,6 +488,31 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
         }
         const uint32_t poff = rp.slot * kParamBytes;
         const uint32_t cbase = crow + rs.slot * CHUNK;
+        // the params of one 32-code block as fp16 pairs: (1024 + z), D
+        auto block_params = [&](int blk, __half2 (&zsub)[GPB],
+                                __half2 (&dh)[GPB]) {
+          const int gl0 = ((k0 + 32 * blk) >> lg) & (kParamGroups - 1);
+#pragma unroll
+          for (int j = 0; j < GPB; ++j) {
+            const int gl = gl0 + j;
+            const float dl = __uint_as_float(ld_shared_u32(
+                drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
+                4 * (gl & 3)));
+            const uint32_t zj = ld_shared_u8(zrow + poff + gl);
+            dh[j] = __float2half2_rn(dl);
+            zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
+          }
+        };
+        if constexpr (kParts == 4) {
+          // one 32-code block per warp and stage
+          uint32_t o[16];
+          uint32_t cw[BITS];
+          load_block<BITS>(cbase + h * 4 * BITS, cw);
+          __half2 zsub[GPB], dh[GPB];
+          block_params(h, zsub, dh);
+          dequant_block<BITS, GMODE>(cw, zsub, dh, o);
+          tmem_st16(acol + 16u * h, o);
+        } else {
 #pragma unroll
         for (int half = half_lo; half < half_hi; ++half) {
           uint32_t o[32];
@@ -470,28 +521,19 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
             const int blk = 2 * half + h;  // 32-code block of the stage
             uint32_t cw[BITS];
             load_block<BITS>(cbase + blk * 4 * BITS, cw);
-            const int gl0 = ((k0 + 32 * blk) >> lg) & (kParamGroups - 1);
             __half2 zsub[GPB], dh[GPB];
-#pragma unroll
-            for (int j = 0; j < GPB; ++j) {
-              const int gl = gl0 + j;
-              const float dl = __uint_as_float(ld_shared_u32(
-                  drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
-                  4 * (gl & 3)));
-              const uint32_t zj = ld_shared_u8(zrow + poff + gl);
-              dh[j] = __float2half2_rn(dl);
-              zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);  // 1024 + z
-            }
+            block_params(blk, zsub, dh);
             dequant_block<BITS, GMODE>(cw, zsub, dh, o + 16 * h);
           }
           tmem_st32(acol + 32u * half, o);
+        }
         }
         // release the params once their last stage is read
         if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
           mbar_arrive(b_empty_p + 8 * rp.slot);
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
-        if (half_lo == 0) {
+        if (h == 0) {
           uint32_t o[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -516,13 +558,35 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
     __syncwarp();
 
     // ------------------------------------------------------ epilogue ----
+    // the first two parts' warps drain the accumulator (with 16
+    // dequantisers the other eight are done)
+    if (kParts == 4 && h >= 2) goto done;
+    {  // the epilogue's scope
     const bool acc_ok = mbar_wait(b_accum, 0, p.err);
     tc_fence_after();
     const bool ok = acc_ok && !*aborted && n_total > 0;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+    if constexpr (NACC > 1) {
+      // add the issuers' accumulators into the first, in issuer order
+      for (int c = 0; c < bn; c += 16) {
+        float v[16], w[16];
+        tmem_ld16(t_lane + (uint32_t)c, v);
+#pragma unroll
+        for (int jj = 1; jj < NACC; ++jj) {
+          tmem_ld16(t_lane + (uint32_t)(jj * bn + c), w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] += w[e];
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(v[e]);
+        tmem_st16(t_lane + (uint32_t)c, o);
+      }
+      tmem_wait_st();
+    }
     // columns of the accumulator this warp drains
-    const int c_lo = DQW == 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
-    const int c_hi = DQW == 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
+    const int c_lo = DQW >= 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
+    const int c_hi = DQW >= 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
                               : bn;
     if (split == 1 && p.y_mode == 0) {
       // Y rows not 16-byte aligned: each thread stores its row directly
@@ -651,6 +715,8 @@ __global__ void __launch_bounds__(cta_threads(DQW), 2)
         for (int c = 0; c < 16; ++c) part[(j + c) * kBM + i] = ok ? v[c] : 0.f;
       }
     }
+    }
+  done:;
   }
 
   if (split > 1) {
@@ -813,32 +879,30 @@ struct Maps {
   CUtensorMap x, u, c, d, z, y;
 };
 
-template <int BITS, int GMODE, int DQW>
+template <int BITS, int GMODE, int DQW, int NACC>
 ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
-  auto kern = lowbit_gemm_kernel<BITS, GMODE, DQW>;
+  auto kern = lowbit_gemm_kernel<BITS, GMODE, DQW, NACC>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return TTQ_ERR_CUDA;
   LaunchShape ls;
   ls.grid = grid;
-  ls.block = dim3(cta_threads(DQW), 1, 1);
+  ls.block = dim3(cta_threads(DQW, NACC), 1, 1);
   ls.smem = smem;
   ls.cluster_z = (unsigned)split;
   return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, m.y, a);
 }
 
-template <int GMODE, int DQW>
+template <int GMODE, int DQW, int NACC>
 ttq_status dispatch_bits(int bits, const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
   switch (bits) {
-    case 2: return launch_kernel<2, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 3: return launch_kernel<3, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 4: return launch_kernel<4, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 5: return launch_kernel<5, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 6: return launch_kernel<6, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 7: return launch_kernel<7, GMODE, DQW>(m, a, grid, split, smem, st);
-    case 8: return launch_kernel<8, GMODE, DQW>(m, a, grid, split, smem, st);
+#define TTQ_LK(B)                                                       \
+  case B:                                                               \
+    return launch_kernel<B, GMODE, DQW, NACC>(m, a, grid, split, smem, st);
+    TTQ_LK(2) TTQ_LK(3) TTQ_LK(4) TTQ_LK(5) TTQ_LK(6) TTQ_LK(7) TTQ_LK(8)
+#undef TTQ_LK
   }
   return TTQ_ERR_INVALID_ARG;
 }
@@ -902,7 +966,7 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 int64_t N, int bits, int group, const void* B,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
                                 int64_t ldy, cudaStream_t st) {
-  // one or two tokens: the CUDA-core matrix-vector product (gemv.cu)
+  // up to four tokens: the CUDA-core matrix-vector product (gemv.cu)
   if (gemv_applies(T, K))
     return launch_gemv(Xs, U, T, K, codes, delta, zero, N, bits, group, B, bt,
                        r, Y, yt, ldy, st);
@@ -913,7 +977,9 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   // Prefill: all 512 TMEM columns; the token tile is picked by a model of
   // waves x (fixed cost + stages x max(MMA, dequant)), an MMA of N tokens
   // costing about max(45, N/2) cycles (eight per stage) and a stage about
-  // 600 cycles of dequantisation.
+  // 600 cycles of dequantisation. (Costing every MMA at least 128 cycles,
+  // which moves every large layer to N = 256, measured slower: 390 against
+  // 346 us on the Llama up layer, with one shared-memory stage less.)
   const int sms = sm_count();
   const int64_t tiles_m = (N + kBM - 1) / kBM;
   const int k_stages = (int)((K + kSK - 1) / kSK);
@@ -926,7 +992,8 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   };
   if (T <= 32) {
     bn = T <= 16 ? 16 : 32;
-    acc_cols = 32;
+    // one accumulator per MMA issuer: 4 x 16 or 2 x 32 columns
+    acc_cols = (bn == 16 ? kDecodeIssuers : kDecodeIssuers / 2) * bn;
     tmem_cols = 256;
     SA = (tmem_cols - acc_cols) / kSCols;
     // the shared-memory ring runs deeper than the TMEM weight ring so that
@@ -993,8 +1060,8 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   // tokens one group of four dequantiser warps drains (half the tile with
   // eight dequantisers); the split-K form reduces through the cluster
   // instead and never reads this map
-  const int dqw = dual ? 4 : 8;
-  const int box_t = (dqw == 8 && bn >= 32) ? bn / 2 : bn;
+  const int dqw = dual ? 4 : kPrefillDequantWarps;
+  const int box_t = (dqw >= 8 && bn >= 32) ? bn / 2 : bn;
   int y_mode = 0;
   if (split == 1 && ((uint64_t)ldy * dtype_bytes(yt)) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(Y) % 16 == 0)
@@ -1037,15 +1104,28 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
   // decode packs two CTAs per SM with four dequant warps each; prefill runs
-  // one CTA per SM with eight
+  // one CTA per SM with sixteen
 
   if (dual) {
-    if (group == 16)
-      return dispatch_bits<0, 4>(bits, m, a, grid, split, smem, st);
-    return dispatch_bits<1, 4>(bits, m, a, grid, split, smem, st);
+    // decode: several MMA issuers (their per-instruction cost dominates at
+    // 16 or 32 tokens), one accumulator each
+    if (bn == 16)
+      return group == 16
+                 ? dispatch_bits<0, 4, kDecodeIssuers>(bits, m, a, grid, split,
+                                                       smem, st)
+                 : dispatch_bits<1, 4, kDecodeIssuers>(bits, m, a, grid, split,
+                                                       smem, st);
+    return group == 16
+               ? dispatch_bits<0, 4, kDecodeIssuers / 2>(bits, m, a, grid,
+                                                         split, smem, st)
+               : dispatch_bits<1, 4, kDecodeIssuers / 2>(bits, m, a, grid,
+                                                         split, smem, st);
   }
-  if (group == 16) return dispatch_bits<0, 8>(bits, m, a, grid, split, smem, st);
-  return dispatch_bits<1, 8>(bits, m, a, grid, split, smem, st);
+  if (group == 16)
+    return dispatch_bits<0, kPrefillDequantWarps, 1>(bits, m, a, grid, split,
+                                                     smem, st);
+  return dispatch_bits<1, kPrefillDequantWarps, 1>(bits, m, a, grid, split,
+                                                   smem, st);
 }
 
 ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,

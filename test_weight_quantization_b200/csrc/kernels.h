@@ -20,6 +20,13 @@ ttq_status launch_act_stats_scales(const void* X, ttq_dtype xt, int64_t T,
                                    float* s, float* inv_s,
                                    unsigned int* counter, cudaStream_t st);
 
+ttq_status launch_channel_total(const float* sum, int64_t T_total, int64_t K,
+                                double* out, cudaStream_t st);
+ttq_status launch_awq_scales_sharded(const float* sum, int64_t T_total,
+                                     int64_t K, int64_t K_total,
+                                     const double* total, double alpha,
+                                     double lambda, double p, float* s,
+                                     float* inv_s, cudaStream_t st);
 ttq_status launch_awq_scales(const float* sum, int64_t T_total, int64_t K,
                              double alpha, double lambda, double p, float* s,
                              float* inv_s, cudaStream_t st);
@@ -48,7 +55,7 @@ ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                           const void* A, int r, void* Xs, void* U,
                           cudaStream_t st);
 
-// The decode projection on CUDA cores (T <= 2), used by
+// The decode projection on CUDA cores (T <= 4), used by
 // launch_gemm_prepared when it applies.
 bool gemv_applies(int64_t T, int64_t K);
 ttq_status launch_gemv(const void* Xs, const void* U, int64_t T, int64_t K,

@@ -6,11 +6,12 @@
 // contraction into FMA), as ttq.h states:
 //   w = W*s;  mn = min(0, min w);  mx = max(0, max w);
 //   D = (mx - mn)/(2^b - 1) (1 if 0);
-//   z = clamp(rint(-mn/D));  q = clamp(rint(w*r) + z),  r = RN(1/D).
-// The zero point takes the IEEE quotient, once per group. The codes take
-// the product with the rounded reciprocal: it lies within one fp32 step of
-// the IEEE quotient w/D, so a code can differ from rint(w/D) + z only where
-// that quotient is within one step of a half-integer (a near-tie).
+//   z = clamp(rint(-mn/D));  q = clamp(rint(w*r) + z),  r = RN(1/D),
+// where rint(w*r) rounds the exact product (one fused multiply-add with the
+// round-to-integer offset below). The zero point takes the IEEE quotient,
+// once per group. The exact product w*r lies within 2^-24 |w/D| of the
+// quotient w/D, so a code can differ from rint(w/D) + z only where the
+// IEEE quotient is within one fp32 step of a half-integer (a near-tie).
 //
 // Design (HBM-bound, kept below the instruction budget): one lane per
 // 32-code block, i.e. 32 consecutive channels of one weight row, loaded as
@@ -192,10 +193,15 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
       const float4 sv =
           STAGED ? *reinterpret_cast<const float4*>(sb + 4 * i)
                  : __ldg(reinterpret_cast<const float4*>(c.s + col0) + i);
-      w[4 * i] = __fmul_rn(w[4 * i], sv.x);
-      w[4 * i + 1] = __fmul_rn(w[4 * i + 1], sv.y);
-      w[4 * i + 2] = __fmul_rn(w[4 * i + 2], sv.z);
-      w[4 * i + 3] = __fmul_rn(w[4 * i + 3], sv.w);
+      // two correctly rounded products per packed multiply
+      const float2 p01 = __fmul2_rn(make_float2(w[4 * i], w[4 * i + 1]),
+                                    make_float2(sv.x, sv.y));
+      const float2 p23 = __fmul2_rn(make_float2(w[4 * i + 2], w[4 * i + 3]),
+                                    make_float2(sv.z, sv.w));
+      w[4 * i] = p01.x;
+      w[4 * i + 1] = p01.y;
+      w[4 * i + 2] = p23.x;
+      w[4 * i + 3] = p23.y;
     }
   }
   // groups never straddle warp-items (32 is a multiple of group/32 and a
@@ -244,7 +250,7 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
   for (int e = 0; e < 32; ++e) {
     const int gi = e / E;
     const float t =
-        fminf(__fadd_rn(__fmul_rn(w[e], r[gi]), kMagic), topz[gi]);
+        fminf(__fmaf_rn(w[e], r[gi], kMagic), topz[gi]);
     const uint32_t tb = __float_as_uint(t);  // bits(M) + q - z
     const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
     if (sh + BITS <= 32) {

@@ -5,6 +5,11 @@
     python -m test_weight_quantization_b200.measure quantize N K bits group
     python -m test_weight_quantization_b200.measure gemm     T N K bits group
     python -m test_weight_quantization_b200.measure table    (the shapes below)
+    python -m test_weight_quantization_b200.measure [--eager] KIND ...
+        (--eager launches directly instead of replaying a CUDA graph)
+    python -m test_weight_quantization_b200.measure decode   [T ...]
+        (the decode sweep: 14336x4096 and 4096x14336, b in 2..5, g in
+        16..128, at each T given; default T = 1 2 4 16)
 
 Each call is captured REPS times in a CUDA graph and timed with CUDA events
 around a replay, after three warm-up calls. Inputs are seeded and
@@ -40,8 +45,30 @@ def peaks():
     return 6650.0, 1400.0
 
 
+EAGER = False  # --eager: launch directly instead of replaying a graph
+
+
+def eager_us(fns):
+    """Mean device time of one call, launched directly (for profilers)."""
+    st = torch.cuda.Stream()
+    n = max(REPS, len(fns))
+    with torch.cuda.stream(st):
+        for f in fns[:3]:
+            f()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for i in range(n):
+            fns[i % len(fns)]()
+        b.record()
+    st.synchronize()
+    return a.elapsed_time(b) / n * 1e3
+
+
 def graph_us(fns):
     """Mean device time of one call, the calls in ``fns`` replayed in turn."""
+    if EAGER:
+        return eager_us(fns)
     st = torch.cuda.Stream()
     with torch.cuda.stream(st):
         for f in fns[:3]:
@@ -174,7 +201,24 @@ TABLE = [
 FNS = {"stats": stats, "prepare": prepare, "quantize": quantize, "gemm": gemm}
 
 
+def decode(*Ts):
+    """The decode sweep's shapes at the given token counts."""
+    for T in Ts or (1, 2, 4, 16):
+        for N, K in ((14336, 4096), (4096, 14336)):
+            for bits in (2, 3, 4, 5):
+                for group in (16, 32, 64, 128):
+                    gemm(T, N, K, bits, group)
+                    torch.cuda.empty_cache()
+
+
 def main(argv):
+    global EAGER
+    if argv and argv[0] == "--eager":
+        EAGER = True
+        argv = argv[1:]
+    if argv and argv[0] == "decode":
+        decode(*[int(a) for a in argv[1:]])
+        return
     if not argv or argv[0] == "table":
         for kind, args in TABLE:
             FNS[kind](*args)

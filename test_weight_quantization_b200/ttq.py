@@ -60,6 +60,8 @@ def _load() -> ctypes.CDLL:
         "ttq_codes_ld": [I64, I],
         "ttq_groups_ld": [I64, I],
         "ttq_selftest_bounded_wait": [I, P, P],
+        "ttq_channel_moment_total": [P, I64, I64, P, P],
+        "ttq_awq_scales_sharded": [P, I64, I64, I64, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -81,7 +83,8 @@ EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_act_stats_scales",
            "ttq_prepare_activations", "ttq_w_lowbit_gemm_prepared",
            "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
            "ttq_device_error", "ttq_abi_version", "ttq_codes_ld",
-           "ttq_groups_ld", "ttq_selftest_bounded_wait")
+           "ttq_groups_ld", "ttq_selftest_bounded_wait",
+           "ttq_channel_moment_total", "ttq_awq_scales_sharded")
 
 
 class _Params(ctypes.Structure):
@@ -265,6 +268,44 @@ def awq_scales(sums: torch.Tensor, T_total: int, alpha: float = 0.5,
     return s, inv_s
 
 
+def channel_moment_total(sums: torch.Tensor, T_total: int,
+                         out: torch.Tensor | None = None) -> torch.Tensor:
+    """sum_j sums[j] / T_total of one shard's channels, fp64 [1] on the
+    device (the shard's part of the shrinkage mean)."""
+    _buf(sums, "sums", torch.float32, 0)
+    K = sums.shape[0]
+    out = torch.empty(1, dtype=torch.float64, device=sums.device) \
+        if out is None else out
+    _buf(out, "out", torch.float64, 1)
+    _check(_lib.ttq_channel_moment_total(sums.data_ptr(), int(T_total), K,
+                                         out.data_ptr(), _stream()),
+           "ttq_channel_moment_total")
+    return out
+
+
+def awq_scales_sharded(sums: torch.Tensor, T_total: int, K_total: int,
+                       total: torch.Tensor, alpha: float = 0.5,
+                       lam: float = 0.1, p: float = 2.0, s=None, inv_s=None):
+    """Step 2 of one shard of the input channels: (s, inv_s) fp32 [K] with
+    the shrinkage mean total / K_total, total being the fp64 [1] sum of every
+    shard's channel_moment_total."""
+    _buf(sums, "sums", torch.float32, 0)
+    _buf(total, "total", torch.float64, 1)
+    K = sums.shape[0]
+    s = torch.empty(K, dtype=torch.float32, device=sums.device) if s is None \
+        else s
+    inv_s = torch.empty_like(s) if inv_s is None else inv_s
+    _buf(s, "s", torch.float32, K)
+    _buf(inv_s, "inv_s", torch.float32, K)
+    prm = _Params(0, 0, alpha, lam, p)
+    _check(_lib.ttq_awq_scales_sharded(sums.data_ptr(), int(T_total), K,
+                                       int(K_total), ctypes.addressof(prm),
+                                       total.data_ptr(), s.data_ptr(),
+                                       inv_s.data_ptr(), _stream()),
+           "ttq_awq_scales_sharded")
+    return s, inv_s
+
+
 def new_counter(device=None) -> torch.Tensor:
     """A zeroed device word for act_stats_scales (one per concurrent
     stream; each call leaves it zero again)."""
@@ -386,7 +427,7 @@ def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
                            B: torch.Tensor | None = None,
                            out: torch.Tensor | None = None,
                            out_dtype=torch.bfloat16) -> torch.Tensor:
-    """The projection on prepared operands (one kernel launch; one or two
+    """The projection on prepared operands (one kernel launch; up to four
     tokens run on CUDA cores, more on tensor cores)."""
     _dev(Xs, "Xs")
     if Xs.dim() != 2:

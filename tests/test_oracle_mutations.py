@@ -27,6 +27,9 @@ MISTAKES = [
     ("shrink_weights_swapped",
      "(1.0 - lambda) * m[j] + lambda * mbar",
      "lambda * m[j] + (1.0 - lambda) * mbar"),
+    ("given_mean_replaced_by_own_statistic",
+     "double c = (1.0 - lambda) * m + lambda * mbar;",
+     "double c = (1.0 - lambda) * m + lambda * m;"),
     ("exponent_alpha_times_p",
      "sj = pow(c, alpha / p);", "sj = pow(c, alpha * p);"),
     ("range_not_widened_to_zero",

@@ -116,6 +116,28 @@ def test_scales_monotone_in_statistic():
     assert np.all(np.diff(s[order]) >= 0)
 
 
+def test_scales_of_channel_shards_with_the_global_mean_equal_the_whole():
+    """Splitting the channels into shards and giving every shard the mean
+    over all channels reproduces the scales of the unsplit layer; giving it
+    its own shard's mean does not (the shrinkage mixes in all channels)."""
+    rng = np.random.default_rng(21)
+    T, K = 40, 96
+    X = rng.standard_normal((T, K)) * np.exp(rng.standard_normal(K))
+    sums = oracle.act_sums(X)
+    s, inv = oracle.awq_scales(sums, T, 0.5, 0.3, 2.0)
+    mbar = float(np.mean(sums / T))
+    parts = [oracle.awq_scales_given_mean(sums[a:b], T, mbar, 0.5, 0.3, 2.0)
+             for a, b in ((0, 32), (32, 96))]
+    np.testing.assert_allclose(np.concatenate([p[0] for p in parts]), s,
+                               rtol=1e-13)
+    np.testing.assert_allclose(np.concatenate([p[1] for p in parts]), inv,
+                               rtol=1e-13)
+    own, _ = oracle.awq_scales_given_mean(sums[:32], T,
+                                          float(np.mean(sums[:32] / T)), 0.5,
+                                          0.3, 2.0)
+    assert np.max(np.abs(own / s[:32] - 1)) > 1e-3
+
+
 def test_scales_degenerate_zero_statistic():
     s, inv = oracle.awq_scales(np.zeros(32), 10, 0.5, 0.0, 2.0)
     assert np.all(s == 1.0) and np.all(inv == 1.0)

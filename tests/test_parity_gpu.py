@@ -141,6 +141,59 @@ def test_stats_scales_fused_zero_input(ttq):
     assert torch.all(sums == 0) and torch.all(s == 1) and torch.all(inv == 1)
 
 
+# ------------------------------------------- sharded (row-parallel) scales ----
+
+def test_channel_total_and_sharded_scales(ttq):
+    """Input channels split in two shards: each shard's channel total, added
+    (the all-reduce of a row-parallel layer, here on one GPU), gives every
+    shard the scales the unsplit layer has."""
+    T, K = 300, 1152
+    X = acts(T, K, 71, torch.bfloat16).cuda()
+    sums = ttq.act_stats(X)
+    s_full, inv_full = ttq.awq_scales(sums, T, 0.5, 0.1, 2.0)
+    parts, totals = [], []
+    for a, b in ((0, 512), (512, 1152)):
+        sh = ttq.act_stats(X[:, a:b].contiguous())
+        parts.append(sh)
+        totals.append(ttq.channel_moment_total(sh, T))
+    total = totals[0] + totals[1]
+    ref_total = np.sum(np32(sums).astype(np.float64) / T)
+    assert abs(total.item() - ref_total) <= 1e-12 * abs(ref_total)
+    got = [ttq.awq_scales_sharded(sh, T, K, total, 0.5, 0.1, 2.0)
+           for sh in parts]
+    s = torch.cat([g[0] for g in got])
+    inv = torch.cat([g[1] for g in got])
+    rs, rinv = oracle.awq_scales(np32(sums).astype(np.float64), T, 0.5, 0.1,
+                                 2.0)
+    assert_rel_close(np32(s), rs, what="sharded s")
+    assert_rel_close(np32(inv), rinv, what="sharded inv_s")
+    assert torch.allclose(s, s_full, rtol=1e-6, atol=0)
+
+
+def test_row_parallel_projection_on_one_gpu(ttq):
+    """The row-parallel layer's arithmetic, its two ranks run one after the
+    other on one GPU and their fp32 partial outputs added: the oracle's
+    unsplit projection within the projection tolerance."""
+    T, N, K, bits, group = 200, 320, 1024, 4, 128
+    X = acts(T, K, 72, torch.bfloat16).cuda()
+    W = weights(N, K, 73, torch.bfloat16).cuda()
+    shards = ((0, 512), (512, 1024))
+    sums = [ttq.act_stats(X[:, a:b].contiguous()) for a, b in shards]
+    total = sum(ttq.channel_moment_total(sh, T) for sh in sums)
+    Y = torch.zeros(T, N, dtype=torch.float32, device="cuda")
+    for (a, b), sh in zip(shards, sums):
+        s, inv = ttq.awq_scales_sharded(sh, T, K, total)
+        c, d, z = ttq.quantize_rtn_grouped(W[:, a:b].contiguous(), s, bits,
+                                           group)
+        Y += ttq.w_lowbit_gemm(X[:, a:b].contiguous(), inv, c, d, z, N, bits,
+                               group, out_dtype=torch.float32)
+    # the oracle's unsplit layer on the GPU's scales
+    s_full, inv_full = ttq.awq_scales(ttq.act_stats(X), T)
+    c, d, z = ttq.quantize_rtn_grouped(W, s_full, bits, group)
+    ref = oracle_y(X.cpu(), inv_full, c, d, z, N, bits, group)
+    assert_gemm_close(np32(Y), ref, "row-parallel on one GPU", Y.dtype)
+
+
 # ---------------------------------------------------------- quantize ----
 
 def dense(c, d, z, K, bits, group):
@@ -301,13 +354,13 @@ def test_one_and_two_tokens_with_very_long_rows(ttq):
                           f"long rows T={T}", Y.dtype)
 
 
-@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("group", [16, 32, 128])
 def test_decode_gemv(ttq, T, bits, group):
-    """One or two tokens take the CUDA-core matrix-vector path; every code
-    width and group size against the oracle (K spans 10 row passes of a
-    warp's lanes and a ragged one)."""
+    """Up to four tokens take the CUDA-core matrix-vector path; every code
+    width and group size against the oracle (K spans several work units of
+    a warp's lanes and a ragged one)."""
     N, K = 300, 1408
     X = acts(T, K, 40 + T + bits, torch.bfloat16)
     W = weights(N, K, 41 + bits, torch.bfloat16)
@@ -316,8 +369,27 @@ def test_decode_gemv(ttq, T, bits, group):
     assert_gemm_close(np32(Y), ref, f"gemv T={T} b={bits} g={group}", Y.dtype)
 
 
+def test_decode_gemv_many_rows_per_block(ttq):
+    """160000 rows of K = 256: each CTA owns more rows than its shared
+    memory holds partial sums for, so it works through them in chunks.
+    Sampled output channels (first and last included) against the oracle."""
+    N, K, bits, group = 160000, 256, 4, 32
+    rng = np.random.default_rng(61)
+    W = torch.from_numpy((rng.standard_normal((N, K)) * 0.02).astype(
+        np.float32)).to(torch.bfloat16)
+    for T in (1, 4):
+        X = acts(T, K, 62 + T, torch.bfloat16)
+        Y, inv, c, d, z = run_path(ttq, X, W, bits, group)
+        rows = np.unique(np.concatenate([[0, N - 1], rng.choice(
+            np.arange(1, N - 1), 2000, replace=False)]))
+        cd, dd, zd = dense(c, d, z, K, bits, group)
+        ref = oracle.lowbit_gemm(np32(X), np32(inv), cd[rows], dd[rows],
+                                 zd[rows], len(rows), bits, group)
+        assert_gemm_close(np32(Y)[:, rows], ref, f"many rows T={T}", Y.dtype)
+
+
 @pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
-@pytest.mark.parametrize("T", [1, 2])
+@pytest.mark.parametrize("T", [1, 2, 4])
 def test_decode_gemv_lowrank_and_dtypes(ttq, out, T):
     N, K, r, bits, group = 200, 512, 16, 4, 64
     X = acts(T, K, 50 + T, torch.bfloat16)
