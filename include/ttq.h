@@ -226,7 +226,7 @@ size_t ttq_w_lowbit_gemm_workspace_size(int64_t T, int64_t K, int r);
  * The tensor cores take fp16 operands: X / s is rounded once to fp16 and
  * each weight (q - z) * D once to fp16; products accumulate in fp32.
  * |X / s| must stay below 65504 (else TTQ_DEVERR_FP16_RANGE is raised).
- * Which kernel runs depends on T: T <= 4 a CUDA-core matrix-vector product
+ * Which kernel runs depends on T: T <= 2 a CUDA-core matrix-vector product
  * (the weight (q - z) D is applied in fp32, the activations are the fp16
  * X / s) when its staged activations (about 4.75 T K bytes) fit its shared
  * memory, otherwise and up to T = 32 the tensor-core decode configuration
@@ -263,7 +263,7 @@ ttq_status ttq_prepare_activations(const void* X, ttq_dtype xt, int64_t T,
                                    void* U, void* stream);
 
 /* ttq_w_lowbit_gemm_prepared: the projection on prepared operands, one
- * kernel launch (T <= 4: CUDA cores, otherwise tensor cores, as above):
+ * kernel launch (T <= 2: CUDA cores, otherwise tensor cores, as above):
  *   Y[t][n] = sum_j Xs[t][j] (q[n][j] - z) D + sum_rho U[t][rho] B[n][rho].
  * Xs, U as written by ttq_prepare_activations for the same bits; B [N, r]
  * of dtype bt. */
@@ -275,6 +275,61 @@ ttq_status ttq_w_lowbit_gemm_prepared(const void* Xs, const void* U,
                                       const void* B, ttq_dtype bt, int r,
                                       void* Y, ttq_dtype yt, int64_t ldy,
                                       void* stream);
+
+/* Steps 3 and 4 in one launch: the projection quantizes the weights
+ * itself (TTQ review, Proposed method, bullet 1: group-wise RTN with QDQ,
+ * quantize then dequantize inside the projection). The tensor-core
+ * producer loads bf16 tiles of W; the dequantiser warps quantize each
+ * 128-channel stage exactly as ttq_quantize_rtn_grouped does (same codes,
+ * delta and zero, the same near-tie behaviour), dequantise as the codes
+ * path does and feed the tensor cores; Y equals ttq_w_lowbit_gemm_prepared
+ * on ttq_quantize_rtn_grouped's output bit for bit.
+ *   W        [N, K] bf16, row pitch ldw (16-byte aligned rows); s [K]
+ *            float32 scales (ttq_awq_scales), 16-byte aligned.
+ *   Xs, U, B, r, Y, yt, ldy   as for ttq_w_lowbit_gemm_prepared.
+ *   codes, delta, zero   where to store the quantized weights for later
+ *            (decode) use, in the layout above, written once by the CTAs of
+ *            the first token tile; all three NULL to skip. Row padding is
+ *            left untouched.
+ * Every token tile quantizes its weight tiles again, so the form pays off
+ * where the prompt spans few token tiles. Only the prefill tile (T > 32)
+ * runs it, and W must be bf16: otherwise TTQ_ERR_UNSUPPORTED. */
+ttq_status ttq_quantize_gemm_prepared(
+    const void* W, ttq_dtype wt, int64_t ldw, const float* s, const void* Xs,
+    const void* U, int64_t T, int64_t K, int64_t N, int bits, int group,
+    const void* B, ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy,
+    uint32_t* codes, float* delta, uint8_t* zero, void* stream);
+
+/* The projection on prepared operands that also emits the statistic of
+ * its own output for the layer that takes that output as input (TTQ
+ * review, Proposed method, bullets 2-3: the next layer's per-channel
+ * statistic, here computed in the projection's epilogue instead of by a
+ * separate pass over Y). Same arguments and Y as
+ * ttq_w_lowbit_gemm_prepared, plus:
+ *   p        moment order (> 0) of the statistic;
+ *   stats    [stats_rows][N] float32 device buffer of partial sums:
+ *            row i holds, for every output channel n, the sum of
+ *            |Y[t][n]|^p over one range of tokens, Y[t][n] being the value
+ *            stored in Y (after rounding to yt); ranges are disjoint and
+ *            cover all T tokens;
+ *   stats_rows  must equal ttq_projection_stats_rows(T, N, K, bits).
+ * ttq_stats_reduce then gives sum_out[n] = sum_t |Y[t][n]|^p, the input
+ * of ttq_awq_scales for that layer. Only the tensor-core prefill form
+ * (T > 32) computes it: for T <= 32 ttq_projection_stats_rows returns 0 and
+ * the call returns TTQ_ERR_UNSUPPORTED. A wrong stats_rows or a bad p
+ * returns TTQ_ERR_INVALID_ARG. */
+int64_t ttq_projection_stats_rows(int64_t T, int64_t N, int64_t K, int bits);
+ttq_status ttq_w_lowbit_gemm_prepared_stats(
+    const void* Xs, const void* U, int64_t T, int64_t K, const uint32_t* codes,
+    const float* delta, const uint8_t* zero, int64_t N, int bits, int group,
+    const void* B, ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy,
+    float p, float* stats, int64_t stats_rows, void* stream);
+
+/* sum_out[n] (+)= sum_i partials[i][n] over the P rows in order (fp32,
+ * deterministic). partials [P][N], sum_out [N], device; accumulate 0 or 1.
+ * Invalid arguments return TTQ_ERR_INVALID_ARG. */
+ttq_status ttq_stats_reduce(const float* partials, int64_t P, int64_t N,
+                            int accumulate, float* sum_out, void* stream);
 
 /* ttq_w_lowbit_gemm without a workspace argument, for callers that cannot
  * allocate device memory where they run the projection (a plugin called by
@@ -342,7 +397,9 @@ ttq_status ttq_selftest_bounded_wait(int arrive, uint32_t* out, void* stream);
 
 /* ABI version of this header (3: ttq_act_stats_scales added; 4:
  * ttq_selftest_bounded_wait added; 5: ttq_channel_moment_total and
- * ttq_awq_scales_sharded added). */
+ * ttq_awq_scales_sharded added; 6: ttq_projection_stats_rows,
+ * ttq_w_lowbit_gemm_prepared_stats and ttq_stats_reduce added; 7:
+ * ttq_quantize_gemm_prepared added). */
 int ttq_abi_version(void);
 
 #ifdef __cplusplus

@@ -92,7 +92,7 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 5; }
+TTQ_EXPORT int ttq_abi_version(void) { return 7; }
 
 TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
   if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
@@ -282,6 +282,76 @@ TTQ_EXPORT ttq_status ttq_w_lowbit_gemm_prepared(
     return TTQ_ERR_INVALID_ARG;
   return launch_gemm_prepared(Xs, U, T, K, codes, delta, zero, N, bits, group,
                               B, bt, r, Y, yt, ldy, as_stream(stream));
+}
+
+TTQ_EXPORT int64_t ttq_projection_stats_rows(int64_t T, int64_t N, int64_t K,
+                                            int bits) {
+  if (T < 1 || N < 1 || K < 32 || K % 32 != 0 || bits < 2 || bits > 8 ||
+      T >= ((int64_t)1 << 31) || N >= ((int64_t)1 << 31) ||
+      K >= ((int64_t)1 << 31))
+    return 0;
+  return gemm_stats_rows(T, N, K, bits);
+}
+
+TTQ_EXPORT ttq_status ttq_w_lowbit_gemm_prepared_stats(
+    const void* Xs, const void* U, int64_t T, int64_t K, const uint32_t* codes,
+    const float* delta, const uint8_t* zero, int64_t N, int bits, int group,
+    const void* B, ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy,
+    float p, float* stats, int64_t stats_rows, void* stream) {
+  if (!stats || !(p > 0.f) || !isfinite(p) || !aligned(stats, 4))
+    return TTQ_ERR_INVALID_ARG;
+  const int64_t rows = ttq_projection_stats_rows(T, N, K, bits);
+  if (rows == 0) return TTQ_ERR_UNSUPPORTED;
+  if (stats_rows != rows) return TTQ_ERR_INVALID_ARG;
+  if (!Xs || !codes || !delta || !zero || !Y || !valid_dtype(yt) ||
+      !valid_group(group) || K % group != 0 || r < 0 || r > 64 ||
+      ((r > 0) != (U && B)) || (r == 0 && (U || B)) ||
+      (r > 0 && !valid_dtype(bt)) || ldy < N || !aligned(Xs, 16) ||
+      (U && !aligned(U, 16)) || !aligned(codes, 16) || !aligned(delta, 16) ||
+      !aligned(zero, 16) || !aligned(Y, dtype_bytes(yt)) ||
+      (r > 0 && !aligned(B, dtype_bytes(bt))))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_gemm_prepared(Xs, U, T, K, codes, delta, zero, N, bits, group,
+                              B, bt, r, Y, yt, ldy, as_stream(stream), stats,
+                              p);
+}
+
+TTQ_EXPORT ttq_status ttq_quantize_gemm_prepared(
+    const void* W, ttq_dtype wt, int64_t ldw, const float* s, const void* Xs,
+    const void* U, int64_t T, int64_t K, int64_t N, int bits, int group,
+    const void* B, ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy,
+    uint32_t* codes, float* delta, uint8_t* zero, void* stream) {
+  if (!W || !s || !Xs || !Y || !valid_dtype(wt) || !valid_dtype(yt) || T < 1 ||
+      N < 1 || K < 32 || K % 32 != 0 || bits < 2 || bits > 8 ||
+      !valid_group(group) || K % group != 0 || r < 0 || r > 64 ||
+      ((r > 0) != (U && B)) || (r == 0 && (U || B)) ||
+      (r > 0 && !valid_dtype(bt)) || ldw < K || ldy < N ||
+      !rows_aligned(W, wt, ldw) || !aligned(s, 16) || !aligned(Xs, 16) ||
+      (U && !aligned(U, 16)) || !aligned(Y, dtype_bytes(yt)) ||
+      (r > 0 && !aligned(B, dtype_bytes(bt))) ||
+      ((codes != nullptr) != (delta != nullptr)) ||
+      ((codes != nullptr) != (zero != nullptr)) ||
+      (codes && (!aligned(codes, 16) || !aligned(delta, 16) ||
+                 !aligned(zero, 16))) ||
+      T >= ((int64_t)1 << 31) || K >= ((int64_t)1 << 31) ||
+      N >= ((int64_t)1 << 31))
+    return TTQ_ERR_INVALID_ARG;
+  // the fused form reads bf16 weight tiles and runs the prefill tile only
+  if (wt != TTQ_BF16 || T <= 32) return TTQ_ERR_UNSUPPORTED;
+  return launch_quantize_gemm_prepared(W, ldw, s, Xs, U, T, K, N, bits, group,
+                                       B, bt, r, Y, yt, ldy, codes, delta,
+                                       zero, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_stats_reduce(const float* partials, int64_t P,
+                                       int64_t N, int accumulate,
+                                       float* sum_out, void* stream) {
+  if (!partials || !sum_out || P < 1 || N < 1 ||
+      (accumulate != 0 && accumulate != 1) || !aligned(partials, 4) ||
+      !aligned(sum_out, 4))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_stats_reduce(partials, P, N, accumulate, sum_out,
+                             as_stream(stream));
 }
 
 TTQ_EXPORT ttq_status ttq_lowrank_add(const void* X, ttq_dtype xt, int64_t T,

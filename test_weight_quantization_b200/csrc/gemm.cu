@@ -25,7 +25,7 @@
 // accumulator leaves TMEM in 16x256b fragment order, is packed to 16-bit
 // pairs and written transposed by stmatrix into 128-byte-swizzled boxes of
 // the idle activation ring, and a TMA tensor store writes Y. Decode
-// (T <= 32 where gemv.cu, which takes up to four tokens, does not apply)
+// (T <= 32 where gemv.cu, which takes one or two tokens, does not apply)
 // splits K over a cluster of up to 8 CTAs whose partial tiles every rank
 // reduces in part through distributed shared memory, in rank order. The rank-r low-rank term is one
 // extra K stage, [X~ | U] [W_hat | B]^T with U = X A^T (fp16, from
@@ -52,19 +52,13 @@ constexpr int kParamGroups = 16;   // groups per params chunk
 // CTA = producer warp + MMA warp + DQW dequantiser warps (4, 8 or 16; with
 // 8 or 16, two or four warps share each TMEM lane quarter and split every
 // stage into parts of 64 or 32 channels)
-// Warps: 0 the TMA producer, 1 .. NACC the MMA issuers (NACC accumulators,
-// one per issuer), then the dequantisers.
-__host__ __device__ constexpr int dq_warp0(int nacc) { return 1 + nacc; }
+constexpr int kDqWarp0 = 2;  // first dequantiser warp
 // dequantiser warps of the prefill form (four per SM sub-partition, so that
 // one warp's dependent chain of shared-memory loads, unpacking and TMEM
 // stores overlaps the others')
 constexpr int kPrefillDequantWarps = 16;
-// MMA issuers of the decode form at 16 tokens (half as many at 32): one
-// thread issues an M = 128, N = 16 MMA only every ~140 cycles whatever the
-// accumulator, while issuers in different warps overlap
-constexpr int kDecodeIssuers = 4;
-__host__ __device__ constexpr int cta_threads(int dqw, int nacc) {
-  return 32 * (dq_warp0(nacc) + dqw);
+__host__ __device__ constexpr int cta_threads(int dqw) {
+  return 32 * (kDqWarp0 + dqw);
 }
 constexpr int kParamDeltaBytes = kBM * kParamGroups * 4;
 constexpr int kParamBytes = kParamDeltaBytes + kBM * kParamGroups;
@@ -86,6 +80,16 @@ struct GemmArgs {
   int group;
   int k_stages;   // ceil(K / 128)
   int per;        // stages per split rank
+  // fused quantization (QDQ form): the scales, and where the first token
+  // tile's CTAs store the codes, delta and zero (null: not stored)
+  const float* qs;
+  uint32_t* q_codes;
+  float* q_delta;
+  uint8_t* q_zero;
+  long long q_ldc, q_ldg;
+  float* stats;   // per-row partial sums of |Y|^stats_p, or null
+  float stats_p;
+  int stats_parts;  // partial rows per token tile (1 or 2)
   int y_mode;     // 0: per-row stores (rows not 16-byte aligned);
                   // 1: staged tile [tokens][128] stored through tm_y;
                   // 2: 16-bit Y staged by stmatrix in 128-byte swizzled
@@ -101,19 +105,29 @@ struct Layout {
   uint32_t x, c, p, part, bars, tmem, abort_flag, total, stage_x;
 };
 
+// bf16 weight tile of one stage in the fused (QDQ) form: two 64-channel
+// boxes of 128 rows, 128-byte swizzled
+constexpr uint32_t kWStageBytes = 2u * kBM * 128u;
+// group-range exchange of the fused form: [2 stage parities][4 parts]
+// [128 rows] (min, max)
+constexpr uint32_t kXchgBytes = 2u * 4u * kBM * 8u;
+
 // Shared memory: per stage two 64-channel activation boxes and one codes
-// chunk; two params slots; the split-K partial tile (decode); barriers.
-// The fp16 weight stages live in TMEM.
+// chunk (the bf16 weight tile in the fused form); two params slots (the
+// group-range exchange in the fused form); the split-K partial tile
+// (decode); barriers. The fp16 weight stages live in TMEM.
 __host__ __device__ inline Layout make_layout(int bits, int bn, int S,
-                                              bool split) {
+                                              bool split, bool qdq = false) {
   Layout L;
   L.stage_x = (uint32_t)(2 * bn * 128);
   L.x = 0;
   L.c = L.x + (uint32_t)S * L.stage_x;
-  L.p = L.c + (uint32_t)S * code_chunk_bytes(bits);
-  L.part = L.p + 2u * kParamBytes;
+  L.p = L.c + (uint32_t)S * (qdq ? kWStageBytes : code_chunk_bytes(bits));
+  L.part = L.p + (qdq ? kXchgBytes : 2u * kParamBytes);
   L.bars = L.part + (split ? (uint32_t)(bn * kBM * 4) : 0u);
-  const int nbars = 3 * S + S + 4 + 1;  // loaded, ready, empty, a_free
+  // loaded, ready, empty, a_free; params; accumulator; the fused form's
+  // group-range exchange (4 lane quarters x 2 stage parities)
+  const int nbars = 3 * S + S + 4 + 1 + (qdq ? 8 : 0);
   L.tmem = L.bars + 8u * nbars;
   L.abort_flag = L.tmem + 4;
   L.total = L.abort_flag + 4;
@@ -172,6 +186,20 @@ __device__ __forceinline__ void store_y(void* Y, int yt, long long idx,
     static_cast<__half*>(Y)[idx] = __float2half_rn(v);
   else
     static_cast<float*>(Y)[idx] = v;
+}
+
+// The value Y stores for v (rounded to its dtype), as fp32.
+__device__ __forceinline__ float stored_y(int yt, float v) {
+  if (yt == TTQ_BF16) return __bfloat162float(__float2bfloat16_rn(v));
+  if (yt == TTQ_F16) return __half2float(__float2half_rn(v));
+  return v;
+}
+
+// |y|^p of the fused output statistic.
+__device__ __forceinline__ float y_moment(float y, float p) {
+  if (p == 2.f) return y * y;
+  if (p == 1.f) return fabsf(y);
+  return powf(fabsf(y), p);
 }
 
 __device__ __forceinline__ float load_any(const void* p, int t, long long idx) {
@@ -254,20 +282,24 @@ struct Ring {
 //   MMA        waits `ready`, issues 8 MMAs, commits to `empty`, which frees
 //              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
-template <int BITS, int GMODE, int DQW, int NACC>
-__global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
+// QDQ: the fused form. The producer loads bf16 weight tiles instead of
+// codes, and the dequantiser warps quantize them on the fly (the same
+// arithmetic as quantize.cu), store the codes, delta and zero of the first
+// token tile for later use, and hand the dequantised fp16 weights to the
+// tensor cores as usual (TTQ review, Proposed method, bullet 1: QDQ).
+template <int BITS, int GMODE, int DQW, bool QDQ>
+__global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
     lowbit_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
                        const __grid_constant__ CUtensorMap tm_u,
                        const __grid_constant__ CUtensorMap tm_c,
                        const __grid_constant__ CUtensorMap tm_d,
                        const __grid_constant__ CUtensorMap tm_z,
                        const __grid_constant__ CUtensorMap tm_y,
+                       const __grid_constant__ CUtensorMap tm_w,
                        const GemmArgs p) {
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
-  constexpr uint32_t CHUNK = kBM * 16 * BITS;
+  constexpr uint32_t CHUNK = QDQ ? kWStageBytes : kBM * 16 * BITS;
   constexpr int kDq = 32 * DQW;            // dequantiser threads
-  constexpr int kDqWarp0 = dq_warp0(NACC);
-  static_assert(NACC == 1 || DQW == 4, "several accumulators: decode form");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -276,7 +308,7 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
 
   const int S = p.S, SA = p.SA, bn = p.bn;
   const int split = (int)gridDim.z;
-  const Layout L = make_layout(BITS, bn, S, split > 1);
+  const Layout L = make_layout(BITS, bn, S, split > 1, QDQ);
   const uint32_t b_loaded = base + L.bars;
   const uint32_t b_ready = b_loaded + 8 * S;
   const uint32_t b_empty = b_ready + 8 * S;
@@ -284,6 +316,7 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
   const uint32_t b_full_p = b_afree + 8 * S;
   const uint32_t b_empty_p = b_full_p + 16;
   const uint32_t b_accum = b_empty_p + 16;
+  const uint32_t b_xchg = b_accum + 8;  // fused form: [lane quarter][parity]
   volatile uint32_t* tmem_slot =
       reinterpret_cast<volatile uint32_t*>(gbase + L.tmem);
   volatile int* aborted = reinterpret_cast<volatile int*>(gbase + L.abort_flag);
@@ -303,21 +336,28 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
     for (int i = 0; i < S; ++i) {
       mbar_init(b_loaded + 8 * i, 1);
       mbar_init(b_ready + 8 * i, kDq);
-      mbar_init(b_empty + 8 * i, NACC);
-      mbar_init(b_afree + 8 * i, NACC);
+      mbar_init(b_empty + 8 * i, 1);
+      mbar_init(b_afree + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
       mbar_init(b_empty_p + 8 * i, kDq);
     }
-    mbar_init(b_accum, NACC);
+    mbar_init(b_accum, 1);
+    if constexpr (QDQ) {
+      for (int i = 0; i < 8; ++i) mbar_init(b_xchg + 8 * i, 128);
+    }
     *aborted = 0;
     fence_barrier_init();
     // the tensor maps are kernel parameters: no need to wait for them
     tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_c);
-    tma_prefetch_desc(&tm_d);
-    tma_prefetch_desc(&tm_z);
+    if constexpr (QDQ) {
+      tma_prefetch_desc(&tm_w);
+    } else {
+      tma_prefetch_desc(&tm_c);
+      tma_prefetch_desc(&tm_d);
+      tma_prefetch_desc(&tm_z);
+    }
     if (p.r > 0) tma_prefetch_desc(&tm_u);
   }
   // The set-up above and the TMEM allocation touch no global memory, so
@@ -345,7 +385,7 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
       bool ok = true;
       for (int s = 0; s < n_total; ++s) {
         const int k0 = (ks_begin + s) * kSK;
-        if (s < n_main) {
+        if (!QDQ && s < n_main) {
           const int pc = k0 >> (lg + 4);  // params chunk: 16 groups
           if (pc != pchunk) {
             if (pchunk >= 0) rp.next(2);
@@ -374,8 +414,13 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
         const uint32_t xdst = base + L.x + rs.slot * L.stage_x;
         if (s < n_main) {
           mbar_arrive_expect_tx(bar, CHUNK + 2 * xbytes);
-          tma_load_2d(base + L.c + rs.slot * CHUNK, &tm_c, (k0 >> 7) * 4 * BITS,
-                      m0, bar);
+          const uint32_t cdst = base + L.c + rs.slot * CHUNK;
+          if constexpr (QDQ) {
+            tma_load_2d(cdst, &tm_w, k0, m0, bar);
+            tma_load_2d(cdst + CHUNK / 2, &tm_w, k0 + 64, m0, bar);
+          } else {
+            tma_load_2d(cdst, &tm_c, (k0 >> 7) * 4 * BITS, m0, bar);
+          }
           tma_load_2d(xdst, &tm_x, k0, t0, bar);
           tma_load_2d(xdst + xbytes, &tm_x, k0 + 64, t0, bar);
         } else {
@@ -397,20 +442,15 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
         mbar_wait(b_full_p + 8 * (q & 1), (uint32_t)(q >> 1) & 1, p.err);
       }
     }
-  } else if (warp <= NACC) {
-    // ------------------------------------------------ MMA issuers -----
-    // A stage is eight K steps of 16 channels. With NACC issuers, issuer j
-    // (one elected thread of warp 1 + j) issues K steps j*8/NACC .. into
-    // its own accumulator at column j*bn, so the issuers' MMAs overlap; the
-    // accumulators are added in order before the epilogue.
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer -----
+    // (Issuing a stage's MMAs from several warps into separate accumulators
+    // was measured slower for the decode tile: 21.9 against 19.3 us on
+    // 14336 x 4096 at 16 tokens.)
     if (lane == 0) {
-      constexpr int KPI = 8 / NACC;  // K steps per issuer and stage
-      const int j = warp - 1;
-      const uint32_t acc = tmem + (uint32_t)(j * bn);
       const uint32_t idesc = idesc_f16_f32(kBM, bn);
       const uint32_t xbytes = (uint32_t)bn * 128u;
       Ring rs, ra;
-      bool first = true;
       for (int s = 0; s < n_total; ++s) {
         if (!mbar_wait(b_ready + 8 * rs.slot, rs.round & 1, p.err)) {
           *aborted = 1;
@@ -421,17 +461,16 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
         const uint32_t xs = base + L.x + rs.slot * L.stage_x;
         const uint64_t bd0 = smem_desc_sw128(xs);
         const uint64_t bd1 = smem_desc_sw128(xs + xbytes);
-        // the low-rank stage has only the four K steps of its first box
-        const int steps = s < n_main ? 8 : 4;
+        // the stage's eight K steps back to back (four for the low-rank
+        // stage)
 #pragma unroll
-        for (int u = 0; u < KPI; ++u) {
-          const int kidx = j * KPI + u;
-          if (kidx < steps) {
-            const uint64_t bd =
-                kidx < 4 ? bd0 + 2 * kidx : bd1 + 2 * (kidx - 4);
-            tc_mma_f16_ts(acc, ad + 8 * kidx, bd, idesc, first ? 0u : 1u);
-            first = false;
-          }
+        for (int k = 0; k < 4; ++k)
+          tc_mma_f16_ts(tmem, ad + 8 * k, bd0 + 2 * k, idesc,
+                        (s > 0 || k > 0) ? 1u : 0u);
+        if (s < n_main) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ts(tmem, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
         }
         tc_commit(b_empty + 8 * rs.slot);
         tc_commit(b_afree + 8 * ra.slot);
@@ -463,6 +502,164 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
     int pchunk = -1;
     bool ok_loop = true;
 
+    // The fused (QDQ) form of a main stage: this warp's 32 channels (block
+    // h of the stage) of row i, quantized from the bf16 tile exactly as
+    // quantize.cu does, dequantised as the codes path does, stored to TMEM;
+    // the first token tile also stores the codes, delta and zero.
+    auto qdq_stage = [&](int s, int k0, uint32_t acol) {
+      if constexpr (QDQ) {
+        static_assert(DQW == 16, "the fused form uses 16 dequantiser warps");
+        constexpr int QMAX = (1 << BITS) - 1;
+        constexpr float kMagic = 12582912.0f;  // rint by 1.5 * 2^23
+        constexpr float kTop = kMagic + (float)QMAX;
+        constexpr int NG = GMODE == 0 ? 2 : 1;  // groups in the block
+        constexpr int E = 32 / NG;
+        constexpr int PERM = (BITS == 2 || BITS == 4 || BITS == 8) ? BITS : 0;
+        // raw bf16 weights: box h >> 1, 16-byte chunks (h & 1) * 4 .. + 3
+        // of row i, stored at chunk ^ (i % 8) (128-byte swizzle)
+        const uint32_t wrow = base + L.c + rs.slot * CHUNK +
+                              (uint32_t)(h >> 1) * (CHUNK / 2) +
+                              (uint32_t)i * 128u;
+        float w[32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t c = (uint32_t)((h & 1) * 4 + cc);
+          uint32_t v[4];
+          asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                       : "r"(wrow + ((c ^ ((uint32_t)i & 7u)) << 4))
+                       : "memory");
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            w[8 * cc + 2 * e] = __uint_as_float(v[e] << 16);
+            w[8 * cc + 2 * e + 1] = __uint_as_float(v[e] & 0xFFFF0000u);
+          }
+        }
+        // w = W * s (the same scale for every row: broadcast loads); a
+        // block past K (the last stage's tail) holds zeros from the tile
+        // load and keeps them
+        const bool in_k = k0 + 32 * h < p.K;
+        const float4* sp = reinterpret_cast<const float4*>(
+            p.qs + (in_k ? k0 + 32 * h : 0));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 sv = in_k ? __ldg(sp + q) : make_float4(0.f, 0.f, 0.f,
+                                                               0.f);
+          const float2 a = __fmul2_rn(make_float2(w[4 * q], w[4 * q + 1]),
+                                      make_float2(sv.x, sv.y));
+          const float2 b = __fmul2_rn(make_float2(w[4 * q + 2], w[4 * q + 3]),
+                                      make_float2(sv.z, sv.w));
+          w[4 * q] = a.x;
+          w[4 * q + 1] = a.y;
+          w[4 * q + 2] = b.x;
+          w[4 * q + 3] = b.y;
+        }
+        // group ranges widened to contain 0; groups of 64 or 128 channels
+        // span two or four warps of this lane quarter, which exchange their
+        // parts through shared memory (two slots by stage parity)
+        float mn[NG], mx[NG];
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+          mn[gi] = 0.f;
+          mx[gi] = 0.f;
+#pragma unroll
+          for (int e = gi * E; e < (gi + 1) * E; ++e) {
+            mn[gi] = fminf(mn[gi], w[e]);
+            mx[gi] = fmaxf(mx[gi], w[e]);
+          }
+        }
+        if (NG == 1 && p.group >= 64) {
+          const uint32_t xslot =
+              base + L.p + (uint32_t)((s & 1) * 4) * kBM * 8u;
+          const uint32_t mine = xslot + (uint32_t)(h * kBM + i) * 8u;
+          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(mine),
+                       "f"(mn[0]), "f"(mx[0])
+                       : "memory");
+          // the lane quarter's four warps meet on a bounded barrier (its
+          // phase of use s >> 1); a wait that gives up flags the error word
+          const uint32_t bx = b_xchg + 8u * (uint32_t)(2 * q4 + (s & 1));
+          mbar_arrive(bx);
+          mbar_wait(bx, (uint32_t)(s >> 1) & 1u, p.err);
+          const int gp = p.group >> 5;  // parts per group: 2 or 4
+          const int h0 = h & ~(gp - 1);
+          for (int j = 0; j < gp; ++j) {
+            float a, b;
+            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];"
+                         : "=f"(a), "=f"(b)
+                         : "r"(xslot + (uint32_t)((h0 + j) * kBM + i) * 8u)
+                         : "memory");
+            mn[0] = fminf(mn[0], a);
+            mx[0] = fmaxf(mx[0], b);
+          }
+        }
+        float dd[NG], r[NG], zf[NG], topz[NG], botz[NG];
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+          float d0 = __fdiv_rn(__fsub_rn(mx[gi], mn[gi]), (float)QMAX);
+          if (d0 == 0.f) d0 = 1.f;
+          dd[gi] = d0;
+          r[gi] = __frcp_rn(d0);
+          zf[gi] = fminf(fmaxf(__fadd_rn(__fdiv_rn(-mn[gi], d0), kMagic),
+                               kMagic),
+                         kTop) - kMagic;
+          topz[gi] = kTop - zf[gi];
+          botz[gi] = kMagic - zf[gi];
+        }
+        uint32_t qv[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int gi = e / E;
+          const float t = fmaxf(
+              fminf(__fmaf_rn(w[e], r[gi], kMagic), topz[gi]), botz[gi]);
+          qv[e] = __float_as_uint(t) - 0x4B400000u + (uint32_t)zf[gi];
+        }
+        // fp16 pairs in the codes path's TMEM order: position p of a span
+        // holds channel k_perm(p); (1024 + q) - (1024 + z), then times D
+        // rounded to fp16: the codes path's exact operations
+        uint32_t o[16];
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) {
+          const int pa = 2 * pp, pb = 2 * pp + 1;
+          const int ca = 16 * (pa >> 4) + k_perm<PERM>(pa & 15);
+          const int cb = 16 * (pb >> 4) + k_perm<PERM>(pb & 15);
+          const int gi = ca / E;
+          const uint32_t x = (0x6400u | qv[ca]) | ((0x6400u | qv[cb]) << 16);
+          const uint32_t zz = (0x6400u | (uint32_t)zf[gi]) * 0x00010001u;
+          o[pp] = h2_bits(__hmul2(__hsub2(bits_h2(x), bits_h2(zz)),
+                                  __float2half2_rn(dd[gi])));
+        }
+        tmem_st16(acol + 16u * h, o);
+        // the codes, delta and zero, once (the first token tile)
+        if (blockIdx.y == 0 && p.q_codes != nullptr && row_ok && in_k) {
+          uint32_t cw[BITS];
+#pragma unroll
+          for (int k = 0; k < BITS; ++k) cw[k] = 0u;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
+            cw[wd] |= qv[e] << sh;
+            if (sh + BITS > 32) cw[wd + 1] |= qv[e] >> (32 - sh);
+          }
+          uint32_t* dst = p.q_codes + (long long)n * p.q_ldc +
+                          (long long)(k0 / 32 + h) * BITS;
+#pragma unroll
+          for (int k = 0; k < BITS; ++k) dst[k] = cw[k];
+          const int c0 = k0 + 32 * h;
+          if (NG == 2) {
+            const long long gidx = (long long)n * p.q_ldg + c0 / 16;
+            p.q_delta[gidx] = dd[0];
+            p.q_delta[gidx + 1] = dd[NG - 1];
+            p.q_zero[gidx] = (uint8_t)zf[0];
+            p.q_zero[gidx + 1] = (uint8_t)zf[NG - 1];
+          } else if (c0 % p.group == 0) {
+            const long long gidx = (long long)n * p.q_ldg + c0 / p.group;
+            p.q_delta[gidx] = dd[0];
+            p.q_zero[gidx] = (uint8_t)zf[0];
+          }
+        }
+      }
+    };
+
     for (int s = 0; s < n_total && ok_loop; ++s) {
       const int k0 = (ks_begin + s) * kSK;
       // codes and activations of this stage have landed; its TMEM weight
@@ -477,6 +674,9 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
       tc_fence_after();
       const uint32_t acol = arow + (uint32_t)(ra.slot * kSCols);
       if (s < n_main) {
+        if constexpr (QDQ) {
+          qdq_stage(s, k0, acol);
+        } else {
         const int pc = k0 >> (lg + 4);
         if (pc != pchunk) {
           if (pchunk >= 0) rp.next(2);
@@ -531,6 +731,7 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
         // release the params once their last stage is read
         if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
           mbar_arrive(b_empty_p + 8 * rp.slot);
+        }
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
         if (h == 0) {
@@ -566,30 +767,21 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
     tc_fence_after();
     const bool ok = acc_ok && !*aborted && n_total > 0;
     const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
-    if constexpr (NACC > 1) {
-      // add the issuers' accumulators into the first, in issuer order
-      for (int c = 0; c < bn; c += 16) {
-        float v[16], w[16];
-        tmem_ld16(t_lane + (uint32_t)c, v);
-#pragma unroll
-        for (int jj = 1; jj < NACC; ++jj) {
-          tmem_ld16(t_lane + (uint32_t)(jj * bn + c), w);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] += w[e];
-        }
-        uint32_t o[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(v[e]);
-        tmem_st16(t_lane + (uint32_t)c, o);
-      }
-      tmem_wait_st();
-    }
+
     // columns of the accumulator this warp drains
     const int c_lo = DQW >= 8 ? (bn >= 32 ? h * (bn / 2) : 0) : 0;
     const int c_hi = DQW >= 8 ? (bn >= 32 ? c_lo + bn / 2 : (h == 0 ? bn : 0))
                               : bn;
+    // The statistic of the stored output over this warp's columns (the
+    // next layer's input statistic, Proposed method bullets 2-3): row n's
+    // sum of |Y[t][n]|^p goes to partial row (tile, part) of p.stats.
+    float* const stats_row =
+        p.stats ? p.stats + ((int64_t)blockIdx.y * p.stats_parts +
+                             (p.stats_parts > 1 ? h : 0)) * p.N
+                : nullptr;
     if (split == 1 && p.y_mode == 0) {
       // Y rows not 16-byte aligned: each thread stores its row directly
+      float st = 0.f;
       for (int j = c_lo; j < c_hi; j += 16) {
         float v[16];
         tmem_ld16(t_lane + (uint32_t)j, v);
@@ -597,10 +789,14 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int t = t0 + j + c;
-            if (t < p.T) store_y(p.Y, p.yt, (long long)t * p.ldy + n, v[c]);
+            if (t < p.T) {
+              store_y(p.Y, p.yt, (long long)t * p.ldy + n, v[c]);
+              if (stats_row) st += y_moment(stored_y(p.yt, v[c]), p.stats_p);
+            }
           }
         }
       }
+      if (stats_row && ok && row_ok && c_hi > c_lo) stats_row[n] = st;
     } else if (split == 1 && p.y_mode == 2) {
       // 16-bit Y. Each warp reads its 32 rows in two halves of 16 lanes in
       // the 16x256b fragment order, packs column pairs, and writes 8x8
@@ -618,6 +814,7 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
         const int nb = 32 * q4 + 16 * lh;  // first row of this lane half
         const uint32_t box = gtile + (uint32_t)(nb >> 6) * (uint32_t)box_t * 128u;
         const int chunk = ((nb & 63) >> 3) + (mi & 1);
+        float st_lo = 0.f, st_hi = 0.f;  // rows nb + lane/4 and + 8
         for (int j = 0; j < box_t; j += 32) {
           uint32_t rr[16];
           tmem_ld_16x256b_x4(
@@ -636,6 +833,21 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
               pk[2 * k] = h2_bits(__floats2half2_rn(a0, a1));
               pk[2 * k + 1] = h2_bits(__floats2half2_rn(b0, b1));
             }
+            if (stats_row) {
+              // the stored values (columns past T hold zeros)
+              float2 lo, hi;
+              if (bf) {
+                lo = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(
+                    &pk[2 * k]));
+                hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(
+                    &pk[2 * k + 1]));
+              } else {
+                lo = __half22float2(bits_h2(pk[2 * k]));
+                hi = __half22float2(bits_h2(pk[2 * k + 1]));
+              }
+              st_lo += y_moment(lo.x, p.stats_p) + y_moment(lo.y, p.stats_p);
+              st_hi += y_moment(hi.x, p.stats_p) + y_moment(hi.y, p.stats_p);
+            }
           }
           if (ok) {
 #pragma unroll
@@ -646,6 +858,19 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
               stmatrix_x4_trans(addr, pk[4 * q], pk[4 * q + 1],
                                 pk[4 * q + 2], pk[4 * q + 3]);
             }
+          }
+        }
+        if (stats_row) {
+          // the four lanes that hold a row's columns add their sums
+#pragma unroll
+          for (int o = 1; o < 4; o <<= 1) {
+            st_lo += __shfl_xor_sync(0xffffffffu, st_lo, o);
+            st_hi += __shfl_xor_sync(0xffffffffu, st_hi, o);
+          }
+          const int r_lo = m0 + nb + (lane >> 2);
+          if (ok && box_t > 0 && (lane & 3) == 0) {
+            if (r_lo < p.N) stats_row[r_lo] = st_lo;
+            if (r_lo + 8 < p.N) stats_row[r_lo + 8] = st_hi;
           }
         }
       }
@@ -670,7 +895,9 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
       // rows beyond N and tokens beyond T are clipped by the store.
       const uint32_t esz = p.yt == TTQ_F32 ? 4u : 2u;
       const uint32_t ytile = base + L.x;
+      float st = 0.f;
       auto put = [&](int col, float v) {
+        if (stats_row) st += y_moment(stored_y(p.yt, v), p.stats_p);
         const uint32_t a = ytile + ((uint32_t)col * kBM + (uint32_t)i) * esz;
         if (p.yt == TTQ_F32)
           st_shared_f32(a, v);
@@ -696,6 +923,8 @@ __global__ void __launch_bounds__(cta_threads(DQW, NACC), DQW >= 16 ? 1 : 2)
           for (int c = 0; c < 16; ++c) put(j + c, v[c]);
         }
       }
+      // (columns past T hold zeros, which add nothing)
+      if (stats_row && ok && row_ok && c_hi > c_lo) stats_row[n] = st;
       fence_proxy_async_smem();
       if (h == 0)
         named_bar_sync<1>(128);
@@ -876,31 +1105,31 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr,
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Maps {
-  CUtensorMap x, u, c, d, z, y;
+  CUtensorMap x, u, c, d, z, y, w;
 };
 
-template <int BITS, int GMODE, int DQW, int NACC>
+template <int BITS, int GMODE, int DQW, bool QDQ = false>
 ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
-  auto kern = lowbit_gemm_kernel<BITS, GMODE, DQW, NACC>;
+  auto kern = lowbit_gemm_kernel<BITS, GMODE, DQW, QDQ>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return TTQ_ERR_CUDA;
   LaunchShape ls;
   ls.grid = grid;
-  ls.block = dim3(cta_threads(DQW, NACC), 1, 1);
+  ls.block = dim3(cta_threads(DQW), 1, 1);
   ls.smem = smem;
   ls.cluster_z = (unsigned)split;
-  return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, m.y, a);
+  return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, m.y, m.w, a);
 }
 
-template <int GMODE, int DQW, int NACC>
+template <int GMODE, int DQW, bool QDQ = false>
 ttq_status dispatch_bits(int bits, const Maps& m, const GemmArgs& a, dim3 grid,
                          int split, size_t smem, cudaStream_t st) {
   switch (bits) {
 #define TTQ_LK(B)                                                       \
   case B:                                                               \
-    return launch_kernel<B, GMODE, DQW, NACC>(m, a, grid, split, smem, st);
+    return launch_kernel<B, GMODE, DQW, QDQ>(m, a, grid, split, smem, st);
     TTQ_LK(2) TTQ_LK(3) TTQ_LK(4) TTQ_LK(5) TTQ_LK(6) TTQ_LK(7) TTQ_LK(8)
 #undef TTQ_LK
   }
@@ -936,6 +1165,10 @@ ttq_status launch_pre(const void* X, int64_t T, int64_t K, int64_t ldx,
 
 }  // namespace
 
+// Partial statistic rows per token tile: one per column part of the
+// epilogue (two halves with eight or more dequantisers and 32+ tokens).
+int stats_parts_of(int dqw, int bn) { return (dqw >= 8 && bn >= 32) ? 2 : 1; }
+
 size_t gemm_workspace_bytes(int64_t T, int64_t K, int r) {
   size_t b = align_up((size_t)T * (size_t)K * 2, 1024);
   if (r > 0) b += align_up((size_t)T * 64 * 2, 1024);
@@ -960,47 +1193,27 @@ ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
   return TTQ_ERR_INVALID_ARG;
 }
 
-ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
-                                int64_t K, const uint32_t* codes,
-                                const float* delta, const uint8_t* zero,
-                                int64_t N, int bits, int group, const void* B,
-                                ttq_dtype bt, int r, void* Y, ttq_dtype yt,
-                                int64_t ldy, cudaStream_t st) {
-  // up to four tokens: the CUDA-core matrix-vector product (gemv.cu)
-  if (gemv_applies(T, K))
-    return launch_gemv(Xs, U, T, K, codes, delta, zero, N, bits, group, B, bt,
-                       r, Y, yt, ldy, st);
-  // Tile shape. A stage is 128 channels: a codes chunk, two 64-channel
-  // activation boxes, one 64-column fp16 weight stage in TMEM.
-  // Decode (T <= 32): 256 TMEM columns per CTA (two CTAs per SM), K split
-  // over a cluster so that about one wave covers the GPU.
-  // Prefill: all 512 TMEM columns; the token tile is picked by a model of
-  // waves x (fixed cost + stages x max(MMA, dequant)), an MMA of N tokens
-  // costing about max(45, N/2) cycles (eight per stage) and a stage about
-  // 600 cycles of dequantisation. (Costing every MMA at least 128 cycles,
-  // which moves every large layer to N = 256, measured slower: 390 against
-  // 346 us on the Llama up layer, with one shared-memory stage less.)
+// Tile shape of the tensor-core projection: token tile bn, shared-memory
+// ring depth S, TMEM weight ring depth SA, TMEM columns (S < 2: no shape).
+void plan_tiles(int64_t T, int64_t N, int64_t K, int bits, int& bn, int& S,
+                int& SA, int& tmem_cols, int& acc_cols, bool qdq = false) {
   const int sms = sm_count();
   const int64_t tiles_m = (N + kBM - 1) / kBM;
   const int k_stages = (int)((K + kSK - 1) / kSK);
-  const uint32_t cchunk = code_chunk_bytes(bits);
-  int bn, S, SA, tmem_cols, acc_cols, split = 1;
-  // dual: two CTAs per SM, four dequantiser warps and 256 TMEM columns each
-  bool dual = T <= 32;
+  S = 0;
   auto fits = [&](int bn_, int S_, bool sp, size_t lim) {
-    return (size_t)make_layout(bits, bn_, S_, sp).total + 1024 <= lim;
+    return (size_t)make_layout(bits, bn_, S_, sp, qdq).total + 1024 <= lim;
   };
   if (T <= 32) {
     bn = T <= 16 ? 16 : 32;
-    // one accumulator per MMA issuer: 4 x 16 or 2 x 32 columns
-    acc_cols = (bn == 16 ? kDecodeIssuers : kDecodeIssuers / 2) * bn;
+    acc_cols = 32;
     tmem_cols = 256;
     SA = (tmem_cols - acc_cols) / kSCols;
     // the shared-memory ring runs deeper than the TMEM weight ring so that
     // loads are issued well ahead of the dequantisers
     S = 8;
     while (S > SA && !fits(bn, S, true, 110 * 1024)) --S;
-  } else if (!dual) {
+  } else {
     bn = 64;
     double best = 1e30;
     for (int c : {256, 192, 128, 64}) {
@@ -1024,6 +1237,59 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
     while (S > 1 && !fits(bn, S, false, kMaxSmem)) --S;
     SA = S;
   }
+}
+
+// Partial statistic rows of the fused output statistic for a prefill
+// projection of T x N x K (0 when there is none: T <= 32 or no shape).
+int64_t gemm_stats_rows(int64_t T, int64_t N, int64_t K, int bits) {
+  if (T <= 32) return 0;
+  int bn, S, SA, tmem_cols, acc_cols;
+  plan_tiles(T, N, K, bits, bn, S, SA, tmem_cols, acc_cols);
+  if (S < 2) return 0;
+  return ((T + bn - 1) / bn) * stats_parts_of(kPrefillDequantWarps, bn);
+}
+
+// The fused (QDQ) form's extra inputs and outputs.
+struct QdqInputs {
+  const void* W;  // bf16 [N, K], row pitch ldw elements
+  int64_t ldw;
+  const float* s;
+  uint32_t* codes;  // outputs (null: not stored)
+  float* delta;
+  uint8_t* zero;
+};
+
+ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
+                            int64_t K, const uint32_t* codes,
+                            const float* delta, const uint8_t* zero,
+                            int64_t N, int bits, int group, const void* B,
+                            ttq_dtype bt, int r, void* Y, ttq_dtype yt,
+                            int64_t ldy, cudaStream_t st, float* stats,
+                            float stats_p, const QdqInputs* q) {
+  // one or two tokens: the CUDA-core matrix-vector product (gemv.cu)
+  if (!q && gemv_applies(T, K)) {
+    if (stats) return TTQ_ERR_UNSUPPORTED;
+    return launch_gemv(Xs, U, T, K, codes, delta, zero, N, bits, group, B, bt,
+                       r, Y, yt, ldy, st);
+  }
+  if ((stats || q) && T <= 32) return TTQ_ERR_UNSUPPORTED;
+  // Tile shape. A stage is 128 channels: a codes chunk, two 64-channel
+  // activation boxes, one 64-column fp16 weight stage in TMEM.
+  // Decode (T <= 32): 256 TMEM columns per CTA (two CTAs per SM), K split
+  // over a cluster so that about one wave covers the GPU.
+  // Prefill: all 512 TMEM columns; the token tile is picked by a model of
+  // waves x (fixed cost + stages x max(MMA, dequant)), an MMA of N tokens
+  // costing about max(45, N/2) cycles (eight per stage) and a stage about
+  // 600 cycles of dequantisation. (Costing every MMA at least 128 cycles,
+  // which moves every large layer to N = 256, measured slower: 390 against
+  // 346 us on the Llama up layer, with one shared-memory stage less.)
+  const int sms = sm_count();
+  const int64_t tiles_m = (N + kBM - 1) / kBM;
+  const int k_stages = (int)((K + kSK - 1) / kSK);
+  int bn, S, SA, tmem_cols, acc_cols, split = 1;
+  // dual: two CTAs per SM, four dequantiser warps and 256 TMEM columns each
+  const bool dual = T <= 32;
+  plan_tiles(T, N, K, bits, bn, S, SA, tmem_cols, acc_cols, q != nullptr);
   if (S < 2) return TTQ_ERR_UNSUPPORTED;
   if (T <= 32) {
     const size_t sm1 = make_layout(bits, bn, S, true).total + 1024;
@@ -1034,26 +1300,37 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   }
   const int per = (k_stages + split - 1) / split;
   split = (k_stages + per - 1) / per;  // every rank gets at least one stage
-  const Layout L = make_layout(bits, bn, S, split > 1);
+  const Layout L = make_layout(bits, bn, S, split > 1, q != nullptr);
   const size_t smem = L.total + 1024;
   const int64_t tiles_t = (T + bn - 1) / bn;
 
   Maps m;
   const int64_t G = K / group;
-  const bool ok =
+  bool ok =
       make_tmap(&m.x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Xs, K, T, K * 2, 64,
                 bn, CU_TENSOR_MAP_SWIZZLE_128B) &&
-      make_tmap(&m.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32, N,
-                codes_ld(K, bits) * 4, 4 * bits, kBM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) &&
-      make_tmap(&m.d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, delta, G, N,
-                groups_ld(K, group) * 4, kParamGroups, kBM,
-                CU_TENSOR_MAP_SWIZZLE_64B) &&
-      make_tmap(&m.z, CU_TENSOR_MAP_DATA_TYPE_UINT8, zero, G, N,
-                groups_ld(K, group), kParamGroups, kBM,
-                CU_TENSOR_MAP_SWIZZLE_NONE) &&
       (r == 0 || make_tmap(&m.u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U, 64, T,
                            128, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B));
+  if (q) {
+    // bf16 weight tiles of 64 channels x 128 rows, 128-byte swizzled; the
+    // codes maps are not read
+    ok = ok && make_tmap(&m.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q->W, K, N,
+                         (uint64_t)q->ldw * 2, 64, kBM,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    m.c = m.d = m.z = m.x;
+  } else {
+    ok = ok &&
+         make_tmap(&m.c, CU_TENSOR_MAP_DATA_TYPE_UINT32, codes, K * bits / 32,
+                   N, codes_ld(K, bits) * 4, 4 * bits, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_tmap(&m.d, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, delta, G, N,
+                   groups_ld(K, group) * 4, kParamGroups, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_64B) &&
+         make_tmap(&m.z, CU_TENSOR_MAP_DATA_TYPE_UINT8, zero, G, N,
+                   groups_ld(K, group), kParamGroups, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    m.w = m.x;
+  }
   if (!ok) return TTQ_ERR_CUDA;
   if (r == 0) m.u = m.x;  // never read without a low-rank stage
   // Y is stored by the tensor memory accelerator in boxes of 128 rows x the
@@ -1101,31 +1378,57 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
   a.k_stages = k_stages;
   a.per = per;
   a.y_mode = y_mode;
+  a.qs = q ? q->s : nullptr;
+  a.q_codes = q ? q->codes : nullptr;
+  a.q_delta = q ? q->delta : nullptr;
+  a.q_zero = q ? q->zero : nullptr;
+  a.q_ldc = codes_ld(K, bits);
+  a.q_ldg = groups_ld(K, group);
+  a.stats = stats;
+  a.stats_p = stats_p;
+  a.stats_parts = stats_parts_of(dqw, bn);
   a.err = device_error_word();
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
   // decode packs two CTAs per SM with four dequant warps each; prefill runs
   // one CTA per SM with sixteen
 
   if (dual) {
-    // decode: several MMA issuers (their per-instruction cost dominates at
-    // 16 or 32 tokens), one accumulator each
-    if (bn == 16)
-      return group == 16
-                 ? dispatch_bits<0, 4, kDecodeIssuers>(bits, m, a, grid, split,
-                                                       smem, st)
-                 : dispatch_bits<1, 4, kDecodeIssuers>(bits, m, a, grid, split,
-                                                       smem, st);
-    return group == 16
-               ? dispatch_bits<0, 4, kDecodeIssuers / 2>(bits, m, a, grid,
-                                                         split, smem, st)
-               : dispatch_bits<1, 4, kDecodeIssuers / 2>(bits, m, a, grid,
-                                                         split, smem, st);
+    if (group == 16)
+      return dispatch_bits<0, 4>(bits, m, a, grid, split, smem, st);
+    return dispatch_bits<1, 4>(bits, m, a, grid, split, smem, st);
   }
+  if (q)
+    return group == 16
+               ? dispatch_bits<0, kPrefillDequantWarps, true>(
+                     bits, m, a, grid, split, smem, st)
+               : dispatch_bits<1, kPrefillDequantWarps, true>(
+                     bits, m, a, grid, split, smem, st);
   if (group == 16)
-    return dispatch_bits<0, kPrefillDequantWarps, 1>(bits, m, a, grid, split,
+    return dispatch_bits<0, kPrefillDequantWarps>(bits, m, a, grid, split,
                                                      smem, st);
-  return dispatch_bits<1, kPrefillDequantWarps, 1>(bits, m, a, grid, split,
+  return dispatch_bits<1, kPrefillDequantWarps>(bits, m, a, grid, split,
                                                    smem, st);
+}
+
+ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
+                                int64_t K, const uint32_t* codes,
+                                const float* delta, const uint8_t* zero,
+                                int64_t N, int bits, int group, const void* B,
+                                ttq_dtype bt, int r, void* Y, ttq_dtype yt,
+                                int64_t ldy, cudaStream_t st, float* stats,
+                                float stats_p) {
+  return launch_gemm_impl(Xs, U, T, K, codes, delta, zero, N, bits, group, B,
+                          bt, r, Y, yt, ldy, st, stats, stats_p, nullptr);
+}
+
+ttq_status launch_quantize_gemm_prepared(
+    const void* W, int64_t ldw, const float* s, const void* Xs, const void* U,
+    int64_t T, int64_t K, int64_t N, int bits, int group, const void* B,
+    ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy, uint32_t* codes,
+    float* delta, uint8_t* zero, cudaStream_t st) {
+  const QdqInputs q = {W, ldw, s, codes, delta, zero};
+  return launch_gemm_impl(Xs, U, T, K, nullptr, nullptr, nullptr, N, bits,
+                          group, B, bt, r, Y, yt, ldy, st, nullptr, 2.f, &q);
 }
 
 ttq_status launch_lowbit_gemm(const void* X, ttq_dtype xt, int64_t T,

@@ -55,7 +55,7 @@ ttq_status launch_prepare(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                           const void* A, int r, void* Xs, void* U,
                           cudaStream_t st);
 
-// The decode projection on CUDA cores (T <= 4), used by
+// The decode projection on CUDA cores (T <= 2), used by
 // launch_gemm_prepared when it applies.
 bool gemv_applies(int64_t T, int64_t K);
 ttq_status launch_gemv(const void* Xs, const void* U, int64_t T, int64_t K,
@@ -69,7 +69,24 @@ ttq_status launch_gemm_prepared(const void* Xs, const void* U, int64_t T,
                                 const float* delta, const uint8_t* zero,
                                 int64_t N, int bits, int group, const void* B,
                                 ttq_dtype bt, int r, void* Y, ttq_dtype yt,
-                                int64_t ldy, cudaStream_t st);
+                                int64_t ldy, cudaStream_t st,
+                                float* stats = nullptr, float stats_p = 2.f);
+// The fused (QDQ) projection: group RTN of the bf16 weights W (pitch ldw)
+// with scales s inside the tensor-core projection; codes, delta and zero of
+// the quantized weights are stored when not null. Prefill (T > 32) only.
+ttq_status launch_quantize_gemm_prepared(
+    const void* W, int64_t ldw, const float* s, const void* Xs, const void* U,
+    int64_t T, int64_t K, int64_t N, int bits, int group, const void* B,
+    ttq_dtype bt, int r, void* Y, ttq_dtype yt, int64_t ldy, uint32_t* codes,
+    float* delta, uint8_t* zero, cudaStream_t st);
+// Partial rows of the fused output statistic for a prefill projection
+// (0 when the shape has none), and the rows per token tile.
+int64_t gemm_stats_rows(int64_t T, int64_t N, int64_t K, int bits);
+int stats_parts_of(int dqw, int bn);
+// sum_out[n] (+)= sum_p partials[p][n], p in order.
+ttq_status launch_stats_reduce(const float* partials, int64_t P, int64_t N,
+                               int accumulate, float* sum_out,
+                               cudaStream_t st);
 
 // One thread runs the library's bounded mbarrier wait; *out = 1 if the
 // phase completed, 0 if the wait gave up (selftest.cu).

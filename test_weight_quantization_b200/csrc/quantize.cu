@@ -208,7 +208,7 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
   // row holds whole groups), so a lane past the end never shares one with
   // a live lane
 
-  float d[NG], r[NG], zf[NG], topz[NG];
+  float d[NG], r[NG], zf[NG], topz[NG], botz[NG];
 #pragma unroll
   for (int gi = 0; gi < NG; ++gi) {
     // group range, widened to contain 0 (min and max are exact, so the
@@ -236,9 +236,12 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
     // already because -mn <= mx - mn, the clamp matches the definition
     zf[gi] = fminf(fmaxf(__fadd_rn(__fdiv_rn(-mn, dd), kMagic), kMagic),
                    kTop) - kMagic;
-    // q = min(rint(w*r) + z, 2^b - 1) <=> M + q - z = min(M + rint(w*r),
-    // M + 2^b - 1 - z); q >= 0 since rint(w*r) >= rint(mn*r) = -z
+    // q = clamp(rint(w*r) + z, 0, 2^b - 1) <=> M + q - z =
+    // clamp(M + rint(w*r), M - z, M + 2^b - 1 - z). The lower clamp matters:
+    // z is the IEEE quotient's rint(-mn/D), and where that is a near-tie
+    // rint(mn*r) can fall one below -z.
     topz[gi] = kTop - zf[gi];
+    botz[gi] = kMagic - zf[gi];
   }
 
   // code e at bits [e*BITS, e*BITS + BITS) of the block's little-endian
@@ -250,7 +253,7 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
   for (int e = 0; e < 32; ++e) {
     const int gi = e / E;
     const float t =
-        fminf(__fmaf_rn(w[e], r[gi], kMagic), topz[gi]);
+        fmaxf(fminf(__fmaf_rn(w[e], r[gi], kMagic), topz[gi]), botz[gi]);
     const uint32_t tb = __float_as_uint(t);  // bits(M) + q - z
     const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
     if (sh + BITS <= 32) {

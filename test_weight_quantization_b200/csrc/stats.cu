@@ -306,7 +306,30 @@ ttq_status launch_x(const void* X, ttq_dtype xt, int64_t T, int64_t K,
   return TTQ_ERR_INVALID_ARG;
 }
 
+// sum_out[n] (+)= sum_p partials[p][n] over the P partial rows in order:
+// one thread per channel, consecutive threads on consecutive channels.
+__global__ void stats_reduce_kernel(const float* __restrict__ partials,
+                                    int64_t P, int64_t N, int accumulate,
+                                    float* __restrict__ sum_out) {
+  griddep_enter();
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float acc = 0.f;
+  for (int64_t q = 0; q < P; ++q) acc += __ldcg(partials + q * N + n);
+  sum_out[n] = accumulate ? sum_out[n] + acc : acc;
+}
+
 }  // namespace
+
+ttq_status launch_stats_reduce(const float* partials, int64_t P, int64_t N,
+                               int accumulate, float* sum_out,
+                               cudaStream_t st) {
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)((N + 255) / 256));
+  ls.block = dim3(256);
+  return launch(ls, st, stats_reduce_kernel, partials, P, N, accumulate,
+                sum_out);
+}
 
 ttq_status launch_act_stats(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                             int64_t ldx, float p, int accumulate,

@@ -4,6 +4,7 @@
     python -m test_weight_quantization_b200.measure prepare  T K bits
     python -m test_weight_quantization_b200.measure quantize N K bits group
     python -m test_weight_quantization_b200.measure gemm     T N K bits group
+    python -m test_weight_quantization_b200.measure qgemm    T N K bits group
     python -m test_weight_quantization_b200.measure table    (the shapes below)
     python -m test_weight_quantization_b200.measure [--eager] KIND ...
         (--eager launches directly instead of replaying a CUDA graph)
@@ -198,7 +199,29 @@ TABLE = [
     ("gemm", (16, 4096, 14336, 2, 16)),
 ]
 
-FNS = {"stats": stats, "prepare": prepare, "quantize": quantize, "gemm": gemm}
+
+
+def qgemm(T, N, K, bits, group):
+    """Quantize + projection as two launches against the fused launch that
+    quantizes the bf16 weights inside the projection (codes stored)."""
+    W = weights(N, K)
+    X = acts(T, K)
+    s = torch.ones(K, device="cuda")
+    Xs, _ = ttq.prepare_activations(X, s, bits)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, bits, group)
+    Y = torch.empty(T, N, dtype=torch.bfloat16, device="cuda")
+
+    def two():
+        ttq.quantize_rtn_grouped(W, s, bits, group, c, d, z)
+        ttq.w_lowbit_gemm_prepared(Xs, None, c, d, z, N, bits, group, out=Y)
+
+    def fused():
+        ttq.quantize_gemm_prepared(W, s, Xs, None, bits, group, out=Y,
+                                   codes=c, delta=d, zero=z)
+    flops = 2 * T * N * K
+    name = f"T={T:5d} N={N:6d} K={K:6d} b={bits} g={group:3d}"
+    report("quantize+gemm  " + name, graph_us([two]), flops=flops)
+    report("fused qdq gemm " + name, graph_us([fused]), flops=flops)
 
 
 def decode(*Ts):
@@ -209,6 +232,10 @@ def decode(*Ts):
                 for group in (16, 32, 64, 128):
                     gemm(T, N, K, bits, group)
                     torch.cuda.empty_cache()
+
+
+FNS = {"stats": stats, "prepare": prepare, "quantize": quantize, "gemm": gemm,
+       "qgemm": qgemm}
 
 
 def main(argv):

@@ -62,6 +62,13 @@ def _load() -> ctypes.CDLL:
         "ttq_selftest_bounded_wait": [I, P, P],
         "ttq_channel_moment_total": [P, I64, I64, P, P],
         "ttq_awq_scales_sharded": [P, I64, I64, I64, P, P, P, P, P],
+        "ttq_projection_stats_rows": [I64, I64, I64, I],
+        "ttq_w_lowbit_gemm_prepared_stats": [P, P, I64, I64, P, P, P, I64, I,
+                                             I, P, I, I, P, I, I64, F, P,
+                                             I64, P],
+        "ttq_stats_reduce": [P, I64, I64, I, P, P],
+        "ttq_quantize_gemm_prepared": [P, I, I64, P, P, P, I64, I64, I64, I,
+                                       I, P, I, I, P, I, I64, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -71,6 +78,7 @@ def _load() -> ctypes.CDLL:
     lib.ttq_w_lowbit_gemm_workspace_size.restype = SZ
     lib.ttq_codes_ld.restype = I64
     lib.ttq_groups_ld.restype = I64
+    lib.ttq_projection_stats_rows.restype = I64
     return lib
 
 
@@ -84,7 +92,9 @@ EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_act_stats_scales",
            "ttq_lowrank_add", "ttq_unpack_codes", "ttq_status_string",
            "ttq_device_error", "ttq_abi_version", "ttq_codes_ld",
            "ttq_groups_ld", "ttq_selftest_bounded_wait",
-           "ttq_channel_moment_total", "ttq_awq_scales_sharded")
+           "ttq_channel_moment_total", "ttq_awq_scales_sharded",
+           "ttq_projection_stats_rows", "ttq_w_lowbit_gemm_prepared_stats",
+           "ttq_stats_reduce", "ttq_quantize_gemm_prepared")
 
 
 class _Params(ctypes.Structure):
@@ -427,7 +437,7 @@ def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
                            B: torch.Tensor | None = None,
                            out: torch.Tensor | None = None,
                            out_dtype=torch.bfloat16) -> torch.Tensor:
-    """The projection on prepared operands (one kernel launch; up to four
+    """The projection on prepared operands (one kernel launch; one or two
     tokens run on CUDA cores, more on tensor cores)."""
     _dev(Xs, "Xs")
     if Xs.dim() != 2:
@@ -453,6 +463,122 @@ def w_lowbit_gemm_prepared(Xs: torch.Tensor, U: torch.Tensor | None,
         delta.data_ptr(), zero.data_ptr(), N, bits, group, _ptr(B),
         _code(B, "B") if r else 0, r, out.data_ptr(), _code(out, "out"),
         ldy, _stream()), "ttq_w_lowbit_gemm_prepared")
+    return out
+
+
+def quantize_gemm_prepared(W: torch.Tensor, s: torch.Tensor, Xs: torch.Tensor,
+                           U: torch.Tensor | None, bits: int, group: int,
+                           B: torch.Tensor | None = None,
+                           out: torch.Tensor | None = None,
+                           out_dtype=torch.bfloat16, store_codes: bool = True,
+                           codes=None, delta=None, zero=None):
+    """Steps 3 and 4 in one launch (the projection quantizes the bf16 W
+    itself): Y [T, N], and (codes, delta, zero) of the quantized weights
+    unless store_codes is False (then None)."""
+    ldw = _rows(W, "W")
+    N, K = W.shape
+    _buf(s, "s", torch.float32, K)
+    _dev(Xs, "Xs")
+    T = Xs.shape[0]
+    _buf(Xs, "Xs", torch.float16, T, K)
+    r = 0
+    if B is not None:
+        r = B.shape[1] if B.dim() == 2 else -1
+        _buf(B, "B", B.dtype, N, r)
+        if B.shape[0] != N:
+            raise TTQError(f"B must have {N} rows, got {B.shape[0]}")
+        if U is None:
+            raise TTQError("a low-rank projection needs U")
+        _buf(U, "U", torch.float16, T, 64)
+    if store_codes:
+        dev = W.device
+        cl, gl = codes_ld(K, bits), groups_ld(K, group)
+        codes = torch.zeros((N, cl), dtype=torch.int32, device=dev) \
+            if codes is None else codes
+        delta = torch.zeros((N, gl), dtype=torch.float32, device=dev) \
+            if delta is None else delta
+        zero = torch.zeros((N, gl), dtype=torch.uint8, device=dev) \
+            if zero is None else zero
+        _packed(codes, delta, zero, N, K, bits, group)
+    if out is None:
+        out = torch.empty((T, N), dtype=out_dtype, device=Xs.device)
+    ldy = _out(out, "out", T, N)
+    _check(_lib.ttq_quantize_gemm_prepared(
+        W.data_ptr(), _code(W, "W"), ldw, s.data_ptr(), Xs.data_ptr(),
+        _ptr(U) if r else None, T, K, N, bits, group, _ptr(B),
+        _code(B, "B") if r else 0, r, out.data_ptr(), _code(out, "out"), ldy,
+        _ptr(codes) if store_codes else None,
+        _ptr(delta) if store_codes else None,
+        _ptr(zero) if store_codes else None, _stream()),
+        "ttq_quantize_gemm_prepared")
+    return out, ((codes, delta, zero) if store_codes else None)
+
+
+def projection_stats_rows(T: int, N: int, K: int, bits: int) -> int:
+    """Partial rows the fused output statistic needs (0: none for T)."""
+    return int(_lib.ttq_projection_stats_rows(T, N, K, bits))
+
+
+def w_lowbit_gemm_prepared_stats(Xs: torch.Tensor, U: torch.Tensor | None,
+                                 codes: torch.Tensor, delta: torch.Tensor,
+                                 zero: torch.Tensor, N: int, bits: int,
+                                 group: int, B: torch.Tensor | None = None,
+                                 p: float = 2.0, out: torch.Tensor | None = None,
+                                 out_dtype=torch.bfloat16,
+                                 stats: torch.Tensor | None = None):
+    """The projection on prepared operands plus the partial statistic of its
+    stored output: (Y [T, N], stats [rows, N] fp32); stats_reduce adds the
+    rows into the next layer's channel sums."""
+    _dev(Xs, "Xs")
+    if Xs.dim() != 2:
+        raise TTQError("Xs must be 2D")
+    T, K = Xs.shape
+    _buf(Xs, "Xs", torch.float16, T, K)
+    rows = projection_stats_rows(T, N, K, bits)
+    if rows == 0:
+        raise TTQError(f"no fused statistic for T = {T} (prefill only)")
+    r = 0
+    if B is not None:
+        r = B.shape[1] if B.dim() == 2 else -1
+        _buf(B, "B", B.dtype, N, r)
+        _code(B, "B")
+        if B.shape[0] != N:
+            raise TTQError(f"B must have {N} rows, got {B.shape[0]}")
+        if U is None:
+            raise TTQError("a low-rank projection needs U")
+        _buf(U, "U", torch.float16, T, 64)
+    _packed(codes, delta, zero, N, K, bits, group)
+    if out is None:
+        out = torch.empty((T, N), dtype=out_dtype, device=Xs.device)
+    ldy = _out(out, "out", T, N)
+    if stats is None:
+        stats = torch.empty((rows, N), dtype=torch.float32, device=Xs.device)
+    _buf(stats, "stats", torch.float32, rows, N)
+    if stats.shape[0] != rows:
+        raise TTQError(f"stats must have {rows} rows")
+    _check(_lib.ttq_w_lowbit_gemm_prepared_stats(
+        Xs.data_ptr(), _ptr(U) if r else None, T, K, codes.data_ptr(),
+        delta.data_ptr(), zero.data_ptr(), N, bits, group, _ptr(B),
+        _code(B, "B") if r else 0, r, out.data_ptr(), _code(out, "out"),
+        ldy, float(p), stats.data_ptr(), rows, _stream()),
+        "ttq_w_lowbit_gemm_prepared_stats")
+    return out, stats
+
+
+def stats_reduce(partials: torch.Tensor, out: torch.Tensor | None = None,
+                 accumulate: bool = False) -> torch.Tensor:
+    """out[n] (+)= sum_i partials[i][n], fp32 [N]."""
+    _dev(partials, "partials")
+    if partials.dim() != 2:
+        raise TTQError("partials must be 2D")
+    P, N = partials.shape
+    _buf(partials, "partials", torch.float32, P, N)
+    if out is None:
+        out = torch.empty(N, dtype=torch.float32, device=partials.device)
+    _buf(out, "out", torch.float32, N)
+    _check(_lib.ttq_stats_reduce(partials.data_ptr(), P, N, int(accumulate),
+                                 out.data_ptr(), _stream()),
+           "ttq_stats_reduce")
     return out
 
 

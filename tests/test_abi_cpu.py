@@ -45,7 +45,7 @@ def test_status_strings_and_version(lib):
     assert lib.ttq_status_string(0) == b"TTQ_OK"
     assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
     assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
-    assert lib.ttq_abi_version() == 5
+    assert lib.ttq_abi_version() == 7
 
 
 def test_workspace_size(lib):

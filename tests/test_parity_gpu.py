@@ -157,7 +157,10 @@ def test_channel_total_and_sharded_scales(ttq):
         parts.append(sh)
         totals.append(ttq.channel_moment_total(sh, T))
     total = totals[0] + totals[1]
-    ref_total = np.sum(np32(sums).astype(np.float64) / T)
+    # each shard's total is the fp64 sum of its own channel sums (which
+    # differ from the unsplit statistics' in the last fp32 bits: another
+    # accumulation order)
+    ref_total = sum(np.sum(np32(sh).astype(np.float64) / T) for sh in parts)
     assert abs(total.item() - ref_total) <= 1e-12 * abs(ref_total)
     got = [ttq.awq_scales_sharded(sh, T, K, total, 0.5, 0.1, 2.0)
            for sh in parts]
@@ -192,6 +195,123 @@ def test_row_parallel_projection_on_one_gpu(ttq):
     c, d, z = ttq.quantize_rtn_grouped(W, s_full, bits, group)
     ref = oracle_y(X.cpu(), inv_full, c, d, z, N, bits, group)
     assert_gemm_close(np32(Y), ref, "row-parallel on one GPU", Y.dtype)
+
+
+# ------------------------------- quantization fused into the projection ----
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (3, 32), (2, 16), (5, 64),
+                                        (8, 128), (4, 64), (6, 16)])
+@pytest.mark.parametrize("T,N,K", [(300, 272, 1152), (64, 130, 1056)])
+def test_fused_quantize_projection_equals_two_passes(ttq, bits, group, T, N,
+                                                     K):
+    """The projection that quantizes the bf16 weights itself gives the two-
+    pass result (quantize, then project) bit for bit, and stores the same
+    codes, delta and zero; several token tiles, ragged N, a K whose last
+    128-channel stage is partial, every group size (64 and 128 span several
+    dequantiser warps)."""
+    if K % group:
+        pytest.skip("K not a multiple of g")
+    X = acts(T, K, 100 + bits, torch.bfloat16).cuda()
+    W = weights(N, K, 101 + group, torch.bfloat16).cuda()
+    sums = ttq.act_stats(X)
+    s, inv = ttq.awq_scales(sums, T)
+    Xs, _ = ttq.prepare_activations(X, inv, bits)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, bits, group)
+    ref = ttq.w_lowbit_gemm_prepared(Xs, None, c, d, z, N, bits, group)
+    Y, (fc, fd, fz) = ttq.quantize_gemm_prepared(W, s, Xs, None, bits, group)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, ref)
+    w, G = K * bits // 32, K // group
+    assert torch.equal(fc[:, :w], c[:, :w])
+    assert torch.equal(fd[:, :G], d[:, :G])
+    assert torch.equal(fz[:, :G], z[:, :G])
+    Y2, none = ttq.quantize_gemm_prepared(W, s, Xs, None, bits, group,
+                                          store_codes=False)
+    assert none is None and torch.equal(Y2, ref)
+
+
+def test_fused_quantize_projection_lowrank_and_oracle(ttq):
+    """With the low-rank stage, against the oracle's projection."""
+    T, N, K, r, bits, group = 200, 272, 384, 16, 4, 64
+    X = acts(T, K, 110, torch.bfloat16)
+    W = weights(N, K, 111, torch.bfloat16)
+    rng = np.random.default_rng(112)
+    A = torch.from_numpy(rng.standard_normal((r, K)).astype(np.float32) * .05
+                         ).to(torch.bfloat16).cuda()
+    B = torch.from_numpy(rng.standard_normal((N, r)).astype(np.float32) * .05
+                         ).to(torch.bfloat16).cuda()
+    Xg, Wg = X.cuda(), W.cuda()
+    s, inv = ttq.awq_scales(ttq.act_stats(Xg), T)
+    Xs, U = ttq.prepare_activations(Xg, inv, bits, A)
+    Y, (c, d, z) = ttq.quantize_gemm_prepared(Wg, s, Xs, U, bits, group, B=B)
+    torch.cuda.synchronize()
+    ref = oracle_y(X, inv, c, d, z, N, bits, group, A.cpu(), B.cpu())
+    assert_gemm_close(np32(Y), ref, "fused quantize + low rank", Y.dtype)
+    check_quantized(ttq, W, s.cpu(), bits, group, "fused codes source")
+
+
+def test_fused_quantize_projection_refusals(ttq):
+    X = acts(16, 256, 113, torch.bfloat16).cuda()
+    W = weights(128, 256, 114, torch.bfloat16).cuda()
+    s, inv = ttq.awq_scales(ttq.act_stats(X), 16)
+    Xs, _ = ttq.prepare_activations(X, inv, 4)
+    with pytest.raises(ttq.TTQError):      # decode sizes: not this form
+        ttq.quantize_gemm_prepared(W, s, Xs, None, 4, 64)
+    X2 = acts(64, 256, 115, torch.bfloat16).cuda()
+    Xs2, _ = ttq.prepare_activations(X2, inv, 4)
+    with pytest.raises(ttq.TTQError):      # fp16 weights: not this form
+        ttq.quantize_gemm_prepared(W.half(), s, Xs2, None, 4, 64)
+
+
+# ------------------------------------- statistic fused into the epilogue ----
+
+@pytest.mark.parametrize("T,N,K,out,pk", [
+    (300, 272, 384, "bf16", 2.0),    # two token tiles, ragged N and T
+    (4096, 1152, 1152, "bf16", 2.0), # many tiles, the 16-bit tensor store
+    (200, 264, 256, "f32", 2.0),     # fp32 Y: the staged-tile store
+    (300, 300, 256, "f16", 1.0),     # Y rows not 16-byte aligned; p = 1
+    (100, 128, 256, "bf16", 3.0),
+])
+def test_projection_output_statistic(ttq, T, N, K, out, pk):
+    """The projection's epilogue adds |Y|^p of the stored outputs per output
+    channel: reduced, it equals the statistics pass over Y (the oracle's
+    fp64 sums of the stored values, and the CUDA statistics kernel)."""
+    X = acts(T, K, 80 + T, torch.bfloat16).cuda()
+    W = weights(N, K, 81, torch.bfloat16).cuda()
+    sums = ttq.act_stats(X)
+    s, inv = ttq.awq_scales(sums, T)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, 4, 64)
+    Xs, _ = ttq.prepare_activations(X, inv, 4)
+    if N == 300:  # a pitch whose rows are not 16-byte aligned
+        big = torch.zeros((T, 301), dtype=DT[out], device="cuda")
+        Y = big[:, :N]
+    else:
+        Y = torch.empty((T, N), dtype=DT[out], device="cuda")
+    Y2, part = ttq.w_lowbit_gemm_prepared_stats(Xs, None, c, d, z, N, 4, 64,
+                                                p=pk, out=Y)
+    got = ttq.stats_reduce(part)
+    torch.cuda.synchronize()
+    Yc = np32(Y)
+    ref = oracle.act_sums(Yc, pk)
+    assert_rel_close(np32(got), ref, what="fused statistic")
+    if N % 8 == 0:  # the statistics pass takes K % 8 == 0
+        assert_rel_close(np32(got), np32(ttq.act_stats(Y.contiguous(), pk)),
+                         what="fused vs statistics pass")
+    # the projection itself is the plain one's
+    Yp = ttq.w_lowbit_gemm_prepared(Xs, None, c, d, z, N, 4, 64,
+                                    out_dtype=DT[out])
+    assert torch.equal(Yp, Y.contiguous())
+
+
+def test_projection_output_statistic_refusals(ttq):
+    X = acts(16, 256, 90, torch.bfloat16).cuda()
+    W = weights(128, 256, 91, torch.bfloat16).cuda()
+    s, inv = ttq.awq_scales(ttq.act_stats(X), 16)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, 4, 64)
+    Xs, _ = ttq.prepare_activations(X, inv, 4)
+    assert ttq.projection_stats_rows(16, 128, 256, 4) == 0
+    with pytest.raises(ttq.TTQError):
+        ttq.w_lowbit_gemm_prepared_stats(Xs, None, c, d, z, 128, 4, 64)
 
 
 # ---------------------------------------------------------- quantize ----
@@ -254,6 +374,29 @@ def test_quantize_unstaged_scales_for_very_long_rows(ttq):
         28672) * 0.7).astype(np.float32))
     for bits, group in ((4, 128), (3, 16)):
         check_quantized(ttq, W, s, bits, group, f"K=28672 b={bits} g={group}")
+
+
+@pytest.mark.parametrize("bits,seed", [(8, 40), (7, 41)])
+def test_quantize_zero_point_near_ties_keep_codes_in_range(ttq, bits, seed):
+    """Groups whose zero point is a near-tie (the oracle's pin search:
+    rint(-mn * (1/D)) and rint(-mn / D) differ): every GPU code lies in
+    [0, 2^b - 1], differs from the oracle's only at counted near-ties, and
+    dequantizes within half a step of its weight."""
+    from test_oracle_pins import _reciprocal_disagreements
+    W, n_zero, _ = _reciprocal_disagreements(seed, bits, 12)
+    assert n_zero >= 3
+    Wt = torch.from_numpy(W)
+    c, d, z, rc, rd, rz = quantize_both(ttq, Wt, None, bits, 16)
+    assert_codes_match(c, d, z, rc, rd, rz, W, None, bits, 16, "zero ties")
+    q = oracle.unpack_codes(c, 32, bits).astype(np.float64)
+    assert q.max() <= (1 << bits) - 1
+    dq = (q - np.repeat(z, 16, axis=1)) * np.repeat(d.astype(np.float64), 16,
+                                                    axis=1)
+    # half a step, plus the quotient's fp32 rounding at a near-tie (up to
+    # one step of w/D, which reaches 2^b)
+    bound = np.repeat(d.astype(np.float64), 16, axis=1) * (
+        0.5 + 2.0 ** (bits - 22))
+    assert np.all(np.abs(dq - W) <= bound)
 
 
 @pytest.mark.parametrize("dt", ["f32", "f16"])
@@ -358,9 +501,10 @@ def test_one_and_two_tokens_with_very_long_rows(ttq):
 @pytest.mark.parametrize("bits", [2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("group", [16, 32, 128])
 def test_decode_gemv(ttq, T, bits, group):
-    """Up to four tokens take the CUDA-core matrix-vector path; every code
-    width and group size against the oracle (K spans several work units of
-    a warp's lanes and a ragged one)."""
+    """One or two tokens take the CUDA-core matrix-vector path, three and
+    four the tensor-core decode tile; every code width and group size
+    against the oracle (K spans 10 row passes of a warp's lanes and a
+    ragged one)."""
     N, K = 300, 1408
     X = acts(T, K, 40 + T + bits, torch.bfloat16)
     W = weights(N, K, 41 + bits, torch.bfloat16)
