@@ -125,6 +125,30 @@ def weights(N: int, K: int, seed: int, std: float = 0.02) -> np.ndarray:
     return (rng.standard_normal((N, K)) * std).astype(np.float32)
 
 
+def spectral_weights(N: int, K: int, seed: int, strong: int = 32,
+                     sigma0: float = 20.0, decay: float = 0.85,
+                     std: float = 0.02) -> np.ndarray:
+    """[N, K] float32 weights with a planted decaying spectrum: ``strong``
+    rank-one components of sizes sigma0 * decay^i along seeded Gaussian
+    directions (normalised by sqrt(N) and sqrt(K), so nearly orthonormal),
+    plus i.i.d. N(0, std^2) noise. Stands in for trained projections, whose
+    spectra have a few large singular values above a flat bulk."""
+    rng = np.random.default_rng(seed)
+    G = rng.standard_normal((N, strong)) / math.sqrt(N)
+    H = rng.standard_normal((strong, K)) / math.sqrt(K)
+    sig = sigma0 * decay ** np.arange(strong)
+    W = (G * sig[None, :]) @ H + rng.standard_normal((N, K)) * std
+    return W.astype(np.float32)
+
+
+def probe_vectors(r: int, K: int, seed: int) -> np.ndarray:
+    """[r, K] float32 standard Gaussian vectors: the random draws of a
+    randomized factorisation, generated once and handed to both the kernels
+    and the oracle as an input."""
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((r, K)).astype(np.float32)
+
+
 def lowrank_checkpoint(W: np.ndarray, r: int, dtype=torch.bfloat16):
     """Stores a layer as residual + rank-r factors, the way a checkpoint in
     the W = W_q + B A form would ship it (TTQ review, Proposed method,
