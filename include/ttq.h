@@ -370,6 +370,49 @@ ttq_status ttq_lowrank_add(const void* X, ttq_dtype xt, int64_t T, int64_t K,
                            int64_t N, void* Y, ttq_dtype yt, int64_t ldy,
                            void* stream);
 
+/* Per-prompt ("dynamic") low-rank factors (TTQ review, Proposed method,
+ * bullet 5: W = W_q + B A with dynamic B, A and W_q quantized on the fly;
+ * Main results, bullet 4: TTQ quantizes the residual). With TTQ's scales s
+ * of the prompt, the factors span the dominant r-dimensional column space
+ * of W_s = W diag(s), found by randomized subspace iteration (Halko,
+ * Martinsson and Tropp 2011, Algorithm 4.4) from r probe vectors omega:
+ *   Q = orth(W_s omega^T);  iters times: Z = orth(W_s^T Q), Q = orth(W_s Z)
+ *   B = bf16(Q) [N, r],  A = bf16(Q^T W) [r, K]     (B A = Q Q^T W)
+ * orth() orthonormalises the columns in order (Gram-Schmidt's order) and
+ * drops a column whose part orthogonal to the kept ones has a norm of at
+ * most 2^-10 of the input's largest column (that column of B is zero).
+ *   W      bf16 [N, K], row pitch ldw (ldw >= K, ldw % 8 == 0), 16-byte
+ *          aligned (read by TMA).
+ *   s      fp32 [K] scales of step 2 (positive).
+ *   omega  fp32 [r, K] probe vectors the caller draws (standard Gaussian);
+ *          the call is deterministic given them.
+ *   B, A   bf16 outputs, dense [N, r] and [r, K], 2-byte aligned; the
+ *          layout ttq_w_lowbit_gemm takes for its low-rank term.
+ *   1 <= r <= 64, 0 <= iters <= 16.
+ * workspace: ttq_lowrank_factors_workspace_size(N, K, r) bytes, 256-byte
+ * aligned, caller-owned, not used concurrently by another call. The
+ * products with W run on the tensor cores with fp16 operands (W and the
+ * basis rounded to fp16), fp32 accumulation; the orthonormalisation runs a
+ * Cholesky factorisation in fp64. Argument errors return
+ * TTQ_ERR_INVALID_ARG before anything is enqueued; a weight beyond fp16's
+ * range raises TTQ_DEVERR_FP16_RANGE. */
+size_t ttq_lowrank_factors_workspace_size(int64_t N, int64_t K, int r);
+ttq_status ttq_lowrank_factors(const void* W, int64_t N, int64_t K,
+                               int64_t ldw, const float* s, const float* omega,
+                               int r, int iters, void* B, void* A,
+                               void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* The residual TTQ quantizes when W = W_q + B A (TTQ review, Main results,
+ * bullet 4): R = bf16(W - B A), each element accumulated from W in fp32 by
+ * fused multiply-adds in the order j = 0 .. r-1 and rounded to bf16 once.
+ * W, R bf16 [N, K] with pitches ldw, ldr (multiples of 8, rows 16-byte
+ * aligned); B bf16 [N, r], A bf16 [r, K] dense; 1 <= r <= 64. R may be W
+ * itself (ldr == ldw) but must not overlap it otherwise, nor B or A. */
+ttq_status ttq_lowrank_residual(const void* W, int64_t N, int64_t K,
+                                int64_t ldw, const void* B, const void* A,
+                                int r, void* R, int64_t ldr, void* stream);
+
 /* Expand packed codes to one uint8 per weight: q_out [N][K] (device).
  * Inverse of the packing in ttq_quantize_rtn_grouped. */
 ttq_status ttq_unpack_codes(const uint32_t* codes, int64_t N, int64_t K,
@@ -399,7 +442,8 @@ ttq_status ttq_selftest_bounded_wait(int arrive, uint32_t* out, void* stream);
  * ttq_selftest_bounded_wait added; 5: ttq_channel_moment_total and
  * ttq_awq_scales_sharded added; 6: ttq_projection_stats_rows,
  * ttq_w_lowbit_gemm_prepared_stats and ttq_stats_reduce added; 7:
- * ttq_quantize_gemm_prepared added). */
+ * ttq_quantize_gemm_prepared added; 8: ttq_lowrank_factors,
+ * ttq_lowrank_factors_workspace_size and ttq_lowrank_residual added). */
 int ttq_abi_version(void);
 
 #ifdef __cplusplus

@@ -96,3 +96,26 @@ def residual(W, B, A) -> np.ndarray:
     B = np.asarray(B, dtype=np.float64)
     A = np.asarray(A, dtype=np.float64)
     return round_bf16(W - B @ A)
+
+
+def residual_near_ties(W, B, A) -> np.ndarray:
+    """Where a residual computed in fp32 may round to the other bf16
+    neighbour: the exact W - B A lies within the bound of an fp32
+    multiply-add chain over r terms, (r + 1) 2^-24 (|W| + sum_j |B_j A_j|),
+    of a point halfway between two bf16 values. Elsewhere every such
+    computation gives the bf16 value of ``residual``."""
+    W = np.asarray(W, dtype=np.float64)
+    B = np.asarray(B, dtype=np.float64)
+    A = np.asarray(A, dtype=np.float64)
+    r = B.shape[1]
+    v = W - B @ A
+    bound = (r + 1) * 2.0 ** -24 * (np.abs(W) + np.abs(B) @ np.abs(A))
+    m, e = np.frexp(v)
+    e = np.maximum(e, -125)
+    step = np.ldexp(1.0, e - 8)
+    # distance to the nearest midpoint between bf16 neighbours
+    frac = v / step - np.floor(v / step)
+    dist = np.abs(frac - 0.5) * step
+    # (a value within the bound of zero may round to any of the tiny bf16
+    # values around it)
+    return (dist <= bound) | (np.abs(v) <= bound)

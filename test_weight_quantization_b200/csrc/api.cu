@@ -92,7 +92,7 @@ int sm_count() {
 
 using namespace ttq;
 
-TTQ_EXPORT int ttq_abi_version(void) { return 7; }
+TTQ_EXPORT int ttq_abi_version(void) { return 8; }
 
 TTQ_EXPORT int64_t ttq_codes_ld(int64_t K, int bits) {
   if (K < 32 || K % 32 != 0 || bits < 2 || bits > 8) return 0;
@@ -366,6 +366,57 @@ TTQ_EXPORT ttq_status ttq_lowrank_add(const void* X, ttq_dtype xt, int64_t T,
     return TTQ_ERR_INVALID_ARG;
   return launch_lowrank_add(X, xt, T, K, ldx, A, B, r, N, Y, yt, ldy,
                             as_stream(stream));
+}
+
+TTQ_EXPORT size_t ttq_lowrank_factors_workspace_size(int64_t N, int64_t K,
+                                                     int r) {
+  if (N < 1 || K < 1 || r < 1 || r > 64 || N > (1LL << 30) ||
+      K > (1LL << 30))
+    return 0;
+  return lowrank_factors_workspace_bytes(N, K, r);
+}
+
+TTQ_EXPORT ttq_status ttq_lowrank_factors(const void* W, int64_t N, int64_t K,
+                                          int64_t ldw, const float* s,
+                                          const float* omega, int r, int iters,
+                                          void* B, void* A, void* workspace,
+                                          size_t workspace_bytes,
+                                          void* stream) {
+  if (!W || !s || !omega || !B || !A || !workspace || N < 1 || K < 1 ||
+      N > (1LL << 30) || K > (1LL << 30) || r < 1 || r > 64 || iters < 0 ||
+      iters > 16 || ldw < K || !rows_aligned(W, TTQ_BF16, ldw) ||
+      !aligned(s, 4) || !aligned(omega, 4) || !aligned(B, 2) ||
+      !aligned(A, 2) || !aligned(workspace, 256) ||
+      workspace_bytes < lowrank_factors_workspace_bytes(N, K, r))
+    return TTQ_ERR_INVALID_ARG;
+  const size_t nb = (size_t)N * r * 2, na = (size_t)r * K * 2,
+               nw = (size_t)((N - 1) * ldw + K) * 2;
+  if (overlaps(B, nb, A, na) || overlaps(B, nb, W, nw) ||
+      overlaps(A, na, W, nw) || overlaps(workspace, workspace_bytes, B, nb) ||
+      overlaps(workspace, workspace_bytes, A, na))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_lowrank_factors(W, N, K, ldw, s, omega, r, iters, B, A,
+                                workspace, as_stream(stream));
+}
+
+TTQ_EXPORT ttq_status ttq_lowrank_residual(const void* W, int64_t N, int64_t K,
+                                           int64_t ldw, const void* B,
+                                           const void* A, int r, void* R,
+                                           int64_t ldr, void* stream) {
+  if (!W || !B || !A || !R || N < 1 || K < 1 || N > (1LL << 30) ||
+      K > (1LL << 30) || r < 1 || r > 64 || ldw < K || ldr < K ||
+      !rows_aligned(W, TTQ_BF16, ldw) || !rows_aligned(R, TTQ_BF16, ldr) ||
+      !aligned(B, 2) || !aligned(A, 2))
+    return TTQ_ERR_INVALID_ARG;
+  const size_t nb = (size_t)N * r * 2, na = (size_t)r * K * 2,
+               nw = (size_t)((N - 1) * ldw + K) * 2,
+               nr = (size_t)((N - 1) * ldr + K) * 2;
+  const bool in_place = R == W && ldr == ldw;
+  if ((!in_place && overlaps(R, nr, W, nw)) || overlaps(R, nr, B, nb) ||
+      overlaps(R, nr, A, na))
+    return TTQ_ERR_INVALID_ARG;
+  return launch_lowrank_residual(W, N, K, ldw, B, A, r, R, ldr,
+                                 as_stream(stream));
 }
 
 TTQ_EXPORT ttq_status ttq_unpack_codes(const uint32_t* codes, int64_t N,

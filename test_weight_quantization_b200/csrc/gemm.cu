@@ -1169,6 +1169,14 @@ ttq_status launch_pre(const void* X, int64_t T, int64_t K, int64_t ldx,
 // epilogue (two halves with eight or more dequantisers and 32+ tokens).
 int stats_parts_of(int dqw, int bn) { return (dqw >= 8 && bn >= 32) ? 2 : 1; }
 
+bool make_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt,
+                        const void* ptr, uint64_t inner, uint64_t rows,
+                        uint64_t pitch_bytes, uint32_t box_inner,
+                        uint32_t box_rows, CUtensorMapSwizzle swz) {
+  return make_tmap(m, dt, ptr, inner, rows, pitch_bytes, box_inner, box_rows,
+                   swz);
+}
+
 size_t gemm_workspace_bytes(int64_t T, int64_t K, int r) {
   size_t b = align_up((size_t)T * (size_t)K * 2, 1024);
   if (r > 0) b += align_up((size_t)T * 64 * 2, 1024);

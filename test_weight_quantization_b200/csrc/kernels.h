@@ -1,6 +1,7 @@
 // kernels.h — internal launchers behind the C ABI (not exported).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -97,5 +98,25 @@ ttq_status launch_lowrank_add(const void* X, ttq_dtype xt, int64_t T,
                               int64_t K, int64_t ldx, const void* A,
                               const void* B, int r, int64_t N, void* Y,
                               ttq_dtype yt, int64_t ldy, cudaStream_t st);
+
+// 2D TMA descriptor of a [rows][inner] tensor with a row pitch of
+// pitch_bytes, copied in boxes of box_inner x box_rows; out-of-range
+// elements read as zero (gemm.cu).
+bool make_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt,
+                        const void* ptr, uint64_t inner, uint64_t rows,
+                        uint64_t pitch_bytes, uint32_t box_inner,
+                        uint32_t box_rows, CUtensorMapSwizzle swz);
+
+// Per-prompt low-rank factors of the bf16 weight W (lowrank_dyn.cu).
+size_t lowrank_factors_workspace_bytes(int64_t N, int64_t K, int r);
+ttq_status launch_lowrank_factors(const void* W, int64_t N, int64_t K,
+                                  int64_t ldw, const float* s,
+                                  const float* omega, int r, int iters,
+                                  void* B, void* A, void* workspace,
+                                  cudaStream_t st);
+ttq_status launch_lowrank_residual(const void* W, int64_t N, int64_t K,
+                                   int64_t ldw, const void* B, const void* A,
+                                   int r, void* R, int64_t ldr,
+                                   cudaStream_t st);
 
 }  // namespace ttq

@@ -1,0 +1,814 @@
+// lowrank_dyn.cu — per-prompt ("dynamic") low-rank factors of a weight and
+// the residual that TTQ then quantizes.
+//
+// TTQ review, "Proposed method", bullet 5: when needed, W is written as
+// W_q + B A with dynamic factors B and A and W_q is quantized on the fly;
+// "Main results", bullet 4: TTQ quantizes the residual and adds the
+// low-rank projection. The factors are found per prompt, once TTQ's scales
+// s are known, by randomized subspace iteration (Halko, Martinsson and
+// Tropp, "Finding structure with randomness", Algorithm 4.4) on the matrix
+// TTQ quantizes, W_s = W diag(s), from r caller-drawn probe vectors Omega:
+//   Q = orth(W_s Omega^T);  iters x { Z = orth(W_s^T Q); Q = orth(W_s Z) }
+//   B = bf16(Q),  A = bf16(Q^T W)
+// orth() keeps Gram-Schmidt's column order and drops a column whose part
+// orthogonal to the kept columns is at most 2^-10 of the input's largest
+// column norm (its output column is zero).
+//
+// Kernels:
+//  skinny_kernel<TRANS>  out[j][m] = sum_c W[m][c] P[j][c] (TRANS: W[c][m]),
+//      the r <= 64 columns of a product with the weight on tcgen05. W is
+//      read once by TMA in 128 x 128 bf16 stages; eight converter warps move
+//      a stage into TMEM as fp16 pairs (the A operand: a thread per output
+//      row m = TMEM lane; TRANS reads a column of the stage per thread), and
+//      one thread issues M=128, N=rpad, K=16 MMAs against the fp16 P tile.
+//      The contraction is split over gridDim.y; each split writes its
+//      partial sums, which the next kernel adds in split order.
+//  gram_kernel           partial Gram matrices of y_m = sc_m sum_p parts
+//      (fp32 entries, fp64 products and sums); the last CTA to
+//      arrive adds the partials in CTA order and factors the Gram matrix
+//      (Cholesky with the drop rule) into R, fp64.
+//  apply_kernel          q_m = y_m R^-1 by forward substitution: Q in fp32,
+//      and the fp16 operand P = (post_m q_m) of the next product. Two
+//      gram/apply rounds (CholeskyQR2) orthonormalise a block of columns.
+//  factors_out_kernel    B = bf16(Q_N)^T and A = bf16(sum_p parts).
+//  residual_kernel       R = bf16(W - B A), fp32 accumulation in j order.
+// Every mbarrier wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds
+// down); nothing spins on another CTA (the Gram tail uses an arrival count).
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ttq {
+namespace {
+
+constexpr int kBM = 128;                  // output rows per CTA (TMEM lanes)
+constexpr int kSC = 128;                  // contraction per stage
+constexpr uint32_t kWBox = kBM * 128u;    // one 128 x 64 bf16 box, bytes
+constexpr uint32_t kWStage = 2u * kWBox;  // two boxes per stage
+constexpr int kConvWarps = 8;
+constexpr int kSkinnyThreads = 32 * (2 + kConvWarps);
+constexpr int kTmemCols = 256;            // accumulator (64) + 3 stages
+constexpr int kAccCols = 64;
+constexpr float kDropTol = 0.0009765625f;  // 2^-10
+
+struct SkinnyArgs {
+  int M, C;          // output rows, contraction length
+  int rpad, r;       // MMA N (16..64) and rows j of the output
+  int c_stages;      // ceil(C / 128)
+  int per;           // stages per split
+  int S;             // shared-memory ring depth (2 or 3)
+  float* out;        // [split][r][ldo]
+  long long ldo;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ uint32_t bf16_pair_to_f16_pair(uint32_t v,
+                                                          bool& range) {
+  const float a = __uint_as_float(v << 16);
+  const float b = __uint_as_float(v & 0xFFFF0000u);
+  range |= !(fabsf(a) < 65504.f) || !(fabsf(b) < 65504.f);
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+template <bool TRANS>
+__global__ void __launch_bounds__(kSkinnyThreads, 2)
+    skinny_kernel(const __grid_constant__ CUtensorMap tm_w,
+                  const __grid_constant__ CUtensorMap tm_p,
+                  const SkinnyArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const gbase = smem_raw + (base - raw);
+  const int S = a.S;
+  const uint32_t pbox = (uint32_t)a.rpad * 128u;  // one 64-column P box
+  const uint32_t p_off = (uint32_t)S * kWStage;
+  const uint32_t bar_off = p_off + (uint32_t)S * 2u * pbox;
+  const uint32_t b_loaded = base + bar_off;
+  const uint32_t b_ready = b_loaded + 8u * S;
+  const uint32_t b_empty = b_ready + 8u * S;
+  const uint32_t b_acc = b_empty + 8u * S;
+  volatile uint32_t* tmem_slot =
+      reinterpret_cast<volatile uint32_t*>(gbase + bar_off + 24u * S + 8u);
+  volatile int* aborted =
+      reinterpret_cast<volatile int*>(gbase + bar_off + 24u * S + 12u);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int split = blockIdx.y;
+  const int s_begin = min(split * a.per, a.c_stages);
+  const int n = min(s_begin + a.per, a.c_stages) - s_begin;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(b_loaded + 8 * i, 1);
+      mbar_init(b_ready + 8 * i, 32 * kConvWarps);
+      mbar_init(b_empty + 8 * i, 1);
+    }
+    mbar_init(b_acc, 1);
+    *aborted = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_p);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  griddep_enter();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_w = tmem + kAccCols;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer ----
+    if (lane == 0) {
+      int issued = 0;
+      for (int s = 0; s < n; ++s) {
+        const int slot = s % S;
+        if (s >= S &&
+            !mbar_wait(b_empty + 8 * slot, (uint32_t)(s / S - 1) & 1u, a.err)) {
+          *aborted = 1;
+          break;
+        }
+        if (*aborted) break;
+        const int c0 = (s_begin + s) * kSC;
+        const uint32_t bar = b_loaded + 8 * slot;
+        const uint32_t wdst = base + (uint32_t)slot * kWStage;
+        const uint32_t pdst = base + p_off + (uint32_t)slot * 2u * pbox;
+        mbar_arrive_expect_tx(bar, kWStage + 2u * pbox);
+        if constexpr (TRANS) {
+          tma_load_2d(wdst, &tm_w, m0, c0, bar);
+          tma_load_2d(wdst + kWBox, &tm_w, m0 + 64, c0, bar);
+        } else {
+          tma_load_2d(wdst, &tm_w, c0, m0, bar);
+          tma_load_2d(wdst + kWBox, &tm_w, c0 + 64, m0, bar);
+        }
+        tma_load_2d(pdst, &tm_p, c0, 0, bar);
+        tma_load_2d(pdst + pbox, &tm_p, c0 + 64, 0, bar);
+        issued = s + 1;
+      }
+      // no bulk copy may still be writing shared memory at exit
+      for (int i = 0; i < S && i < issued; ++i) {
+        const int q = issued - 1 - i;
+        mbar_wait(b_loaded + 8 * (q % S), (uint32_t)(q / S) & 1u, a.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kBM, a.rpad);
+      for (int s = 0; s < n; ++s) {
+        const int slot = s % S;
+        if (!mbar_wait(b_ready + 8 * slot, (uint32_t)(s / S) & 1u, a.err)) {
+          *aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ad = tmem_w + (uint32_t)slot * 64u;
+        const uint32_t pd = base + p_off + (uint32_t)slot * 2u * pbox;
+        const uint64_t bd0 = smem_desc_sw128(pd);
+        const uint64_t bd1 = smem_desc_sw128(pd + pbox);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc_mma_f16_ts(tmem, ad + 8 * k, bd0 + 2 * k, idesc,
+                        (s > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          tc_mma_f16_ts(tmem, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
+        tc_commit(b_empty + 8 * slot);
+      }
+      tc_commit(b_acc);
+    }
+  } else {
+    // ---------------------------------------------- converter warps ---
+    // thread = output row i of the tile = TMEM lane; the two warps of a
+    // lane quarter take the two 64-wide halves of a stage's contraction
+    const int q4 = warp & 3;
+    const int h = (warp - 2) >> 2;
+    const int i = 32 * q4 + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+    bool range = false;
+    for (int s = 0; s < n; ++s) {
+      const int slot = s % S;
+      // the load of stage s follows the MMA of stage s - S (the producer
+      // waited for it), so this TMEM slot is free once `loaded` completes
+      const bool ok =
+          mbar_wait(b_loaded + 8 * slot, (uint32_t)(s / S) & 1u, a.err) &&
+          !*aborted;
+      if (!__all_sync(0xffffffffu, ok)) break;  // the TMEM store is per warp
+      const uint32_t wst = base + (uint32_t)slot * kWStage;
+      uint32_t o[32];
+      if constexpr (!TRANS) {
+        // row i of box h: 8 chunks of 16 bytes at chunk ^ (i % 8)
+        const uint32_t row = wst + (uint32_t)h * kWBox + (uint32_t)i * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[4];
+          asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
+                       : "r"(row + (((uint32_t)c ^ ((uint32_t)i & 7u)) << 4))
+                       : "memory");
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            o[4 * c + e] = bf16_pair_to_f16_pair(v[e], range);
+        }
+      } else {
+        // column i (box i / 64, column i % 64) of stage rows 64h .. 64h+63
+        const uint32_t col = wst + (uint32_t)(i >> 6) * kWBox +
+                             (uint32_t)(i & 7) * 2u;
+        const uint32_t chunk = (uint32_t)((i & 63) >> 3);
+#pragma unroll
+        for (int pp = 0; pp < 32; ++pp) {
+          const uint32_t c0 = (uint32_t)(64 * h + 2 * pp);
+          const uint32_t lo = ld_shared_u16(col + c0 * 128u +
+                                            ((chunk ^ (c0 & 7u)) << 4));
+          const uint32_t hi = ld_shared_u16(col + (c0 + 1u) * 128u +
+                                            ((chunk ^ ((c0 + 1u) & 7u)) << 4));
+          o[pp] = bf16_pair_to_f16_pair(lo | (hi << 16), range);
+        }
+      }
+      tmem_st32(tmem_w + (uint32_t)slot * 64u + lane_base + 32u * h, o);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(b_ready + 8 * slot);
+    }
+    if (range) flag_error(a.err, TTQ_DEVERR_FP16_RANGE);
+    // epilogue: every issued MMA has completed once b_acc does (the MMA
+    // thread commits it on every path)
+    const bool done = mbar_wait(b_acc, 0, a.err);
+    tc_fence_after();
+    const bool go = __all_sync(0xffffffffu, done && !*aborted);
+    if (go && h == 0) {
+      const int m = m0 + i;
+      float* out = a.out + (long long)split * a.r * a.ldo + m;
+      for (int j0 = 0; j0 < a.rpad; j0 += 16) {
+        float v[16];
+        tmem_ld16(tmem + lane_base + (uint32_t)j0, v);
+        if (m < a.M) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (j0 + j < a.r) out[(long long)(j0 + j) * a.ldo] = v[j];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------- orthonormalisation ---
+
+constexpr int kGramThreads = 256;
+constexpr int kGramRows = 128;
+constexpr int kMaxGramCtas = 64;
+constexpr int kMaxPairs = 64 * 65 / 2;
+
+struct GramArgs {
+  const float* parts;  // [nparts][r][ld]
+  int nparts;
+  long long ld;
+  int M, r;
+  const float* sc;     // row scales (null: 1)
+  double* partials;    // [gridDim.x][npairs]
+  double* R;           // [64][64] upper triangular, output
+  unsigned int* counter;
+  uint32_t* err;
+};
+
+// y_m[j] for one row, summed over the parts in order and scaled
+__device__ __forceinline__ float y_entry(const GramArgs& g, int j, int m) {
+  float v = 0.f;
+  for (int p = 0; p < g.nparts; ++p)
+    v += g.parts[((long long)p * g.r + j) * g.ld + m];
+  return g.sc ? v * g.sc[m] : v;
+}
+
+__global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
+  // rows of y (fp32) during the partial sums; the Gram matrix (fp64) in
+  // the tail
+  __shared__ __align__(16) uint8_t buf[kGramRows * 65 * 4 > 64 * 65 * 8
+                                           ? kGramRows * 65 * 4
+                                           : 64 * 65 * 8];
+  __shared__ uint16_t pa[kMaxPairs], pb[kMaxPairs];
+  __shared__ double diag_max;
+  __shared__ bool is_last;
+  griddep_enter();
+  const int r = g.r, npairs = r * (r + 1) / 2;
+  for (int e = threadIdx.x; e < r; e += kGramThreads) {
+    // pairs of row a start at a*r - a(a-1)/2
+    const int s0 = e * r - e * (e - 1) / 2;
+    for (int b = e; b < r; ++b) {
+      pa[s0 + b - e] = (uint16_t)e;
+      pb[s0 + b - e] = (uint16_t)b;
+    }
+  }
+  float* ys = reinterpret_cast<float*>(buf);  // [kGramRows][65]
+  constexpr int kPer = (kMaxPairs + kGramThreads - 1) / kGramThreads;
+  double acc[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) acc[q] = 0.0;
+  const int nblk = (g.M + kGramRows - 1) / kGramRows;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kGramRows * r; e += kGramThreads) {
+      const int row = e % kGramRows, j = e / kGramRows;
+      const int m = blk * kGramRows + row;
+      ys[row * 65 + j] = m < g.M ? y_entry(g, j, m) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int e = threadIdx.x + q * kGramThreads;
+      if (e < npairs) {
+        const int ea = pa[e], eb = pb[e];
+        // fp64 products of fp32 entries are exact: the Gram matrix keeps
+        // the resolution the drop rule needs (a column's remaining squared
+        // norm is a difference of such sums)
+        double d = 0.0;
+        for (int row = 0; row < kGramRows; ++row)
+          d = fma((double)ys[row * 65 + ea], (double)ys[row * 65 + eb], d);
+        acc[q] += d;
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int e = threadIdx.x + q * kGramThreads;
+    if (e < npairs) g.partials[(long long)blockIdx.x * npairs + e] = acc[q];
+  }
+  // the last CTA to arrive factors the sum of the partials
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    is_last = atomicAdd(g.counter, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  double* G = reinterpret_cast<double*>(buf);  // [64][65], upper part
+  for (int e = threadIdx.x; e < npairs; e += kGramThreads) {
+    double v = 0.0;
+    for (int c = 0; c < (int)gridDim.x; ++c)
+      v += __ldcg(g.partials + (long long)c * npairs + e);
+    G[pa[e] * 65 + pb[e]] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double mx = 0.0;
+    for (int j = 0; j < r; ++j) mx = fmax(mx, G[j * 65 + j]);
+    diag_max = mx;
+  }
+  __syncthreads();
+  // right-looking Cholesky, upper factor in place; a column is dropped when
+  // its remaining squared norm is at most (tol * largest column norm)^2
+  const double thresh = (double)kDropTol * (double)kDropTol * diag_max;
+  for (int j = 0; j < r; ++j) {
+    const double d = G[j * 65 + j];
+    const bool keep = diag_max > 0.0 && d > thresh;
+    const double rjj = keep ? sqrt(d) : 0.0;
+    __syncthreads();
+    for (int b = j + 1 + threadIdx.x; b < r; b += kGramThreads)
+      G[j * 65 + b] = keep ? G[j * 65 + b] / rjj : 0.0;
+    if (threadIdx.x == 0) G[j * 65 + j] = rjj;
+    __syncthreads();
+    const int rest = r - j - 1;
+    for (int e = threadIdx.x; e < rest * rest; e += kGramThreads) {
+      const int ia = j + 1 + e / rest, ib = j + 1 + e % rest;
+      if (ia <= ib) G[ia * 65 + ib] -= G[j * 65 + ia] * G[j * 65 + ib];
+    }
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < 64 * 64; e += kGramThreads) {
+    const int ia = e / 64, ib = e % 64;
+    g.R[e] = (ia < r && ib < r && ia <= ib) ? G[ia * 65 + ib] : 0.0;
+  }
+  if (threadIdx.x == 0) *g.counter = 0u;  // ready for the next launch
+}
+
+struct ApplyArgs {
+  GramArgs in;         // the same y as the Gram kernel read
+  const double* R;
+  float* Q;            // [r][ldq] or null
+  long long ldq;
+  __half* P;           // [rpad][ldp] fp16 operand or null
+  long long ldp;
+  int rpad, Mp;        // P rows and the padded columns written
+  const float* post;   // scales of P's columns (null: 1)
+};
+
+template <int RT>
+__global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
+  __shared__ float Rs[RT][RT + 1];
+  griddep_enter();
+  const int r = a.in.r;
+  for (int e = threadIdx.x; e < RT * RT; e += blockDim.x) {
+    const int ia = e / RT, ib = e % RT;
+    Rs[ia][ib] = (ia < r && ib < r) ? (float)a.R[ia * 64 + ib] : 0.f;
+  }
+  __syncthreads();
+  const int m = blockIdx.x * blockDim.x + threadIdx.x;
+  if (m >= a.Mp) return;
+  if (m >= a.in.M) {
+    if (a.P)
+      for (int j = 0; j < a.rpad; ++j) a.P[(long long)j * a.ldp + m] =
+          __float2half_rn(0.f);
+    return;
+  }
+  float q[RT];
+#pragma unroll
+  for (int j = 0; j < RT; ++j) {
+    q[j] = 0.f;
+    if (j < r && Rs[j][j] > 0.f) {
+      float v = y_entry(a.in, j, m);
+#pragma unroll
+      for (int k = 0; k < j; ++k) v = fmaf(-Rs[k][j], q[k], v);
+      q[j] = v / Rs[j][j];
+    }
+  }
+  const float post = a.post ? a.post[m] : 1.f;
+#pragma unroll
+  for (int j = 0; j < RT; ++j) {
+    if (j < r) {
+      if (a.Q) a.Q[(long long)j * a.ldq + m] = q[j];
+      if (a.P) a.P[(long long)j * a.ldp + m] = __float2half_rn(post * q[j]);
+    } else if (a.P && j < a.rpad) {
+      a.P[(long long)j * a.ldp + m] = __float2half_rn(0.f);
+    }
+  }
+  if (a.P)
+    for (int j = RT; j < a.rpad; ++j)
+      a.P[(long long)j * a.ldp + m] = __float2half_rn(0.f);
+}
+
+// P[j][k] = fp16(s_k omega[j][k]); zeros past r rows and K columns
+__global__ void probe_kernel(const float* __restrict__ omega,
+                             const float* __restrict__ s, int r, int K,
+                             int rpad, int Kp, __half* __restrict__ P) {
+  griddep_enter();
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (long long)rpad * Kp) return;
+  const int j = (int)(e / Kp), k = (int)(e % Kp);
+  const float v = (j < r && k < K) ? s[k] * omega[(long long)j * K + k] : 0.f;
+  P[e] = __float2half_rn(v);
+}
+
+// B[n][j] = bf16(Q[j][n]) and A[j][k] = bf16(sum_p parts[p][j][k])
+__global__ void factors_out_kernel(const float* __restrict__ Qn, int N,
+                                   const float* __restrict__ parts, int nparts,
+                                   int K, int r, __nv_bfloat16* __restrict__ B,
+                                   __nv_bfloat16* __restrict__ A) {
+  griddep_enter();
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nb = (long long)N * r;
+  if (e < nb) {
+    const int nn = (int)(e / r), j = (int)(e % r);
+    B[e] = __float2bfloat16_rn(Qn[(long long)j * N + nn]);
+  } else if (e < nb + (long long)r * K) {
+    const long long f = e - nb;
+    float v = 0.f;
+    for (int p = 0; p < nparts; ++p) v += parts[(long long)p * r * K + f];
+    A[f] = __float2bfloat16_rn(v);
+  }
+}
+
+// --------------------------------------------------------- residual ----
+
+// R[n][k] = bf16(W[n][k] - sum_j B[n][j] A[j][k]), accumulated from W in j
+// order with fused multiply-adds. A thread owns CPT consecutive channels
+// of kResRows rows and holds their column of A in registers.
+constexpr int kResThreads = 256;
+constexpr int kResRows = 32;
+
+template <int RT, int CPT>
+__global__ void __launch_bounds__(kResThreads)
+    residual_kernel(const __nv_bfloat16* __restrict__ W, int N, int K,
+                    long long ldw, const __nv_bfloat16* __restrict__ B,
+                    const __nv_bfloat16* __restrict__ A, int r,
+                    __nv_bfloat16* __restrict__ R, long long ldr) {
+  __shared__ float Bs[kResRows][RT];
+  griddep_enter();
+  const int n0 = blockIdx.y * kResRows;
+  const int k0 = (blockIdx.x * kResThreads + threadIdx.x) * CPT;
+  for (int e = threadIdx.x; e < kResRows * RT; e += kResThreads) {
+    const int rr = e / RT, j = e % RT;
+    const int nn = n0 + rr;
+    Bs[rr][j] = (nn < N && j < r) ? __bfloat162float(B[(long long)nn * r + j])
+                                  : 0.f;
+  }
+  __syncthreads();
+  if (k0 >= K) return;
+  float av[RT][CPT];
+#pragma unroll
+  for (int j = 0; j < RT; ++j)
+#pragma unroll
+    for (int c = 0; c < CPT; ++c)
+      av[j][c] = (j < r && k0 + c < K)
+                     ? __bfloat162float(A[(long long)j * K + k0 + c])
+                     : 0.f;
+  const int rows = min(kResRows, N - n0);
+  for (int rr = 0; rr < rows; ++rr) {
+    const long long off = (long long)(n0 + rr) * ldw + k0;
+    const long long oo = (long long)(n0 + rr) * ldr + k0;
+    float acc[CPT];
+    const bool whole = k0 + CPT <= K;
+    if constexpr (CPT == 4) {
+      if (whole) {
+        const uint2 v = *reinterpret_cast<const uint2*>(W + off);
+        acc[0] = __uint_as_float(v.x << 16);
+        acc[1] = __uint_as_float(v.x & 0xFFFF0000u);
+        acc[2] = __uint_as_float(v.y << 16);
+        acc[3] = __uint_as_float(v.y & 0xFFFF0000u);
+      }
+    } else if constexpr (CPT == 2) {
+      if (whole) {
+        const uint32_t v = *reinterpret_cast<const uint32_t*>(W + off);
+        acc[0] = __uint_as_float(v << 16);
+        acc[1] = __uint_as_float(v & 0xFFFF0000u);
+      }
+    }
+    if (CPT == 1 || !whole) {
+#pragma unroll
+      for (int c = 0; c < CPT; ++c)
+        acc[c] = k0 + c < K ? __bfloat162float(W[off + c]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < RT; ++j) {
+      if (j < r) {
+        const float b = Bs[rr][j];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[c] = fmaf(-b, av[j][c], acc[c]);
+      }
+    }
+    if constexpr (CPT == 4) {
+      if (whole) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+        uint2 v;
+        v.x = *reinterpret_cast<const uint32_t*>(&lo);
+        v.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(R + oo) = v;
+      }
+    } else if constexpr (CPT == 2) {
+      if (whole)
+        *reinterpret_cast<__nv_bfloat162*>(R + oo) =
+            __floats2bfloat162_rn(acc[0], acc[1]);
+    }
+    if (CPT == 1 || !whole) {
+#pragma unroll
+      for (int c = 0; c < CPT; ++c)
+        if (k0 + c < K) R[oo + c] = __float2bfloat16_rn(acc[c]);
+    }
+  }
+}
+
+// ------------------------------------------------------------ host ------
+
+inline long long round_up(long long v, long long a) { return (v + a - 1) / a * a; }
+
+struct Carve {
+  float* parts;      // [max_splits][r][max(N, K)]
+  float* qn;         // [r][N]
+  float* qk;         // [r][K]
+  float* q1;         // [r][max(N, K)]  first CholeskyQR round
+  __half* pn;        // [rpad][Np]
+  __half* pk;        // [rpad][Kp]
+  double* partials;  // [kMaxGramCtas][kMaxPairs]
+  double* R;         // [64][64]
+  unsigned int* counter;
+  size_t total;
+};
+
+constexpr int kMaxSplits = 16;
+
+Carve carve(void* ws, int64_t N, int64_t K, int r) {
+  const long long rpad = round_up(r, 16), Np = round_up(N, 8),
+                  Kp = round_up(K, 8), MX = std::max(N, K);
+  Carve c{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = (size_t)round_up((long long)(off + bytes), 256);
+    return at;
+  };
+  const size_t o_parts = take((size_t)kMaxSplits * r * MX * 4);
+  const size_t o_qn = take((size_t)r * N * 4);
+  const size_t o_qk = take((size_t)r * K * 4);
+  const size_t o_q1 = take((size_t)r * MX * 4);
+  const size_t o_pn = take((size_t)rpad * Np * 2);
+  const size_t o_pk = take((size_t)rpad * Kp * 2);
+  const size_t o_part = take((size_t)kMaxGramCtas * kMaxPairs * 8);
+  const size_t o_R = take(64 * 64 * 8);
+  const size_t o_cnt = take(16);
+  c.total = off;
+  if (ws) {
+    uint8_t* b = static_cast<uint8_t*>(ws);
+    c.parts = reinterpret_cast<float*>(b + o_parts);
+    c.qn = reinterpret_cast<float*>(b + o_qn);
+    c.qk = reinterpret_cast<float*>(b + o_qk);
+    c.q1 = reinterpret_cast<float*>(b + o_q1);
+    c.pn = reinterpret_cast<__half*>(b + o_pn);
+    c.pk = reinterpret_cast<__half*>(b + o_pk);
+    c.partials = reinterpret_cast<double*>(b + o_part);
+    c.R = reinterpret_cast<double*>(b + o_R);
+    c.counter = reinterpret_cast<unsigned int*>(b + o_cnt);
+  }
+  return c;
+}
+
+size_t skinny_smem(int rpad, int S) {
+  return 1024 + (size_t)S * (kWStage + 2u * (uint32_t)rpad * 128u) +
+         24u * S + 16;
+}
+
+// out[split][j][m] partial products of W (bf16 [N][K], pitch ldw) with the
+// fp16 operand P [rpad][Cp]; returns the number of splits written.
+ttq_status run_skinny(bool trans, const void* W, int64_t N, int64_t K,
+                      int64_t ldw, const __half* P, int r, float* out,
+                      int* splits_out, cudaStream_t st) {
+  const int rpad = (int)round_up(r, 16);
+  const int64_t M = trans ? K : N, C = trans ? N : K;
+  const int64_t Cp = round_up(C, 8);
+  const int mtiles = (int)((M + kBM - 1) / kBM);
+  const int cst = (int)((C + kSC - 1) / kSC);
+  const int want = std::max(1, 2 * sm_count() / mtiles);
+  int splits = std::min({want, cst, kMaxSplits});
+  const int per = (cst + splits - 1) / splits;
+  splits = (cst + per - 1) / per;
+  const int S = rpad <= 16 ? 3 : 2;
+  CUtensorMap tw, tp;
+  if (!make_tensor_map_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W,
+                          (uint64_t)K, (uint64_t)N, (uint64_t)ldw * 2, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tensor_map_2d(&tp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, P,
+                          (uint64_t)Cp, (uint64_t)rpad, (uint64_t)Cp * 2, 64,
+                          (uint32_t)rpad, CU_TENSOR_MAP_SWIZZLE_128B))
+    return TTQ_ERR_CUDA;
+  SkinnyArgs a;
+  a.M = (int)M;
+  a.C = (int)C;
+  a.rpad = rpad;
+  a.r = r;
+  a.c_stages = cst;
+  a.per = per;
+  a.S = S;
+  a.out = out;
+  a.ldo = M;
+  a.err = device_error_word();
+  const size_t smem = skinny_smem(rpad, S);
+  auto kern = trans ? skinny_kernel<true> : skinny_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return TTQ_ERR_CUDA;
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)mtiles, (unsigned)splits, 1);
+  ls.block = dim3(kSkinnyThreads);
+  ls.smem = smem;
+  *splits_out = splits;
+  return launch(ls, st, kern, tw, tp, a);
+}
+
+template <int RT>
+ttq_status launch_apply(const ApplyArgs& a, cudaStream_t st) {
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)((a.Mp + 255) / 256));
+  ls.block = dim3(256);
+  return launch(ls, st, apply_kernel<RT>, a);
+}
+
+// Orthonormal columns of y (the summed, row-scaled parts) by two
+// Gram/Cholesky/apply rounds: Q fp32 [r][M] and the fp16 operand P
+// [rpad][Mp] = post * Q.
+ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
+                  int r, const float* sc, float* Q, __half* P,
+                  const float* post, cudaStream_t st) {
+  const int rpad = (int)round_up(r, 16);
+  const int64_t Mp = round_up(M, 8);
+  const int ctas = (int)std::min<int64_t>(kMaxGramCtas, (M + kGramRows - 1) /
+                                                            kGramRows);
+  for (int round = 0; round < 2; ++round) {
+    GramArgs g;
+    g.parts = round == 0 ? parts : c.q1;
+    g.nparts = round == 0 ? nparts : 1;
+    g.ld = M;
+    g.M = (int)M;
+    g.r = r;
+    g.sc = round == 0 ? sc : nullptr;
+    g.partials = c.partials;
+    g.R = c.R;
+    g.counter = c.counter;
+    g.err = device_error_word();
+    LaunchShape ls;
+    ls.grid = dim3((unsigned)ctas);
+    ls.block = dim3(kGramThreads);
+    ttq_status e = launch(ls, st, gram_kernel, g);
+    if (e != TTQ_OK) return e;
+    ApplyArgs a;
+    a.in = g;
+    a.R = c.R;
+    a.Q = round == 0 ? c.q1 : Q;
+    a.ldq = M;
+    a.P = round == 0 ? nullptr : P;
+    a.ldp = Mp;
+    a.rpad = rpad;
+    a.Mp = (int)(round == 0 ? M : Mp);
+    a.post = round == 0 ? nullptr : post;
+    e = r <= 16 ? launch_apply<16>(a, st)
+        : r <= 32 ? launch_apply<32>(a, st) : launch_apply<64>(a, st);
+    if (e != TTQ_OK) return e;
+  }
+  return TTQ_OK;
+}
+
+template <int RT, int CPT>
+ttq_status launch_residual_t(const void* W, int64_t N, int64_t K,
+                             int64_t ldw, const void* B, const void* A, int r,
+                             void* R, int64_t ldr, cudaStream_t st) {
+  LaunchShape ls;
+  const int64_t cols = (K + CPT - 1) / CPT;
+  ls.grid = dim3((unsigned)((cols + kResThreads - 1) / kResThreads),
+                 (unsigned)((N + kResRows - 1) / kResRows));
+  ls.block = dim3(kResThreads);
+  return launch(ls, st, residual_kernel<RT, CPT>,
+                static_cast<const __nv_bfloat16*>(W), (int)N, (int)K,
+                (long long)ldw, static_cast<const __nv_bfloat16*>(B),
+                static_cast<const __nv_bfloat16*>(A), r,
+                static_cast<__nv_bfloat16*>(R), (long long)ldr);
+}
+
+}  // namespace
+
+size_t lowrank_factors_workspace_bytes(int64_t N, int64_t K, int r) {
+  return carve(nullptr, N, K, r).total;
+}
+
+ttq_status launch_lowrank_factors(const void* W, int64_t N, int64_t K,
+                                  int64_t ldw, const float* s,
+                                  const float* omega, int r, int iters,
+                                  void* B, void* A, void* workspace,
+                                  cudaStream_t st) {
+  const Carve c = carve(workspace, N, K, r);
+  const int rpad = (int)round_up(r, 16);
+  const int64_t Kp = round_up(K, 8);
+  // the counter must start at zero; the Gram tail leaves it at zero
+  if (cudaMemsetAsync(c.counter, 0, 16, st) != cudaSuccess)
+    return TTQ_ERR_CUDA;
+  {
+    LaunchShape ls;
+    const long long total = (long long)rpad * Kp;
+    ls.grid = dim3((unsigned)((total + 255) / 256));
+    ls.block = dim3(256);
+    ttq_status e = launch(ls, st, probe_kernel, omega, s, r, (int)K, rpad,
+                          (int)Kp, c.pk);
+    if (e != TTQ_OK) return e;
+  }
+  int splits = 0;
+  ttq_status e = run_skinny(false, W, N, K, ldw, c.pk, r, c.parts, &splits, st);
+  if (e != TTQ_OK) return e;
+  e = run_qr(c, c.parts, splits, N, r, nullptr, c.qn, c.pn, nullptr, st);
+  if (e != TTQ_OK) return e;
+  for (int it = 0; it < iters; ++it) {
+    e = run_skinny(true, W, N, K, ldw, c.pn, r, c.parts, &splits, st);
+    if (e != TTQ_OK) return e;
+    e = run_qr(c, c.parts, splits, K, r, s, c.qk, c.pk, s, st);
+    if (e != TTQ_OK) return e;
+    e = run_skinny(false, W, N, K, ldw, c.pk, r, c.parts, &splits, st);
+    if (e != TTQ_OK) return e;
+    e = run_qr(c, c.parts, splits, N, r, nullptr, c.qn, c.pn, nullptr, st);
+    if (e != TTQ_OK) return e;
+  }
+  e = run_skinny(true, W, N, K, ldw, c.pn, r, c.parts, &splits, st);
+  if (e != TTQ_OK) return e;
+  LaunchShape ls;
+  const long long total = (long long)N * r + (long long)r * K;
+  ls.grid = dim3((unsigned)((total + 255) / 256));
+  ls.block = dim3(256);
+  return launch(ls, st, factors_out_kernel, (const float*)c.qn, (int)N,
+                (const float*)c.parts, splits, (int)K, r,
+                static_cast<__nv_bfloat16*>(B), static_cast<__nv_bfloat16*>(A));
+}
+
+ttq_status launch_lowrank_residual(const void* W, int64_t N, int64_t K,
+                                   int64_t ldw, const void* B, const void* A,
+                                   int r, void* R, int64_t ldr,
+                                   cudaStream_t st) {
+  if (r <= 16)
+    return launch_residual_t<16, 4>(W, N, K, ldw, B, A, r, R, ldr, st);
+  if (r <= 32)
+    return launch_residual_t<32, 2>(W, N, K, ldw, B, A, r, R, ldr, st);
+  return launch_residual_t<64, 1>(W, N, K, ldw, B, A, r, R, ldr, st);
+}
+
+}  // namespace ttq

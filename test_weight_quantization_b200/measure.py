@@ -5,6 +5,7 @@
     python -m test_weight_quantization_b200.measure quantize N K bits group
     python -m test_weight_quantization_b200.measure gemm     T N K bits group
     python -m test_weight_quantization_b200.measure qgemm    T N K bits group
+    python -m test_weight_quantization_b200.measure lowrank  N K r iters
     python -m test_weight_quantization_b200.measure table    (the shapes below)
     python -m test_weight_quantization_b200.measure [--eager] KIND ...
         (--eager launches directly instead of replaying a CUDA graph)
@@ -224,6 +225,30 @@ def qgemm(T, N, K, bits, group):
     report("fused qdq gemm " + name, graph_us([fused]), flops=flops)
 
 
+def lowrank(N, K, r, iters):
+    """Per-prompt low-rank factors (randomized subspace iteration, iters
+    rounds) and the residual W - B A of an N x K bf16 weight. Algorithmic
+    bytes of the factors: 2 + 2 iters reads of W; of the residual: W read
+    and R written."""
+    Wr = [weights(N, K)]
+    Wr += [Wr[0].clone() for _ in range(rotation(N * K * 2) - 1)]
+    s = torch.ones(K, device="cuda")
+    om = torch.randn(r, K, device="cuda", generator=_gen(3))
+    ws = torch.empty(ttq.lowrank_factors_workspace_size(N, K, r),
+                     dtype=torch.uint8, device="cuda")
+    B, A = ttq.lowrank_factors(Wr[0], s, om, iters, workspace=ws)
+    R = torch.empty_like(Wr[0])
+    name = f"N={N:6d} K={K:6d} r={r:2d}"
+    us = graph_us([lambda W=W: ttq.lowrank_factors(W, s, om, iters,
+                                                   workspace=ws)
+                   for W in Wr])
+    report(f"lowrank factors {name} iters={iters}", us,
+           (2 + 2 * iters) * N * K * 2 + (N + K) * r * 2)
+    us = graph_us([lambda W=W: ttq.lowrank_residual(W, B, A, out=R)
+                   for W in Wr])
+    report(f"lowrank residual {name}", us, 4 * N * K + (N + K) * r * 2)
+
+
 def decode(*Ts):
     """The decode sweep's shapes at the given token counts."""
     for T in Ts or (1, 2, 4, 16):
@@ -235,7 +260,7 @@ def decode(*Ts):
 
 
 FNS = {"stats": stats, "prepare": prepare, "quantize": quantize, "gemm": gemm,
-       "qgemm": qgemm}
+       "qgemm": qgemm, "lowrank": lowrank}
 
 
 def main(argv):

@@ -69,6 +69,9 @@ def _load() -> ctypes.CDLL:
         "ttq_stats_reduce": [P, I64, I64, I, P, P],
         "ttq_quantize_gemm_prepared": [P, I, I64, P, P, P, I64, I64, I64, I,
                                        I, P, I, I, P, I, I64, P, P, P, P],
+        "ttq_lowrank_factors_workspace_size": [I64, I64, I],
+        "ttq_lowrank_factors": [P, I64, I64, I64, P, P, I, I, P, P, P, SZ, P],
+        "ttq_lowrank_residual": [P, I64, I64, I64, P, P, I, P, I64, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -79,6 +82,7 @@ def _load() -> ctypes.CDLL:
     lib.ttq_codes_ld.restype = I64
     lib.ttq_groups_ld.restype = I64
     lib.ttq_projection_stats_rows.restype = I64
+    lib.ttq_lowrank_factors_workspace_size.restype = SZ
     return lib
 
 
@@ -94,7 +98,9 @@ EXPORTS = ("ttq_act_stats", "ttq_awq_scales", "ttq_act_stats_scales",
            "ttq_groups_ld", "ttq_selftest_bounded_wait",
            "ttq_channel_moment_total", "ttq_awq_scales_sharded",
            "ttq_projection_stats_rows", "ttq_w_lowbit_gemm_prepared_stats",
-           "ttq_stats_reduce", "ttq_quantize_gemm_prepared")
+           "ttq_stats_reduce", "ttq_quantize_gemm_prepared",
+           "ttq_lowrank_factors_workspace_size", "ttq_lowrank_factors",
+           "ttq_lowrank_residual")
 
 
 class _Params(ctypes.Structure):
@@ -596,6 +602,59 @@ def lowrank_add(X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
                                 _code(Y, "Y"), ldy, _stream()),
            "ttq_lowrank_add")
     return Y
+
+
+def lowrank_factors_workspace_size(N: int, K: int, r: int) -> int:
+    return int(_lib.ttq_lowrank_factors_workspace_size(N, K, r))
+
+
+def lowrank_factors(W: torch.Tensor, s: torch.Tensor, omega: torch.Tensor,
+                    iters: int = 1, workspace: torch.Tensor | None = None):
+    """Per-prompt low-rank factors (B [N, r], A [r, K], bf16) of the bf16
+    weight W for the scales s, from the probe vectors omega [r, K] (fp32):
+    randomized subspace iteration on W diag(s), B = Q, A = Q^T W."""
+    ldw = _rows(W, "W")
+    N, K = W.shape
+    if W.dtype != torch.bfloat16:
+        raise TTQError("W must be bfloat16")
+    _buf(s, "s", torch.float32, K)
+    if omega.dim() != 2 or omega.shape[1] != K:
+        raise TTQError(f"omega must be [r, {K}], got {tuple(omega.shape)}")
+    r = omega.shape[0]
+    _buf(omega, "omega", torch.float32, r, K)
+    need = lowrank_factors_workspace_size(N, K, r)
+    if need == 0:
+        raise TTQError(f"no factor workspace for N={N}, K={K}, r={r}")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _buf(workspace, "workspace", torch.uint8, need)
+    B = torch.empty((N, r), dtype=torch.bfloat16, device=W.device)
+    A = torch.empty((r, K), dtype=torch.bfloat16, device=W.device)
+    _check(_lib.ttq_lowrank_factors(W.data_ptr(), N, K, ldw, s.data_ptr(),
+                                    omega.data_ptr(), r, int(iters),
+                                    B.data_ptr(), A.data_ptr(),
+                                    workspace.data_ptr(), workspace.numel(),
+                                    _stream()), "ttq_lowrank_factors")
+    return B, A
+
+
+def lowrank_residual(W: torch.Tensor, B: torch.Tensor, A: torch.Tensor,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """R = bf16(W - B A) (bf16 W [N, K], B [N, r], A [r, K])."""
+    ldw = _rows(W, "W")
+    N, K = W.shape
+    if W.dtype != torch.bfloat16:
+        raise TTQError("W must be bfloat16")
+    r = _factors(A, B, N, K, torch.bfloat16)
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.bfloat16, device=W.device)
+    ldr = _out(out, "out", N, K)
+    if out.dtype != torch.bfloat16:
+        raise TTQError("out must be bfloat16")
+    _check(_lib.ttq_lowrank_residual(W.data_ptr(), N, K, ldw, B.data_ptr(),
+                                     A.data_ptr(), r, out.data_ptr(), ldr,
+                                     _stream()), "ttq_lowrank_residual")
+    return out
 
 
 def unpack_codes(codes: torch.Tensor, K: int, bits: int) -> torch.Tensor:

@@ -45,7 +45,7 @@ def test_status_strings_and_version(lib):
     assert lib.ttq_status_string(0) == b"TTQ_OK"
     assert lib.ttq_status_string(1) == b"TTQ_ERR_INVALID_ARG"
     assert lib.ttq_status_string(99) == b"TTQ_ERR_UNKNOWN"
-    assert lib.ttq_abi_version() == 7
+    assert lib.ttq_abi_version() == 8
 
 
 def test_workspace_size(lib):
@@ -113,6 +113,45 @@ def test_bad_arguments_are_rejected_before_launch(lib):
              None, 8, fake, 1, 32, fake, 1 << 20, None) == 1
     lib.ttq_unpack_codes.argtypes = [P, I64, I64, I, P, P]
     assert lib.ttq_unpack_codes(None, 4, 64, 4, fake, None) == 1
+    SZ = ctypes.c_size_t
+    ws = lib.ttq_lowrank_factors_workspace_size
+    ws.argtypes = [I64, I64, I]
+    ws.restype = SZ
+    assert ws(256, 512, 16) > 0 and ws(256, 512, 0) == 0
+    assert ws(256, 512, 65) == 0
+    lf = lib.ttq_lowrank_factors
+    lf.argtypes = [P, I64, I64, I64, P, P, I, I, P, P, P, SZ, P]
+    big = 1 << 30
+    a16 = ctypes.c_void_p(0x1000000)     # 16-byte aligned, never touched
+    Bp, Ap = ctypes.c_void_p(0x2000000), ctypes.c_void_p(0x3000000)
+    wsp = ctypes.c_void_p(0x4000000)
+    need = ws(256, 512, 16)
+    assert lf(a16, 256, 512, 512, a16, a16, 0, 1, Bp, Ap, wsp, big,
+              None) == 1                                  # r = 0
+    assert lf(a16, 256, 512, 512, a16, a16, 16, 17, Bp, Ap, wsp, big,
+              None) == 1                                  # iters > 16
+    assert lf(a16, 256, 512, 500, a16, a16, 16, 1, Bp, Ap, wsp, big,
+              None) == 1                                  # ldw < K
+    assert lf(a16, 256, 512, 516, a16, a16, 16, 1, Bp, Ap, wsp, big,
+              None) == 1                                  # ldw % 8
+    assert lf(ctypes.c_void_p(0x1000008), 256, 512, 512, a16, a16, 16, 1, Bp,
+              Ap, wsp, big, None) == 1                    # W not 16-aligned
+    assert lf(a16, 256, 512, 512, a16, a16, 16, 1, Bp, Ap, wsp, need - 1,
+              None) == 1                                  # workspace short
+    assert lf(a16, 256, 512, 512, a16, a16, 16, 1, Bp, Ap,
+              ctypes.c_void_p(0x4000080), big, None) == 1  # ws not 256-aligned
+    assert lf(a16, 256, 512, 512, a16, a16, 16, 1, Bp,
+              ctypes.c_void_p(0x2000000 + 256 * 16), wsp, big,
+              None) == 1                                  # A overlaps B
+    lr = lib.ttq_lowrank_residual
+    lr.argtypes = [P, I64, I64, I64, P, P, I, P, I64, P]
+    Rp = ctypes.c_void_p(0x5000000)
+    assert lr(a16, 64, 512, 512, Bp, Ap, 0, Rp, 512, None) == 1   # r = 0
+    assert lr(a16, 64, 512, 512, Bp, Ap, 65, Rp, 512, None) == 1  # r > 64
+    assert lr(a16, 64, 512, 512, Bp, Ap, 16, Rp, 508, None) == 1  # ldr < K
+    assert lr(a16, 64, 512, 512, Bp, Ap, 16,
+              ctypes.c_void_p(0x1000000 + 1024), 512, None) == 1  # R inside W
+    assert lr(a16, 64, 512, 512, Bp, Ap, 16, a16, 520, None) == 1  # W, other ld
 
 
 def test_oracle_and_cuda_path_share_no_code():

@@ -41,6 +41,11 @@ MISTAKES = [
     ("bf16_rounding_half_up",
      "np.rint(np.ldexp(x, -step_exp))", "np.floor(np.ldexp(x, -step_exp) + 0.5)"),
     ("no_subnormal_floor", "e = np.maximum(e, -125)", "e = e"),
+    ("near_ties_without_the_chain_bound",
+     "bound = (r + 1) * 2.0 ** -24 * (np.abs(W) + np.abs(B) @ np.abs(A))",
+     "bound = 0.0 * np.abs(W)"),
+    ("near_ties_at_representable_values",
+     "dist = np.abs(frac - 0.5) * step", "dist = np.minimum(frac, 1 - frac) * step"),
 ]
 
 

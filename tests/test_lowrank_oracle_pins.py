@@ -214,6 +214,18 @@ def pin_residual_is_rounded_once(lr):
                                               np.zeros((2, 3))), W)
 
 
+def pin_residual_near_ties_mark_midpoints_only(lr):
+    """Exact midpoints and values within the fp32 chain bound of one are
+    marked; values a bf16 quarter-step away, and exact results of
+    representable values, are not; a cancellation to (almost) zero is."""
+    W = np.array([[1.0, 2.0, 1.0, 3.0, 1.0, 1.0]])
+    B = np.array([[1.0]])
+    A = np.array([[-2.0 ** -8, 0.5, -2.0 ** -8 - 2.0 ** -30,
+                   -2.0 ** -9, 1.0 - 2.0 ** -40, 1.0]])
+    np.testing.assert_array_equal(lr.residual_near_ties(W, B, A),
+                                  [[1, 0, 1, 0, 1, 1]])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
