@@ -27,7 +27,8 @@
 //      (fp32 entries, fp64 products and sums); the last CTA to
 //      arrive adds the partials in CTA order and factors the Gram matrix
 //      (Cholesky with the drop rule) into R, fp64.
-//  apply_kernel          q_m = y_m R^-1 by forward substitution: Q in fp32,
+//  apply_kernel          q_m = y_m R^-1 by forward substitution (y as the
+//      Gram kernel summed it): Q in fp32,
 //      and the fp16 operand P = (post_m q_m) of the next product. Two
 //      gram/apply rounds (CholeskyQR2) orthonormalise a block of columns.
 //  factors_out_kernel    B = bf16(Q_N)^T and A = bf16(sum_p parts).
@@ -35,6 +36,7 @@
 // Every mbarrier wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds
 // down); nothing spins on another CTA (the Gram tail uses an arrival count).
 #include <algorithm>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -278,24 +280,20 @@ constexpr int kMaxGramCtas = 64;
 constexpr int kMaxPairs = 64 * 65 / 2;
 
 struct GramArgs {
-  const float* parts;  // [nparts][r][ld]
+  const float* parts;  // [nparts][r][ld], nparts <= kMaxParts
   int nparts;
   long long ld;
   int M, r;
   const float* sc;     // row scales (null: 1)
+  float* ysum;         // if not null: the summed, scaled y, [r][ld]
   double* partials;    // [gridDim.x][npairs]
   double* R;           // [64][64] upper triangular, output
   unsigned int* counter;
   uint32_t* err;
 };
 
-// y_m[j] for one row, summed over the parts in order and scaled
-__device__ __forceinline__ float y_entry(const GramArgs& g, int j, int m) {
-  float v = 0.f;
-  for (int p = 0; p < g.nparts; ++p)
-    v += g.parts[((long long)p * g.r + j) * g.ld + m];
-  return g.sc ? v * g.sc[m] : v;
-}
+constexpr int kMaxParts = 16;  // partial products per y (the splits)
+constexpr int kYBatch = 8;     // y entries a thread sums at once
 
 __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   // rows of y (fp32) during the partial sums; the Gram matrix (fp64) in
@@ -324,10 +322,53 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   const int nblk = (g.M + kGramRows - 1) / kGramRows;
   for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kGramRows * r; e += kGramThreads) {
-      const int row = e % kGramRows, j = e / kGramRows;
-      const int m = blk * kGramRows + row;
-      ys[row * 65 + j] = m < g.M ? y_entry(g, j, m) : 0.f;
+    // y = sc_m sum_p parts[p], parts added in order. Loads are issued in
+    // batches of four parts x kYBatch entries before any of them is added
+    // (issue is in order: an add between two loads would serialise them);
+    // entries past the block read a valid address and are discarded.
+    for (int e0 = threadIdx.x; e0 < kGramRows * r;
+         e0 += kYBatch * kGramThreads) {
+      float v[kYBatch];
+      long long off[kYBatch];
+#pragma unroll
+      for (int u = 0; u < kYBatch; ++u) {
+        v[u] = 0.f;
+        const int e = e0 + u * kGramThreads;
+        const int m = blk * kGramRows + e % kGramRows;
+        off[u] = (e < kGramRows * r && m < g.M)
+                     ? (long long)(e / kGramRows) * g.ld + m
+                     : 0;
+      }
+      for (int p0 = 0; p0 < g.nparts; p0 += 4) {
+        float raw[4][kYBatch];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+          const long long pb =
+              (long long)min(p0 + pp, g.nparts - 1) * r * g.ld;
+#pragma unroll
+          for (int u = 0; u < kYBatch; ++u)
+            raw[pp][u] = __ldcg(g.parts + pb + off[u]);
+        }
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp)
+          if (p0 + pp < g.nparts)
+#pragma unroll
+            for (int u = 0; u < kYBatch; ++u) v[u] += raw[pp][u];
+      }
+#pragma unroll
+      for (int u = 0; u < kYBatch; ++u) {
+        const int e = e0 + u * kGramThreads;
+        if (e < kGramRows * r) {
+          const int row = e % kGramRows, j = e / kGramRows;
+          const int m = blk * kGramRows + row;
+          float y = 0.f;
+          if (m < g.M) {
+            y = g.sc ? v[u] * g.sc[m] : v[u];
+            if (g.ysum) g.ysum[(long long)j * g.ld + m] = y;
+          }
+          ys[row * 65 + j] = y;
+        }
+      }
     }
     __syncthreads();
 #pragma unroll
@@ -360,9 +401,19 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   __threadfence();
   double* G = reinterpret_cast<double*>(buf);  // [64][65], upper part
   for (int e = threadIdx.x; e < npairs; e += kGramThreads) {
+    // the CTAs' partials in CTA order, loads issued eight at a time
     double v = 0.0;
-    for (int c = 0; c < (int)gridDim.x; ++c)
-      v += __ldcg(g.partials + (long long)c * npairs + e);
+    const int nc = (int)gridDim.x;
+    for (int c0 = 0; c0 < nc; c0 += 8) {
+      double raw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        raw[u] = __ldcg(g.partials + (long long)min(c0 + u, nc - 1) * npairs +
+                        e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (c0 + u < nc) v += raw[u];
+    }
     G[pa[e] * 65 + pb[e]] = v;
   }
   __syncthreads();
@@ -399,7 +450,9 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
 }
 
 struct ApplyArgs {
-  GramArgs in;         // the same y as the Gram kernel read
+  const float* y;      // [r][ldy]: the rows the Gram kernel factored
+  long long ldy;
+  int M, r;
   const double* R;
   float* Q;            // [r][ldq] or null
   long long ldq;
@@ -412,30 +465,36 @@ struct ApplyArgs {
 template <int RT>
 __global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
   __shared__ float Rs[RT][RT + 1];
+  __shared__ float Rinv[RT];  // 1 / R_jj (0 for a dropped column)
   griddep_enter();
-  const int r = a.in.r;
+  const int r = a.r;
   for (int e = threadIdx.x; e < RT * RT; e += blockDim.x) {
     const int ia = e / RT, ib = e % RT;
-    Rs[ia][ib] = (ia < r && ib < r) ? (float)a.R[ia * 64 + ib] : 0.f;
+    const double v = (ia < r && ib < r) ? a.R[ia * 64 + ib] : 0.0;
+    Rs[ia][ib] = (float)v;
+    if (ia == ib) Rinv[ia] = v > 0.0 ? (float)(1.0 / v) : 0.f;
   }
   __syncthreads();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
   if (m >= a.Mp) return;
-  if (m >= a.in.M) {
+  if (m >= a.M) {
     if (a.P)
       for (int j = 0; j < a.rpad; ++j) a.P[(long long)j * a.ldp + m] =
           __float2half_rn(0.f);
     return;
   }
-  float q[RT];
+  float yv[RT], q[RT];
+#pragma unroll
+  for (int j = 0; j < RT; ++j)
+    yv[j] = j < r ? __ldcg(a.y + (long long)j * a.ldy + m) : 0.f;
 #pragma unroll
   for (int j = 0; j < RT; ++j) {
     q[j] = 0.f;
     if (j < r && Rs[j][j] > 0.f) {
-      float v = y_entry(a.in, j, m);
+      float v = yv[j];
 #pragma unroll
       for (int k = 0; k < j; ++k) v = fmaf(-Rs[k][j], q[k], v);
-      q[j] = v / Rs[j][j];
+      q[j] = v * Rinv[j];
     }
   }
   const float post = a.post ? a.post[m] : 1.f;
@@ -477,9 +536,19 @@ __global__ void factors_out_kernel(const float* __restrict__ Qn, int N,
     const int nn = (int)(e / r), j = (int)(e % r);
     B[e] = __float2bfloat16_rn(Qn[(long long)j * N + nn]);
   } else if (e < nb + (long long)r * K) {
+    // the parts in order, their loads issued four at a time
     const long long f = e - nb;
     float v = 0.f;
-    for (int p = 0; p < nparts; ++p) v += parts[(long long)p * r * K + f];
+    for (int p0 = 0; p0 < nparts; p0 += 4) {
+      float raw[4];
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp)
+        raw[pp] = __ldcg(parts + (long long)min(p0 + pp, nparts - 1) * r * K +
+                         f);
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp)
+        if (p0 + pp < nparts) v += raw[pp];
+    }
     A[f] = __float2bfloat16_rn(v);
   }
 }
@@ -488,9 +557,35 @@ __global__ void factors_out_kernel(const float* __restrict__ Qn, int N,
 
 // R[n][k] = bf16(W[n][k] - sum_j B[n][j] A[j][k]), accumulated from W in j
 // order with fused multiply-adds. A thread owns CPT consecutive channels
-// of kResRows rows and holds their column of A in registers.
+// of kResRows rows and holds their column of A in registers; it keeps the
+// weights of 32 / CPT rows in flight (loads issued before any arithmetic),
+// so that enough bytes are outstanding to stream W at HBM rate.
 constexpr int kResThreads = 256;
 constexpr int kResRows = 32;
+
+template <int CPT>
+__device__ __forceinline__ void store_r(__nv_bfloat16* __restrict__ p,
+                                        int left, const float (&v)[CPT]) {
+  if constexpr (CPT == 4) {
+    if (left >= 4) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(v[2], v[3]);
+      uint2 u;
+      u.x = *reinterpret_cast<const uint32_t*>(&lo);
+      u.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(p) = u;
+      return;
+    }
+  } else if constexpr (CPT == 2) {
+    if (left >= 2) {
+      *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v[0], v[1]);
+      return;
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < CPT; ++c)
+    if (c < left) p[c] = __float2bfloat16_rn(v[c]);
+}
 
 template <int RT, int CPT>
 __global__ void __launch_bounds__(kResThreads)
@@ -498,7 +593,8 @@ __global__ void __launch_bounds__(kResThreads)
                     long long ldw, const __nv_bfloat16* __restrict__ B,
                     const __nv_bfloat16* __restrict__ A, int r,
                     __nv_bfloat16* __restrict__ R, long long ldr) {
-  __shared__ float Bs[kResRows][RT];
+  constexpr int RB = 32 / CPT;  // rows in flight per thread
+  __shared__ __align__(16) float Bs[kResRows][RT];
   griddep_enter();
   const int n0 = blockIdx.y * kResRows;
   const int k0 = (blockIdx.x * kResThreads + threadIdx.x) * CPT;
@@ -510,66 +606,103 @@ __global__ void __launch_bounds__(kResThreads)
   }
   __syncthreads();
   if (k0 >= K) return;
+  const int left = K - k0;
   float av[RT][CPT];
 #pragma unroll
   for (int j = 0; j < RT; ++j)
 #pragma unroll
     for (int c = 0; c < CPT; ++c)
-      av[j][c] = (j < r && k0 + c < K)
+      av[j][c] = (j < r && c < left)
                      ? __bfloat162float(A[(long long)j * K + k0 + c])
                      : 0.f;
   const int rows = min(kResRows, N - n0);
-  for (int rr = 0; rr < rows; ++rr) {
-    const long long off = (long long)(n0 + rr) * ldw + k0;
-    const long long oo = (long long)(n0 + rr) * ldr + k0;
-    float acc[CPT];
-    const bool whole = k0 + CPT <= K;
-    if constexpr (CPT == 4) {
-      if (whole) {
-        const uint2 v = *reinterpret_cast<const uint2*>(W + off);
-        acc[0] = __uint_as_float(v.x << 16);
-        acc[1] = __uint_as_float(v.x & 0xFFFF0000u);
-        acc[2] = __uint_as_float(v.y << 16);
-        acc[3] = __uint_as_float(v.y & 0xFFFF0000u);
-      }
-    } else if constexpr (CPT == 2) {
-      if (whole) {
-        const uint32_t v = *reinterpret_cast<const uint32_t*>(W + off);
-        acc[0] = __uint_as_float(v << 16);
-        acc[1] = __uint_as_float(v & 0xFFFF0000u);
-      }
-    }
-    if (CPT == 1 || !whole) {
+  for (int rr0 = 0; rr0 < rows; rr0 += RB) {
+    float w[RB][CPT];
+    if (left >= CPT && CPT > 1) {
+      // the RB rows' loads are issued before any of them is used (rows
+      // past the end re-read the last row and are not stored): issue is in
+      // order, so a use between two loads would serialise them
+      using Raw = typename std::conditional<CPT == 4, uint2, uint32_t>::type;
+      Raw raw[RB];
 #pragma unroll
-      for (int c = 0; c < CPT; ++c)
-        acc[c] = k0 + c < K ? __bfloat162float(W[off + c]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < RT; ++j) {
-      if (j < r) {
-        const float b = Bs[rr][j];
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) acc[c] = fmaf(-b, av[j][c], acc[c]);
+      for (int u = 0; u < RB; ++u) {
+        const int rr = min(rr0 + u, rows - 1);
+        raw[u] = *reinterpret_cast<const Raw*>(
+            W + (long long)(n0 + rr) * ldw + k0);
       }
-    }
-    if constexpr (CPT == 4) {
-      if (whole) {
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
-        uint2 v;
-        v.x = *reinterpret_cast<const uint32_t*>(&lo);
-        v.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(R + oo) = v;
-      }
-    } else if constexpr (CPT == 2) {
-      if (whole)
-        *reinterpret_cast<__nv_bfloat162*>(R + oo) =
-            __floats2bfloat162_rn(acc[0], acc[1]);
-    }
-    if (CPT == 1 || !whole) {
 #pragma unroll
-      for (int c = 0; c < CPT; ++c)
-        if (k0 + c < K) R[oo + c] = __float2bfloat16_rn(acc[c]);
+      for (int u = 0; u < RB; ++u) {
+        if constexpr (CPT == 4) {
+          const uint2 v = *reinterpret_cast<const uint2*>(&raw[u]);
+          w[u][0] = __uint_as_float(v.x << 16);
+          w[u][1] = __uint_as_float(v.x & 0xFFFF0000u);
+          w[u][2] = __uint_as_float(v.y << 16);
+          w[u][3] = __uint_as_float(v.y & 0xFFFF0000u);
+        } else {
+          const uint32_t v = *reinterpret_cast<const uint32_t*>(&raw[u]);
+          w[u][0] = __uint_as_float(v << 16);
+          w[u][CPT - 1] = __uint_as_float(v & 0xFFFF0000u);
+        }
+      }
+    } else {
+      // one channel per thread, or the ragged end of a row: scalar loads,
+      // again all issued before the arithmetic
+      uint16_t raw[RB][CPT];
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const int rr = min(rr0 + u, rows - 1);
+        const unsigned short* src = reinterpret_cast<const unsigned short*>(
+            W + (long long)(n0 + rr) * ldw + k0);
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) raw[u][c] = src[c < left ? c : 0];
+      }
+#pragma unroll
+      for (int u = 0; u < RB; ++u)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c)
+          w[u][c] = c < left ? __uint_as_float((uint32_t)raw[u][c] << 16)
+                             : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      if (rr0 + u < rows) {
+        // B's row as float4s; entries past r are zero and so are A's, so
+        // the padded steps add exact zeros and need no test
+        float bj[RT];
+#pragma unroll
+        for (int q = 0; q < RT / 4; ++q) {
+          const float4 t = *reinterpret_cast<const float4*>(&Bs[rr0 + u][4 * q]);
+          bj[4 * q] = t.x;
+          bj[4 * q + 1] = t.y;
+          bj[4 * q + 2] = t.z;
+          bj[4 * q + 3] = t.w;
+        }
+        if constexpr (CPT >= 2) {
+          // two channels per instruction (two independent fp32 fused
+          // multiply-adds, each rounded as fmaf would round it)
+          float2 acc[CPT / 2];
+#pragma unroll
+          for (int c = 0; c < CPT / 2; ++c)
+            acc[c] = make_float2(w[u][2 * c], w[u][2 * c + 1]);
+#pragma unroll
+          for (int j = 0; j < RT; ++j) {
+            const float2 nb = make_float2(-bj[j], -bj[j]);
+#pragma unroll
+            for (int c = 0; c < CPT / 2; ++c)
+              acc[c] = __ffma2_rn(
+                  nb, make_float2(av[j][2 * c], av[j][2 * c + 1]), acc[c]);
+          }
+#pragma unroll
+          for (int c = 0; c < CPT / 2; ++c) {
+            w[u][2 * c] = acc[c].x;
+            w[u][2 * c + 1] = acc[c].y;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < RT; ++j) w[u][0] = fmaf(-bj[j], av[j][0], w[u][0]);
+        }
+        store_r<CPT>(R + (long long)(n0 + rr0 + u) * ldr + k0, left, w[u]);
+      }
     }
   }
 }
@@ -583,6 +716,7 @@ struct Carve {
   float* qn;         // [r][N]
   float* qk;         // [r][K]
   float* q1;         // [r][max(N, K)]  first CholeskyQR round
+  float* ysum;       // [r][max(N, K)]  summed products
   __half* pn;        // [rpad][Np]
   __half* pk;        // [rpad][Kp]
   double* partials;  // [kMaxGramCtas][kMaxPairs]
@@ -591,7 +725,7 @@ struct Carve {
   size_t total;
 };
 
-constexpr int kMaxSplits = 16;
+constexpr int kMaxSplits = kMaxParts;
 
 Carve carve(void* ws, int64_t N, int64_t K, int r) {
   const long long rpad = round_up(r, 16), Np = round_up(N, 8),
@@ -607,6 +741,7 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
   const size_t o_qn = take((size_t)r * N * 4);
   const size_t o_qk = take((size_t)r * K * 4);
   const size_t o_q1 = take((size_t)r * MX * 4);
+  const size_t o_ys = take((size_t)r * MX * 4);
   const size_t o_pn = take((size_t)rpad * Np * 2);
   const size_t o_pk = take((size_t)rpad * Kp * 2);
   const size_t o_part = take((size_t)kMaxGramCtas * kMaxPairs * 8);
@@ -619,6 +754,7 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
     c.qn = reinterpret_cast<float*>(b + o_qn);
     c.qk = reinterpret_cast<float*>(b + o_qk);
     c.q1 = reinterpret_cast<float*>(b + o_q1);
+    c.ysum = reinterpret_cast<float*>(b + o_ys);
     c.pn = reinterpret_cast<__half*>(b + o_pn);
     c.pk = reinterpret_cast<__half*>(b + o_pk);
     c.partials = reinterpret_cast<double*>(b + o_part);
@@ -699,6 +835,8 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
   const int ctas = (int)std::min<int64_t>(kMaxGramCtas, (M + kGramRows - 1) /
                                                             kGramRows);
   for (int round = 0; round < 2; ++round) {
+    // round 0 sums the parts into y (kept in c.ysum), round 1 factors the
+    // first round's basis q1
     GramArgs g;
     g.parts = round == 0 ? parts : c.q1;
     g.nparts = round == 0 ? nparts : 1;
@@ -706,6 +844,7 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
     g.M = (int)M;
     g.r = r;
     g.sc = round == 0 ? sc : nullptr;
+    g.ysum = round == 0 ? c.ysum : nullptr;
     g.partials = c.partials;
     g.R = c.R;
     g.counter = c.counter;
@@ -716,7 +855,10 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
     ttq_status e = launch(ls, st, gram_kernel, g);
     if (e != TTQ_OK) return e;
     ApplyArgs a;
-    a.in = g;
+    a.y = round == 0 ? c.ysum : c.q1;
+    a.ldy = M;
+    a.M = (int)M;
+    a.r = r;
     a.R = c.R;
     a.Q = round == 0 ? c.q1 : Q;
     a.ldq = M;

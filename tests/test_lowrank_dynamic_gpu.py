@@ -60,7 +60,7 @@ def _run_factors(ttq, Wb, s, om, iters):
     return B.double().cpu().numpy(), A.double().cpu().numpy()
 
 
-def _check_factors(Bg, Ag, Bo, Ao, W, s, what):
+def _check_factors(Bg, Ag, Bo, Ao, W, s, what, energy=True):
     P_g, P_o = Bg @ Ag, Bo @ Ao
     rel = np.linalg.norm(P_g - P_o) / max(np.linalg.norm(P_o), 1e-30)
     kept = np.linalg.norm(Bg, axis=0) > 0.5
@@ -74,7 +74,8 @@ def _check_factors(Bg, Ag, Bo, Ao, W, s, what):
           f"residual energy rel {erel:.2e}, kept {int(kept.sum())}")
     assert rel < 1e-2, what
     assert orth < 1e-2, what
-    assert erel < 1e-3, what
+    if energy:
+        assert erel < 1e-3, what
 
 
 @pytest.mark.parametrize("N,K,r,iters", [
@@ -116,7 +117,10 @@ def test_factors_of_exactly_low_rank_weight_drop_columns(ttq):
     assert kept.sum() == 3 and not Bg[:, ~kept].any() and not Ag[~kept].any()
     np.testing.assert_allclose(Bg @ Ag, W, rtol=0, atol=2e-2 * np.abs(W).max())
     Bo, Ao = lr_oracle.dynamic_factors(W, s, om, 1)
-    _check_factors(Bg, Ag, Bo, Ao, W, s.astype(np.float64), "rank 3")
+    # the residual of an exactly low-rank weight is the rounding of B and A
+    # alone, different on the two sides: its energy is not compared
+    _check_factors(Bg, Ag, Bo, Ao, W, s.astype(np.float64), "rank 3",
+                   energy=False)
 
 
 def test_factors_with_rank_above_the_dimension(ttq):
