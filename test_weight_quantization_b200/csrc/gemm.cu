@@ -1305,6 +1305,23 @@ ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
     split = (int)std::min<int64_t>(
         8, std::max<int64_t>(1, per_sm * sms / tiles_m));
     split = std::min(split, k_stages);
+  } else if (q && !stats && T <= bn && 2 * tiles_m <= sms) {
+    // The fused form with one token tile: each CTA would quantize a whole
+    // 128-row slab of the weight alone, on a few dozen SMs. Splitting K
+    // over a cluster spreads the quantization over about one wave; the
+    // ranks' partial tiles are reduced in rank order as in decode.
+    int s_ = S;
+    while (s_ > 1 && make_layout(bits, bn, s_, true, true).total + 1024 >
+                         (size_t)kMaxSmem)
+      --s_;
+    if (s_ >= 2) {
+      split = (int)std::min<int64_t>(8, sms / tiles_m);
+      split = std::min(split, k_stages);
+      if (split > 1) {
+        S = s_;
+        SA = std::min(SA, S);
+      }
+    }
   }
   const int per = (k_stages + split - 1) / split;
   split = (k_stages + per - 1) / per;  // every rank gets at least one stage

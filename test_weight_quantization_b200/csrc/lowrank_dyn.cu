@@ -27,10 +27,13 @@
 //      (fp32 entries, fp64 products and sums); the last CTA to
 //      arrive adds the partials in CTA order and factors the Gram matrix
 //      (Cholesky with the drop rule) into R, fp64.
-//  apply_kernel          q_m = y_m R^-1 by forward substitution (y as the
-//      Gram kernel summed it): Q in fp32,
-//      and the fp16 operand P = (post_m q_m) of the next product. Two
-//      gram/apply rounds (CholeskyQR2) orthonormalise a block of columns.
+//  apply_kernel          q_m = y_m R^-1 by forward substitution in fp64 (y
+//      as the Gram kernel summed it): Q in fp32,
+//      and the fp16 operand P = (post_m q_m) of the next product. One
+//      gram/apply round orthonormalises a block of columns: the Gram
+//      matrix is exact up to fp64 sums of exact products, so Q is
+//      orthonormal to about cond(Y)^2 x 1e-16 (cond(Y) stays below about
+//      4 x 2^10 because of the drop rule).
 //  factors_out_kernel    B = bf16(Q_N)^T and A = bf16(sum_p parts).
 //  residual_kernel       R = bf16(W - B A), fp32 accumulation in j order.
 // Every mbarrier wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds
@@ -276,7 +279,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 2)
 
 constexpr int kGramThreads = 256;
 constexpr int kGramRows = 128;
-constexpr int kMaxGramCtas = 64;
+constexpr int kMaxGramCtas = 32;
 constexpr int kMaxPairs = 64 * 65 / 2;
 
 struct GramArgs {
@@ -379,10 +382,18 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
         // fp64 products of fp32 entries are exact: the Gram matrix keeps
         // the resolution the drop rule needs (a column's remaining squared
         // norm is a difference of such sums)
-        double d = 0.0;
-        for (int row = 0; row < kGramRows; ++row)
-          d = fma((double)ys[row * 65 + ea], (double)ys[row * 65 + eb], d);
-        acc[q] += d;
+        // four independent sums over rows 4i .. 4i+3 (the multiply-adds
+        // of one sum would otherwise wait on each other), added in a fixed
+        // order
+        double d[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+        for (int row = 0; row < kGramRows; row += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            d[u] = fma((double)ys[(row + u) * 65 + ea],
+                       (double)ys[(row + u) * 65 + eb], d[u]);
+        }
+        acc[q] += (d[0] + d[1]) + (d[2] + d[3]);
       }
     }
   }
@@ -392,7 +403,7 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
     if (e < npairs) g.partials[(long long)blockIdx.x * npairs + e] = acc[q];
   }
   // the last CTA to arrive factors the sum of the partials
-  __threadfence();
+  if (threadIdx.x < npairs) __threadfence();
   __syncthreads();
   if (threadIdx.x == 0)
     is_last = atomicAdd(g.counter, 1u) == gridDim.x - 1;
@@ -401,19 +412,17 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   __threadfence();
   double* G = reinterpret_cast<double*>(buf);  // [64][65], upper part
   for (int e = threadIdx.x; e < npairs; e += kGramThreads) {
-    // the CTAs' partials in CTA order, loads issued eight at a time
-    double v = 0.0;
+    // the CTAs' partials (at most kMaxGramCtas) in CTA order, their loads
+    // issued together
     const int nc = (int)gridDim.x;
-    for (int c0 = 0; c0 < nc; c0 += 8) {
-      double raw[8];
+    double raw[kMaxGramCtas];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        raw[u] = __ldcg(g.partials + (long long)min(c0 + u, nc - 1) * npairs +
-                        e);
+    for (int u = 0; u < kMaxGramCtas; ++u)
+      raw[u] = __ldcg(g.partials + (long long)min(u, nc - 1) * npairs + e);
+    double v = 0.0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c0 + u < nc) v += raw[u];
-    }
+    for (int u = 0; u < kMaxGramCtas; ++u)
+      if (u < nc) v += raw[u];
     G[pa[e] * 65 + pb[e]] = v;
   }
   __syncthreads();
@@ -429,10 +438,24 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   for (int j = 0; j < r; ++j) {
     const double d = G[j * 65 + j];
     const bool keep = diag_max > 0.0 && d > thresh;
-    const double rjj = keep ? sqrt(d) : 0.0;
+    // 1/sqrt(d): the fp32 estimate refined by two Newton steps in fp64
+    // (each squares the relative error: 2^-22 -> 2^-44 -> below fp64's
+    // precision), then sqrt(d) = d / sqrt(d); no fp64 divide or square
+    // root on the factorisation's critical path
+    double rinv = 0.0, rjj = 0.0;
+    if (keep) {
+      if (d > 1e-30 && d < 1e30) {  // inside fp32's range
+        rinv = (double)rsqrtf((float)d);
+        rinv = rinv * fma(-0.5 * d, rinv * rinv, 1.5);
+        rinv = rinv * fma(-0.5 * d, rinv * rinv, 1.5);
+      } else {
+        rinv = 1.0 / sqrt(d);
+      }
+      rjj = d * rinv;
+    }
     __syncthreads();
     for (int b = j + 1 + threadIdx.x; b < r; b += kGramThreads)
-      G[j * 65 + b] = keep ? G[j * 65 + b] / rjj : 0.0;
+      G[j * 65 + b] = keep ? G[j * 65 + b] * rinv : 0.0;
     if (threadIdx.x == 0) G[j * 65 + j] = rjj;
     __syncthreads();
     const int rest = r - j - 1;
@@ -464,15 +487,15 @@ struct ApplyArgs {
 
 template <int RT>
 __global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
-  __shared__ float Rs[RT][RT + 1];
-  __shared__ float Rinv[RT];  // 1 / R_jj (0 for a dropped column)
+  __shared__ double Rs[RT][RT + 1];
+  __shared__ double Rinv[RT];  // 1 / R_jj (0 for a dropped column)
   griddep_enter();
   const int r = a.r;
   for (int e = threadIdx.x; e < RT * RT; e += blockDim.x) {
     const int ia = e / RT, ib = e % RT;
     const double v = (ia < r && ib < r) ? a.R[ia * 64 + ib] : 0.0;
-    Rs[ia][ib] = (float)v;
-    if (ia == ib) Rinv[ia] = v > 0.0 ? (float)(1.0 / v) : 0.f;
+    Rs[ia][ib] = v;
+    if (ia == ib) Rinv[ia] = v > 0.0 ? 1.0 / v : 0.0;
   }
   __syncthreads();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
@@ -483,17 +506,21 @@ __global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
           __float2half_rn(0.f);
     return;
   }
-  float yv[RT], q[RT];
+  // forward substitution in fp64: with R from an fp64 Gram matrix, one
+  // Cholesky-QR round leaves Q orthonormal to about cond(Y)^2 x 1e-16,
+  // far below the fp32 and bf16 roundings that follow
+  float yv[RT];
+  double q[RT];
 #pragma unroll
   for (int j = 0; j < RT; ++j)
     yv[j] = j < r ? __ldcg(a.y + (long long)j * a.ldy + m) : 0.f;
 #pragma unroll
   for (int j = 0; j < RT; ++j) {
-    q[j] = 0.f;
-    if (j < r && Rs[j][j] > 0.f) {
-      float v = yv[j];
+    q[j] = 0.0;
+    if (j < r && Rinv[j] > 0.0) {
+      double v = (double)yv[j];
 #pragma unroll
-      for (int k = 0; k < j; ++k) v = fmaf(-Rs[k][j], q[k], v);
+      for (int k = 0; k < j; ++k) v = fma(-Rs[k][j], q[k], v);
       q[j] = v * Rinv[j];
     }
   }
@@ -501,8 +528,9 @@ __global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
 #pragma unroll
   for (int j = 0; j < RT; ++j) {
     if (j < r) {
-      if (a.Q) a.Q[(long long)j * a.ldq + m] = q[j];
-      if (a.P) a.P[(long long)j * a.ldp + m] = __float2half_rn(post * q[j]);
+      const float qf = (float)q[j];
+      if (a.Q) a.Q[(long long)j * a.ldq + m] = qf;
+      if (a.P) a.P[(long long)j * a.ldp + m] = __float2half_rn(post * qf);
     } else if (a.P && j < a.rpad) {
       a.P[(long long)j * a.ldp + m] = __float2half_rn(0.f);
     }
@@ -715,7 +743,6 @@ struct Carve {
   float* parts;      // [max_splits][r][max(N, K)]
   float* qn;         // [r][N]
   float* qk;         // [r][K]
-  float* q1;         // [r][max(N, K)]  first CholeskyQR round
   float* ysum;       // [r][max(N, K)]  summed products
   __half* pn;        // [rpad][Np]
   __half* pk;        // [rpad][Kp]
@@ -740,7 +767,6 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
   const size_t o_parts = take((size_t)kMaxSplits * r * MX * 4);
   const size_t o_qn = take((size_t)r * N * 4);
   const size_t o_qk = take((size_t)r * K * 4);
-  const size_t o_q1 = take((size_t)r * MX * 4);
   const size_t o_ys = take((size_t)r * MX * 4);
   const size_t o_pn = take((size_t)rpad * Np * 2);
   const size_t o_pk = take((size_t)rpad * Kp * 2);
@@ -753,7 +779,6 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
     c.parts = reinterpret_cast<float*>(b + o_parts);
     c.qn = reinterpret_cast<float*>(b + o_qn);
     c.qk = reinterpret_cast<float*>(b + o_qk);
-    c.q1 = reinterpret_cast<float*>(b + o_q1);
     c.ysum = reinterpret_cast<float*>(b + o_ys);
     c.pn = reinterpret_cast<__half*>(b + o_pn);
     c.pk = reinterpret_cast<__half*>(b + o_pk);
@@ -824,8 +849,9 @@ ttq_status launch_apply(const ApplyArgs& a, cudaStream_t st) {
   return launch(ls, st, apply_kernel<RT>, a);
 }
 
-// Orthonormal columns of y (the summed, row-scaled parts) by two
-// Gram/Cholesky/apply rounds: Q fp32 [r][M] and the fp16 operand P
+// Orthonormal columns of y (the summed, row-scaled parts) by one
+// Gram/Cholesky/apply round (Cholesky-QR with an fp64 Gram matrix and an
+// fp64 forward substitution): Q fp32 [r][M] and the fp16 operand P
 // [rpad][Mp] = post * Q.
 ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
                   int r, const float* sc, float* Q, __half* P,
@@ -834,44 +860,38 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
   const int64_t Mp = round_up(M, 8);
   const int ctas = (int)std::min<int64_t>(kMaxGramCtas, (M + kGramRows - 1) /
                                                             kGramRows);
-  for (int round = 0; round < 2; ++round) {
-    // round 0 sums the parts into y (kept in c.ysum), round 1 factors the
-    // first round's basis q1
-    GramArgs g;
-    g.parts = round == 0 ? parts : c.q1;
-    g.nparts = round == 0 ? nparts : 1;
-    g.ld = M;
-    g.M = (int)M;
-    g.r = r;
-    g.sc = round == 0 ? sc : nullptr;
-    g.ysum = round == 0 ? c.ysum : nullptr;
-    g.partials = c.partials;
-    g.R = c.R;
-    g.counter = c.counter;
-    g.err = device_error_word();
-    LaunchShape ls;
-    ls.grid = dim3((unsigned)ctas);
-    ls.block = dim3(kGramThreads);
-    ttq_status e = launch(ls, st, gram_kernel, g);
-    if (e != TTQ_OK) return e;
-    ApplyArgs a;
-    a.y = round == 0 ? c.ysum : c.q1;
-    a.ldy = M;
-    a.M = (int)M;
-    a.r = r;
-    a.R = c.R;
-    a.Q = round == 0 ? c.q1 : Q;
-    a.ldq = M;
-    a.P = round == 0 ? nullptr : P;
-    a.ldp = Mp;
-    a.rpad = rpad;
-    a.Mp = (int)(round == 0 ? M : Mp);
-    a.post = round == 0 ? nullptr : post;
-    e = r <= 16 ? launch_apply<16>(a, st)
-        : r <= 32 ? launch_apply<32>(a, st) : launch_apply<64>(a, st);
-    if (e != TTQ_OK) return e;
-  }
-  return TTQ_OK;
+  GramArgs g;
+  g.parts = parts;
+  g.nparts = nparts;
+  g.ld = M;
+  g.M = (int)M;
+  g.r = r;
+  g.sc = sc;
+  g.ysum = c.ysum;
+  g.partials = c.partials;
+  g.R = c.R;
+  g.counter = c.counter;
+  g.err = device_error_word();
+  LaunchShape ls;
+  ls.grid = dim3((unsigned)ctas);
+  ls.block = dim3(kGramThreads);
+  ttq_status e = launch(ls, st, gram_kernel, g);
+  if (e != TTQ_OK) return e;
+  ApplyArgs a;
+  a.y = c.ysum;
+  a.ldy = M;
+  a.M = (int)M;
+  a.r = r;
+  a.R = c.R;
+  a.Q = Q;
+  a.ldq = M;
+  a.P = P;
+  a.ldp = Mp;
+  a.rpad = rpad;
+  a.Mp = (int)Mp;
+  a.post = post;
+  return r <= 16 ? launch_apply<16>(a, st)
+         : r <= 32 ? launch_apply<32>(a, st) : launch_apply<64>(a, st);
 }
 
 template <int RT, int CPT>

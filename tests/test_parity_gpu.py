@@ -220,14 +220,23 @@ def test_fused_quantize_projection_equals_two_passes(ttq, bits, group, T, N,
     ref = ttq.w_lowbit_gemm_prepared(Xs, None, c, d, z, N, bits, group)
     Y, (fc, fd, fz) = ttq.quantize_gemm_prepared(W, s, Xs, None, bits, group)
     torch.cuda.synchronize()
-    assert torch.equal(Y, ref)
     w, G = K * bits // 32, K // group
     assert torch.equal(fc[:, :w], c[:, :w])
     assert torch.equal(fd[:, :G], d[:, :G])
     assert torch.equal(fz[:, :G], z[:, :G])
     Y2, none = ttq.quantize_gemm_prepared(W, s, Xs, None, bits, group,
                                           store_codes=False)
-    assert none is None and torch.equal(Y2, ref)
+    assert none is None and torch.equal(Y2, Y)
+    if T > 256:
+        # several token tiles: the same tiles in the same order, bit for bit
+        assert torch.equal(Y, ref)
+    else:
+        # one token tile: the fused form splits K over a cluster, so the
+        # fp32 sums run in another order; against the oracle's projection
+        ref_o = oracle_y(X.cpu(), inv.cpu(), c.cpu(), d.cpu(), z.cpu(), N,
+                         bits, group)
+        assert_gemm_close(np32(Y), ref_o, "fused, K split", Y.dtype)
+        assert_gemm_close(np32(ref), ref_o, "two passes", ref.dtype)
 
 
 def test_fused_quantize_projection_lowrank_and_oracle(ttq):
