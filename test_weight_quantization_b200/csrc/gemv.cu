@@ -50,20 +50,26 @@ __host__ __device__ constexpr int code_pos(int bits, int i) {
              : ((i * bits) & 31) + bits <= 32 ? ((i * bits) & 31) - 9 : 0;
 }
 
-// q * 2^(pos - 23) for code I (exact).
+// q * 2^(pos - 23) for code I (exact). cwo and cw9o are the code words
+// (and the words shifted right by 9) with the exponent bits of 1.0 already
+// OR-ed in, once per word: since those bits lie outside every field's mask,
+// (w | E) & (mask | E) = (w & mask) | E, and a code in place costs a single
+// AND with one immediate.
 template <int BITS, int I>
 __device__ __forceinline__ float code_val(const uint32_t (&cw)[BITS],
-                                          const uint32_t (&cw9)[BITS]) {
+                                          const uint32_t (&cwo)[BITS],
+                                          const uint32_t (&cw9o)[BITS]) {
   using C = CodeAt<BITS, I>;
+  constexpr uint32_t kOne = 0x3F800000u;
   constexpr uint32_t mask = ((1u << BITS) - 1u) << C::pos;
-  uint32_t src;
+  uint32_t bits;
   if constexpr (C::kind == 0)
-    src = cw[C::wd];
+    bits = cwo[C::wd] & (mask | kOne);
   else if constexpr (C::kind == 1)
-    src = cw9[C::wd];
+    bits = cw9o[C::wd] & (mask | kOne);
   else
-    src = __funnelshift_r(cw[C::wd], cw[C::wd + 1], C::sh);
-  return __fsub_rn(__uint_as_float((src & mask) | 0x3F800000u), 1.f);
+    bits = (__funnelshift_r(cw[C::wd], cw[C::wd + 1], C::sh) & mask) | kOne;
+  return __fsub_rn(__uint_as_float(bits), 1.f);
 }
 
 template <int BITS>
@@ -95,7 +101,8 @@ __device__ __forceinline__ void load_codes(const uint32_t* p,
 // for the NT tokens whose staged (pre-scaled) blocks start at xb[t].
 template <int BITS, int NT, int I, int HI>
 __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
-                                          const uint32_t (&cw9)[BITS],
+                                          const uint32_t (&cwo)[BITS],
+                                          const uint32_t (&cw9o)[BITS],
                                           const float* const (&xb)[NT],
                                           float (&acc)[NT]) {
   if constexpr (I < HI) {
@@ -103,10 +110,10 @@ __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
 #pragma unroll
     for (int t = 0; t < NT; ++t)
       xv[t] = *reinterpret_cast<const float4*>(xb[t] + I);
-    const float f0 = code_val<BITS, I>(cw, cw9);
-    const float f1 = code_val<BITS, I + 1>(cw, cw9);
-    const float f2 = code_val<BITS, I + 2>(cw, cw9);
-    const float f3 = code_val<BITS, I + 3>(cw, cw9);
+    const float f0 = code_val<BITS, I>(cw, cwo, cw9o);
+    const float f1 = code_val<BITS, I + 1>(cw, cwo, cw9o);
+    const float f2 = code_val<BITS, I + 2>(cw, cwo, cw9o);
+    const float f3 = code_val<BITS, I + 3>(cw, cwo, cw9o);
 #pragma unroll
     for (int t = 0; t < NT; ++t) {
       acc[t] = fmaf(f0, xv[t].x, acc[t]);
@@ -114,7 +121,7 @@ __device__ __forceinline__ void dot_range(const uint32_t (&cw)[BITS],
       acc[t] = fmaf(f2, xv[t].z, acc[t]);
       acc[t] = fmaf(f3, xv[t].w, acc[t]);
     }
-    dot_range<BITS, NT, I + 4, HI>(cw, cw9, xb, acc);
+    dot_range<BITS, NT, I + 4, HI>(cw, cwo, cw9o, xb, acc);
   }
 }
 
@@ -209,9 +216,12 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     for (int u = 0; u < U_BLK; ++u) {
       const int bk = ch * 32 * U_BLK + lane + 32 * u;
       if (bk < bpr) {
-        uint32_t cw9[BITS];
+        uint32_t cwo[BITS], cw9o[BITS];
 #pragma unroll
-        for (int w = 0; w < BITS; ++w) cw9[w] = it.cw[u][w] >> 9;
+        for (int w = 0; w < BITS; ++w) {
+          cwo[w] = it.cw[u][w] | 0x3F800000u;
+          cw9o[w] = (it.cw[u][w] >> 9) | 0x3F800000u;
+        }
         const float* xb[NT];
 #pragma unroll
         for (int t = 0; t < NT; ++t) xb[t] = xs_sm + (t * bpr + bk) * kBlkPitch;
@@ -221,8 +231,8 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           float a0[NT], a1[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) a0[t] = a1[t] = 0.f;
-          dot_range<BITS, NT, 0, 16>(it.cw[u], cw9, xb, a0);
-          dot_range<BITS, NT, 16, 32>(it.cw[u], cw9, xb, a1);
+          dot_range<BITS, NT, 0, 16>(it.cw[u], cwo, cw9o, xb, a0);
+          dot_range<BITS, NT, 16, 32>(it.cw[u], cwo, cw9o, xb, a1);
           const float z0 = (float)(it.zz[u] & 0xFFu);
           const float z1 = (float)(it.zz[u] >> 8);
 #pragma unroll
@@ -234,7 +244,7 @@ __global__ void __launch_bounds__(kGvThreads, 1)
           float a[NT];
 #pragma unroll
           for (int t = 0; t < NT; ++t) a[t] = 0.f;
-          dot_range<BITS, NT, 0, 32>(it.cw[u], cw9, xb, a);
+          dot_range<BITS, NT, 0, 32>(it.cw[u], cwo, cw9o, xb, a);
           const float z = (float)it.zz[u];
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
