@@ -24,11 +24,11 @@
 //      The contraction is split over gridDim.y; each split writes its
 //      partial sums, which the next kernel adds in split order.
 //  gram_kernel           partial Gram matrices of y_m = sc_m sum_p parts
-//      (fp32 entries, fp64 products and sums); the last CTA to
-//      arrive adds the partials in CTA order and factors the Gram matrix
-//      (Cholesky with the drop rule) into R, fp64.
-//  apply_kernel          q_m = y_m R^-1 by forward substitution in fp64 (y
-//      as the Gram kernel summed it): Q in fp32,
+//      (fp32 entries, fp64 products and sums), one per CTA.
+//  apply_kernel          every CTA adds the partials in CTA order and
+//      factors the Gram matrix (Cholesky with the drop rule, fp64) into R,
+//      then q_m = y_m R^-1 by forward substitution in fp64 (y as the Gram
+//      kernel summed it): Q in fp32,
 //      and the fp16 operand P = (post_m q_m) of the next product. One
 //      gram/apply round orthonormalises a block of columns: the Gram
 //      matrix is exact up to fp64 sums of exact products, so Q is
@@ -37,7 +37,7 @@
 //  factors_out_kernel    B = bf16(Q_N)^T and A = bf16(sum_p parts).
 //  residual_kernel       R = bf16(W - B A), fp32 accumulation in j order.
 // Every mbarrier wait is bounded (TTQ_DEVERR_TIMEOUT, then the CTA winds
-// down); nothing spins on another CTA (the Gram tail uses an arrival count).
+// down); nothing spins on another CTA.
 #include <algorithm>
 #include <type_traits>
 
@@ -290,13 +290,23 @@ struct GramArgs {
   const float* sc;     // row scales (null: 1)
   float* ysum;         // if not null: the summed, scaled y, [r][ld]
   double* partials;    // [gridDim.x][npairs]
-  double* R;           // [64][64] upper triangular, output
-  unsigned int* counter;
   uint32_t* err;
 };
 
 constexpr int kMaxParts = 16;  // partial products per y (the splits)
 constexpr int kYBatch = 8;     // y entries a thread sums at once
+
+// The (a, b) pairs a <= b of an r x r upper triangle in row order, into
+// shared tables (entry s0(a) + b - a, s0(a) = a r - a (a - 1) / 2).
+__device__ __forceinline__ void pair_tables(int r, uint16_t* pa, uint16_t* pb) {
+  for (int e = threadIdx.x; e < r; e += blockDim.x) {
+    const int s0 = e * r - e * (e - 1) / 2;
+    for (int b = e; b < r; ++b) {
+      pa[s0 + b - e] = (uint16_t)e;
+      pb[s0 + b - e] = (uint16_t)b;
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
   // rows of y (fp32) during the partial sums; the Gram matrix (fp64) in
@@ -305,18 +315,9 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
                                            ? kGramRows * 65 * 4
                                            : 64 * 65 * 8];
   __shared__ uint16_t pa[kMaxPairs], pb[kMaxPairs];
-  __shared__ double diag_max;
-  __shared__ bool is_last;
   griddep_enter();
   const int r = g.r, npairs = r * (r + 1) / 2;
-  for (int e = threadIdx.x; e < r; e += kGramThreads) {
-    // pairs of row a start at a*r - a(a-1)/2
-    const int s0 = e * r - e * (e - 1) / 2;
-    for (int b = e; b < r; ++b) {
-      pa[s0 + b - e] = (uint16_t)e;
-      pb[s0 + b - e] = (uint16_t)b;
-    }
-  }
+  pair_tables(r, pa, pb);
   float* ys = reinterpret_cast<float*>(buf);  // [kGramRows][65]
   constexpr int kPer = (kMaxPairs + kGramThreads - 1) / kGramThreads;
   double acc[kPer];
@@ -402,42 +403,43 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
     const int e = threadIdx.x + q * kGramThreads;
     if (e < npairs) g.partials[(long long)blockIdx.x * npairs + e] = acc[q];
   }
-  // the last CTA to arrive factors the sum of the partials
-  if (threadIdx.x < npairs) __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0)
-    is_last = atomicAdd(g.counter, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  double* G = reinterpret_cast<double*>(buf);  // [64][65], upper part
-  for (int e = threadIdx.x; e < npairs; e += kGramThreads) {
+}
+
+// R (upper, in G[a * ld + b], a <= b) of the Cholesky factorisation with the
+// drop rule of the Gram matrix sum_c partials[c] (nc partials, added in
+// order). Every thread of the CTA takes part; every CTA that runs it on
+// the same partials gets the same R.
+__device__ void factor_gram(const double* __restrict__ partials, int nc,
+                            int r, const uint16_t* pa, const uint16_t* pb,
+                            double* G, int ld, double* diag_max) {
+  const int npairs = r * (r + 1) / 2;
+  for (int e = threadIdx.x; e < npairs; e += blockDim.x) {
     // the CTAs' partials (at most kMaxGramCtas) in CTA order, their loads
     // issued together
-    const int nc = (int)gridDim.x;
     double raw[kMaxGramCtas];
 #pragma unroll
     for (int u = 0; u < kMaxGramCtas; ++u)
-      raw[u] = __ldcg(g.partials + (long long)min(u, nc - 1) * npairs + e);
+      raw[u] = __ldcg(partials + (long long)min(u, nc - 1) * npairs + e);
     double v = 0.0;
 #pragma unroll
     for (int u = 0; u < kMaxGramCtas; ++u)
       if (u < nc) v += raw[u];
-    G[pa[e] * 65 + pb[e]] = v;
+    G[pa[e] * ld + pb[e]] = v;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     double mx = 0.0;
-    for (int j = 0; j < r; ++j) mx = fmax(mx, G[j * 65 + j]);
-    diag_max = mx;
+    for (int j = 0; j < r; ++j) mx = fmax(mx, G[j * ld + j]);
+    *diag_max = mx;
   }
   __syncthreads();
   // right-looking Cholesky, upper factor in place; a column is dropped when
   // its remaining squared norm is at most (tol * largest column norm)^2
-  const double thresh = (double)kDropTol * (double)kDropTol * diag_max;
+  const double dmax = *diag_max;
+  const double thresh = (double)kDropTol * (double)kDropTol * dmax;
   for (int j = 0; j < r; ++j) {
-    const double d = G[j * 65 + j];
-    const bool keep = diag_max > 0.0 && d > thresh;
+    const double d = G[j * ld + j];
+    const bool keep = dmax > 0.0 && d > thresh;
     // 1/sqrt(d): the fp32 estimate refined by two Newton steps in fp64
     // (each squares the relative error: 2^-22 -> 2^-44 -> below fp64's
     // precision), then sqrt(d) = d / sqrt(d); no fp64 divide or square
@@ -454,29 +456,25 @@ __global__ void __launch_bounds__(kGramThreads) gram_kernel(const GramArgs g) {
       rjj = d * rinv;
     }
     __syncthreads();
-    for (int b = j + 1 + threadIdx.x; b < r; b += kGramThreads)
-      G[j * 65 + b] = keep ? G[j * 65 + b] * rinv : 0.0;
-    if (threadIdx.x == 0) G[j * 65 + j] = rjj;
+    for (int b = j + 1 + threadIdx.x; b < r; b += blockDim.x)
+      G[j * ld + b] = keep ? G[j * ld + b] * rinv : 0.0;
+    if (threadIdx.x == 0) G[j * ld + j] = rjj;
     __syncthreads();
     const int rest = r - j - 1;
-    for (int e = threadIdx.x; e < rest * rest; e += kGramThreads) {
+    for (int e = threadIdx.x; e < rest * rest; e += blockDim.x) {
       const int ia = j + 1 + e / rest, ib = j + 1 + e % rest;
-      if (ia <= ib) G[ia * 65 + ib] -= G[j * 65 + ia] * G[j * 65 + ib];
+      if (ia <= ib) G[ia * ld + ib] -= G[j * ld + ia] * G[j * ld + ib];
     }
     __syncthreads();
   }
-  for (int e = threadIdx.x; e < 64 * 64; e += kGramThreads) {
-    const int ia = e / 64, ib = e % 64;
-    g.R[e] = (ia < r && ib < r && ia <= ib) ? G[ia * 65 + ib] : 0.0;
-  }
-  if (threadIdx.x == 0) *g.counter = 0u;  // ready for the next launch
 }
 
 struct ApplyArgs {
   const float* y;      // [r][ldy]: the rows the Gram kernel factored
   long long ldy;
   int M, r;
-  const double* R;
+  const double* partials;  // the Gram kernel's [nc][npairs] partial sums
+  int nc;
   float* Q;            // [r][ldq] or null
   long long ldq;
   __half* P;           // [rpad][ldp] fp16 operand or null
@@ -487,16 +485,21 @@ struct ApplyArgs {
 
 template <int RT>
 __global__ void __launch_bounds__(256) apply_kernel(const ApplyArgs a) {
+  // every CTA factors the Gram matrix itself (no CTA waits for another),
+  // then substitutes its rows
   __shared__ double Rs[RT][RT + 1];
   __shared__ double Rinv[RT];  // 1 / R_jj (0 for a dropped column)
+  __shared__ uint16_t pa[RT * (RT + 1) / 2], pb[RT * (RT + 1) / 2];
+  __shared__ double diag_max;
   griddep_enter();
   const int r = a.r;
-  for (int e = threadIdx.x; e < RT * RT; e += blockDim.x) {
-    const int ia = e / RT, ib = e % RT;
-    const double v = (ia < r && ib < r) ? a.R[ia * 64 + ib] : 0.0;
-    Rs[ia][ib] = v;
-    if (ia == ib) Rinv[ia] = v > 0.0 ? 1.0 / v : 0.0;
-  }
+  pair_tables(r, pa, pb);
+  for (int e = threadIdx.x; e < RT * (RT + 1); e += blockDim.x)
+    (&Rs[0][0])[e] = 0.0;
+  __syncthreads();
+  factor_gram(a.partials, a.nc, r, pa, pb, &Rs[0][0], RT + 1, &diag_max);
+  for (int j = threadIdx.x; j < RT; j += blockDim.x)
+    Rinv[j] = Rs[j][j] > 0.0 ? 1.0 / Rs[j][j] : 0.0;
   __syncthreads();
   const int m = blockIdx.x * blockDim.x + threadIdx.x;
   if (m >= a.Mp) return;
@@ -747,8 +750,6 @@ struct Carve {
   __half* pn;        // [rpad][Np]
   __half* pk;        // [rpad][Kp]
   double* partials;  // [kMaxGramCtas][kMaxPairs]
-  double* R;         // [64][64]
-  unsigned int* counter;
   size_t total;
 };
 
@@ -771,8 +772,6 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
   const size_t o_pn = take((size_t)rpad * Np * 2);
   const size_t o_pk = take((size_t)rpad * Kp * 2);
   const size_t o_part = take((size_t)kMaxGramCtas * kMaxPairs * 8);
-  const size_t o_R = take(64 * 64 * 8);
-  const size_t o_cnt = take(16);
   c.total = off;
   if (ws) {
     uint8_t* b = static_cast<uint8_t*>(ws);
@@ -783,8 +782,6 @@ Carve carve(void* ws, int64_t N, int64_t K, int r) {
     c.pn = reinterpret_cast<__half*>(b + o_pn);
     c.pk = reinterpret_cast<__half*>(b + o_pk);
     c.partials = reinterpret_cast<double*>(b + o_part);
-    c.R = reinterpret_cast<double*>(b + o_R);
-    c.counter = reinterpret_cast<unsigned int*>(b + o_cnt);
   }
   return c;
 }
@@ -869,8 +866,6 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
   g.sc = sc;
   g.ysum = c.ysum;
   g.partials = c.partials;
-  g.R = c.R;
-  g.counter = c.counter;
   g.err = device_error_word();
   LaunchShape ls;
   ls.grid = dim3((unsigned)ctas);
@@ -882,7 +877,8 @@ ttq_status run_qr(const Carve& c, const float* parts, int nparts, int64_t M,
   a.ldy = M;
   a.M = (int)M;
   a.r = r;
-  a.R = c.R;
+  a.partials = c.partials;
+  a.nc = ctas;
   a.Q = Q;
   a.ldq = M;
   a.P = P;
@@ -924,9 +920,6 @@ ttq_status launch_lowrank_factors(const void* W, int64_t N, int64_t K,
   const Carve c = carve(workspace, N, K, r);
   const int rpad = (int)round_up(r, 16);
   const int64_t Kp = round_up(K, 8);
-  // the counter must start at zero; the Gram tail leaves it at zero
-  if (cudaMemsetAsync(c.counter, 0, 16, st) != cudaSuccess)
-    return TTQ_ERR_CUDA;
   {
     LaunchShape ls;
     const long long total = (long long)rpad * Kp;
