@@ -117,7 +117,8 @@ constexpr uint32_t kXchgBytes = 2u * 4u * kBM * 8u;
 // group-range exchange in the fused form); the split-K partial tile
 // (decode); barriers. The fp16 weight stages live in TMEM.
 __host__ __device__ inline Layout make_layout(int bits, int bn, int S,
-                                              bool split, bool qdq = false) {
+                                              bool split, bool qdq = false,
+                                              int extra_bars = 0) {
   Layout L;
   L.stage_x = (uint32_t)(2 * bn * 128);
   L.x = 0;
@@ -127,7 +128,7 @@ __host__ __device__ inline Layout make_layout(int bits, int bn, int S,
   L.bars = L.part + (split ? (uint32_t)(bn * kBM * 4) : 0u);
   // loaded, ready, empty, a_free; params; accumulator; the fused form's
   // group-range exchange (4 lane quarters x 2 stage parities)
-  const int nbars = 3 * S + S + 4 + 1 + (qdq ? 8 : 0);
+  const int nbars = 3 * S + S + 4 + 1 + (qdq ? 8 : 0) + extra_bars;
   L.tmem = L.bars + 8u * nbars;
   L.abort_flag = L.tmem + 4;
   L.total = L.abort_flag + 4;
@@ -995,6 +996,362 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
   if (warp == 1) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
 }
 
+// The prefill projection as a persistent kernel: one CTA per SM walks the
+// output tiles (tile = blockIdx.x + i * gridDim.x, weight tiles fastest),
+// so the TMA ring, the dequantisers and the MMA thread run on without a
+// break between tiles. The accumulator is double-buffered in TMEM and four
+// extra epilogue warps drain tile i (TMEM -> registers -> Y, coalesced
+// across a warp's 32 rows for each token) while the MMAs of tile i+1 run.
+// Roles and stage protocol are those of lowbit_gemm_kernel (codes path,
+// sixteen dequantiser warps, one token tile per CTA at a time); the rings'
+// slots and phases count stages over all of a CTA's tiles.
+constexpr int kPersistEpiWarps = 4;
+constexpr int kPersistBars = 4;  // accumulator full and empty, two buffers
+__host__ __device__ constexpr int persist_threads() {
+  return cta_threads(kPrefillDequantWarps) + 32 * kPersistEpiWarps;
+}
+
+template <int BITS, int GMODE>
+__global__ void __launch_bounds__(persist_threads(), 1)
+    lowbit_gemm_persist_kernel(const __grid_constant__ CUtensorMap tm_x,
+                               const __grid_constant__ CUtensorMap tm_u,
+                               const __grid_constant__ CUtensorMap tm_c,
+                               const __grid_constant__ CUtensorMap tm_d,
+                               const __grid_constant__ CUtensorMap tm_z,
+                               const GemmArgs p) {
+  constexpr int DQW = kPrefillDequantWarps;
+  constexpr int GPB = GMODE == 0 ? 2 : 1;
+  constexpr uint32_t CHUNK = kBM * 16 * BITS;
+  constexpr int kDq = 32 * DQW;
+  constexpr int kEpiWarp0 = kDqWarp0 + DQW;
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* const gbase = smem_raw + (base - raw_base);
+
+  const int S = p.S, SA = p.SA, bn = p.bn;
+  const Layout L = make_layout(BITS, bn, S, false, false, kPersistBars);
+  const uint32_t b_loaded = base + L.bars;
+  const uint32_t b_ready = b_loaded + 8 * S;
+  const uint32_t b_empty = b_ready + 8 * S;
+  const uint32_t b_afree = b_empty + 8 * S;
+  const uint32_t b_full_p = b_afree + 8 * S;
+  const uint32_t b_empty_p = b_full_p + 16;
+  // accumulator buffers: full (MMA -> epilogue), empty (epilogue -> MMA),
+  // after the single-tile form's accumulator barrier
+  const uint32_t b_acc_full = b_empty_p + 16 + 8;
+  const uint32_t b_acc_empty = b_acc_full + 16;
+  volatile uint32_t* tmem_slot =
+      reinterpret_cast<volatile uint32_t*>(gbase + L.tmem);
+  volatile int* aborted = reinterpret_cast<volatile int*>(gbase + L.abort_flag);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_main = p.k_stages;
+  const int n_total = n_main + (p.r > 0 ? 1 : 0);
+  const int lg = 31 - __clz(p.group);
+  const int tiles_m = (p.N + kBM - 1) / kBM;
+  const int n_tiles = tiles_m * ((p.T + bn - 1) / bn);
+  auto tile_of = [&](int it, int& m0, int& t0) -> bool {
+    const int tile = (int)blockIdx.x + it * (int)gridDim.x;
+    if (tile >= n_tiles) return false;
+    m0 = (tile % tiles_m) * kBM;
+    t0 = (tile / tiles_m) * bn;
+    return true;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(b_loaded + 8 * i, 1);
+      mbar_init(b_ready + 8 * i, kDq);
+      mbar_init(b_empty + 8 * i, 1);
+      mbar_init(b_afree + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_full_p + 8 * i, 1);
+      mbar_init(b_empty_p + 8 * i, kDq);
+      mbar_init(b_acc_full + 8 * i, 1);
+      mbar_init(b_acc_empty + 8 * i, 32 * kPersistEpiWarps);
+    }
+    *aborted = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_c);
+    tma_prefetch_desc(&tm_d);
+    tma_prefetch_desc(&tm_z);
+    if (p.r > 0) tma_prefetch_desc(&tm_u);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + L.tmem, (uint32_t)p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  griddep_enter();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_a = tmem + (uint32_t)p.acc_cols;  // weight-stage ring
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer ----
+    if (lane == 0) {
+      const uint32_t xbytes = (uint32_t)bn * 128u;
+      Ring rs, rp;
+      int issued = 0, np = 0, pchunk = -1;
+      bool ok = true;
+      int m0, t0;
+      for (int it = 0; ok && tile_of(it, m0, t0); ++it) {
+        if (pchunk >= 0) rp.next(2);  // a new row tile: a new params chunk
+        pchunk = -1;
+        for (int s = 0; s < n_total; ++s) {
+          const int k0 = s * kSK;
+          if (s < n_main) {
+            const int pc = k0 >> (lg + 4);
+            if (pc != pchunk) {
+              if (pchunk >= 0) rp.next(2);
+              pchunk = pc;
+              if (np >= 2 && !mbar_wait(b_empty_p + 8 * rp.slot,
+                                        (rp.round & 1) ^ 1, p.err)) {
+                ok = false;
+                break;
+              }
+              const uint32_t bar = b_full_p + 8 * rp.slot;
+              const uint32_t dst = base + L.p + rp.slot * kParamBytes;
+              mbar_arrive_expect_tx(bar, kParamBytes);
+              tma_load_2d(dst, &tm_d, pc * kParamGroups, m0, bar);
+              tma_load_2d(dst + kParamDeltaBytes, &tm_z, pc * kParamGroups,
+                          m0, bar);
+              ++np;
+            }
+          }
+          if (issued >= S && !mbar_wait(b_empty + 8 * rs.slot,
+                                        (rs.round & 1) ^ 1, p.err)) {
+            ok = false;
+            break;
+          }
+          if (*aborted) {
+            ok = false;
+            break;
+          }
+          const uint32_t bar = b_loaded + 8 * rs.slot;
+          const uint32_t xdst = base + L.x + rs.slot * L.stage_x;
+          if (s < n_main) {
+            mbar_arrive_expect_tx(bar, CHUNK + 2 * xbytes);
+            tma_load_2d(base + L.c + rs.slot * CHUNK, &tm_c,
+                        (k0 >> 7) * 4 * BITS, m0, bar);
+            tma_load_2d(xdst, &tm_x, k0, t0, bar);
+            tma_load_2d(xdst + xbytes, &tm_x, k0 + 64, t0, bar);
+          } else {
+            mbar_arrive_expect_tx(bar, xbytes);
+            tma_load_2d(xdst, &tm_u, 0, t0, bar);
+          }
+          rs.next(S);
+          ++issued;
+        }
+      }
+      if (!ok) *aborted = 1;
+      // no bulk copy may still be writing shared memory at exit
+      for (int i = 0; i < S && i < issued; ++i) {
+        const int q = issued - 1 - i;
+        mbar_wait(b_loaded + 8 * (q % S), (uint32_t)(q / S) & 1, p.err);
+      }
+      for (int i = 0; i < 2 && i < np; ++i) {
+        const int q = np - 1 - i;
+        mbar_wait(b_full_p + 8 * (q & 1), (uint32_t)(q >> 1) & 1, p.err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer -----
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kBM, bn);
+      const uint32_t xbytes = (uint32_t)bn * 128u;
+      Ring rs, ra;
+      bool ok = true;
+      int m0, t0, it = 0;
+      for (; ok && tile_of(it, m0, t0); ++it) {
+        const int buf = it & 1;
+        // the epilogue has drained this buffer's previous tile
+        if (it >= 2 && !mbar_wait(b_acc_empty + 8 * buf,
+                                  (uint32_t)((it >> 1) - 1) & 1u, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * bn);
+        for (int s = 0; s < n_total; ++s) {
+          if (!mbar_wait(b_ready + 8 * rs.slot, rs.round & 1, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ad = tmem_a + (uint32_t)(ra.slot * kSCols);
+          const uint32_t xs = base + L.x + rs.slot * L.stage_x;
+          const uint64_t bd0 = smem_desc_sw128(xs);
+          const uint64_t bd1 = smem_desc_sw128(xs + xbytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_f16_ts(acc, ad + 8 * k, bd0 + 2 * k, idesc,
+                          (s > 0 || k > 0) ? 1u : 0u);
+          if (s < n_main) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma_f16_ts(acc, ad + 32 + 8 * k, bd1 + 2 * k, idesc, 1u);
+          }
+          tc_commit(b_empty + 8 * rs.slot);
+          tc_commit(b_afree + 8 * ra.slot);
+          rs.next(S);
+          ra.next(SA);
+        }
+        tc_commit(b_acc_full + 8 * buf);  // every MMA of the tile done
+      }
+      if (!ok) *aborted = 1;
+    }
+  } else if (warp < kEpiWarp0) {
+    // ------------------------------------------------ dequantisers ----
+    // One 32-code block of one weight row per thread and stage. A stage's
+    // weights are computed from shared memory before the wait for its TMEM
+    // slot. (Handing a stage to the MMA only after the next one is computed,
+    // to hide the TMEM store wait, measured slower: 392 against 331 us on
+    // the Llama-7B up layer, even when done only while the next stage's
+    // data had already landed; the MMA waits on each stage's hand-over.)
+    const int q4 = warp & 3;
+    const int h = (warp - kDqWarp0) >> 2;   // block of the stage
+    const int i = 32 * q4 + lane;           // row in the tile = TMEM lane
+    const uint32_t crow = base + L.c + i * 16 * BITS;
+    const uint32_t drow = base + L.p + i * 64;
+    const uint32_t dswz = (uint32_t)((i >> 1) & 3);
+    const uint32_t zrow = base + L.p + kParamDeltaBytes + i * 16;
+    const uint32_t arow = tmem_a + ((uint32_t)(32 * q4) << 16);
+    Ring rs, ra, rp;
+    int pchunk = -1, done = 0;
+    bool ok = true;
+    // the TMEM weight slot of this stage is free (the MMA of stage
+    // done - SA completed)
+    auto slot_free = [&]() -> bool {
+      if (done >= SA &&
+          !mbar_wait(b_afree + 8 * ra.slot, (ra.round & 1) ^ 1, p.err))
+        return false;
+      tc_fence_after();
+      return true;
+    };
+    int m0, t0;
+    for (int it = 0; ok && tile_of(it, m0, t0); ++it) {
+      if (pchunk >= 0) rp.next(2);
+      pchunk = -1;
+      const int n = m0 + i;
+      const bool row_ok = n < p.N;
+      for (int s = 0; s < n_total; ++s) {
+        const int k0 = s * kSK;
+        if (!mbar_wait(b_loaded + 8 * rs.slot, rs.round & 1, p.err) ||
+            *aborted) {
+          ok = false;
+          break;
+        }
+        const uint32_t acol = arow + (uint32_t)(ra.slot * kSCols);
+        if (s < n_main) {
+          const int pc = k0 >> (lg + 4);
+          if (pc != pchunk) {
+            if (pchunk >= 0) rp.next(2);
+            pchunk = pc;
+            if (!mbar_wait(b_full_p + 8 * rp.slot, rp.round & 1, p.err)) {
+              ok = false;
+              break;
+            }
+          }
+          const uint32_t poff = rp.slot * kParamBytes;
+          const int gl0 = ((k0 + 32 * h) >> lg) & (kParamGroups - 1);
+          __half2 zsub[GPB], dh[GPB];
+#pragma unroll
+          for (int j = 0; j < GPB; ++j) {
+            const int gl = gl0 + j;
+            const float dl = __uint_as_float(ld_shared_u32(
+                drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
+                4 * (gl & 3)));
+            const uint32_t zj = ld_shared_u8(zrow + poff + gl);
+            dh[j] = __float2half2_rn(dl);
+            zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);
+          }
+          uint32_t o[16];
+          uint32_t cw[BITS];
+          load_block<BITS>(crow + rs.slot * CHUNK + h * 4 * BITS, cw);
+          dequant_block<BITS, GMODE>(cw, zsub, dh, o);
+          // release the params once their last stage is read
+          if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
+            mbar_arrive(b_empty_p + 8 * rp.slot);
+          if (!slot_free()) {
+            ok = false;
+            break;
+          }
+          tmem_st16(acol + 16u * h, o);
+        } else {
+          if (!slot_free()) {
+            ok = false;
+            break;
+          }
+          if (h == 0) {
+            // low-rank stage: row n of B (r <= 64 values) as fp16, zero
+            // padded
+            uint32_t o[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int rho = 2 * e;
+              float lo = 0.f, hi = 0.f;
+              if (row_ok && rho < p.r)
+                lo = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho);
+              if (row_ok && rho + 1 < p.r)
+                hi = load_any(p.Blr, p.blr_t, (long long)n * p.r + rho + 1);
+              o[e] = h2_bits(__floats2half2_rn(lo, hi));
+            }
+            tmem_st32(acol, o);
+          }
+        }
+        // hand the stage to the MMA once its TMEM stores landed
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(b_ready + 8 * rs.slot);
+        rs.next(S);
+        ra.next(SA);
+        ++done;
+      }
+    }
+    if (!ok) *aborted = 1;
+  } else {
+    // -------------------------------------------------- epilogue -------
+    // thread = output row (TMEM lane) of its quarter; per token column the
+    // warp's 32 lanes store 32 consecutive rows of Y
+    const int q4 = warp & 3;
+    const int i = 32 * q4 + lane;
+    const uint32_t t_lane = tmem + ((uint32_t)(32 * q4) << 16);
+    int m0, t0;
+    for (int it = 0; tile_of(it, m0, t0); ++it) {
+      const int buf = it & 1;
+      if (!mbar_wait(b_acc_full + 8 * buf, (uint32_t)(it >> 1) & 1u, p.err))
+        break;
+      tc_fence_after();
+      const int n = m0 + i;
+      const bool ok = !*aborted;
+      for (int j = 0; j < bn; j += 16) {
+        float v[16];
+        tmem_ld16(t_lane + (uint32_t)(buf * bn + j), v);
+        if (ok && n < p.N) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int t = t0 + j + c;
+            if (t < p.T) store_y(p.Y, p.yt, (long long)t * p.ldy + n, v[c]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(b_acc_empty + 8 * buf);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, (uint32_t)p.tmem_cols);
+}
+
 // X~ = fp16(X * inv_s), one thread per 16 channels, K-permuted for PERM.
 template <typename TX, int PERM>
 __global__ void prescale_kernel(const TX* __restrict__ X, int64_t T, int64_t K,
@@ -1121,6 +1478,33 @@ ttq_status launch_kernel(const Maps& m, const GemmArgs& a, dim3 grid,
   ls.smem = smem;
   ls.cluster_z = (unsigned)split;
   return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, m.y, m.w, a);
+}
+
+template <int BITS, int GMODE>
+ttq_status launch_persist(const Maps& m, const GemmArgs& a, unsigned ctas,
+                          size_t smem, cudaStream_t st) {
+  auto kern = lowbit_gemm_persist_kernel<BITS, GMODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return TTQ_ERR_CUDA;
+  LaunchShape ls;
+  ls.grid = dim3(ctas, 1, 1);
+  ls.block = dim3(persist_threads(), 1, 1);
+  ls.smem = smem;
+  return launch(ls, st, kern, m.x, m.u, m.c, m.d, m.z, a);
+}
+
+template <int GMODE>
+ttq_status dispatch_persist(int bits, const Maps& m, const GemmArgs& a,
+                            unsigned ctas, size_t smem, cudaStream_t st) {
+  switch (bits) {
+#define TTQ_LP(B) \
+  case B:         \
+    return launch_persist<B, GMODE>(m, a, ctas, smem, st);
+    TTQ_LP(2) TTQ_LP(3) TTQ_LP(4) TTQ_LP(5) TTQ_LP(6) TTQ_LP(7) TTQ_LP(8)
+#undef TTQ_LP
+  }
+  return TTQ_ERR_INVALID_ARG;
 }
 
 template <int GMODE, int DQW, bool QDQ = false>
@@ -1323,9 +1707,51 @@ ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
       }
     }
   }
+  // The persistent form (four or more output tiles per SM, plain codes, no
+  // fused statistic): two accumulator buffers of bn columns and SA weight
+  // stages share the 512 TMEM columns. The token tile minimises the tiles
+  // per SM times the stage cost of the same model as above. (With fewer
+  // tiles per SM the one-tile-per-CTA grid measured faster: 32.1 against
+  // 38.9 us on 1024 x 6912 x 1152, 13.2 against 24.6 us on 2048 x 2304 x
+  // 768. On the Llama-7B up layer the token tiles 192, 160 and 128
+  // measured 332, 362 and 416 us: a stage costs nearly the same whatever
+  // the tile, so the widest tile that leaves two weight stages wins.)
+  bool persist = false;
+  if (!dual && !q && !stats) {
+    double best = 1e30;
+    int pbn = 0, pS = 0, pSA = 0;
+    for (int c : {192, 160, 128}) {
+      const int sa = std::min(4, (512 - 2 * c) / kSCols);
+      int s_ = 5;
+      while (s_ > 1 && make_layout(bits, c, s_, false, false, kPersistBars)
+                               .total + 1024 > (size_t)kMaxSmem)
+        --s_;
+      if (s_ < 2 || sa < 2) continue;
+      const int64_t tiles = tiles_m * ((T + c - 1) / c);
+      if (tiles < 4 * (int64_t)sms) continue;
+      const int64_t per_sm = (tiles + sms - 1) / sms;
+      const double stage = std::max(8.0 * std::max(45.0, c / 2.0), 600.0);
+      const double t = (double)per_sm * k_stages * stage;
+      if (t < best) {
+        best = t;
+        pbn = c;
+        pS = s_;
+        pSA = std::min(sa, s_);
+      }
+    }
+    if (pbn > 0) {
+      persist = true;
+      bn = pbn;
+      S = pS;
+      SA = pSA;
+      acc_cols = 2 * bn;
+      tmem_cols = 512;
+    }
+  }
   const int per = (k_stages + split - 1) / split;
   split = (k_stages + per - 1) / per;  // every rank gets at least one stage
-  const Layout L = make_layout(bits, bn, S, split > 1, q != nullptr);
+  const Layout L = persist ? make_layout(bits, bn, S, false, false, kPersistBars)
+                           : make_layout(bits, bn, S, split > 1, q != nullptr);
   const size_t smem = L.total + 1024;
   const int64_t tiles_t = (T + bn - 1) / bn;
 
@@ -1365,7 +1791,7 @@ ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
   const int dqw = dual ? 4 : kPrefillDequantWarps;
   const int box_t = (dqw >= 8 && bn >= 32) ? bn / 2 : bn;
   int y_mode = 0;
-  if (split == 1 && ((uint64_t)ldy * dtype_bytes(yt)) % 16 == 0 &&
+  if (!persist && split == 1 && ((uint64_t)ldy * dtype_bytes(yt)) % 16 == 0 &&
       reinterpret_cast<uintptr_t>(Y) % 16 == 0)
     y_mode = (yt != TTQ_F32 && box_t % 32 == 0) ? 2 : 1;
   if (y_mode > 0) {
@@ -1413,6 +1839,12 @@ ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
   a.stats_p = stats_p;
   a.stats_parts = stats_parts_of(dqw, bn);
   a.err = device_error_word();
+  if (persist) {
+    const unsigned ctas =
+        (unsigned)std::min<int64_t>(tiles_m * tiles_t, (int64_t)sms);
+    return group == 16 ? dispatch_persist<0>(bits, m, a, ctas, smem, st)
+                       : dispatch_persist<1>(bits, m, a, ctas, smem, st);
+  }
   const dim3 grid((unsigned)tiles_m, (unsigned)tiles_t, (unsigned)split);
   // decode packs two CTAs per SM with four dequant warps each; prefill runs
   // one CTA per SM with sixteen

@@ -577,6 +577,51 @@ def test_gemm_ragged_k(ttq, K):
                           dtype=Y.dtype)
 
 
+@pytest.mark.parametrize("T,N,K,bits,group,r,out", [
+    (1542, 5770, 640, 4, 128, 0, "bf16"),   # token tile 128
+    (2416, 4657, 640, 3, 32, 0, "f32"),     # token tile 160
+    (2899, 4657, 640, 2, 16, 16, "f16"),    # token tile 192, low-rank stage
+    (2899, 4657, 2304, 5, 128, 0, "bf16"),  # two params chunks per row tile
+    (1542, 5770, 384, 8, 64, 7, "bf16"),
+])
+def test_gemm_many_tiles_per_sm(ttq, T, N, K, bits, group, r, out):
+    """Four or more output tiles per SM: each CTA walks its tiles with a
+    double-buffered accumulator. Ragged N and T, into a pitched Y whose
+    pad columns must stay untouched; every element written (the output is
+    pre-filled with NaN), sampled token rows against the oracle."""
+    X = acts(T, K, 60 + bits, torch.bfloat16)
+    W = weights(N, K, 61 + bits, torch.bfloat16)
+    A = B = None
+    if r:
+        rng = np.random.default_rng(62)
+        A = torch.from_numpy(rng.standard_normal((r, K)).astype(np.float32) *
+                             0.05).to(torch.bfloat16)
+        B = torch.from_numpy(rng.standard_normal((N, r)).astype(np.float32) *
+                             0.05).to(torch.bfloat16)
+    Xg, Wg = X.cuda(), W.cuda()
+    sums = ttq.act_stats(Xg)
+    s, inv = ttq.awq_scales(sums, T)
+    c, d, z = ttq.quantize_rtn_grouped(Wg, s, bits, group)
+    pitch = N + 13
+    big = torch.full((T, pitch), float("nan"), dtype=DT[out], device="cuda")
+    big[:, N:] = 7.0
+    Y = big[:, :N]
+    ttq.w_lowbit_gemm(Xg, inv, c, d, z, N, bits, group,
+                      None if A is None else A.cuda(),
+                      None if B is None else B.cuda(), out=Y)
+    torch.cuda.synchronize()
+    assert not torch.isnan(Y).any(), "output elements left unwritten"
+    assert torch.all(big[:, N:] == 7.0)
+    rng = np.random.default_rng(63)
+    rows = np.unique(np.concatenate([
+        rng.choice(T, 40, replace=False), np.arange(T - 8, T), [0, 127, 128,
+                                                               159, 160, 191,
+                                                               192]]))
+    ref = oracle_y(X, inv, c, d, z, N, bits, group, A, B, rows=rows)
+    assert_gemm_close(np32(Y)[rows], ref, f"T={T} N={N} K={K} b={bits}",
+                      Y.dtype)
+
+
 @pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("xin", ["f32", "bf16", "f16"])
 def test_gemm_dtypes(ttq, xin, out):
