@@ -261,6 +261,14 @@ __device__ __forceinline__ void dequant_block(const uint32_t (&cw)[BITS],
   for (int pp = 0; pp < 16; ++pp) o[pp] = h2_bits(__hmul2(t[pp], dh[grp(pp)]));
 }
 
+// One arrival on `bar` for the whole warp, made by lane 0 once every lane
+// has come here: a barrier then counts warps, not threads, and takes one
+// shared-memory update per warp instead of 32.
+__device__ __forceinline__ void warp_arrive(uint32_t bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Position in a ring of `depth` slots: the slot and how many times the
 // ring has wrapped (its parity is the mbarrier phase of the slot's use).
 struct Ring {
@@ -278,8 +286,8 @@ struct Ring {
 //   producer   waits `empty` (previous use done), then loads the codes
 //              chunk and both activation boxes, completing on `loaded`;
 //   dequant    waits `loaded`, writes the fp16 weight stage to TMEM, then
-//              arrives on `ready` (this also vouches that the activations
-//              have landed, since it observed `loaded`);
+//              arrives on `ready`, once per warp (this also vouches that
+//              the activations have landed, since it observed `loaded`);
 //   MMA        waits `ready`, issues 8 MMAs, commits to `empty`, which frees
 //              the codes, the activations and the TMEM weight stage at once.
 // GMODE: 0 -> g = 16 (a 32-code block spans 2 groups), 1 -> g >= 32.
@@ -300,7 +308,6 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
                        const GemmArgs p) {
   constexpr int GPB = GMODE == 0 ? 2 : 1;  // groups per 32-code block
   constexpr uint32_t CHUNK = QDQ ? kWStageBytes : kBM * 16 * BITS;
-  constexpr int kDq = 32 * DQW;            // dequantiser threads
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -336,13 +343,13 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(b_loaded + 8 * i, 1);
-      mbar_init(b_ready + 8 * i, kDq);
+      mbar_init(b_ready + 8 * i, DQW);
       mbar_init(b_empty + 8 * i, 1);
       mbar_init(b_afree + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
-      mbar_init(b_empty_p + 8 * i, kDq);
+      mbar_init(b_empty_p + 8 * i, DQW);
     }
     mbar_init(b_accum, 1);
     if constexpr (QDQ) {
@@ -731,7 +738,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
         }
         // release the params once their last stage is read
         if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
-          mbar_arrive(b_empty_p + 8 * rp.slot);
+          warp_arrive(b_empty_p + 8 * rp.slot);
         }
       } else {
         // low-rank stage: row n of B (r <= 64 values) as fp16, zero padded
@@ -752,7 +759,7 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(b_ready + 8 * rs.slot);
+      warp_arrive(b_ready + 8 * rs.slot);
       rs.next(S);
       ra.next(SA);
     }
@@ -1022,7 +1029,6 @@ __global__ void __launch_bounds__(persist_threads(), 1)
   constexpr int DQW = kPrefillDequantWarps;
   constexpr int GPB = GMODE == 0 ? 2 : 1;
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
-  constexpr int kDq = 32 * DQW;
   constexpr int kEpiWarp0 = kDqWarp0 + DQW;
 
   extern __shared__ uint8_t smem_raw[];
@@ -1064,15 +1070,15 @@ __global__ void __launch_bounds__(persist_threads(), 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(b_loaded + 8 * i, 1);
-      mbar_init(b_ready + 8 * i, kDq);
+      mbar_init(b_ready + 8 * i, DQW);
       mbar_init(b_empty + 8 * i, 1);
       mbar_init(b_afree + 8 * i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(b_full_p + 8 * i, 1);
-      mbar_init(b_empty_p + 8 * i, kDq);
+      mbar_init(b_empty_p + 8 * i, DQW);
       mbar_init(b_acc_full + 8 * i, 1);
-      mbar_init(b_acc_empty + 8 * i, 32 * kPersistEpiWarps);
+      mbar_init(b_acc_empty + 8 * i, kPersistEpiWarps);
     }
     *aborted = 0;
     fence_barrier_init();
@@ -1278,7 +1284,7 @@ __global__ void __launch_bounds__(persist_threads(), 1)
           dequant_block<BITS, GMODE>(cw, zsub, dh, o);
           // release the params once their last stage is read
           if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
-            mbar_arrive(b_empty_p + 8 * rp.slot);
+            warp_arrive(b_empty_p + 8 * rp.slot);
           if (!slot_free()) {
             ok = false;
             break;
@@ -1309,7 +1315,7 @@ __global__ void __launch_bounds__(persist_threads(), 1)
         // hand the stage to the MMA once its TMEM stores landed
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(b_ready + 8 * rs.slot);
+        warp_arrive(b_ready + 8 * rs.slot);
         rs.next(S);
         ra.next(SA);
         ++done;
@@ -1343,7 +1349,7 @@ __global__ void __launch_bounds__(persist_threads(), 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(b_acc_empty + 8 * buf);
+      warp_arrive(b_acc_empty + 8 * buf);
     }
   }
 
