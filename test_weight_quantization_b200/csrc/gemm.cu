@@ -1010,12 +1010,19 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
 // extra epilogue warps drain tile i (TMEM -> registers -> Y, coalesced
 // across a warp's 32 rows for each token) while the MMAs of tile i+1 run.
 // Roles and stage protocol are those of lowbit_gemm_kernel (codes path,
-// sixteen dequantiser warps, one token tile per CTA at a time); the rings'
-// slots and phases count stages over all of a CTA's tiles.
+// one token tile per CTA at a time); the rings' slots and phases count
+// stages over all of a CTA's tiles.
 constexpr int kPersistEpiWarps = 4;
 constexpr int kPersistBars = 4;  // accumulator full and empty, two buffers
+// Eight dequantiser warps, two 32-code blocks per thread and stage. (Sixteen
+// warps with one block each measured 327 against 318 us on the Llama-7B up
+// layer, 351 against 324 us at b = 2, g = 16: per stage the fixed work of
+// a warp, its waits and bookkeeping, weighs as much as a block's
+// arithmetic, and issue slots are the busiest resource. Four warps with
+// four blocks each were slower again for b = 2, 3 and 8.)
+constexpr int kPersistDequantWarps = 8;
 __host__ __device__ constexpr int persist_threads() {
-  return cta_threads(kPrefillDequantWarps) + 32 * kPersistEpiWarps;
+  return cta_threads(kPersistDequantWarps) + 32 * kPersistEpiWarps;
 }
 
 template <int BITS, int GMODE>
@@ -1026,7 +1033,8 @@ __global__ void __launch_bounds__(persist_threads(), 1)
                                const __grid_constant__ CUtensorMap tm_d,
                                const __grid_constant__ CUtensorMap tm_z,
                                const GemmArgs p) {
-  constexpr int DQW = kPrefillDequantWarps;
+  constexpr int DQW = kPersistDequantWarps;
+  constexpr int NB = 16 / DQW;  // 32-code blocks per thread and stage
   constexpr int GPB = GMODE == 0 ? 2 : 1;
   constexpr uint32_t CHUNK = kBM * 16 * BITS;
   constexpr int kEpiWarp0 = kDqWarp0 + DQW;
@@ -1215,14 +1223,14 @@ __global__ void __launch_bounds__(persist_threads(), 1)
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------------------------ dequantisers ----
-    // One 32-code block of one weight row per thread and stage. A stage's
+    // Two 32-code blocks of one weight row per thread and stage. A stage's
     // weights are computed from shared memory before the wait for its TMEM
     // slot. (Handing a stage to the MMA only after the next one is computed,
     // to hide the TMEM store wait, measured slower: 392 against 331 us on
     // the Llama-7B up layer, even when done only while the next stage's
     // data had already landed; the MMA waits on each stage's hand-over.)
     const int q4 = warp & 3;
-    const int h = (warp - kDqWarp0) >> 2;   // block of the stage
+    const int h = (warp - kDqWarp0) >> 2;   // blocks NB h .. NB h + NB - 1
     const int i = 32 * q4 + lane;           // row in the tile = TMEM lane
     const uint32_t crow = base + L.c + i * 16 * BITS;
     const uint32_t drow = base + L.p + i * 64;
@@ -1266,22 +1274,26 @@ __global__ void __launch_bounds__(persist_threads(), 1)
             }
           }
           const uint32_t poff = rp.slot * kParamBytes;
-          const int gl0 = ((k0 + 32 * h) >> lg) & (kParamGroups - 1);
-          __half2 zsub[GPB], dh[GPB];
+          uint32_t o[16 * NB];
 #pragma unroll
-          for (int j = 0; j < GPB; ++j) {
-            const int gl = gl0 + j;
-            const float dl = __uint_as_float(ld_shared_u32(
-                drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
-                4 * (gl & 3)));
-            const uint32_t zj = ld_shared_u8(zrow + poff + gl);
-            dh[j] = __float2half2_rn(dl);
-            zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);
+          for (int b = 0; b < NB; ++b) {
+            const int blk = NB * h + b;
+            const int gl0 = ((k0 + 32 * blk) >> lg) & (kParamGroups - 1);
+            __half2 zsub[GPB], dh[GPB];
+#pragma unroll
+            for (int j = 0; j < GPB; ++j) {
+              const int gl = gl0 + j;
+              const float dl = __uint_as_float(ld_shared_u32(
+                  drow + poff + ((((uint32_t)gl >> 2) ^ dswz) << 4) +
+                  4 * (gl & 3)));
+              const uint32_t zj = ld_shared_u8(zrow + poff + gl);
+              dh[j] = __float2half2_rn(dl);
+              zsub[j] = bits_h2((0x6400u | zj) * 0x00010001u);
+            }
+            uint32_t cw[BITS];
+            load_block<BITS>(crow + rs.slot * CHUNK + blk * 4 * BITS, cw);
+            dequant_block<BITS, GMODE>(cw, zsub, dh, o + 16 * b);
           }
-          uint32_t o[16];
-          uint32_t cw[BITS];
-          load_block<BITS>(crow + rs.slot * CHUNK + h * 4 * BITS, cw);
-          dequant_block<BITS, GMODE>(cw, zsub, dh, o);
           // release the params once their last stage is read
           if (s + 1 >= n_main || ((k0 + kSK) >> (lg + 4)) != pc)
             warp_arrive(b_empty_p + 8 * rp.slot);
@@ -1289,7 +1301,8 @@ __global__ void __launch_bounds__(persist_threads(), 1)
             ok = false;
             break;
           }
-          tmem_st16(acol + 16u * h, o);
+          static_assert(NB == 2, "one 32-column TMEM store per thread");
+          tmem_st32(acol + 32u * h, o);
         } else {
           if (!slot_free()) {
             ok = false;
