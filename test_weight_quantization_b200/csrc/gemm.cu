@@ -1733,7 +1733,7 @@ ttq_status launch_gemm_impl(const void* Xs, const void* U, int64_t T,
   // tiles per SM the one-tile-per-CTA grid measured faster: 32.1 against
   // 38.9 us on 1024 x 6912 x 1152, 13.2 against 24.6 us on 2048 x 2304 x
   // 768. On the Llama-7B up layer the token tiles 192, 160 and 128
-  // measured 332, 362 and 416 us: a stage costs nearly the same whatever
+  // measured 322, 356 and 418 us: a stage costs nearly the same whatever
   // the tile, so the widest tile that leaves two weight stages wins.)
   bool persist = false;
   if (!dual && !q && !stats) {
