@@ -622,6 +622,29 @@ def test_gemm_many_tiles_per_sm(ttq, T, N, K, bits, group, r, out):
                       Y.dtype)
 
 
+@pytest.mark.parametrize("out", ["bf16", "f32"])
+def test_gemm_persistent_matches_one_tile_grid(ttq, out):
+    """The persistent form (here 4096 tokens, 86 x 22 tiles) and the
+    one-tile-per-CTA grid (the first 192 tokens alone: one token tile of the
+    same width) run the same MMAs in the same order for a tile, so the
+    first 192 rows of Y agree bit for bit. Both runs are deterministic."""
+    T, N, K, bits, group = 4096, 11008, 512, 4, 128
+    X = acts(T, K, 71, torch.bfloat16).cuda()
+    W = weights(N, K, 72, torch.bfloat16).cuda()
+    sums = ttq.act_stats(X)
+    s, inv = ttq.awq_scales(sums, T)
+    c, d, z = ttq.quantize_rtn_grouped(W, s, bits, group)
+    Y = ttq.w_lowbit_gemm(X, inv, c, d, z, N, bits, group,
+                          out_dtype=DT[out])
+    Y2 = ttq.w_lowbit_gemm(X, inv, c, d, z, N, bits, group,
+                           out_dtype=DT[out])
+    Y192 = ttq.w_lowbit_gemm(X[:192].contiguous(), inv, c, d, z, N, bits,
+                             group, out_dtype=DT[out])
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    assert torch.equal(Y[:192], Y192)
+
+
 @pytest.mark.parametrize("out", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("xin", ["f32", "bf16", "f16"])
 def test_gemm_dtypes(ttq, xin, out):
