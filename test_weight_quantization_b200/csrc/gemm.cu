@@ -1018,8 +1018,9 @@ constexpr int kPersistBars = 4;  // accumulator full and empty, two buffers
 // warps with one block each measured 327 against 318 us on the Llama-7B up
 // layer, 351 against 324 us at b = 2, g = 16: per stage the fixed work of
 // a warp, its waits and bookkeeping, weighs as much as a block's
-// arithmetic, and issue slots are the busiest resource. Four warps with
-// four blocks each were slower again for b = 2, 3 and 8.)
+// arithmetic, and sixteen warps kept 68 % of the issue slots busy against
+// 55 % for eight. Four warps with four blocks each were slower again for
+// b = 2, 3 and 8.)
 constexpr int kPersistDequantWarps = 8;
 __host__ __device__ constexpr int persist_threads() {
   return cta_threads(kPersistDequantWarps) + 32 * kPersistEpiWarps;
