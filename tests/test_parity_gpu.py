@@ -458,6 +458,42 @@ def oracle_y(X, inv, c, d, z, N, bits, group, A=None, B=None, rows=None):
                               None if B is None else np32(B), rows=rows)
 
 
+def _prepared_order(bits):
+    """Position p of a 16-channel span of the prepared operand holds channel
+    order[p] of the span: the pairing of the fp16 weight pairs that b-bit
+    code words unpack to (codes 8, 4 or 2 channels apart for b = 2, 4, 8),
+    the layout ttq.h documents for the prepared activations."""
+    p = np.arange(16)
+    if bits == 2:
+        return (p >> 1) + 8 * (p & 1)
+    if bits == 4:
+        return 8 * (p >> 3) + ((p & 7) >> 1) + 4 * (p & 1)
+    if bits == 8:
+        return 4 * (p >> 2) + ((p & 3) >> 1) + 2 * (p & 1)
+    return p
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("dt", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("T,K,pad", [(37, 288, 32), (300, 2080, 0)])
+def test_prepare_activations_exact(ttq, bits, dt, T, K, pad):
+    """Xs = fp16(fp32(X) * inv_s): one fp32 product rounded to fp16, bit for
+    bit, in the channel order of the code width; rows of X with a pitch."""
+    X = acts(T, K + pad, 80 + bits, DT[dt])
+    rng = np.random.default_rng(81)
+    inv = (rng.uniform(0.25, 4.0, K)).astype(np.float32)
+    Xg = X.cuda()[:, :K]
+    Xs, _ = ttq.prepare_activations(Xg, torch.from_numpy(inv).cuda(), bits)
+    torch.cuda.synchronize()
+    xf = X[:, :K].float().numpy()
+    ref = (xf * inv[None, :]).astype(np.float32).astype(np.float16)
+    order = _prepared_order(bits)
+    idx = (np.arange(K) // 16) * 16 + order[np.arange(K) % 16]
+    ref = ref[:, idx]
+    got = Xs.cpu().numpy()
+    np.testing.assert_array_equal(got.view(np.uint16), ref.view(np.uint16))
+
+
 @pytest.mark.parametrize("T", [1, 4, 16, 17, 100, 300])
 @pytest.mark.parametrize("bits,group", [(4, 128), (3, 32), (2, 16), (5, 64)])
 def test_gemm_shapes(ttq, T, bits, group):
