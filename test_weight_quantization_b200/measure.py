@@ -139,6 +139,13 @@ def stats(T, K):
                    for X in Xr])
     report(f"stats+scales   T={T:5d} K={K:6d}", us, T * K * 2 + K * 12)
 
+    def two(X):
+        ttq.act_stats(X, 2.0, out=sums)
+        ttq.awq_scales(sums, T, 0.5, 0.1, 2.0, s, inv)
+    us = graph_us([lambda X=X: two(X) for X in Xr])
+    report(f"stats, scales  T={T:5d} K={K:6d} (two launches)", us,
+           T * K * 2 + K * 12)
+
 
 def prepare(T, K, bits):
     Xr = [acts(T, K)]
