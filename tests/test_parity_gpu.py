@@ -619,6 +619,8 @@ def test_gemm_ragged_k(ttq, K):
     (2899, 4657, 640, 2, 16, 16, "f16"),    # token tile 192, low-rank stage
     (2899, 4657, 2304, 5, 128, 0, "bf16"),  # two params chunks per row tile
     (1542, 5770, 384, 8, 64, 7, "bf16"),
+    (1542, 5770, 672, 3, 32, 0, "bf16"),    # ragged last K stage
+    (2416, 4657, 4160, 4, 64, 16, "f32"),   # ragged K, 5 params chunks
 ])
 def test_gemm_many_tiles_per_sm(ttq, T, N, K, bits, group, r, out):
     """Four or more output tiles per SM: each CTA walks its tiles with a
