@@ -249,11 +249,8 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
   uint32_t cw[BITS];
 #pragma unroll
   for (int i = 0; i < BITS; ++i) cw[i] = 0u;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const int gi = e / E;
-    const float t =
-        fmaxf(fminf(__fmaf_rn(w[e], r[gi], kMagic), topz[gi]), botz[gi]);
+  auto put = [&](int e, int gi, float m) {
+    const float t = fmaxf(fminf(m, topz[gi]), botz[gi]);
     const uint32_t tb = __float_as_uint(t);  // bits(M) + q - z
     const int bit = e * BITS, wd = bit >> 5, sh = bit & 31;
     if (sh + BITS <= 32) {
@@ -263,6 +260,17 @@ __device__ __forceinline__ void quantize_item(const QuantCtx& c,
       cw[wd] += q << sh;
       cw[wd + 1] += q >> (32 - sh);
     }
+  };
+  // M + w r, two correctly rounded fused multiply-adds per instruction
+  // (E is even, so a pair never straddles two groups)
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const int gi = e / E;
+    const float2 m = __ffma2_rn(make_float2(w[e], w[e + 1]),
+                                make_float2(r[gi], r[gi]),
+                                make_float2(kMagic, kMagic));
+    put(e, gi, m.x);
+    put(e + 1, gi, m.y);
   }
   const uint32_t z0 = (uint32_t)zf[0], z1 = (uint32_t)zf[NG - 1];
 #pragma unroll
