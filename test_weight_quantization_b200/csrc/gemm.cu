@@ -722,6 +722,11 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
           dequant_block<BITS, GMODE>(cw, zsub, dh, o);
           tmem_st16(acol + 16u * h, o);
         } else {
+        // a thread's blocks are consecutive in K: the params are loaded
+        // again only where a block starts a new group (every block for
+        // g = 16). Decode at 16 tokens, 14336 x 4096, b = 4, g = 128:
+        // 20.9 against 22.8 us on one box.
+        __half2 zsub[GPB], dh[GPB];
 #pragma unroll
         for (int half = half_lo; half < half_hi; ++half) {
           uint32_t o[32];
@@ -730,8 +735,9 @@ __global__ void __launch_bounds__(cta_threads(DQW), DQW >= 16 ? 1 : 2)
             const int blk = 2 * half + h;  // 32-code block of the stage
             uint32_t cw[BITS];
             load_block<BITS>(cbase + blk * 4 * BITS, cw);
-            __half2 zsub[GPB], dh[GPB];
-            block_params(blk, zsub, dh);
+            if (GMODE == 0 || blk == 2 * half_lo ||
+                ((32 * blk) & (p.group - 1)) == 0)
+              block_params(blk, zsub, dh);
             dequant_block<BITS, GMODE>(cw, zsub, dh, o + 16 * h);
           }
           tmem_st32(acol + 32u * half, o);
